@@ -1,0 +1,57 @@
+"""Oracle: whole-volume decoding of one shape (dense grid or coarse-to-fine).
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).
+
+Wires ``decoder``, ``hierarchy`` and ``adaptive`` together for one shape of a
+workload: the VAE decode stage of the pipeline (techwalker article, section 1:
+image encoding -> diffusion sampling -> VAE decoding -> surface extraction).
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import numpy as np
+
+from . import adaptive as A
+from . import decoder as D
+from . import hierarchy as HV
+
+
+def shape_kv(z: np.ndarray, w: Dict[str, np.ndarray]):
+    """K, V ``[H,N,64]`` of one shape's vecset ``z[N,C]``."""
+    return D.precompute_kv(z, w)
+
+
+def dense_grid(K, V, w, R: int, query_ln: bool, spheres=None, dec_scale: float = 0.0,
+               idx: Optional[np.ndarray] = None) -> np.ndarray:
+    """Field (or raw decoder output without spheres) at grid voxels ``idx``
+    (all R^3 voxels by default), float64."""
+    p = D.grid_points(R, idx)
+    dec = D.decode_points(p, K, V, w, query_ln)
+    return D.field(p, dec, spheres, dec_scale)
+
+
+def hierarchical_volume(K, V, w, r0: int, n_levels: int, query_ln: bool, spheres=None,
+                        dec_scale: float = 0.0, adaptive: bool = False, seed: int = 0,
+                        tile: int = 8, n_probe: int = 64, top_k: int = 1024,
+                        coarse: Optional[np.ndarray] = None, keep_tiles: bool = False) -> Dict:
+    """Hierarchical decoding of one shape, optionally with adaptive KV on the
+    fine levels.  Returns ``hierarchy.hierarchical``'s dict plus, per fine
+    level, the raw decoder outputs (``dec``) and adaptive tile records."""
+    extras = {}
+
+    def decode_level(level: int, R: int, idx: np.ndarray) -> np.ndarray:
+        p = D.grid_points(R, idx)
+        if level == 0 or not adaptive:
+            dec = D.decode_points(p, K, V, w, query_ln)
+            extras[level] = {"dec": dec}
+            return D.field(p, dec, spheres, dec_scale)
+        out = A.adaptive_level(level, R, idx, K, V, w, query_ln, spheres, dec_scale, seed,
+                               tile=tile, n_probe=n_probe, k=top_k, keep_tiles=keep_tiles)
+        extras[level] = out
+        return out["values"]
+
+    res = HV.hierarchical(decode_level, r0, n_levels, coarse=coarse)
+    for lv, e in extras.items():
+        res["levels"][lv].update({k: v for k, v in e.items() if k != "values"})
+    return res
