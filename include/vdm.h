@@ -1,0 +1,237 @@
+/*
+ * vdm.h -- C ABI of the B200 vecset SDF decoder ("lightning vecset decoder").
+ *
+ * A vecset is an unordered set of N latent tokens of width C that encodes one
+ * shape; its decoder is a cross-attention from 3D query points to the token
+ * set followed by the signed distance (SDF) at each point (FlashVDM,
+ * "Unleashing Vecset Diffusion Model for Fast Shape Generation", aipaper.cc
+ * summary, section 3 "foundational concepts: decoder").  Decoding a volume
+ * means running that cross-attention for millions of grid points, which the
+ * pages name the dominant cost of shape generation (section 2; techwalker
+ * article, section 1: VAE decoding is 75.8% of end-to-end time).  The three
+ * accelerations of section 4.1 are exposed here:
+ *   1. hierarchical volume decoding (coarse pass, sign-change + near-surface
+ *      marking, one dilation, refinement of the marked voxels only);
+ *   2. adaptive KV selection (per sub-volume probe queries rank the tokens,
+ *      the rest of the sub-volume attends to the Top-K tokens only);
+ *   3. the efficient (slim) decoder: any width C = 64 H, MLP width F, and the
+ *      query-side LayerNorms optional (query_ln = 0).
+ *
+ * Decoder network, per query point p (W[out][in] row-major, y = x W^T + b):
+ *   pe  = [p, sin(2^k pi p_a), cos(2^k pi p_a)]  k = 0..7; lane 3+8a+k = sin,
+ *         lane 27+8a+k = cos, lanes 51..63 = 0 (64 lanes)
+ *   q   = Wq pe + bq                                        Wq: [C][64]
+ *   K,V = LN_kv(z) Wk^T + bk, LN_kv(z) Wv^T + bv, split into H heads of 64
+ *   a_h = softmax(q_h K_h^T / 8) V_h  (dense, or over a token subset)
+ *   x1  = q + Wo a + bo
+ *   x2  = x1 + W2 GELU(W1 LN1(x1) + b1) + b2                (LN1 iff query_ln)
+ *   dec = w_head . LN2(x2) + b_head                         (LN2 iff query_ln)
+ * LayerNorm: biased variance, eps 1e-5.  GELU: exact erf form.
+ * Optional analytic term (synthetic shapes): field = min_s(|p - c_s| - r_s)
+ *   + dec_scale * tanh(dec); without it the output is dec itself.
+ * Grid: voxel (i,j,k) of an R^3 grid sits at -1 + (2i+1)/R per axis; linear
+ *   index (i R + j) R + k (x slowest).  Children of a voxel at 2R: (2i+di, ...).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named d_* / documented "device" are CUDA device memory owned by
+ *     the caller; the library never allocates device memory.  Host pointers
+ *     are documented as such.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL =
+ *     legacy default stream), except vdm_decode_hierarchical which reads one
+ *     small count back per level (documented there).
+ *   - Errors are returned as vdm_status; nothing aborts, throws across the
+ *     ABI or traps on the device.  vdm_last_error() gives a thread-local
+ *     message for the last failing call.  Launch failures return VDM_ERR_CUDA.
+ *   - Results are bit-identical run to run (no floating-point atomics).
+ *   - Limits: head dim 64; C in {64, 128, 256, 512}; F a multiple of 64 and
+ *     <= 4096; 1 <= N <= 8192; B >= 1.  Other shapes: VDM_ERR_UNSUPPORTED.
+ */
+#ifndef VDM_H
+#define VDM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define VDM_API __attribute__((visibility("default")))
+#else
+#define VDM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* vdm_stream; /* == cudaStream_t */
+
+typedef enum {
+    VDM_OK = 0,
+    VDM_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, negative size ... */
+    VDM_ERR_UNSUPPORTED = 2,   /* shape outside the limits above */
+    VDM_ERR_WORKSPACE = 3,     /* workspace missing or too small */
+    VDM_ERR_CUDA = 4,          /* a CUDA call or launch failed */
+    VDM_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up */
+    VDM_ERR_INTERNAL = 6
+} vdm_status;
+
+typedef enum { VDM_F32 = 0, VDM_BF16 = 1 } vdm_dtype;
+
+#define VDM_HEAD_DIM 64
+#define VDM_PE_LANES 64
+#define VDM_MAX_LEVELS 6
+
+/* Decoder parameters (all device pointers).  Matrices are stored in `dtype`
+ * (float or bf16), row-major W[out][in]; vectors are float32.  K and V
+ * produced by vdm_precompute_kv are stored in `dtype` as well.              */
+typedef struct {
+    int32_t C;          /* width, = 64 * H                                   */
+    int32_t H;          /* heads                                             */
+    int32_t F;          /* MLP hidden width                                  */
+    int32_t query_ln;   /* 1: LayerNorm before the MLP and before the head   */
+    vdm_dtype dtype;
+    const void* Wq;     /* [C][64]; columns 51..63 meet zero embedding lanes */
+    const void* Wk;     /* [C][C] */
+    const void* Wv;     /* [C][C] */
+    const void* Wo;     /* [C][C] */
+    const void* W1;     /* [F][C] */
+    const void* W2;     /* [C][F] */
+    const float *bq, *bk, *bv, *bo, *b1, *b2;            /* [C] ([F] for b1) */
+    const float *ln_kv_g, *ln_kv_b;                      /* [C]              */
+    const float *ln1_g, *ln1_b, *ln2_g, *ln2_b;          /* [C]              */
+    const float* w_head;                                 /* [C]              */
+    const float* b_head;                                 /* [1]              */
+} vdm_decoder;
+
+/* Analytic term of the synthetic field (optional).                         */
+typedef struct {
+    const float* spheres;  /* device [B][n_spheres][4] = (cx, cy, cz, r)     */
+    int32_t n_spheres;     /* >= 1                                           */
+    float dec_scale;       /* field = sphere SDF + dec_scale * tanh(dec)     */
+} vdm_analytic;
+
+/* K/V projection of B vecsets (section 3: the vecset feeds the decoder's
+ * cross-attention as keys and values).
+ *   d_z     [B][N][C] float32 latents
+ *   d_k_out [B][H][N][64] in dec->dtype  (keys)
+ *   d_v_out [B][H][N][64] in dec->dtype  (values)
+ * Errors: INVALID_ARG (null pointer, B/N < 1), UNSUPPORTED (limits).        */
+VDM_API vdm_status vdm_precompute_kv(const vdm_decoder* dec, const float* d_z, int32_t B, int32_t N,
+                             void* d_k_out, void* d_v_out, vdm_stream stream);
+
+/* Dense decode: the decoder at M points per shape, full attention over all
+ * N tokens (section 3; the plain "baseline" decoder of Table 3).
+ *   d_k, d_v  [B][H][N][64] from vdm_precompute_kv
+ *   d_xyz     [B][M][3] float32 points, or NULL: the points are the voxels of
+ *             the grid_R^3 grid in linear order (then M must be grid_R^3)
+ *   analytic  host pointer or NULL (raw decoder output)
+ *   d_out     [B][M] float32
+ * M = 0 is a no-op.  Errors: INVALID_ARG, UNSUPPORTED, CUDA.                */
+VDM_API vdm_status vdm_decode_dense(const vdm_decoder* dec, const void* d_k, const void* d_v,
+                            int32_t B, int32_t N, const float* d_xyz, int64_t M, int32_t grid_R,
+                            const vdm_analytic* analytic, float* d_out, vdm_stream stream);
+
+/* Adaptive KV selection for T sub-volumes of one shape (section 4.1 item 2,
+ * steps 2-4): the probe queries of sub-volume t are
+ * d_probe_xyz[d_tile_off[t] .. d_tile_off[t+1]); every token gets the score
+ * sum over probes and heads of its softmax weight, and the top_k tokens (ties
+ * to the smaller index) are written in ascending index order.
+ *   d_probe_xyz   [P][3] float32, P = d_tile_off[T]
+ *   d_tile_off    [T+1] int32, non-decreasing, d_tile_off[0] = 0 (device)
+ *   P_total       P (host value; must match d_tile_off[T])
+ *   d_sel_out     [T][top_k] int32 (device)
+ *   d_score_out   [T][N] float32 or NULL
+ * Sub-volumes with no probe select tokens 0..top_k-1.  top_k >= N selects
+ * every token.  Errors: INVALID_ARG, UNSUPPORTED (N, top_k > 8192), CUDA.   */
+VDM_API vdm_status vdm_select_kv(const vdm_decoder* dec, const void* d_k, const void* d_v, int32_t N,
+                         const float* d_probe_xyz, const int32_t* d_tile_off, int32_t T,
+                         int64_t P_total, int32_t top_k, int32_t* d_sel_out, float* d_score_out,
+                         vdm_stream stream);
+
+/* Hierarchical volume decoding parameters (section 4.1 items 1-2).        */
+typedef struct {
+    int32_t r0;          /* coarse resolution, multiple of 4                 */
+    int32_t n_levels;    /* >= 1; final resolution r0 * 2^(n_levels-1)      */
+    int32_t adaptive;    /* 1: adaptive KV selection on the fine levels      */
+    int32_t tile;        /* sub-volume edge in fine voxels; must be 8        */
+    int32_t n_probe;     /* probes per sub-volume, 1..512                    */
+    int32_t top_k;       /* kept tokens per sub-volume                       */
+    uint64_t seed;       /* probe sampler seed                               */
+} vdm_hier_params;
+
+/* Per-shape, per-level counts written by vdm_decode_hierarchical (host).   */
+typedef struct {
+    int64_t resolution[VDM_MAX_LEVELS];
+    int64_t decoded[VDM_MAX_LEVELS];        /* queries decoded at the level  */
+    int64_t active_parents[VDM_MAX_LEVELS]; /* refined voxels of level l-1   */
+    int64_t tiles[VDM_MAX_LEVELS];          /* non-empty sub-volumes         */
+    int64_t selected_tiles[VDM_MAX_LEVELS]; /* sub-volumes with selection    */
+    int64_t probes[VDM_MAX_LEVELS];         /* queries decoded over all N
+                                               tokens: probes plus every query
+                                               of sub-volumes with <= n_probe
+                                               queries (adaptive levels)      */
+} vdm_hier_stats;
+
+/* Optional per-level copies for testing (all device pointers, nullable; a
+ * NULL entry skips that copy).  Shapes are handled one after the other, so
+ * each array holds shape b at offset b * (its per-shape size).             */
+typedef struct {
+    float* grid[VDM_MAX_LEVELS];        /* [B][R_l^3] dense field of level l */
+    uint64_t* active[VDM_MAX_LEVELS];   /* [B][(R_l/4)^3] refine mask of level
+                                           l (l < n_levels-1): word w = block
+                                           (bi,bj,bk) of 4^3 voxels in linear
+                                           block order, bit (di*4+dj)*4+dk   */
+    float* dec[VDM_MAX_LEVELS];         /* [B][R_l^3] raw decoder output at the
+                                           voxels decoded at level l; other
+                                           voxels are left untouched         */
+    int32_t* tile_ids[VDM_MAX_LEVELS];  /* [B][max_tiles] ids of sub-volumes
+                                           with a selection (adaptive)       */
+    int32_t* sel[VDM_MAX_LEVELS];       /* [B][max_tiles][top_k] their tokens */
+    int64_t max_tiles;                  /* capacity of tile_ids / sel        */
+} vdm_hier_debug;
+
+/* Workspace bytes needed by vdm_decode_hierarchical (host output).         */
+VDM_API vdm_status vdm_hierarchical_workspace_size(const vdm_decoder* dec, const vdm_hier_params* p,
+                                           int32_t N, size_t* bytes);
+
+/* Hierarchical volume decoding of B shapes (section 4.1 item 1, with item 2
+ * on the fine levels when p->adaptive):
+ *   level 0: dense decode of the r0^3 grid;
+ *   level l -> l+1: mark voxels with a sign change in their 3x3x3
+ *   neighbourhood or |f| < 2h (h = 2/R_l, threshold float32(4/R_l)), dilate
+ *   once (3x3x3), decode the 8 children of every marked voxel at 2R_l, and let
+ *   the other fine voxels inherit their parent's value.
+ *   d_grid_out [B][Rf^3] float32 final field, Rf = r0 * 2^(n_levels-1)
+ *   d_ws/ws_bytes  device workspace >= vdm_hierarchical_workspace_size
+ *   stats    host, B entries, nullable;  debug  host, nullable
+ * Synchronisation: after each level's marking the call copies two counts to
+ * the host and synchronises `stream` (one round trip per level).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA, TIMEOUT.              */
+VDM_API vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, const void* d_v,
+                                   int32_t B, int32_t N, const vdm_hier_params* p,
+                                   const vdm_analytic* analytic, float* d_grid_out,
+                                   void* d_ws, size_t ws_bytes, vdm_hier_stats* stats,
+                                   const vdm_hier_debug* debug, vdm_stream stream);
+
+/* Kernel timing for measurement (not needed for decoding).  Between
+ * vdm_profile_begin() and vdm_profile_end() the calling thread's launches are
+ * bracketed by CUDA events on their stream; vdm_profile_end() waits for those
+ * events and returns, per kernel class, the launch count and the summed
+ * device time.  Classes: 0 K/V projection, 1 decode, 2 probe scoring + Top-K,
+ * 3 mark + dilate, 4 scan, 5 parent list / offsets, 6 inherit fill,
+ * 7 probe ordering.                                                         */
+#define VDM_PROF_CLASSES 8
+typedef struct {
+    int64_t launches[VDM_PROF_CLASSES];
+    double ms[VDM_PROF_CLASSES];
+} vdm_profile;
+VDM_API vdm_status vdm_profile_begin(void);
+VDM_API vdm_status vdm_profile_end(vdm_profile* out);
+
+VDM_API const char* vdm_status_string(vdm_status s);
+VDM_API const char* vdm_last_error(void);   /* thread-local message of the last error */
+VDM_API int32_t vdm_abi_version(void);      /* 1                                      */
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VDM_H */

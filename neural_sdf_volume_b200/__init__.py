@@ -1,0 +1,291 @@
+"""Python binding of the B200 vecset SDF decoder library (``libvdm.so``).
+
+Argument marshalling only: every step of the decoder runs in the library's
+CUDA kernels.  PyTorch provides device memory and the current stream.  The
+functions carry the C names declared in ``include/vdm.h``:
+
+    vdm_precompute_kv, vdm_decode_dense, vdm_select_kv,
+    vdm_hierarchical_workspace_size, vdm_decode_hierarchical
+
+Importing this package loads ``libvdm.so``; if the library is missing the
+import fails (there is no fallback implementation).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+from typing import Dict, Optional
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvdm.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m neural_sdf_volume_b200.build` "
+        "(the CUDA library is required; there is no CPU path)")
+_lib = C.CDLL(LIB_PATH)
+
+MAX_LEVELS = 6
+VDM_F32, VDM_BF16 = 0, 1
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "workspace", 4: "cuda",
+          5: "timeout", 6: "internal"}
+
+EXPORTS = ("vdm_precompute_kv", "vdm_decode_dense", "vdm_select_kv",
+           "vdm_hierarchical_workspace_size", "vdm_decode_hierarchical",
+           "vdm_profile_begin", "vdm_profile_end",
+           "vdm_status_string", "vdm_last_error", "vdm_abi_version")
+PROF_CLASSES = ("kv", "decode", "select", "mark", "scan", "list", "fill", "probe")
+
+
+class VdmError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"vdm status {status} ({STATUS.get(status, '?')}): {msg}")
+        self.status = status
+
+
+class CDecoder(C.Structure):
+    _fields_ = [("C", C.c_int32), ("H", C.c_int32), ("F", C.c_int32), ("query_ln", C.c_int32),
+                ("dtype", C.c_int32),
+                ("Wq", C.c_void_p), ("Wk", C.c_void_p), ("Wv", C.c_void_p), ("Wo", C.c_void_p),
+                ("W1", C.c_void_p), ("W2", C.c_void_p),
+                ("bq", C.c_void_p), ("bk", C.c_void_p), ("bv", C.c_void_p), ("bo", C.c_void_p),
+                ("b1", C.c_void_p), ("b2", C.c_void_p),
+                ("ln_kv_g", C.c_void_p), ("ln_kv_b", C.c_void_p),
+                ("ln1_g", C.c_void_p), ("ln1_b", C.c_void_p), ("ln2_g", C.c_void_p), ("ln2_b", C.c_void_p),
+                ("w_head", C.c_void_p), ("b_head", C.c_void_p)]
+
+
+class CAnalytic(C.Structure):
+    _fields_ = [("spheres", C.c_void_p), ("n_spheres", C.c_int32), ("dec_scale", C.c_float)]
+
+
+class CHierParams(C.Structure):
+    _fields_ = [("r0", C.c_int32), ("n_levels", C.c_int32), ("adaptive", C.c_int32),
+                ("tile", C.c_int32), ("n_probe", C.c_int32), ("top_k", C.c_int32),
+                ("seed", C.c_uint64)]
+
+
+class CHierStats(C.Structure):
+    _fields_ = [(n, C.c_int64 * MAX_LEVELS) for n in
+                ("resolution", "decoded", "active_parents", "tiles", "selected_tiles", "probes")]
+
+
+class CHierDebug(C.Structure):
+    _fields_ = [("grid", C.c_void_p * MAX_LEVELS), ("active", C.c_void_p * MAX_LEVELS),
+                ("dec", C.c_void_p * MAX_LEVELS), ("tile_ids", C.c_void_p * MAX_LEVELS),
+                ("sel", C.c_void_p * MAX_LEVELS), ("max_tiles", C.c_int64)]
+
+
+class CProfile(C.Structure):
+    _fields_ = [("launches", C.c_int64 * 8), ("ms", C.c_double * 8)]
+
+
+_vp, _i32, _i64 = C.c_void_p, C.c_int32, C.c_int64
+_lib.vdm_precompute_kv.argtypes = [C.POINTER(CDecoder), _vp, _i32, _i32, _vp, _vp, _vp]
+_lib.vdm_decode_dense.argtypes = [C.POINTER(CDecoder), _vp, _vp, _i32, _i32, _vp, _i64, _i32,
+                                  C.POINTER(CAnalytic), _vp, _vp]
+_lib.vdm_select_kv.argtypes = [C.POINTER(CDecoder), _vp, _vp, _i32, _vp, _vp, _i32, _i64, _i32,
+                               _vp, _vp, _vp]
+_lib.vdm_hierarchical_workspace_size.argtypes = [C.POINTER(CDecoder), C.POINTER(CHierParams), _i32,
+                                                 C.POINTER(C.c_size_t)]
+_lib.vdm_decode_hierarchical.argtypes = [C.POINTER(CDecoder), _vp, _vp, _i32, _i32,
+                                         C.POINTER(CHierParams), C.POINTER(CAnalytic), _vp, _vp,
+                                         C.c_size_t, C.POINTER(CHierStats), C.POINTER(CHierDebug), _vp]
+_lib.vdm_profile_begin.argtypes = []
+_lib.vdm_profile_end.argtypes = [C.POINTER(CProfile)]
+for _f in ("vdm_precompute_kv", "vdm_decode_dense", "vdm_select_kv",
+           "vdm_hierarchical_workspace_size", "vdm_decode_hierarchical",
+           "vdm_profile_begin", "vdm_profile_end"):
+    getattr(_lib, _f).restype = C.c_int
+_lib.vdm_status_string.argtypes = [C.c_int]
+_lib.vdm_status_string.restype = C.c_char_p
+_lib.vdm_last_error.restype = C.c_char_p
+_lib.vdm_abi_version.restype = C.c_int32
+
+
+def _check(status: int):
+    if status != 0:
+        raise VdmError(status, _lib.vdm_last_error().decode(errors="replace"))
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+# ----------------------------------------------------------------- decoder parameters
+_MATS = ("Wq", "Wk", "Wv", "Wo", "W1", "W2")
+_VECS = ("bq", "bk", "bv", "bo", "b1", "b2", "ln_kv_g", "ln_kv_b", "ln1_g", "ln1_b",
+         "ln2_g", "ln2_b", "w_head", "b_head")
+
+
+@dataclass
+class Decoder:
+    """Device-resident decoder parameters plus the C struct pointing at them."""
+    C: int
+    H: int
+    F: int
+    query_ln: bool
+    dtype: str
+    tensors: Dict[str, "object"]
+
+    @staticmethod
+    def from_numpy(weights: Dict[str, np.ndarray], C: int, H: int, F: int, query_ln: bool,
+                   dtype: str, device="cuda") -> "Decoder":
+        torch = _torch()
+        tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+        t = {}
+        for k in _MATS:
+            t[k] = torch.from_numpy(np.ascontiguousarray(weights[k], np.float32)).to(device=device, dtype=tdt)
+        for k in _VECS:
+            t[k] = torch.from_numpy(np.ascontiguousarray(weights[k], np.float32).reshape(-1)).to(device)
+        return Decoder(C, H, F, bool(query_ln), dtype, t)
+
+    @property
+    def torch_dtype(self):
+        torch = _torch()
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def cstruct(self) -> CDecoder:
+        d = CDecoder()
+        d.C, d.H, d.F, d.query_ln = self.C, self.H, self.F, int(self.query_ln)
+        d.dtype = VDM_F32 if self.dtype == "f32" else VDM_BF16
+        for k in _MATS + _VECS:
+            setattr(d, k, self.tensors[k].data_ptr())
+        return d
+
+
+def _analytic(spheres, dec_scale: float):
+    if spheres is None:
+        return None
+    a = CAnalytic()
+    a.spheres = spheres.data_ptr()
+    a.n_spheres = int(spheres.shape[1])
+    a.dec_scale = float(dec_scale)
+    return a
+
+
+# ----------------------------------------------------------------- entry points
+def vdm_precompute_kv(dec: Decoder, z, stream=None):
+    """``z[B,N,C]`` float32 (device) -> ``K, V [B,H,N,64]`` in the decoder dtype."""
+    torch = _torch()
+    B, N, Cw = z.shape
+    K = torch.empty((B, dec.H, N, 64), device=z.device, dtype=dec.torch_dtype)
+    V = torch.empty_like(K)
+    cd = dec.cstruct()
+    _check(_lib.vdm_precompute_kv(C.byref(cd), z.data_ptr(), B, N, K.data_ptr(), V.data_ptr(),
+                                  _stream(stream)))
+    return K, V
+
+
+def vdm_decode_dense(dec: Decoder, K, V, xyz=None, grid_R: int = 0, spheres=None,
+                     dec_scale: float = 0.0, out=None, stream=None):
+    """Decoder output at ``xyz[B,M,3]`` or at the voxels of the ``grid_R^3`` grid."""
+    torch = _torch()
+    B, H, N, _ = K.shape
+    M = xyz.shape[1] if xyz is not None else grid_R ** 3
+    if out is None:
+        out = torch.empty((B, M), device=K.device, dtype=torch.float32)
+    cd = dec.cstruct()
+    an = _analytic(spheres, dec_scale)
+    _check(_lib.vdm_decode_dense(C.byref(cd), K.data_ptr(), V.data_ptr(), B, N, _ptr(xyz), M,
+                                 grid_R, C.byref(an) if an else None, out.data_ptr(), _stream(stream)))
+    return out
+
+
+def vdm_select_kv(dec: Decoder, K, V, probe_xyz, tile_off, top_k: int, want_scores: bool = False,
+                  stream=None):
+    """Per sub-volume Top-K token ids ``[T, top_k]`` (and scores ``[T, N]``)."""
+    torch = _torch()
+    N = K.shape[-2]
+    T = int(tile_off.numel()) - 1
+    P = int(probe_xyz.shape[0]) if probe_xyz is not None else 0
+    sel = torch.empty((max(T, 0), top_k), device=K.device, dtype=torch.int32)
+    score = torch.empty((max(T, 0), N), device=K.device, dtype=torch.float32) if want_scores else None
+    cd = dec.cstruct()
+    _check(_lib.vdm_select_kv(C.byref(cd), K.data_ptr(), V.data_ptr(), N, _ptr(probe_xyz),
+                              tile_off.data_ptr(), T, P, top_k, sel.data_ptr(), _ptr(score),
+                              _stream(stream)))
+    return (sel, score) if want_scores else sel
+
+
+def hier_params(r0: int, n_levels: int, adaptive: bool = False, tile: int = 8, n_probe: int = 64,
+                top_k: int = 1024, seed: int = 0) -> CHierParams:
+    p = CHierParams()
+    p.r0, p.n_levels, p.adaptive, p.tile = r0, n_levels, int(adaptive), tile
+    p.n_probe, p.top_k, p.seed = n_probe, top_k, seed
+    return p
+
+
+def vdm_hierarchical_workspace_size(dec: Decoder, params: CHierParams, N: int) -> int:
+    n = C.c_size_t(0)
+    cd = dec.cstruct()
+    _check(_lib.vdm_hierarchical_workspace_size(C.byref(cd), C.byref(params), N, C.byref(n)))
+    return int(n.value)
+
+
+def vdm_decode_hierarchical(dec: Decoder, K, V, params: CHierParams, spheres=None,
+                            dec_scale: float = 0.0, workspace=None, out=None, debug=None,
+                            stream=None):
+    """Coarse-to-fine decoding of B shapes -> (grid ``[B,Rf,Rf,Rf]``, per-shape stats).
+
+    ``debug`` is an optional dict of device tensors keyed like ``vdm_hier_debug``
+    (``grid``, ``active``, ``dec``, ``tile_ids``, ``sel``: lists indexed by level,
+    plus ``max_tiles``)."""
+    torch = _torch()
+    B, H, N, _ = K.shape
+    Rf = params.r0 << (params.n_levels - 1)
+    if out is None:
+        out = torch.empty((B, Rf, Rf, Rf), device=K.device, dtype=torch.float32)
+    if workspace is None:
+        nbytes = vdm_hierarchical_workspace_size(dec, params, N)
+        workspace = torch.empty((nbytes,), device=K.device, dtype=torch.uint8)
+    stats = (CHierStats * B)()
+    dbg = None
+    if debug is not None:
+        dbg = CHierDebug()
+        for key in ("grid", "active", "dec", "tile_ids", "sel"):
+            arr = getattr(dbg, key)
+            for l, t in enumerate(debug.get(key, [])):
+                arr[l] = _ptr(t) or 0
+        dbg.max_tiles = int(debug.get("max_tiles", 0))
+    cd = dec.cstruct()
+    an = _analytic(spheres, dec_scale)
+    _check(_lib.vdm_decode_hierarchical(C.byref(cd), K.data_ptr(), V.data_ptr(), B, N,
+                                        C.byref(params), C.byref(an) if an else None,
+                                        out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                        stats, C.byref(dbg) if dbg else None, _stream(stream)))
+    st = [{k: list(getattr(stats[b], k)) for k in ("resolution", "decoded", "active_parents",
+                                                    "tiles", "selected_tiles", "probes")}
+          for b in range(B)]
+    return out, st
+
+
+def vdm_profile_begin():
+    """Start bracketing this thread's kernel launches with CUDA events."""
+    _check(_lib.vdm_profile_begin())
+
+
+def vdm_profile_end() -> Dict[str, Dict[str, float]]:
+    """Wait for the recorded events; per kernel class: launches and device ms."""
+    p = CProfile()
+    _check(_lib.vdm_profile_end(C.byref(p)))
+    return {n: {"launches": int(p.launches[i]), "ms": float(p.ms[i])}
+            for i, n in enumerate(PROF_CLASSES)}
+
+
+def abi_version() -> int:
+    return int(_lib.vdm_abi_version())

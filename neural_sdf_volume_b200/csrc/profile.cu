@@ -1,0 +1,85 @@
+// Optional per-launch CUDA-event timing (vdm_profile_begin / vdm_profile_end).
+#include <string.h>
+
+#include <vector>
+
+#include "vdm_internal.cuh"
+
+namespace vdm {
+namespace {
+
+struct Rec {
+    cudaEvent_t a, b;
+    int cls;
+};
+
+thread_local bool g_on = false;
+thread_local std::vector<Rec> g_recs;
+thread_local std::vector<cudaEvent_t> g_pool;
+thread_local int64_t g_launch[VDM_PROF_CLASSES];
+
+cudaEvent_t take() {
+    if (!g_pool.empty()) {
+        cudaEvent_t e = g_pool.back();
+        g_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+}  // namespace
+
+void prof_begin(int cls, cudaStream_t s) {
+    if (!g_on) return;
+    ++g_launch[cls];
+    Rec r{take(), take(), cls};
+    cudaEventRecord(r.a, s);
+    g_recs.push_back(r);
+}
+
+void prof_end(int cls, cudaStream_t s) {
+    if (!g_on || g_recs.empty()) return;
+    (void)cls;
+    cudaEventRecord(g_recs.back().b, s);
+}
+
+}  // namespace vdm
+
+using namespace vdm;
+
+extern "C" {
+
+vdm_status vdm_profile_begin(void) {
+    for (auto& r : g_recs) {
+        g_pool.push_back(r.a);
+        g_pool.push_back(r.b);
+    }
+    g_recs.clear();
+    memset(g_launch, 0, sizeof(g_launch));
+    g_on = true;
+    return VDM_OK;
+}
+
+vdm_status vdm_profile_end(vdm_profile* out) {
+    if (!out) return fail(VDM_ERR_INVALID_ARG, "out is NULL");
+    memset(out, 0, sizeof(*out));
+    g_on = false;
+    vdm_status st = VDM_OK;
+    for (auto& r : g_recs) {
+        float ms = 0.f;
+        cudaError_t e = cudaEventSynchronize(r.b);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+        if (e != cudaSuccess && st == VDM_OK)
+            st = fail(VDM_ERR_CUDA, "profile event: %s", cudaGetErrorString(e));
+        out->ms[r.cls] += ms;
+        g_pool.push_back(r.a);
+        g_pool.push_back(r.b);
+    }
+    g_recs.clear();
+    for (int c = 0; c < VDM_PROF_CLASSES; ++c) out->launches[c] = g_launch[c];
+    return st;
+}
+
+}  // extern "C"

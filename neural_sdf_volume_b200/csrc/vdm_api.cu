@@ -1,0 +1,442 @@
+// Host side of the C ABI declared in include/vdm.h: argument checks, workspace
+// planning, the coarse-to-fine level driver and kernel launches.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "vdm_internal.cuh"
+
+namespace vdm {
+
+static thread_local char g_err[512] = "";
+
+void set_error(const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+}
+
+vdm_status fail(vdm_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+vdm_status check_launch(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return VDM_OK;
+}
+
+int decode_simt_chunk();
+
+namespace {
+
+size_t elt_size(vdm_dtype d) { return d == VDM_F32 ? 4 : 2; }
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+vdm_status check_decoder(const vdm_decoder* d, bool need_query_side) {
+    if (!d) return fail(VDM_ERR_INVALID_ARG, "decoder is NULL");
+    if (d->dtype != VDM_F32 && d->dtype != VDM_BF16)
+        return fail(VDM_ERR_INVALID_ARG, "unknown dtype %d", (int)d->dtype);
+    if (d->H < 1 || d->C != d->H * kHeadDim)
+        return fail(VDM_ERR_UNSUPPORTED, "C (%d) must equal 64 * H (H = %d)", d->C, d->H);
+    if (d->C != 64 && d->C != 128 && d->C != 256 && d->C != 512)
+        return fail(VDM_ERR_UNSUPPORTED, "C = %d not in {64, 128, 256, 512}", d->C);
+    if (d->F < 64 || d->F > 4096 || d->F % 64)
+        return fail(VDM_ERR_UNSUPPORTED, "F = %d must be a multiple of 64 in [64, 4096]", d->F);
+    if (d->query_ln != 0 && d->query_ln != 1)
+        return fail(VDM_ERR_INVALID_ARG, "query_ln must be 0 or 1");
+    const size_t al = d->dtype == VDM_F32 ? 16 : 8;
+    const void* mats[] = {d->Wq, d->Wk, d->Wv, d->Wo, d->W1, d->W2};
+    const char* names[] = {"Wq", "Wk", "Wv", "Wo", "W1", "W2"};
+    for (int i = 0; i < 6; ++i) {
+        if (!need_query_side && i != 1 && i != 2) continue;
+        if (!mats[i]) return fail(VDM_ERR_INVALID_ARG, "%s is NULL", names[i]);
+        if (!aligned(mats[i], al)) return fail(VDM_ERR_INVALID_ARG, "%s is not %zu-byte aligned", names[i], al);
+    }
+    const float* vecs[] = {d->bk, d->bv, d->ln_kv_g, d->ln_kv_b, d->bq, d->bo, d->b1, d->b2,
+                           d->ln1_g, d->ln1_b, d->ln2_g, d->ln2_b, d->w_head, d->b_head};
+    const int nvec = need_query_side ? 14 : 4;
+    for (int i = 0; i < nvec; ++i)
+        if (!vecs[i]) return fail(VDM_ERR_INVALID_ARG, "decoder vector %d is NULL", i);
+    return VDM_OK;
+}
+
+DecodeArgs base_args(const vdm_decoder* d, const void* K, const void* V, int N) {
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.C = d->C; a.H = d->H; a.F = d->F; a.query_ln = d->query_ln;
+    a.Wq = d->Wq; a.Wo = d->Wo; a.W1 = d->W1; a.W2 = d->W2;
+    a.bq = d->bq; a.bo = d->bo; a.b1 = d->b1; a.b2 = d->b2;
+    a.ln1_g = d->ln1_g; a.ln1_b = d->ln1_b; a.ln2_g = d->ln2_g; a.ln2_b = d->ln2_b;
+    a.w_head = d->w_head; a.b_head = d->b_head;
+    a.K = K; a.V = V; a.N = N;
+    return a;
+}
+
+size_t kv_shape_bytes(const vdm_decoder* d, int N) {
+    return (size_t)d->H * N * kHeadDim * elt_size(d->dtype);
+}
+
+// ---------------------------------------------------------------- workspace plan
+struct Plan {
+    int L;
+    int R[VDM_MAX_LEVELS];
+    size_t off_grid[VDM_MAX_LEVELS];
+    size_t off_words, off_word_off, off_tile_ids, off_tile_off, off_counts, off_scan, off_plist,
+        off_qorder, off_sel;
+    int nw_max;
+    int k;
+    size_t total;
+};
+
+size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
+
+vdm_status make_plan(const vdm_hier_params* p, int N, Plan& pl) {
+    if (!p) return fail(VDM_ERR_INVALID_ARG, "params is NULL");
+    if (p->n_levels < 1 || p->n_levels > VDM_MAX_LEVELS)
+        return fail(VDM_ERR_UNSUPPORTED, "n_levels = %d not in [1, %d]", p->n_levels, VDM_MAX_LEVELS);
+    if (p->r0 < 4 || p->r0 % 4) return fail(VDM_ERR_UNSUPPORTED, "r0 = %d must be a positive multiple of 4", p->r0);
+    const int64_t rf = (int64_t)p->r0 << (p->n_levels - 1);
+    if (rf > 1024) return fail(VDM_ERR_UNSUPPORTED, "final resolution %lld > 1024", (long long)rf);
+    if (p->adaptive) {
+        if (p->tile != 8) return fail(VDM_ERR_UNSUPPORTED, "sub-volume edge must be 8 (got %d)", p->tile);
+        if (p->n_probe < 1 || p->n_probe > 512) return fail(VDM_ERR_UNSUPPORTED, "n_probe must be in [1, 512]");
+        if (p->top_k < 1) return fail(VDM_ERR_INVALID_ARG, "top_k must be >= 1");
+    }
+    pl.L = p->n_levels;
+    pl.k = p->adaptive ? (p->top_k < N ? p->top_k : N) : 0;
+    size_t o = 0;
+    int nw_max = 0;
+    int64_t vox_max = 0;
+    for (int l = 0; l < pl.L; ++l) {
+        pl.R[l] = p->r0 << l;
+        if (l < pl.L - 1) {
+            pl.off_grid[l] = o;
+            o = align_up(o + (size_t)pl.R[l] * pl.R[l] * pl.R[l] * 4);
+            const int nb = pl.R[l] / 4;
+            if (nb * nb * nb > nw_max) nw_max = nb * nb * nb;
+            const int64_t v = (int64_t)pl.R[l] * pl.R[l] * pl.R[l];
+            if (v > vox_max) vox_max = v;
+        }
+    }
+    pl.nw_max = nw_max;
+    pl.off_words = o;     o = align_up(o + (size_t)nw_max * 8);
+    pl.off_word_off = o;  o = align_up(o + (size_t)(nw_max + 1) * 4);
+    pl.off_tile_ids = o;  o = align_up(o + (size_t)nw_max * 4);
+    pl.off_tile_off = o;  o = align_up(o + (size_t)(nw_max + 1) * 4);
+    pl.off_counts = o;    o = align_up(o + 4 * 4 * VDM_MAX_LEVELS);
+    pl.off_scan = o;      o = align_up(o + scan_tmp_ints(nw_max) * 4);
+    pl.off_plist = o;     o = align_up(o + (size_t)vox_max * 4);
+    pl.off_qorder = o;    o = align_up(o + (p->adaptive ? (size_t)vox_max * 8 * 4 : 0));
+    pl.off_sel = o;       o = align_up(o + (p->adaptive ? (size_t)nw_max * pl.k * 4 : 0));
+    pl.total = o + 256;
+    return VDM_OK;
+}
+
+template <typename T> T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+}  // namespace
+}  // namespace vdm
+
+using namespace vdm;
+
+extern "C" {
+
+int32_t vdm_abi_version(void) { return 1; }
+
+const char* vdm_last_error(void) { return g_err; }
+
+const char* vdm_status_string(vdm_status s) {
+    switch (s) {
+        case VDM_OK: return "ok";
+        case VDM_ERR_INVALID_ARG: return "invalid argument";
+        case VDM_ERR_UNSUPPORTED: return "unsupported shape";
+        case VDM_ERR_WORKSPACE: return "workspace too small";
+        case VDM_ERR_CUDA: return "CUDA error";
+        case VDM_ERR_TIMEOUT: return "device wait timed out";
+        case VDM_ERR_INTERNAL: return "internal error";
+    }
+    return "unknown status";
+}
+
+vdm_status vdm_precompute_kv(const vdm_decoder* dec, const float* d_z, int32_t B, int32_t N,
+                             void* d_k_out, void* d_v_out, vdm_stream stream) {
+    VDM_TRY(check_decoder(dec, false));
+    if (B < 1 || N < 1) return fail(VDM_ERR_INVALID_ARG, "B and N must be >= 1");
+    if (N > kMaxN) return fail(VDM_ERR_UNSUPPORTED, "N = %d > %d", N, kMaxN);
+    if (!d_z || !d_k_out || !d_v_out) return fail(VDM_ERR_INVALID_ARG, "null z / k / v");
+    if (!aligned(d_k_out, 16) || !aligned(d_v_out, 16))
+        return fail(VDM_ERR_INVALID_ARG, "k / v must be 16-byte aligned");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t kvb = kv_shape_bytes(dec, N);
+    for (int b = 0; b < B; ++b) {
+        KvArgs a;
+        a.C = dec->C; a.H = dec->H; a.N = N;
+        a.z = d_z + (size_t)b * N * dec->C;
+        a.Wk = dec->Wk; a.Wv = dec->Wv; a.bk = dec->bk; a.bv = dec->bv;
+        a.g = dec->ln_kv_g; a.b = dec->ln_kv_b;
+        a.K = static_cast<char*>(d_k_out) + b * kvb;
+        a.V = static_cast<char*>(d_v_out) + b * kvb;
+        VDM_TRY(launch_precompute_kv(a, dec->dtype, st));
+    }
+    return VDM_OK;
+}
+
+vdm_status vdm_decode_dense(const vdm_decoder* dec, const void* d_k, const void* d_v, int32_t B,
+                            int32_t N, const float* d_xyz, int64_t M, int32_t grid_R,
+                            const vdm_analytic* an, float* d_out, vdm_stream stream) {
+    VDM_TRY(check_decoder(dec, true));
+    if (B < 1 || N < 1 || M < 0) return fail(VDM_ERR_INVALID_ARG, "B, N must be >= 1 and M >= 0");
+    if (N > kMaxN) return fail(VDM_ERR_UNSUPPORTED, "N = %d > %d", N, kMaxN);
+    if (M == 0) return VDM_OK;
+    if (!d_k || !d_v || !d_out) return fail(VDM_ERR_INVALID_ARG, "null k / v / out");
+    if (!d_xyz) {
+        if (grid_R < 1 || (int64_t)grid_R * grid_R * grid_R != M)
+            return fail(VDM_ERR_INVALID_ARG, "grid mode needs M == grid_R^3 (M = %lld, R = %d)",
+                        (long long)M, grid_R);
+    }
+    if (M > ((int64_t)1 << 31) - 1) return fail(VDM_ERR_UNSUPPORTED, "M too large");
+    if (an && (!an->spheres || an->n_spheres < 1))
+        return fail(VDM_ERR_INVALID_ARG, "analytic term needs spheres and n_spheres >= 1");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t kvb = kv_shape_bytes(dec, N);
+    for (int b = 0; b < B; ++b) {
+        DecodeArgs a = base_args(dec, static_cast<const char*>(d_k) + b * kvb,
+                                 static_cast<const char*>(d_v) + b * kvb, N);
+        a.work = kWorkFlat;
+        a.M = M;
+        if (d_xyz) {
+            a.qmode = kQueryXyz;
+            a.xyz = d_xyz + (size_t)b * M * 3;
+        } else {
+            a.qmode = kQueryGrid;
+            a.R = grid_R;
+        }
+        a.out = d_out + (size_t)b * M;
+        if (an) {
+            a.spheres = an->spheres + (size_t)b * an->n_spheres * 4;
+            a.n_spheres = an->n_spheres;
+            a.dec_scale = an->dec_scale;
+        }
+        VDM_TRY(launch_decode_simt(a, dec->dtype, 0, st));
+    }
+    return VDM_OK;
+}
+
+vdm_status vdm_select_kv(const vdm_decoder* dec, const void* d_k, const void* d_v, int32_t N,
+                         const float* d_probe_xyz, const int32_t* d_tile_off, int32_t T,
+                         int64_t P_total, int32_t top_k, int32_t* d_sel_out, float* d_score_out,
+                         vdm_stream stream) {
+    (void)d_v;
+    VDM_TRY(check_decoder(dec, true));
+    if (N < 1 || T < 0 || P_total < 0) return fail(VDM_ERR_INVALID_ARG, "bad N / T / P");
+    if (N > kMaxN) return fail(VDM_ERR_UNSUPPORTED, "N = %d > %d", N, kMaxN);
+    if (top_k < 1 || top_k > N) return fail(VDM_ERR_INVALID_ARG, "top_k must be in [1, N]");
+    if (T == 0) return VDM_OK;
+    if (!d_k || !d_tile_off || !d_sel_out || (P_total > 0 && !d_probe_xyz))
+        return fail(VDM_ERR_INVALID_ARG, "null k / tile_off / sel / probe_xyz");
+    SelectArgs a;
+    memset(&a, 0, sizeof(a));
+    a.C = dec->C; a.H = dec->H; a.N = N;
+    a.Wq = dec->Wq; a.bq = dec->bq; a.K = d_k;
+    a.T = T;
+    a.probe_xyz = d_probe_xyz ? d_probe_xyz : reinterpret_cast<const float*>(d_tile_off);
+    a.probe_off = d_tile_off;
+    a.top_k = top_k;
+    a.sel = d_sel_out;
+    a.score = d_score_out;
+    return launch_select(a, dec->dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+vdm_status vdm_hierarchical_workspace_size(const vdm_decoder* dec, const vdm_hier_params* p, int32_t N,
+                                           size_t* bytes) {
+    VDM_TRY(check_decoder(dec, true));
+    if (!bytes) return fail(VDM_ERR_INVALID_ARG, "bytes is NULL");
+    if (N < 1 || N > kMaxN) return fail(VDM_ERR_UNSUPPORTED, "N = %d not in [1, %d]", N, kMaxN);
+    Plan pl;
+    VDM_TRY(make_plan(p, N, pl));
+    *bytes = pl.total;
+    return VDM_OK;
+}
+
+vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, const void* d_v,
+                                   int32_t B, int32_t N, const vdm_hier_params* p,
+                                   const vdm_analytic* an, float* d_grid_out, void* d_ws,
+                                   size_t ws_bytes, vdm_hier_stats* stats, const vdm_hier_debug* dbg,
+                                   vdm_stream stream) {
+    VDM_TRY(check_decoder(dec, true));
+    if (B < 1 || N < 1) return fail(VDM_ERR_INVALID_ARG, "B and N must be >= 1");
+    if (N > kMaxN) return fail(VDM_ERR_UNSUPPORTED, "N = %d > %d", N, kMaxN);
+    if (!d_k || !d_v || !d_grid_out) return fail(VDM_ERR_INVALID_ARG, "null k / v / grid_out");
+    if (an && (!an->spheres || an->n_spheres < 1))
+        return fail(VDM_ERR_INVALID_ARG, "analytic term needs spheres and n_spheres >= 1");
+    Plan pl;
+    VDM_TRY(make_plan(p, N, pl));
+    if (pl.L > 1 && (!d_ws || ws_bytes < pl.total))
+        return fail(VDM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.total, ws_bytes);
+    void* ws = d_ws ? reinterpret_cast<void*>(align_up((uintptr_t)d_ws)) : nullptr;
+    if (ws && (uintptr_t)ws - (uintptr_t)d_ws + pl.total - 256 > ws_bytes)
+        return fail(VDM_ERR_WORKSPACE, "workspace too small after alignment");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t kvb = kv_shape_bytes(dec, N);
+    const int L = pl.L;
+    const int64_t Rf = pl.R[L - 1];
+    const int qt = decode_simt_chunk();
+
+    for (int b = 0; b < B; ++b) {
+        const void* K = static_cast<const char*>(d_k) + b * kvb;
+        const void* V = static_cast<const char*>(d_v) + b * kvb;
+        float* grid[VDM_MAX_LEVELS];
+        for (int l = 0; l < L - 1; ++l) grid[l] = at<float>(ws, pl.off_grid[l]);
+        grid[L - 1] = d_grid_out + (size_t)b * Rf * Rf * Rf;
+        DecodeArgs base = base_args(dec, K, V, N);
+        if (an) {
+            base.spheres = an->spheres + (size_t)b * an->n_spheres * 4;
+            base.n_spheres = an->n_spheres;
+            base.dec_scale = an->dec_scale;
+        }
+        vdm_hier_stats* sb = stats ? stats + b : nullptr;
+        if (sb) memset(sb, 0, sizeof(*sb));
+        auto dbg_ptr = [&](float* const* arr, int l, int64_t per) -> float* {
+            return (dbg && arr[l]) ? arr[l] + (size_t)b * per : nullptr;
+        };
+        // ---- level 0: dense
+        {
+            const int R = pl.R[0];
+            DecodeArgs a = base;
+            a.work = kWorkFlat;
+            a.qmode = kQueryGrid;
+            a.R = R;
+            a.M = (int64_t)R * R * R;
+            a.grid = grid[0];
+            a.dec_grid = dbg_ptr(dbg ? dbg->dec : nullptr, 0, a.M);
+            VDM_TRY(launch_decode_simt(a, dec->dtype, 0, st));
+            if (sb) { sb->resolution[0] = R; sb->decoded[0] = a.M; }
+        }
+        for (int l = 0; l + 1 < L; ++l) {
+            const int R = pl.R[l], R2 = 2 * R;
+            const int nb = R / 4;
+            const int nw = nb * nb * nb;
+            uint64_t* words = at<uint64_t>(ws, pl.off_words);
+            int32_t* word_off = at<int32_t>(ws, pl.off_word_off);
+            int32_t* tile_ids = at<int32_t>(ws, pl.off_tile_ids);
+            int32_t* tile_off = at<int32_t>(ws, pl.off_tile_off);
+            int32_t* counts = at<int32_t>(ws, pl.off_counts) + 4 * (l + 1);
+            int32_t* scan_tmp = at<int32_t>(ws, pl.off_scan);
+            int32_t* plist = at<int32_t>(ws, pl.off_plist);
+            int32_t* qorder = at<int32_t>(ws, pl.off_qorder);
+            int32_t* sel = at<int32_t>(ws, pl.off_sel);
+            VDM_TRY(launch_mark_dilate(grid[l], R, words, st));
+            VDM_TRY(launch_word_scan(words, nw, word_off, tile_ids, counts, scan_tmp, st));
+            int32_t hc[2] = {0, 0};
+            VDM_CUDA_TRY(cudaMemcpyAsync(hc, counts, sizeof(hc), cudaMemcpyDeviceToHost, st));
+            VDM_CUDA_TRY(cudaStreamSynchronize(st));
+            const int Mp = hc[0], T = hc[1];
+            if (dbg && dbg->active[l])
+                VDM_CUDA_TRY(cudaMemcpyAsync(dbg->active[l] + (size_t)b * nw, words, (size_t)nw * 8,
+                                             cudaMemcpyDeviceToDevice, st));
+            VDM_TRY(launch_parent_list(words, word_off, nw, R, plist, st));
+            VDM_TRY(launch_tile_offsets(word_off, tile_ids, T, nw, tile_off, st));
+            VDM_TRY(launch_fill(grid[l], words, R, grid[l + 1], st));
+            const int64_t vox2 = (int64_t)R2 * R2 * R2;
+            float* decg = dbg_ptr(dbg ? dbg->dec : nullptr, l + 1, vox2);
+            if (sb) {
+                sb->resolution[l + 1] = R2;
+                sb->active_parents[l + 1] = Mp;
+                sb->tiles[l + 1] = T;
+            }
+            if (Mp == 0) continue;
+            if (!p->adaptive) {
+                DecodeArgs a = base;
+                a.work = kWorkFlat;
+                a.qmode = kQueryChildren;
+                a.R = R2;
+                a.plist = plist;
+                a.M = 8 * (int64_t)Mp;
+                a.grid = grid[l + 1];
+                a.dec_grid = decg;
+                VDM_TRY(launch_decode_simt(a, dec->dtype, 0, st));
+                if (sb) sb->decoded[l + 1] = a.M;
+                continue;
+            }
+            const uint64_t salt = splitmix64(p->seed ^ ((uint64_t)(l + 1) << 32));
+            VDM_CUDA_TRY(cudaMemsetAsync(counts + 2, 0, 2 * sizeof(int32_t), st));
+            VDM_TRY(launch_probe_order(tile_off, T, plist, R2, p->n_probe, salt, qorder, counts + 2, st));
+            DecodeArgs a = base;
+            a.qmode = kQueryChildren;
+            a.R = R2;
+            a.plist = plist;
+            a.qorder = qorder;
+            a.tile_off = tile_off;
+            a.T = T;
+            a.n_probe = p->n_probe;
+            a.grid = grid[l + 1];
+            a.dec_grid = decg;
+            // dense pass: probes and small sub-volumes
+            a.work = kWorkTileDense;
+            a.slots = (std::min(512, p->n_probe) + qt - 1) / qt;
+            VDM_TRY(launch_decode_simt(a, dec->dtype, 0, st));
+            // selection
+            SelectArgs s;
+            memset(&s, 0, sizeof(s));
+            s.C = dec->C; s.H = dec->H; s.N = N;
+            s.Wq = dec->Wq; s.bq = dec->bq; s.K = K;
+            s.T = T;
+            s.tile_off = tile_off; s.plist = plist; s.qorder = qorder; s.R = R2;
+            s.n_probe = p->n_probe;
+            s.top_k = pl.k;
+            s.sel = sel;
+            VDM_TRY(launch_select(s, dec->dtype, st));
+            // sparse pass: the remaining queries over the selected tokens
+            if (p->n_probe < 512) {
+                a.work = kWorkTileSparse;
+                a.slots = (512 - p->n_probe + qt - 1) / qt;
+                a.sel = sel;
+                a.ksel = pl.k;
+                VDM_TRY(launch_decode_simt(a, dec->dtype, 0, st));
+            }
+            if (dbg && dbg->tile_ids[l + 1] && dbg->max_tiles > 0) {
+                const int64_t nt = T < dbg->max_tiles ? T : dbg->max_tiles;
+                VDM_CUDA_TRY(cudaMemcpyAsync(dbg->tile_ids[l + 1] + (size_t)b * dbg->max_tiles, tile_ids,
+                                             nt * 4, cudaMemcpyDeviceToDevice, st));
+                if (dbg->sel[l + 1])
+                    VDM_CUDA_TRY(cudaMemcpyAsync(dbg->sel[l + 1] + (size_t)b * dbg->max_tiles * pl.k, sel,
+                                                 nt * pl.k * 4, cudaMemcpyDeviceToDevice, st));
+            }
+            if (sb) sb->decoded[l + 1] = 8 * (int64_t)Mp;
+        }
+        if (sb && p->adaptive && L > 1) {
+            int32_t hc[4 * VDM_MAX_LEVELS];
+            VDM_CUDA_TRY(cudaMemcpyAsync(hc, at<int32_t>(ws, pl.off_counts), sizeof(int32_t) * 4 * L,
+                                         cudaMemcpyDeviceToHost, st));
+            VDM_CUDA_TRY(cudaStreamSynchronize(st));
+            for (int l = 1; l < L; ++l) {
+                if (sb->active_parents[l] == 0) continue;
+                sb->selected_tiles[l] = hc[4 * l + 2];
+                sb->probes[l] = hc[4 * l + 3];
+            }
+        }
+        if (dbg) {
+            for (int l = 0; l < L; ++l) {
+                if (!dbg->grid[l]) continue;
+                const size_t v = (size_t)pl.R[l] * pl.R[l] * pl.R[l];
+                VDM_CUDA_TRY(cudaMemcpyAsync(dbg->grid[l] + (size_t)b * v, grid[l], v * 4,
+                                             cudaMemcpyDeviceToDevice, st));
+            }
+        }
+    }
+    return VDM_OK;
+}
+
+}  // extern "C"
