@@ -212,6 +212,27 @@ VDM_API vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d
                                    void* d_ws, size_t ws_bytes, vdm_hier_stats* stats,
                                    const vdm_hier_debug* debug, vdm_stream stream);
 
+/* Hierarchical decoding with no device allocation at all (no counterpart in
+ * the paper; a deployment aid).  Same arguments and results as
+ * vdm_decode_hierarchical, minus the workspace: the scratch space is a 32 MiB
+ * array built into the library (held on every GPU that loads it until the
+ * process exits).  For callers that may not call cudaMalloc: applications that
+ * own all device memory themselves, and latency-critical code that avoids
+ * cudaMalloc/cudaFree because they can synchronise the device.
+ *   - Problems whose vdm_hierarchical_workspace_size exceeds 32 MiB return
+ *     VDM_ERR_UNSUPPORTED (a 32 -> 64 -> 128 adaptive decode with top_k 1024
+ *     needs about 26 MiB; 64 -> 128 -> 256 without adaptive KV about 18 MiB).
+ *   - All calls on a device share that scratch: calls that overlap on the GPU
+ *     race; issue them one after another on one stream.
+ *   - The first call on each device looks up the scratch address (no
+ *     allocation); make that first call before any stream capture.          */
+VDM_API vdm_status vdm_decode_hierarchical_noalloc(const vdm_decoder* dec, const void* d_k,
+                                                   const void* d_v, int32_t B, int32_t N,
+                                                   const vdm_hier_params* p,
+                                                   const vdm_analytic* analytic, float* d_grid_out,
+                                                   vdm_hier_stats* stats,
+                                                   const vdm_hier_debug* debug, vdm_stream stream);
+
 /* Kernel timing for measurement (not needed for decoding).  Between
  * vdm_profile_begin() and vdm_profile_end() the calling thread's launches are
  * bracketed by CUDA events on their stream; vdm_profile_end() waits for those

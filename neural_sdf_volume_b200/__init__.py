@@ -35,7 +35,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "workspace", 4: "
 
 EXPORTS = ("vdm_precompute_kv", "vdm_decode_dense", "vdm_select_kv",
            "vdm_hierarchical_workspace_size", "vdm_decode_hierarchical",
-           "vdm_profile_begin", "vdm_profile_end",
+           "vdm_decode_hierarchical_noalloc", "vdm_profile_begin", "vdm_profile_end",
            "vdm_status_string", "vdm_last_error", "vdm_abi_version")
 PROF_CLASSES = ("kv", "decode", "select", "mark", "scan", "list", "fill", "probe")
 
@@ -94,11 +94,14 @@ _lib.vdm_hierarchical_workspace_size.argtypes = [C.POINTER(CDecoder), C.POINTER(
 _lib.vdm_decode_hierarchical.argtypes = [C.POINTER(CDecoder), _vp, _vp, _i32, _i32,
                                          C.POINTER(CHierParams), C.POINTER(CAnalytic), _vp, _vp,
                                          C.c_size_t, C.POINTER(CHierStats), C.POINTER(CHierDebug), _vp]
+_lib.vdm_decode_hierarchical_noalloc.argtypes = [C.POINTER(CDecoder), _vp, _vp, _i32, _i32,
+                                                 C.POINTER(CHierParams), C.POINTER(CAnalytic), _vp,
+                                                 C.POINTER(CHierStats), C.POINTER(CHierDebug), _vp]
 _lib.vdm_profile_begin.argtypes = []
 _lib.vdm_profile_end.argtypes = [C.POINTER(CProfile)]
 for _f in ("vdm_precompute_kv", "vdm_decode_dense", "vdm_select_kv",
            "vdm_hierarchical_workspace_size", "vdm_decode_hierarchical",
-           "vdm_profile_begin", "vdm_profile_end"):
+           "vdm_decode_hierarchical_noalloc", "vdm_profile_begin", "vdm_profile_end"):
     getattr(_lib, _f).restype = C.c_int
 _lib.vdm_status_string.argtypes = [C.c_int]
 _lib.vdm_status_string.restype = C.c_char_p
@@ -272,6 +275,25 @@ def vdm_decode_hierarchical(dec: Decoder, K, V, params: CHierParams, spheres=Non
                                                     "tiles", "selected_tiles", "probes")}
           for b in range(B)]
     return out, st
+
+
+def vdm_decode_hierarchical_noalloc(dec: Decoder, K, V, params: CHierParams, spheres=None,
+                                    dec_scale: float = 0.0, out=None, stream=None):
+    """``vdm_decode_hierarchical`` with the library's built-in 32 MiB scratch
+    instead of a caller workspace (for callers that may not allocate device
+    memory).  Only the output grid is passed in."""
+    torch = _torch()
+    B, H, N, _ = K.shape
+    Rf = params.r0 << (params.n_levels - 1)
+    if out is None:
+        out = torch.empty((B, Rf, Rf, Rf), device=K.device, dtype=torch.float32)
+    stats = (CHierStats * B)()
+    cd = dec.cstruct()
+    an = _analytic(spheres, dec_scale)
+    _check(_lib.vdm_decode_hierarchical_noalloc(C.byref(cd), K.data_ptr(), V.data_ptr(), B, N,
+                                                C.byref(params), C.byref(an) if an else None,
+                                                out.data_ptr(), stats, None, _stream(stream)))
+    return out
 
 
 def vdm_profile_begin():
