@@ -1,0 +1,956 @@
+// Fused vecset decoder on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
+//
+// The decoder of FlashVDM ("Unleashing Vecset Diffusion Model for Fast Shape
+// Generation", aipaper.cc summary, section 3: cross-attention from query
+// points to the latent set, then the SDF; section 4.1 item 2: attention over
+// a per-sub-volume token subset) for bf16 weights and K/V, fp32 accumulation.
+// One persistent CTA per SM decodes 128-query tiles; nothing but the final
+// SDF value (and, for probe queries, their softmax statistics) leaves the SM.
+//
+// Warp roles (192 threads):
+//   warps 0-3  compute: one thread per query row = TMEM lane; embedding,
+//              softmax, LayerNorms, GELU, SDF head;
+//   warp 4     MMA issue (one lane);
+//   warp 5     producer: TMA loads of weights and of contiguous K/V blocks,
+//              cp.async gathers of a sub-volume's selected K/V rows;
+// connected only by mbarriers (no CTA-wide barrier inside a tile).
+//
+// Per tile:
+//   PE (bf16 smem) ; per head h: Q_h = PE Wq_h^T (TMEM) -> bf16 in TMEM;
+//   per 128-token block j: S_j = Q_h K_j^T ; softmax -> P_j (bf16, TMEM) ;
+//   O += P_j V_j ; a[:, h] = O / l (bf16 smem).
+//   X = PE Wq^T + a Wo^T ; LN1 -> bf16 smem ; MLP hidden chunks:
+//   H_c = LN1(x1) W1_c^T, GELU, X += GELU(H_c) W2_c^T ; LN2 . w_head -> SDF.
+//
+// TMEM (512 columns x 128 lanes):
+//   attention: S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384) O [384,448)
+//              Q accumulator / packed bf16 Q [448,512)
+//   output projection: X [0, C)
+//   MLP, C <= 256: acc [0, C); hidden chunks (128 wide) at [256,384) [384,512)
+//   MLP, C == 512: the 128 x 512 fp32 residual alone fills TMEM, so the MLP
+//              output is produced in two 256-wide halves (the hidden projection
+//              is recomputed for the second half); while the first half runs,
+//              x1's second half waits in TMEM as bf16 [256,384); hidden chunks
+//              (64 wide) at [384,448) [448,512).
+//
+// Softmax: logits in log2 units (the 1/8 scale and log2 e folded into Q);
+// the running maximum is only raised when a block exceeds it by more than 8
+// (then O and the sum are rescaled), so P stays <= 2^8.
+//
+// Barrier protocol: waits are parity based, so every waiter observes every
+// phase of the barriers it uses, and no barrier can run two phases ahead of a
+// waiter (each producer step depends on the waiter's previous step).
+// Every wait on an mbarrier is bounded: on expiry the kernel records the site
+// in an error word, flags the CTA and winds down.
+#include <cuda.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "tc_ptx.cuh"
+#include "vdm_internal.cuh"
+
+namespace vdm {
+
+namespace {
+
+using namespace ptx;
+
+constexpr int BM = 128;        // queries per tile (TMEM lanes)
+constexpr int NCOMP = 128;     // compute threads
+constexpr int NT = 192;        // + MMA warp + producer warp
+constexpr int WARP_MMA = 4, WARP_PROD = 5;
+constexpr int SLOT = 16384;    // ring slot bytes
+constexpr int MAX_NS = 8;
+constexpr int GATHER_LAG = 2;  // gathered items in flight before their barrier is signalled
+constexpr float kLog2e = 1.4426950408889634f;
+
+constexpr uint32_t T_S0 = 0, T_S1 = 128, T_P0 = 256, T_P1 = 320, T_O = 384, T_Q = 448;
+
+struct TcArgs {
+    DecodeArgs d;
+    int ns;
+    int* err;
+    long long timeout;   // cycles per bounded wait
+};
+
+struct Shared {
+    uint64_t full[MAX_NS], empty[MAX_NS];
+    // MMA commits (count 1); bar_hd and bar_w2 are waited on by the MMA warp only
+    uint64_t bar_q, bar_s[2], bar_pv, bar_x, bar_h[2], bar_acc, bar_hd, bar_w2;
+    // compute-warp arrivals (count 128)
+    uint64_t bar_pe, bar_qc, bar_p[2], bar_a, bar_hin, bar_r, bar_g[2], bar_cs;
+    uint32_t tmem_base;
+    int abort;
+    float G, Bc;
+};
+
+struct Waiter {
+    Shared* sh;
+    int* err;
+    long long timeout;
+    // Wait for the phase with parity `phase` to complete; flips `phase`.
+    __device__ bool wait(uint64_t* bar, uint32_t& phase, int site) {
+        const uint32_t b = smem_u32(bar);
+        long long t0 = 0;
+        for (uint32_t it = 0;; ++it) {
+            if (mbar_try_wait(b, phase)) {
+                phase ^= 1;
+                return true;
+            }
+            if ((it & 63) == 63) {
+                if (*reinterpret_cast<volatile int*>(&sh->abort)) return false;
+                const long long t = clock64();
+                if (t0 == 0) t0 = t;
+                else if (t - t0 > timeout) {
+                    *reinterpret_cast<volatile int*>(&sh->abort) = 1;
+                    atomicCAS(err, 0, site);
+                    return false;
+                }
+            }
+        }
+    }
+};
+
+__device__ __forceinline__ uint32_t swz(uint32_t base, int r, int c) {
+    return base + r * 128 + ((c ^ (r & 7)) << 4);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t* w) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                 "r"(w[3])
+                 : "memory");
+}
+
+// Work unit -> queries (identical in every role).
+struct Unit {
+    int nq;
+    int64_t qbeg;        // first query slot
+    int t;               // tile (tile modes)
+    int first;           // first position inside the tile's dense / sparse range
+    const int32_t* sel;  // selected tokens (sparse mode)
+};
+
+__device__ __forceinline__ Unit unit_of(const DecodeArgs& a, int64_t unit) {
+    Unit u;
+    u.sel = nullptr;
+    u.t = -1;
+    u.first = 0;
+    if (a.work == kWorkFlat) {
+        u.qbeg = unit * BM;
+        u.nq = (int)(a.M - u.qbeg < BM ? a.M - u.qbeg : BM);
+        return u;
+    }
+    const int t = (int)(unit / a.slots), sl = (int)(unit - (int64_t)t * a.slots);
+    const int cnt = 8 * (a.tile_off[t + 1] - a.tile_off[t]);
+    int lo, n;
+    if (a.work == kWorkTileDense) {
+        lo = 0;
+        n = cnt < a.n_probe ? cnt : a.n_probe;
+    } else {
+        lo = a.n_probe;
+        n = cnt > a.n_probe ? cnt - a.n_probe : 0;
+        u.sel = a.sel + (size_t)t * a.ksel;
+    }
+    const int first = lo + sl * BM;
+    u.nq = first < lo + n ? min(BM, lo + n - first) : 0;
+    u.qbeg = 8 * (int64_t)a.tile_off[t] + first;
+    u.t = t;
+    u.first = first;
+    return u;
+}
+
+// ---------------------------------------------------------------- the kernel
+__global__ void __launch_bounds__(NT, 1)
+decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_wq64,
+                 const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_w1,
+                 const __grid_constant__ CUtensorMap tm_w2, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const TcArgs ta) {
+    const DecodeArgs& a = ta.d;
+    extern __shared__ uint8_t dyn_raw[];
+    __shared__ Shared sh;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int C = a.C, H = a.H, F = a.F, N = a.N;
+    const int NA = C / 64;
+    const bool halves = C > 256;
+    const int HN = halves ? 64 : 128;
+    const int NS = ta.ns;
+    const int CW = halves ? 256 : C;
+    const int n_half = halves ? 2 : 1;
+    const uint32_t T_H0 = halves ? 384 : 256, T_H1 = halves ? 448 : 384;
+    const int n_chunks = F / HN;
+    const int w1_gran = NA;
+    const int w2_gran = (CW / 128) * (HN / 64);
+
+    const uint32_t dyn0 = (smem_u32(dyn_raw) + 1023u) & ~1023u;
+    const uint32_t s_abuf = dyn0;
+    const uint32_t s_pe = s_abuf + NA * 16384;
+    const uint32_t s_ring = s_pe + 16384;
+
+    Waiter W{&sh, ta.err, ta.timeout};
+
+    if (tid == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(smem_u32(&sh.full[i]), 1);
+            mbar_init(smem_u32(&sh.empty[i]), 1);
+        }
+        uint64_t* one[] = {&sh.bar_q, &sh.bar_s[0], &sh.bar_s[1], &sh.bar_pv, &sh.bar_x,
+                           &sh.bar_h[0], &sh.bar_h[1], &sh.bar_acc, &sh.bar_hd, &sh.bar_w2};
+        for (auto* b : one) mbar_init(smem_u32(b), 1);
+        uint64_t* many[] = {&sh.bar_pe, &sh.bar_qc, &sh.bar_p[0], &sh.bar_p[1], &sh.bar_a,
+                            &sh.bar_hin, &sh.bar_r, &sh.bar_g[0], &sh.bar_g[1], &sh.bar_cs};
+        for (auto* b : many) mbar_init(smem_u32(b), NCOMP);
+        sh.abort = 0;
+        fence_mbar_init();
+        fence_proxy_async();
+    }
+    if (warp == 1) {
+        float g = 0.f, bc = 0.f;
+        for (int c = lane; c < C; c += 32) {
+            const float w = a.w_head[c];
+            g += a.query_ln ? w * a.ln2_g[c] : w;
+            bc += a.query_ln ? w * a.ln2_b[c] : 0.f;
+        }
+        for (int o = 16; o; o >>= 1) {
+            g += __shfl_xor_sync(0xffffffffu, g, o);
+            bc += __shfl_xor_sync(0xffffffffu, bc, o);
+        }
+        if (lane == 0) {
+            sh.G = g;
+            sh.Bc = bc + a.b_head[0];
+        }
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&sh.tmem_base), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+
+    const int64_t n_units = a.work == kWorkFlat ? (a.M + BM - 1) / BM : (int64_t)a.T * a.slots;
+
+    // ==================================================================== producer
+    if (warp == WARP_PROD) {
+        uint32_t ring_head = 0;
+        int pend[GATHER_LAG + 1];
+        int n_pend = 0;
+        const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.K);
+        const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.V);
+        bool ok = true;
+        auto signal_oldest = [&]() {
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sh.full[pend[0]]));
+            for (int i = 1; i < n_pend; ++i) pend[i - 1] = pend[i];
+            --n_pend;
+        };
+        auto drain = [&]() {
+            if (n_pend == 0) return;
+            cp_async_wait<0>();
+            while (n_pend > 0) signal_oldest();
+        };
+        auto take_slot = [&](int& slot) -> bool {
+            slot = ring_head % NS;
+            if (ring_head >= (uint32_t)NS) {
+                uint32_t ph = ((ring_head / NS) + 1) & 1;
+                if (!W.wait(&sh.empty[slot], ph, 40)) return false;
+            }
+            ++ring_head;
+            return true;
+        };
+        auto push_tma = [&](const CUtensorMap* m, int x, int y, uint32_t bytes) -> bool {
+            drain();
+            int slot;
+            if (!take_slot(slot)) return false;
+            if (lane == 0) {
+                const uint32_t fb = smem_u32(&sh.full[slot]);
+                mbar_expect_tx(fb, bytes);
+                tma_load_2d(s_ring + slot * SLOT, m, x, y, fb);
+            }
+            __syncwarp();
+            return true;
+        };
+        auto push_gather = [&](const __nv_bfloat16* src, const int32_t* sel, int h, int j, int nk) -> bool {
+            int slot;
+            if (!take_slot(slot)) return false;
+            const uint32_t dst = s_ring + slot * SLOT;
+            for (int i = 0; i < 32; ++i) {   // 128 rows x 8 chunks, 32 lanes
+                const int idx = i * 32 + lane;
+                const int r = idx >> 3, c = idx & 7;
+                const int tok = j * 128 + r;
+                const bool okr = tok < nk;
+                const int row = okr ? sel[tok] : 0;
+                cp_async16(swz(dst, r, c), src + ((size_t)h * N + row) * 64 + c * 8, okr);
+            }
+            cp_async_commit();
+            pend[n_pend++] = slot;
+            if (n_pend > GATHER_LAG) {
+                cp_async_wait<GATHER_LAG>();
+                signal_oldest();
+            }
+            return true;
+        };
+        for (int64_t unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+            const Unit u = unit_of(a, unit);
+            if (u.nq <= 0) continue;
+            const int nk = u.sel ? a.ksel : N;
+            const int nb = (nk + 127) / 128;
+            auto push_kv = [&](bool isv, int h, int j) -> bool {
+                if (u.sel) return push_gather(isv ? Vg : Kg, u.sel, h, j, nk);
+                return push_tma(isv ? &tm_v : &tm_k, 0, h * N + j * 128, SLOT);
+            };
+            for (int h = 0; h < H && ok; ++h) {
+                ok = push_tma(&tm_wq64, 0, h * 64, 64 * 128);
+                ok = ok && push_kv(false, h, 0);
+                if (nb > 1) ok = ok && push_kv(false, h, 1);
+                for (int j = 0; j < nb && ok; ++j) {
+                    ok = push_kv(true, h, j);
+                    if (j + 2 < nb) ok = ok && push_kv(false, h, j + 2);
+                }
+            }
+            // X = PE Wq^T + a Wo^T : granule (nc, ka)
+            const int KA = NA + 1;
+            for (int g = 0; g < (C / 128) * KA && ok; ++g) {
+                const int nc = g / KA, ka = g % KA;
+                ok = ka == 0 ? push_tma(&tm_wq, 0, nc * 128, SLOT) : push_tma(&tm_wo, (ka - 1) * 64, nc * 128, SLOT);
+            }
+            // MLP granules in MMA consumption order
+            for (int hf = 0; hf < n_half && ok; ++hf) {
+                auto w1 = [&](int c) {
+                    for (int s = 0; s < w1_gran && ok; ++s) ok = push_tma(&tm_w1, s * 64, c * HN, HN * 128);
+                };
+                auto w2 = [&](int c) {
+                    for (int q = 0; q < w2_gran && ok; ++q) {
+                        const int nc = q / (HN / 64), kh = q % (HN / 64);
+                        ok = push_tma(&tm_w2, c * HN + kh * 64, hf * 256 + nc * 128, SLOT);
+                    }
+                };
+                w1(0);
+                if (n_chunks > 1) w1(1);
+                for (int c = 0; c < n_chunks && ok; ++c) {
+                    w2(c);
+                    if (c + 2 < n_chunks) w1(c + 2);
+                }
+            }
+        }
+        drain();
+    }
+    // ==================================================================== MMA issue
+    else if (warp == WARP_MMA) {
+        if (lane == 0) {
+            uint32_t ring_tail = 0;
+            uint32_t ph_pe = 0, ph_qc = 0, ph_p[2] = {0, 0}, ph_a = 0, ph_hin = 0, ph_r = 0, ph_g[2] = {0, 0};
+            uint32_t ph_hd = 0, ph_w2 = 0;
+            bool ok = true;
+            auto consume = [&](int& slot) -> bool {
+                slot = ring_tail % NS;
+                uint32_t ph = (ring_tail / NS) & 1;
+                if (!W.wait(&sh.full[slot], ph, 50)) return false;
+                tc_fence_after();
+                ++ring_tail;
+                return true;
+            };
+            auto release = [&](int slot) { mma_commit(smem_u32(&sh.empty[slot])); };
+            for (int64_t unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+                const Unit u = unit_of(a, unit);
+                if (u.nq <= 0) continue;
+                const int nk = u.sel ? a.ksel : N;
+                const int nb = (nk + 127) / 128;
+                if (!(ok = W.wait(&sh.bar_pe, ph_pe, 51))) break;
+                tc_fence_after();
+                for (int h = 0; h < H && ok; ++h) {
+                    int slot;
+                    // Q_h = PE Wq_h^T (M=128, N=64, K=64)
+                    if (!(ok = consume(slot))) break;
+                    {
+                        const uint64_t da = desc_sw128(s_pe), db = desc_sw128(s_ring + slot * SLOT);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ss(tmem + T_Q, da + 2 * kk, db + 2 * kk, idesc_bf16(128, 64, false), kk > 0);
+                        release(slot);
+                        mma_commit(smem_u32(&sh.bar_q));
+                    }
+                    if (!(ok = W.wait(&sh.bar_qc, ph_qc, 52))) break;
+                    tc_fence_after();
+                    auto issue_s = [&](int j) -> bool {
+                        int sl;
+                        if (!consume(sl)) return false;
+                        const uint64_t db = desc_sw128(s_ring + sl * SLOT);
+                        const uint32_t sd = tmem + ((j & 1) ? T_S1 : T_S0);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ts(sd, tmem + T_Q + 8 * kk, db + 2 * kk, idesc_bf16(128, 128, false), kk > 0);
+                        release(sl);
+                        mma_commit(smem_u32(&sh.bar_s[j & 1]));
+                        return true;
+                    };
+                    ok = issue_s(0) && (nb < 2 || issue_s(1));
+                    for (int j = 0; j < nb && ok; ++j) {
+                        if (!(ok = W.wait(&sh.bar_p[j & 1], ph_p[j & 1], 53))) break;
+                        tc_fence_after();
+                        if (!(ok = consume(slot))) break;
+                        const uint32_t pa = tmem + ((j & 1) ? T_P1 : T_P0);
+                        const uint64_t dv = desc_sw128(s_ring + slot * SLOT);
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_ts(tmem + T_O, pa + 8 * kk, dv + 128 * kk, idesc_bf16(128, 64, true), (j > 0 || kk > 0));
+                        release(slot);
+                        mma_commit(smem_u32(&sh.bar_pv));
+                        if (j + 2 < nb) ok = issue_s(j + 2);
+                    }
+                    if (!ok) break;
+                    // the next head's Q projection rewrites T_Q, which this head's S MMAs read
+                    mma_commit(smem_u32(&sh.bar_hd));
+                    if (!(ok = W.wait(&sh.bar_hd, ph_hd, 54))) break;
+                    tc_fence_after();
+                }
+                if (!ok) break;
+                // ---- X = PE Wq^T + a Wo^T
+                if (!(ok = W.wait(&sh.bar_a, ph_a, 55))) break;
+                tc_fence_after();
+                const int KA = NA + 1;
+                for (int g = 0; g < (C / 128) * KA && ok; ++g) {
+                    int slot;
+                    if (!(ok = consume(slot))) break;
+                    const int nc = g / KA, ka = g % KA;
+                    const uint64_t da = desc_sw128(ka == 0 ? s_pe : s_abuf + (ka - 1) * 16384);
+                    const uint64_t db = desc_sw128(s_ring + slot * SLOT);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tmem + nc * 128, da + 2 * kk, db + 2 * kk, idesc_bf16(128, 128, false),
+                               (ka > 0 || kk > 0));
+                    release(slot);
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&sh.bar_x));
+                // ---- MLP
+                if (!(ok = W.wait(&sh.bar_hin, ph_hin, 56))) break;
+                tc_fence_after();
+                for (int hf = 0; hf < n_half && ok; ++hf) {
+                    if (hf == 1) {
+                        if (!(ok = W.wait(&sh.bar_r, ph_r, 57))) break;
+                        tc_fence_after();
+                    }
+                    auto issue_w1 = [&](int c) -> bool {
+                        const uint32_t hd = tmem + ((c & 1) ? T_H1 : T_H0);
+                        for (int ka = 0; ka < NA; ++ka) {
+                            int sl;
+                            if (!consume(sl)) return false;
+                            const uint64_t da = desc_sw128(s_abuf + ka * 16384);
+                            const uint64_t db = desc_sw128(s_ring + sl * SLOT);
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_ss(hd, da + 2 * kk, db + 2 * kk, idesc_bf16(128, HN, false), (ka > 0 || kk > 0));
+                            release(sl);
+                        }
+                        mma_commit(smem_u32(&sh.bar_h[c & 1]));
+                        return true;
+                    };
+                    auto issue_w2 = [&](int c) -> bool {
+                        const uint32_t ha = tmem + ((c & 1) ? T_H1 : T_H0);
+                        for (int q = 0; q < w2_gran; ++q) {
+                            int sl;
+                            if (!consume(sl)) return false;
+                            const int nc = q / (HN / 64), kh = q % (HN / 64);
+                            const uint64_t db = desc_sw128(s_ring + sl * SLOT);
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_ts(tmem + nc * 128, ha + kh * 32 + 8 * kk, db + 2 * kk,
+                                       idesc_bf16(128, 128, false), 1u);
+                            release(sl);
+                        }
+                        return true;
+                    };
+                    ok = issue_w1(0) && (n_chunks < 2 || issue_w1(1));
+                    for (int c = 0; c < n_chunks && ok; ++c) {
+                        if (!(ok = W.wait(&sh.bar_g[c & 1], ph_g[c & 1], 58))) break;
+                        tc_fence_after();
+                        if (!(ok = issue_w2(c))) break;
+                        if (c + 2 < n_chunks) {
+                            // H[c%2] is re-written by W1(c+2): W2(c) must have read it first
+                            mma_commit(smem_u32(&sh.bar_w2));
+                            if (!(ok = W.wait(&sh.bar_w2, ph_w2, 59))) break;
+                            tc_fence_after();
+                            ok = issue_w1(c + 2);
+                        }
+                    }
+                    if (!ok) break;
+                    mma_commit(smem_u32(&sh.bar_acc));   // the half's accumulator is complete
+                }
+            }
+        }
+    }
+    // ==================================================================== compute warps
+    else {
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t trow = tmem + lane_off;
+        uint32_t ph_q = 0, ph_s[2] = {0, 0}, ph_pv = 0, ph_x = 0, ph_h[2] = {0, 0}, ph_acc = 0, ph_cs = 0;
+        const float qscale = 0.125f * kLog2e;
+        bool ok = true;
+        auto arrive = [&](uint64_t* b) { mbar_arrive(smem_u32(b)); };
+        for (int64_t unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+            const Unit u = unit_of(a, unit);
+            if (u.nq <= 0) continue;
+            const int nk = u.sel ? a.ksel : N;
+            const int nb = (nk + 127) / 128;
+            // ---- this row's query
+            float p[3] = {0.f, 0.f, 0.f};
+            int64_t vox = -1, qid = -1;
+            if (tid < u.nq) {
+                const int64_t slot = u.qbeg + tid;
+                qid = slot;
+                if (a.qmode == kQueryXyz) {
+                    p[0] = a.xyz[slot * 3];
+                    p[1] = a.xyz[slot * 3 + 1];
+                    p[2] = a.xyz[slot * 3 + 2];
+                } else if (a.qmode == kQueryGrid) {
+                    vox = slot;
+                    voxel_point(vox, a.R, p);
+                } else {
+                    const int e = a.qorder ? a.qorder[slot] : (int)slot;
+                    vox = child_index(a.plist[e >> 3], e & 7, a.R);
+                    voxel_point(vox, a.R, p);
+                }
+            }
+            for (int c = 0; c < 8; ++c) {
+                uint32_t w[4];
+                for (int v = 0; v < 4; ++v) w[v] = pack_bf16(pe_lane(p, c * 8 + 2 * v), pe_lane(p, c * 8 + 2 * v + 1));
+                st_shared_v4(swz(s_pe, tid, c), w);
+            }
+            fence_proxy_async();
+            arrive(&sh.bar_pe);
+            float* ml_out = (a.probe_ml && a.work == kWorkTileDense && tid < u.nq)
+                                ? a.probe_ml + ((size_t)u.t * a.n_probe + u.first + tid) * H * 2
+                                : nullptr;
+            // ================================================= attention
+            for (int h = 0; h < H && ok; ++h) {
+                if (!(ok = W.wait(&sh.bar_q, ph_q, 60))) break;
+                tc_fence_after();
+                {
+                    float q0[32], q1[32];
+                    tmem_ld32(trow + T_Q, q0);
+                    tmem_ld32(trow + T_Q + 32, q1);
+                    tmem_wait_ld();
+                    reg_fence(q0);
+                    reg_fence(q1);
+                    uint32_t pk[32];
+                    for (int v = 0; v < 16; ++v) {
+                        const int c0 = h * 64 + 2 * v, c1 = h * 64 + 32 + 2 * v;
+                        pk[v] = pack_bf16((q0[2 * v] + a.bq[c0]) * qscale, (q0[2 * v + 1] + a.bq[c0 + 1]) * qscale);
+                        pk[16 + v] = pack_bf16((q1[2 * v] + a.bq[c1]) * qscale, (q1[2 * v + 1] + a.bq[c1 + 1]) * qscale);
+                    }
+                    tmem_st32(trow + T_Q, pk);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                arrive(&sh.bar_qc);
+                float m_ref = -INFINITY, l_run = 0.f;
+                for (int j = 0; j < nb; ++j) {
+                    if (!(ok = W.wait(&sh.bar_s[j & 1], ph_s[j & 1], 61))) break;
+                    tc_fence_after();
+                    const uint32_t sbase = trow + ((j & 1) ? T_S1 : T_S0);
+                    float s0[32], s1[32], s2[32], s3[32];
+                    tmem_ld32(sbase, s0);
+                    tmem_ld32(sbase + 32, s1);
+                    tmem_ld32(sbase + 64, s2);
+                    tmem_ld32(sbase + 96, s3);
+                    tmem_wait_ld();
+                    reg_fence(s0);
+                    reg_fence(s1);
+                    reg_fence(s2);
+                    reg_fence(s3);
+                    const int valid = nk - j * 128;
+                    if (valid < 128) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            if (c >= valid) s0[c] = -INFINITY;
+                            if (c + 32 >= valid) s1[c] = -INFINITY;
+                            if (c + 64 >= valid) s2[c] = -INFINITY;
+                            if (c + 96 >= valid) s3[c] = -INFINITY;
+                        }
+                    }
+                    float mb = -INFINITY;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) mb = fmaxf(mb, fmaxf(fmaxf(s0[c], s1[c]), fmaxf(s2[c], s3[c])));
+                    const bool need = (j == 0) || (mb > m_ref + 8.0f);
+                    const float m_new = need ? fmaxf(mb, m_ref) : m_ref;
+                    const float f = (j == 0) ? 0.f : ex2(m_ref - m_new);
+                    if (need) m_ref = m_new;
+                    float ls = 0.f;
+                    uint32_t pk0[32], pk1[32];
+#pragma unroll
+                    for (int v = 0; v < 16; ++v) {
+                        const float e0 = ex2(s0[2 * v] - m_ref), e1 = ex2(s0[2 * v + 1] - m_ref);
+                        const float e2 = ex2(s1[2 * v] - m_ref), e3 = ex2(s1[2 * v + 1] - m_ref);
+                        const float e4 = ex2(s2[2 * v] - m_ref), e5 = ex2(s2[2 * v + 1] - m_ref);
+                        const float e6 = ex2(s3[2 * v] - m_ref), e7 = ex2(s3[2 * v + 1] - m_ref);
+                        ls += (e0 + e1) + (e2 + e3) + (e4 + e5) + (e6 + e7);
+                        pk0[v] = pack_bf16(e0, e1);
+                        pk0[16 + v] = pack_bf16(e2, e3);
+                        pk1[v] = pack_bf16(e4, e5);
+                        pk1[16 + v] = pack_bf16(e6, e7);
+                    }
+                    // P_j's buffer was read by PV_{j-2}; O is rescaled below: PV_{j-1} must be done
+                    if (j > 0) {
+                        if (!(ok = W.wait(&sh.bar_pv, ph_pv, 62))) break;
+                        tc_fence_after();
+                    }
+                    if (need && j > 0) l_run *= f;
+                    l_run += ls;
+                    if (j > 0 && __any_sync(0xffffffffu, need)) {
+                        float o0[32], o1[32];
+                        tmem_ld32(trow + T_O, o0);
+                        tmem_ld32(trow + T_O + 32, o1);
+                        tmem_wait_ld();
+                        reg_fence(o0);
+                        reg_fence(o1);
+                        const float g = need ? f : 1.0f;
+                        uint32_t u0[32], u1[32];
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            u0[c] = __float_as_uint(o0[c] * g);
+                            u1[c] = __float_as_uint(o1[c] * g);
+                        }
+                        tmem_st32(trow + T_O, u0);
+                        tmem_st32(trow + T_O + 32, u1);
+                    }
+                    const uint32_t pbase = trow + ((j & 1) ? T_P1 : T_P0);
+                    tmem_st32(pbase, pk0);
+                    tmem_st32(pbase + 32, pk1);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    arrive(&sh.bar_p[j & 1]);
+                }
+                if (!ok) break;
+                if (!(ok = W.wait(&sh.bar_pv, ph_pv, 63))) break;   // PV_{nb-1}
+                tc_fence_after();
+                {
+                    float o0[32], o1[32];
+                    tmem_ld32(trow + T_O, o0);
+                    tmem_ld32(trow + T_O + 32, o1);
+                    tmem_wait_ld();
+                    reg_fence(o0);
+                    reg_fence(o1);
+                    const float inv = 1.0f / l_run;
+                    const uint32_t atom = s_abuf + h * 16384;
+                    for (int c = 0; c < 8; ++c) {
+                        const float* src = c < 4 ? &o0[c * 8] : &o1[(c - 4) * 8];
+                        uint32_t w[4];
+                        for (int v = 0; v < 4; ++v) w[v] = pack_bf16(src[2 * v] * inv, src[2 * v + 1] * inv);
+                        st_shared_v4(swz(atom, tid, c), w);
+                    }
+                }
+                if (ml_out) {
+                    ml_out[h * 2] = m_ref;
+                    ml_out[h * 2 + 1] = l_run;
+                }
+            }
+            if (!ok) break;
+            fence_proxy_async();
+            tc_fence_before();
+            arrive(&sh.bar_a);
+            // ================================================= LN1
+            if (!(ok = W.wait(&sh.bar_x, ph_x, 64))) break;
+            tc_fence_after();
+            float mean1 = 0.f, rstd1 = 1.f;
+            {
+                float sum = 0.f;
+                for (int cc = 0; cc < C; cc += 32) {
+                    float v[32];
+                    tmem_ld32_sync(trow + cc, v);
+                    for (int e = 0; e < 32; ++e) sum += v[e] + a.bq[cc + e] + a.bo[cc + e];
+                }
+                mean1 = sum / (float)C;
+                if (a.query_ln) {
+                    float m2 = 0.f;
+                    for (int cc = 0; cc < C; cc += 32) {
+                        float v[32];
+                        tmem_ld32_sync(trow + cc, v);
+                        for (int e = 0; e < 32; ++e) {
+                            const float d = v[e] + a.bq[cc + e] + a.bo[cc + e] - mean1;
+                            m2 = fmaf(d, d, m2);
+                        }
+                    }
+                    rstd1 = rsqrtf(m2 / (float)C + kLnEps);
+                }
+                for (int cc = 0; cc < C; cc += 32) {
+                    float v[32];
+                    tmem_ld32_sync(trow + cc, v);
+                    uint32_t w[16];
+                    for (int e = 0; e < 16; ++e) {
+                        float y0 = v[2 * e] + a.bq[cc + 2 * e] + a.bo[cc + 2 * e];
+                        float y1 = v[2 * e + 1] + a.bq[cc + 2 * e + 1] + a.bo[cc + 2 * e + 1];
+                        if (a.query_ln) {
+                            y0 = (y0 - mean1) * rstd1 * a.ln1_g[cc + 2 * e] + a.ln1_b[cc + 2 * e];
+                            y1 = (y1 - mean1) * rstd1 * a.ln1_g[cc + 2 * e + 1] + a.ln1_b[cc + 2 * e + 1];
+                        }
+                        w[e] = pack_bf16(y0, y1);
+                    }
+                    const uint32_t atom = s_abuf + (cc / 64) * 16384;
+                    const int c0 = (cc % 64) / 8;
+                    for (int q = 0; q < 4; ++q) st_shared_v4(swz(atom, tid, c0 + q), &w[4 * q]);
+                }
+                if (halves) {
+                    for (int i = 0; i < 4; ++i) {
+                        float v0[32], v1[32];
+                        tmem_ld32(trow + 256 + 64 * i, v0);
+                        tmem_ld32(trow + 256 + 64 * i + 32, v1);
+                        tmem_wait_ld();
+                        reg_fence(v0);
+                        reg_fence(v1);
+                        uint32_t w[32];
+                        for (int e = 0; e < 16; ++e) {
+                            w[e] = pack_bf16(v0[2 * e], v0[2 * e + 1]);
+                            w[16 + e] = pack_bf16(v1[2 * e], v1[2 * e + 1]);
+                        }
+                        tmem_st32(trow + 256 + 32 * i, w);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            arrive(&sh.bar_hin);
+            // ================================================= MLP
+            float hs_mean0 = 0.f, hs_m20 = 0.f, hs_dot0 = 0.f, hs_mean1 = 0.f, hs_m21 = 0.f, hs_dot1 = 0.f;
+            for (int hf = 0; hf < n_half && ok; ++hf) {
+                if (hf == 1) {
+                    for (int i = 0; i < 4; ++i) {
+                        float pv[32];
+                        tmem_ld32_sync(trow + 256 + 32 * i, pv);
+                        uint32_t w0[32], w1[32];
+                        for (int e = 0; e < 16; ++e) {
+                            const uint32_t x = __float_as_uint(pv[e]);
+                            w0[2 * e] = __float_as_uint(bf16_lo(x));
+                            w0[2 * e + 1] = __float_as_uint(bf16_hi(x));
+                            const uint32_t y = __float_as_uint(pv[16 + e]);
+                            w1[2 * e] = __float_as_uint(bf16_lo(y));
+                            w1[2 * e + 1] = __float_as_uint(bf16_hi(y));
+                        }
+                        tmem_st32(trow + 64 * i, w0);
+                        tmem_st32(trow + 64 * i + 32, w1);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    arrive(&sh.bar_r);
+                }
+                for (int c = 0; c < n_chunks; ++c) {
+                    if (!(ok = W.wait(&sh.bar_h[c & 1], ph_h[c & 1], 65))) break;
+                    tc_fence_after();
+                    const uint32_t hb = trow + ((c & 1) ? T_H1 : T_H0);
+                    for (int part = 0; part < HN / 64; ++part) {
+                        float v0[32], v1[32];
+                        tmem_ld32(hb + part * 64, v0);
+                        tmem_ld32(hb + part * 64 + 32, v1);
+                        tmem_wait_ld();
+                        reg_fence(v0);
+                        reg_fence(v1);
+                        uint32_t w[32];
+                        const int f0 = c * HN + part * 64;
+                        for (int e = 0; e < 16; ++e) {
+                            w[e] = pack_bf16(gelu_erf(v0[2 * e] + a.b1[f0 + 2 * e]),
+                                             gelu_erf(v0[2 * e + 1] + a.b1[f0 + 2 * e + 1]));
+                            w[16 + e] = pack_bf16(gelu_erf(v1[2 * e] + a.b1[f0 + 32 + 2 * e]),
+                                                  gelu_erf(v1[2 * e + 1] + a.b1[f0 + 32 + 2 * e + 1]));
+                        }
+                        tmem_st32(hb + part * 32, w);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    arrive(&sh.bar_g[c & 1]);
+                }
+                if (!ok) break;
+                if (!(ok = W.wait(&sh.bar_acc, ph_acc, 67))) break;
+                tc_fence_after();
+                const int cb = hf * 256;
+                float sum = 0.f, dot = 0.f;
+                for (int cc = 0; cc < CW; cc += 32) {
+                    float v[32];
+                    tmem_ld32_sync(trow + cc, v);
+                    for (int e = 0; e < 32; ++e) {
+                        const int col = cb + cc + e;
+                        const float x = v[e] + a.bq[col] + a.bo[col] + a.b2[col];
+                        sum += x;
+                        dot = fmaf(x, a.query_ln ? a.w_head[col] * a.ln2_g[col] : a.w_head[col], dot);
+                    }
+                }
+                const float mh = sum / (float)CW;
+                float m2 = 0.f;
+                if (a.query_ln) {
+                    for (int cc = 0; cc < CW; cc += 32) {
+                        float v[32];
+                        tmem_ld32_sync(trow + cc, v);
+                        for (int e = 0; e < 32; ++e) {
+                            const int col = cb + cc + e;
+                            const float d = v[e] + a.bq[col] + a.bo[col] + a.b2[col] - mh;
+                            m2 = fmaf(d, d, m2);
+                        }
+                    }
+                }
+                if (hf == 0) {
+                    hs_mean0 = mh;
+                    hs_m20 = m2;
+                    hs_dot0 = dot;
+                } else {
+                    hs_mean1 = mh;
+                    hs_m21 = m2;
+                    hs_dot1 = dot;
+                }
+            }
+            if (!ok) break;
+            // ================================================= head + output
+            float dec;
+            if (a.query_ln) {
+                float mean, m2;
+                if (n_half == 1) {
+                    mean = hs_mean0;
+                    m2 = hs_m20;
+                } else {
+                    const float d = hs_mean1 - hs_mean0;
+                    mean = 0.5f * (hs_mean0 + hs_mean1);
+                    m2 = hs_m20 + hs_m21 + d * d * 0.25f * (float)C;
+                }
+                const float rstd = rsqrtf(m2 / (float)C + kLnEps);
+                dec = (hs_dot0 + hs_dot1 - mean * sh.G) * rstd + sh.Bc;
+            } else {
+                dec = hs_dot0 + hs_dot1 + sh.Bc;
+            }
+            if (tid < u.nq) {
+                float val = dec;
+                if (a.spheres) val = sphere_union(p, a.spheres, a.n_spheres) + a.dec_scale * tanhf(dec);
+                if (a.out) a.out[qid] = val;
+                if (vox >= 0) {
+                    if (a.grid) a.grid[vox] = val;
+                    if (a.dec_grid) a.dec_grid[vox] = dec;
+                }
+            }
+            // the next tile's first MMA waits for bar_pe, which these threads
+            // only arrive at after every TMEM / smem read of this tile (a bounded
+            // barrier among the compute threads)
+            arrive(&sh.bar_cs);
+            if (!(ok = W.wait(&sh.bar_cs, ph_cs, 68))) break;
+        }
+    }
+
+    // ---------------------------------------------------------------- wind down
+    cp_async_wait<0>();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+__device__ int g_tc_error = 0;
+
+}  // namespace
+
+// 2D bf16 matrix [rows][cols] row-major, box {64 cols, box_rows rows}, 128 B swizzle
+vdm_status make_bf16_map(CUtensorMap* m, const void* base, int64_t rows, int cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(VDM_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(VDM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return VDM_OK;
+}
+
+int* tc_error_word() {
+    int* err = nullptr;
+    if (cudaGetSymbolAddress((void**)&err, g_tc_error) != cudaSuccess) return nullptr;
+    return err;
+}
+
+bool tc_supported(const DecodeArgs& a, vdm_dtype dt) {
+    if (dt != VDM_BF16) return false;
+    if (a.C != 128 && a.C != 256 && a.C != 512) return false;
+    if (a.F % 128 != 0) return false;
+    return true;
+}
+
+size_t tc_smem_bytes(int C, int* ns_out) {
+    const size_t fixed = (size_t)(C / 64) * 16384 + 16384 + 1024;
+    const size_t limit = 227 * 1024;
+    int ns = (int)((limit - fixed - 512) / SLOT);
+    if (ns > MAX_NS) ns = MAX_NS;
+    if (ns_out) *ns_out = ns;
+    return fixed + (size_t)ns * SLOT;
+}
+
+vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
+    int64_t n_units = d.work == kWorkFlat ? (d.M + BM - 1) / BM : (int64_t)d.T * d.slots;
+    if (n_units <= 0) return VDM_OK;
+    int ns = 0;
+    const size_t smem = tc_smem_bytes(d.C, &ns);
+    if (ns < GATHER_LAG + 2) return fail(VDM_ERR_INTERNAL, "not enough shared memory for the ring (%d slots)", ns);
+    CUtensorMap m_wq, m_wq64, m_wo, m_w1, m_w2, m_k, m_v;
+    const int HN = d.C > 256 ? 64 : 128;
+    VDM_TRY(make_bf16_map(&m_wq, d.Wq, d.C, 64, 128));
+    VDM_TRY(make_bf16_map(&m_wq64, d.Wq, d.C, 64, 64));
+    VDM_TRY(make_bf16_map(&m_wo, d.Wo, d.C, d.C, 128));
+    VDM_TRY(make_bf16_map(&m_w1, d.W1, d.F, d.C, HN));
+    VDM_TRY(make_bf16_map(&m_w2, d.W2, d.C, d.F, 128));
+    VDM_TRY(make_bf16_map(&m_k, d.K, (int64_t)d.H * d.N, 64, 128));
+    VDM_TRY(make_bf16_map(&m_v, d.V, (int64_t)d.H * d.N, 64, 128));
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    TcArgs ta;
+    ta.d = d;
+    ta.ns = ns;
+    ta.err = tc_error_word();
+    if (!ta.err) return fail(VDM_ERR_CUDA, "error word lookup failed");
+    ta.timeout = 4000000000ll;
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "decode_tc smem attribute: %s", cudaGetErrorString(e));
+    const unsigned grid = (unsigned)(n_units < sms ? n_units : sms);
+    prof_begin(kProfDecode, st);
+    decode_tc_kernel<<<grid, NT, smem, st>>>(m_wq, m_wq64, m_wo, m_w1, m_w2, m_k, m_v, ta);
+    prof_end(kProfDecode, st);
+    return check_launch("decode_tc_kernel");
+}
+
+int decode_simt_chunk();
+
+vdm_status launch_decode(DecodeArgs a, vdm_dtype dt, cudaStream_t st) {
+    const bool tc = tc_supported(a, dt);
+    if (a.work != kWorkFlat) {
+        const int qt = tc ? kTcTile : decode_simt_chunk();
+        const int most = a.work == kWorkTileDense ? (a.n_probe < 512 ? a.n_probe : 512) : 512 - a.n_probe;
+        a.slots = most > 0 ? (most + qt - 1) / qt : 0;
+        if (a.slots == 0) return VDM_OK;
+    }
+    if (tc) return launch_decode_tc(a, st);
+    return launch_decode_simt(a, dt, 0, st);
+}
+
+// Reads and clears the device error word (call after the stream is synchronised).
+vdm_status tc_check_error() {
+    int h = 0;
+    VDM_CUDA_TRY(cudaMemcpyFromSymbol(&h, g_tc_error, sizeof(int)));
+    if (h) {
+        int z = 0;
+        cudaMemcpyToSymbol(g_tc_error, &z, sizeof(int));
+        return fail(VDM_ERR_TIMEOUT, "tensor-core kernel: bounded wait expired at site %d", h);
+    }
+    return VDM_OK;
+}
+
+}  // namespace vdm

@@ -229,7 +229,7 @@ vdm_status vdm_decode_dense(const vdm_decoder* dec, const void* d_k, const void*
             a.n_spheres = an->n_spheres;
             a.dec_scale = an->dec_scale;
         }
-        VDM_TRY(launch_decode_simt(a, dec->dtype, 0, st));
+        VDM_TRY(launch_decode(a, dec->dtype, st));
     }
     return VDM_OK;
 }
@@ -292,7 +292,6 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
     const size_t kvb = kv_shape_bytes(dec, N);
     const int L = pl.L;
     const int64_t Rf = pl.R[L - 1];
-    const int qt = decode_simt_chunk();
 
     for (int b = 0; b < B; ++b) {
         const void* K = static_cast<const char*>(d_k) + b * kvb;
@@ -321,7 +320,7 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             a.M = (int64_t)R * R * R;
             a.grid = grid[0];
             a.dec_grid = dbg_ptr(dbg ? dbg->dec : nullptr, 0, a.M);
-            VDM_TRY(launch_decode_simt(a, dec->dtype, 0, st));
+            VDM_TRY(launch_decode(a, dec->dtype, st));
             if (sb) { sb->resolution[0] = R; sb->decoded[0] = a.M; }
         }
         for (int l = 0; l + 1 < L; ++l) {
@@ -342,6 +341,7 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             int32_t hc[2] = {0, 0};
             VDM_CUDA_TRY(cudaMemcpyAsync(hc, counts, sizeof(hc), cudaMemcpyDeviceToHost, st));
             VDM_CUDA_TRY(cudaStreamSynchronize(st));
+            VDM_TRY(tc_check_error());
             const int Mp = hc[0], T = hc[1];
             if (dbg && dbg->active[l])
                 VDM_CUDA_TRY(cudaMemcpyAsync(dbg->active[l] + (size_t)b * nw, words, (size_t)nw * 8,
@@ -366,7 +366,7 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
                 a.M = 8 * (int64_t)Mp;
                 a.grid = grid[l + 1];
                 a.dec_grid = decg;
-                VDM_TRY(launch_decode_simt(a, dec->dtype, 0, st));
+                VDM_TRY(launch_decode(a, dec->dtype, st));
                 if (sb) sb->decoded[l + 1] = a.M;
                 continue;
             }
@@ -385,8 +385,7 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             a.dec_grid = decg;
             // dense pass: probes and small sub-volumes
             a.work = kWorkTileDense;
-            a.slots = (std::min(512, p->n_probe) + qt - 1) / qt;
-            VDM_TRY(launch_decode_simt(a, dec->dtype, 0, st));
+            VDM_TRY(launch_decode(a, dec->dtype, st));
             // selection
             SelectArgs s;
             memset(&s, 0, sizeof(s));
@@ -401,10 +400,9 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             // sparse pass: the remaining queries over the selected tokens
             if (p->n_probe < 512) {
                 a.work = kWorkTileSparse;
-                a.slots = (512 - p->n_probe + qt - 1) / qt;
                 a.sel = sel;
                 a.ksel = pl.k;
-                VDM_TRY(launch_decode_simt(a, dec->dtype, 0, st));
+                VDM_TRY(launch_decode(a, dec->dtype, st));
             }
             if (dbg && dbg->tile_ids[l + 1] && dbg->max_tiles > 0) {
                 const int64_t nt = T < dbg->max_tiles ? T : dbg->max_tiles;

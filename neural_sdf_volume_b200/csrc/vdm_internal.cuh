@@ -72,6 +72,7 @@ struct DecodeArgs {
     const int32_t* sel;         // [T][ksel]
     int ksel;
     // outputs
+    float* probe_ml;            // kWorkTileDense: per (tile, probe, head) softmax max and sum (log2 units) or NULL
     float* out;                 // out[q] (flat work only) or NULL
     float* grid;                // scatter field at voxel linear index or NULL
     float* dec_grid;            // debug: raw decoder output at voxel index or NULL
@@ -121,6 +122,13 @@ void prof_end(int cls, cudaStream_t s);
 vdm_status launch_precompute_kv(const KvArgs& a, vdm_dtype dt, cudaStream_t s);
 vdm_status launch_decode_simt(const DecodeArgs& a, vdm_dtype dt, int n_ctas_hint, cudaStream_t s);
 vdm_status launch_select(const SelectArgs& a, vdm_dtype dt, cudaStream_t s);
+// tensor-core decoder (bf16, C in {128, 256, 512}, F % 128 == 0)
+bool tc_supported(const DecodeArgs& a, vdm_dtype dt);
+vdm_status launch_decode_tc(const DecodeArgs& a, cudaStream_t s);
+vdm_status tc_check_error();
+constexpr int kTcTile = 128;
+// picks the kernel for the decoder's dtype and shape; `slots` of tile modes follow its tile size
+vdm_status launch_decode(DecodeArgs a, vdm_dtype dt, cudaStream_t s);
 
 // volume kernels
 vdm_status launch_mark_dilate(const float* f, int R, uint64_t* words, cudaStream_t s);
