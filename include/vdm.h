@@ -81,8 +81,9 @@ typedef enum { VDM_F32 = 0, VDM_BF16 = 1 } vdm_dtype;
 #define VDM_MAX_LEVELS 6
 
 /* Decoder parameters (all device pointers).  Matrices are stored in `dtype`
- * (float or bf16), row-major W[out][in]; vectors are float32.  K and V
- * produced by vdm_precompute_kv are stored in `dtype` as well.              */
+ * (float or bf16), row-major W[out][in]; vectors are float32.  Every matrix
+ * and vector (except b_head) must be 16-byte aligned.  K and V produced by
+ * vdm_precompute_kv are stored in `dtype` as well.                          */
 typedef struct {
     int32_t C;          /* width, = 64 * H                                   */
     int32_t H;          /* heads                                             */

@@ -523,17 +523,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 if (!(ok = W.wait(&sh.bar_q, ph_q, 60))) break;
                 tc_fence_after();
                 {
-                    float q0[32], q1[32];
+                    float q0[32], q1[32], b0[32], b1v[32];
                     tmem_ld32(trow + T_Q, q0);
                     tmem_ld32(trow + T_Q + 32, q1);
+                    ldg32(a.bq + h * 64, b0);
+                    ldg32(a.bq + h * 64 + 32, b1v);
                     tmem_wait_ld();
                     reg_fence(q0);
                     reg_fence(q1);
                     uint32_t pk[32];
+#pragma unroll
                     for (int v = 0; v < 16; ++v) {
-                        const int c0 = h * 64 + 2 * v, c1 = h * 64 + 32 + 2 * v;
-                        pk[v] = pack_bf16((q0[2 * v] + a.bq[c0]) * qscale, (q0[2 * v + 1] + a.bq[c0 + 1]) * qscale);
-                        pk[16 + v] = pack_bf16((q1[2 * v] + a.bq[c1]) * qscale, (q1[2 * v + 1] + a.bq[c1 + 1]) * qscale);
+                        pk[v] = pack_bf16((q0[2 * v] + b0[2 * v]) * qscale, (q0[2 * v + 1] + b0[2 * v + 1]) * qscale);
+                        pk[16 + v] = pack_bf16((q1[2 * v] + b1v[2 * v]) * qscale, (q1[2 * v + 1] + b1v[2 * v + 1]) * qscale);
                     }
                     tmem_st32(trow + T_Q, pk);
                     tmem_wait_st();
@@ -650,35 +652,45 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             tc_fence_after();
             float mean1 = 0.f, rstd1 = 1.f;
             {
-                float sum = 0.f;
+                // x1 = X + bq + bo; statistics in one pass (sums shifted by the row's first value)
+                float shift = 0.f, s1 = 0.f, s2 = 0.f;
                 for (int cc = 0; cc < C; cc += 32) {
-                    float v[32];
-                    tmem_ld32_sync(trow + cc, v);
-                    for (int e = 0; e < 32; ++e) sum += v[e] + a.bq[cc + e] + a.bo[cc + e];
-                }
-                mean1 = sum / (float)C;
-                if (a.query_ln) {
-                    float m2 = 0.f;
-                    for (int cc = 0; cc < C; cc += 32) {
-                        float v[32];
-                        tmem_ld32_sync(trow + cc, v);
-                        for (int e = 0; e < 32; ++e) {
-                            const float d = v[e] + a.bq[cc + e] + a.bo[cc + e] - mean1;
-                            m2 = fmaf(d, d, m2);
-                        }
+                    float v[32], bqv[32], bov[32];
+                    tmem_ld32(trow + cc, v);
+                    ldg32(a.bq + cc, bqv);
+                    ldg32(a.bo + cc, bov);
+                    tmem_wait_ld();
+                    reg_fence(v);
+                    if (cc == 0) shift = v[0] + bqv[0] + bov[0];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float d = v[e] + bqv[e] + bov[e] - shift;
+                        s1 += d;
+                        s2 = fmaf(d, d, s2);
                     }
-                    rstd1 = rsqrtf(m2 / (float)C + kLnEps);
                 }
+                const float m_s = s1 / (float)C;
+                mean1 = shift + m_s;
+                if (a.query_ln) rstd1 = rsqrtf(fmaxf(s2 / (float)C - m_s * m_s, 0.f) + kLnEps);
                 for (int cc = 0; cc < C; cc += 32) {
-                    float v[32];
-                    tmem_ld32_sync(trow + cc, v);
+                    float v[32], bqv[32], bov[32], g[32], be[32];
+                    tmem_ld32(trow + cc, v);
+                    ldg32(a.bq + cc, bqv);
+                    ldg32(a.bo + cc, bov);
+                    if (a.query_ln) {
+                        ldg32(a.ln1_g + cc, g);
+                        ldg32(a.ln1_b + cc, be);
+                    }
+                    tmem_wait_ld();
+                    reg_fence(v);
                     uint32_t w[16];
+#pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        float y0 = v[2 * e] + a.bq[cc + 2 * e] + a.bo[cc + 2 * e];
-                        float y1 = v[2 * e + 1] + a.bq[cc + 2 * e + 1] + a.bo[cc + 2 * e + 1];
+                        float y0 = v[2 * e] + bqv[2 * e] + bov[2 * e];
+                        float y1 = v[2 * e + 1] + bqv[2 * e + 1] + bov[2 * e + 1];
                         if (a.query_ln) {
-                            y0 = (y0 - mean1) * rstd1 * a.ln1_g[cc + 2 * e] + a.ln1_b[cc + 2 * e];
-                            y1 = (y1 - mean1) * rstd1 * a.ln1_g[cc + 2 * e + 1] + a.ln1_b[cc + 2 * e + 1];
+                            y0 = (y0 - mean1) * rstd1 * g[2 * e] + be[2 * e];
+                            y1 = (y1 - mean1) * rstd1 * g[2 * e + 1] + be[2 * e + 1];
                         }
                         w[e] = pack_bf16(y0, y1);
                     }
@@ -735,19 +747,20 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     tc_fence_after();
                     const uint32_t hb = trow + ((c & 1) ? T_H1 : T_H0);
                     for (int part = 0; part < HN / 64; ++part) {
-                        float v0[32], v1[32];
+                        float v0[32], v1[32], c0v[32], c1v[32];
+                        const int f0 = c * HN + part * 64;
                         tmem_ld32(hb + part * 64, v0);
                         tmem_ld32(hb + part * 64 + 32, v1);
+                        ldg32(a.b1 + f0, c0v);
+                        ldg32(a.b1 + f0 + 32, c1v);
                         tmem_wait_ld();
                         reg_fence(v0);
                         reg_fence(v1);
                         uint32_t w[32];
-                        const int f0 = c * HN + part * 64;
+#pragma unroll
                         for (int e = 0; e < 16; ++e) {
-                            w[e] = pack_bf16(gelu_erf(v0[2 * e] + a.b1[f0 + 2 * e]),
-                                             gelu_erf(v0[2 * e + 1] + a.b1[f0 + 2 * e + 1]));
-                            w[16 + e] = pack_bf16(gelu_erf(v1[2 * e] + a.b1[f0 + 32 + 2 * e]),
-                                                  gelu_erf(v1[2 * e + 1] + a.b1[f0 + 32 + 2 * e + 1]));
+                            w[e] = pack_bf16(gelu_as(v0[2 * e] + c0v[2 * e]), gelu_as(v0[2 * e + 1] + c0v[2 * e + 1]));
+                            w[16 + e] = pack_bf16(gelu_as(v1[2 * e] + c1v[2 * e]), gelu_as(v1[2 * e + 1] + c1v[2 * e + 1]));
                         }
                         tmem_st32(hb + part * 32, w);
                     }
@@ -759,30 +772,32 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 if (!(ok = W.wait(&sh.bar_acc, ph_acc, 67))) break;
                 tc_fence_after();
                 const int cb = hf * 256;
-                float sum = 0.f, dot = 0.f;
+                // x2 = acc + bq + bo + b2 on this half's columns: shifted sums and the head dot product
+                float shift = 0.f, s1 = 0.f, s2 = 0.f, dot = 0.f;
                 for (int cc = 0; cc < CW; cc += 32) {
-                    float v[32];
-                    tmem_ld32_sync(trow + cc, v);
+                    const int col0 = cb + cc;
+                    float v[32], bqv[32], bov[32], b2v[32], wv[32], gv[32];
+                    tmem_ld32(trow + cc, v);
+                    ldg32(a.bq + col0, bqv);
+                    ldg32(a.bo + col0, bov);
+                    ldg32(a.b2 + col0, b2v);
+                    ldg32(a.w_head + col0, wv);
+                    if (a.query_ln) ldg32(a.ln2_g + col0, gv);
+                    tmem_wait_ld();
+                    reg_fence(v);
+                    if (cc == 0) shift = v[0] + bqv[0] + bov[0] + b2v[0];
+#pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        const int col = cb + cc + e;
-                        const float x = v[e] + a.bq[col] + a.bo[col] + a.b2[col];
-                        sum += x;
-                        dot = fmaf(x, a.query_ln ? a.w_head[col] * a.ln2_g[col] : a.w_head[col], dot);
+                        const float x = v[e] + bqv[e] + bov[e] + b2v[e];
+                        const float d = x - shift;
+                        s1 += d;
+                        s2 = fmaf(d, d, s2);
+                        dot = fmaf(x, a.query_ln ? wv[e] * gv[e] : wv[e], dot);
                     }
                 }
-                const float mh = sum / (float)CW;
-                float m2 = 0.f;
-                if (a.query_ln) {
-                    for (int cc = 0; cc < CW; cc += 32) {
-                        float v[32];
-                        tmem_ld32_sync(trow + cc, v);
-                        for (int e = 0; e < 32; ++e) {
-                            const int col = cb + cc + e;
-                            const float d = v[e] + a.bq[col] + a.bo[col] + a.b2[col] - mh;
-                            m2 = fmaf(d, d, m2);
-                        }
-                    }
-                }
+                const float m_s = s1 / (float)CW;
+                const float mh = shift + m_s;
+                const float m2 = fmaxf(s2 - s1 * m_s, 0.f);   // sum of squared deviations from mh
                 if (hf == 0) {
                     hs_mean0 = mh;
                     hs_m20 = m2;

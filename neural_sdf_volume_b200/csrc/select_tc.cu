@@ -1,0 +1,513 @@
+// Adaptive KV selection on the tensor cores: probe scoring and Top-K.
+//
+// FlashVDM ("Unleashing Vecset Diffusion Model for Fast Shape Generation",
+// aipaper.cc summary, section 4.1 item 2, steps 2-4): sampled queries of each
+// sub-volume score all vecset tokens by attention; the Top-K tokens are kept.
+//
+// score_t[j] = sum over the probes p of sub-volume t and heads h of
+//              softmax_h(q_p K_h^T / 8)_j
+//
+// The probes were already decoded with full attention by the dense pass of the
+// level, which exported each probe's per-head softmax maximum m and sum l (in
+// log2 units, against the same bf16 Q and K).  One pass suffices here:
+// S = Q K^T on the tensor cores (TMEM), P = 2^(S - m) / l in registers, and
+// the column sums over each sub-volume's probe rows by a warp transpose-reduce
+// (5 shuffle rounds; lane L ends with columns 4L..4L+3) plus a fixed-order sum
+// over the sub-volume's warps -- deterministic.  Then a radix select of the k
+// largest scores (ties to the smaller token) per sub-volume, in shared memory.
+//
+// Rows: 128 TMEM lanes hold 128 / n_probe sub-volumes' probes (n_probe in
+// {32, 64, 128}).  Roles: warps 0-3 compute, warp 4 MMA issue, warp 5 TMA.
+#include <cuda.h>
+
+#include "tc_ptx.cuh"
+#include "vdm_internal.cuh"
+
+namespace vdm {
+
+vdm_status make_bf16_map(CUtensorMap* m, const void* base, int64_t rows, int cols, int box_rows);
+int* tc_error_word();
+
+namespace {
+
+using namespace ptx;
+
+constexpr int NT = 192;
+constexpr int NCOMP = 128;
+constexpr int SLOT = 16384;
+constexpr int NS = 6;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t T_S0 = 0, T_S1 = 128, T_Q = 448;
+
+struct SelArgs {
+    int C, H, N;
+    const void* bq_unused;
+    const float* bq;
+    int n_sel_max;                 // capacity of the tile list
+    const int32_t* n_sel;          // device: number of tiles to score
+    const int32_t* sel_tiles;      // device: their ids
+    const int32_t* tile_off;       // [T+1] parent offsets
+    const int32_t* plist;
+    const int32_t* qorder;
+    const float* probe_ml;         // [T][n_probe][H][2]
+    int R;
+    int n_probe;
+    int tpu;                       // sub-volumes per unit = 128 / n_probe
+    int top_k;
+    int32_t* sel;                  // [T][top_k]
+    int* err;
+    long long timeout;
+};
+
+struct Shared {
+    uint64_t full[NS], empty[NS];
+    uint64_t bar_q, bar_s[2], bar_hd;          // MMA commits
+    uint64_t bar_pe, bar_qc, bar_p[2], bar_cs; // compute arrivals (128)
+    uint32_t tmem_base;
+    int abort;
+    int hist[256];
+    int red[4];
+    int wsum[4];
+};
+
+struct Waiter {
+    Shared* sh;
+    int* err;
+    long long timeout;
+    __device__ bool wait(uint64_t* bar, uint32_t& phase, int site) {
+        const uint32_t b = smem_u32(bar);
+        long long t0 = 0;
+        for (uint32_t it = 0;; ++it) {
+            if (mbar_try_wait(b, phase)) {
+                phase ^= 1;
+                return true;
+            }
+            if ((it & 63) == 63) {
+                if (*reinterpret_cast<volatile int*>(&sh->abort)) return false;
+                const long long t = clock64();
+                if (t0 == 0) t0 = t;
+                else if (t - t0 > timeout) {
+                    *reinterpret_cast<volatile int*>(&sh->abort) = 1;
+                    atomicCAS(err, 0, site);
+                    return false;
+                }
+            }
+        }
+    }
+};
+
+__device__ __forceinline__ uint32_t swz(uint32_t base, int r, int c) {
+    return base + r * 128 + ((c ^ (r & 7)) << 4);
+}
+
+// Sum of v over the 32 lanes for each of 128 columns; lane L returns the sums
+// of columns 4L .. 4L+3 (recursive halving: at offset o a lane keeps the upper
+// half of its current columns if (lane & o), and adds its partner's copy).
+__device__ __forceinline__ void warp_colsum128(const float (&v)[128], int lane, float (&out)[4]) {
+    float a64[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const bool up = lane & 16;
+        const float send = up ? v[i] : v[i + 64];
+        const float keep = up ? v[i + 64] : v[i];
+        a64[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    float a32[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const bool up = lane & 8;
+        const float send = up ? a64[i] : a64[i + 32];
+        const float keep = up ? a64[i + 32] : a64[i];
+        a32[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float a16[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const bool up = lane & 4;
+        const float send = up ? a32[i] : a32[i + 16];
+        const float keep = up ? a32[i + 16] : a32[i];
+        a16[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+    float a8[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const bool up = lane & 2;
+        const float send = up ? a16[i] : a16[i + 8];
+        const float keep = up ? a16[i + 8] : a16[i];
+        a8[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool up = lane & 1;
+        const float send = up ? a8[i] : a8[i + 4];
+        const float keep = up ? a8[i + 4] : a8[i];
+        out[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    }
+}
+
+__global__ void __launch_bounds__(NT, 1)
+select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_constant__ CUtensorMap tm_k,
+                 const SelArgs a) {
+    extern __shared__ uint8_t dyn_raw[];
+    __shared__ Shared sh;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = a.H, N = a.N, np = a.n_probe, tpu = a.tpu;
+    const int nb = (N + 127) / 128;
+    const uint32_t dyn0 = (smem_u32(dyn_raw) + 1023u) & ~1023u;
+    const uint32_t s_pe = dyn0;
+    const uint32_t s_ring = s_pe + 16384;
+    float* score = reinterpret_cast<float*>(dyn_raw + (dyn0 - smem_u32(dyn_raw)) + 16384 + NS * SLOT);  // [tpu][N]
+    float* part = score + (size_t)tpu * N;    // [2][4 warps][128]
+    Waiter W{&sh, a.err, a.timeout};
+
+    if (tid == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(smem_u32(&sh.full[i]), 1);
+            mbar_init(smem_u32(&sh.empty[i]), 1);
+        }
+        mbar_init(smem_u32(&sh.bar_q), 1);
+        mbar_init(smem_u32(&sh.bar_s[0]), 1);
+        mbar_init(smem_u32(&sh.bar_s[1]), 1);
+        mbar_init(smem_u32(&sh.bar_hd), 1);
+        mbar_init(smem_u32(&sh.bar_pe), NCOMP);
+        mbar_init(smem_u32(&sh.bar_qc), NCOMP);
+        mbar_init(smem_u32(&sh.bar_p[0]), NCOMP);
+        mbar_init(smem_u32(&sh.bar_p[1]), NCOMP);
+        mbar_init(smem_u32(&sh.bar_cs), NCOMP);
+        sh.abort = 0;
+        fence_mbar_init();
+        fence_proxy_async();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&sh.tmem_base), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+    const int n_sel = *a.n_sel < a.n_sel_max ? *a.n_sel : a.n_sel_max;
+    const int n_units = (n_sel + tpu - 1) / tpu;
+
+    if (warp == 5) {
+        // ------------------------------------------------------------ producer
+        uint32_t ring_head = 0;
+        bool ok = true;
+        auto push = [&](const CUtensorMap* m, int y, uint32_t bytes) -> bool {
+            const int slot = ring_head % NS;
+            if (ring_head >= (uint32_t)NS) {
+                uint32_t ph = ((ring_head / NS) + 1) & 1;
+                if (!W.wait(&sh.empty[slot], ph, 80)) return false;
+            }
+            ++ring_head;
+            if (lane == 0) {
+                const uint32_t fb = smem_u32(&sh.full[slot]);
+                mbar_expect_tx(fb, bytes);
+                tma_load_2d(s_ring + slot * SLOT, m, 0, y, fb);
+            }
+            __syncwarp();
+            return true;
+        };
+        for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x)
+            for (int h = 0; h < H && ok; ++h) {
+                ok = push(&tm_wq64, h * 64, 64 * 128);
+                for (int j = 0; j < nb && ok; ++j) ok = push(&tm_k, h * N + j * 128, SLOT);
+            }
+    } else if (warp == 4) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            uint32_t ring_tail = 0, ph_pe = 0, ph_qc = 0, ph_p[2] = {0, 0}, ph_hd = 0;
+            bool ok = true;
+            auto consume = [&](int& slot) -> bool {
+                slot = ring_tail % NS;
+                uint32_t ph = (ring_tail / NS) & 1;
+                if (!W.wait(&sh.full[slot], ph, 81)) return false;
+                tc_fence_after();
+                ++ring_tail;
+                return true;
+            };
+            auto issue_s = [&](int j) -> bool {
+                int sl;
+                if (!consume(sl)) return false;
+                const uint64_t db = desc_sw128(s_ring + sl * SLOT);
+                const uint32_t sd = tmem + ((j & 1) ? T_S1 : T_S0);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(sd, tmem + T_Q + 8 * kk, db + 2 * kk, idesc_bf16(128, 128, false), kk > 0);
+                mma_commit(smem_u32(&sh.empty[sl]));
+                mma_commit(smem_u32(&sh.bar_s[j & 1]));
+                return true;
+            };
+            for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+                if (!(ok = W.wait(&sh.bar_pe, ph_pe, 82))) break;
+                tc_fence_after();
+                for (int h = 0; h < H && ok; ++h) {
+                    int slot;
+                    if (!(ok = consume(slot))) break;
+                    const uint64_t da = desc_sw128(s_pe), db = desc_sw128(s_ring + slot * SLOT);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tmem + T_Q, da + 2 * kk, db + 2 * kk, idesc_bf16(128, 64, false), kk > 0);
+                    mma_commit(smem_u32(&sh.empty[slot]));
+                    mma_commit(smem_u32(&sh.bar_q));
+                    if (!(ok = W.wait(&sh.bar_qc, ph_qc, 83))) break;
+                    tc_fence_after();
+                    ok = issue_s(0) && (nb < 2 || issue_s(1));
+                    for (int j = 0; j < nb && ok; ++j) {
+                        if (!(ok = W.wait(&sh.bar_p[j & 1], ph_p[j & 1], 84))) break;
+                        tc_fence_after();
+                        if (j + 2 < nb) ok = issue_s(j + 2);
+                    }
+                    if (!ok) break;
+                    mma_commit(smem_u32(&sh.bar_hd));
+                    if (!(ok = W.wait(&sh.bar_hd, ph_hd, 85))) break;
+                    tc_fence_after();
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ compute
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+        uint32_t ph_q = 0, ph_s[2] = {0, 0}, ph_cs = 0;
+        const float qscale = 0.125f * kLog2e;
+        bool ok = true;
+        auto arrive = [&](uint64_t* b) { mbar_arrive(smem_u32(b)); };
+        auto csync = [&](int site) -> bool {
+            arrive(&sh.bar_cs);
+            return W.wait(&sh.bar_cs, ph_cs, site);
+        };
+        const int my_slot = tid / np;            // sub-volume slot of this row
+        const int my_i = tid % np;               // probe index within it
+        const int warps_per_tile = np >= 32 ? np / 32 : 1;
+        for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+            const int t_idx = unit * tpu + my_slot;
+            const bool valid = my_slot < tpu && t_idx < n_sel;
+            const int t = valid ? a.sel_tiles[t_idx] : -1;
+            float p[3] = {0.f, 0.f, 0.f};
+            if (valid) {
+                const int e = a.qorder[8 * a.tile_off[t] + my_i];
+                voxel_point(child_index(a.plist[e >> 3], e & 7, a.R), a.R, p);
+            }
+            for (int c = 0; c < 8; ++c) {
+                uint32_t w[4];
+                for (int v = 0; v < 4; ++v) w[v] = pack_bf16(pe_lane(p, c * 8 + 2 * v), pe_lane(p, c * 8 + 2 * v + 1));
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(swz(s_pe, tid, c)), "r"(w[0]),
+                             "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
+            }
+            for (int j = tid; j < tpu * N; j += NCOMP) score[j] = 0.f;
+            fence_proxy_async();
+            arrive(&sh.bar_pe);
+            const float* ml = valid ? a.probe_ml + ((size_t)t * np + my_i) * H * 2 : nullptr;
+            int pb = 0;   // partial-sum buffer
+            for (int h = 0; h < H && ok; ++h) {
+                if (!(ok = W.wait(&sh.bar_q, ph_q, 86))) break;
+                tc_fence_after();
+                {
+                    float q0[32], q1[32];
+                    tmem_ld32(trow + T_Q, q0);
+                    tmem_ld32(trow + T_Q + 32, q1);
+                    tmem_wait_ld();
+                    reg_fence(q0);
+                    reg_fence(q1);
+                    uint32_t pk[32];
+                    for (int v = 0; v < 16; ++v) {
+                        const int c0 = h * 64 + 2 * v, c1 = h * 64 + 32 + 2 * v;
+                        pk[v] = pack_bf16((q0[2 * v] + a.bq[c0]) * qscale, (q0[2 * v + 1] + a.bq[c0 + 1]) * qscale);
+                        pk[16 + v] = pack_bf16((q1[2 * v] + a.bq[c1]) * qscale, (q1[2 * v + 1] + a.bq[c1 + 1]) * qscale);
+                    }
+                    tmem_st32(trow + T_Q, pk);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                arrive(&sh.bar_qc);
+                const float m = valid ? ml[h * 2] : 0.f;
+                const float inv_l = valid ? 1.0f / ml[h * 2 + 1] : 0.f;
+                for (int j = 0; j < nb; ++j) {
+                    if (!(ok = W.wait(&sh.bar_s[j & 1], ph_s[j & 1], 87))) break;
+                    tc_fence_after();
+                    float v[128];
+                    {
+                        const uint32_t sb = trow + ((j & 1) ? T_S1 : T_S0);
+                        float s0[32], s1[32], s2[32], s3[32];
+                        tmem_ld32(sb, s0);
+                        tmem_ld32(sb + 32, s1);
+                        tmem_ld32(sb + 64, s2);
+                        tmem_ld32(sb + 96, s3);
+                        tmem_wait_ld();
+                        reg_fence(s0);
+                        reg_fence(s1);
+                        reg_fence(s2);
+                        reg_fence(s3);
+                        tc_fence_before();
+                        arrive(&sh.bar_p[j & 1]);   // S_j consumed
+                        const int vcols = N - j * 128;
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            v[c] = (c < vcols) ? ex2(s0[c] - m) * inv_l : 0.f;
+                            v[32 + c] = (32 + c < vcols) ? ex2(s1[c] - m) * inv_l : 0.f;
+                            v[64 + c] = (64 + c < vcols) ? ex2(s2[c] - m) * inv_l : 0.f;
+                            v[96 + c] = (96 + c < vcols) ? ex2(s3[c] - m) * inv_l : 0.f;
+                        }
+                    }
+                    float cs[4];
+                    warp_colsum128(v, lane, cs);
+                    float* pw = part + (pb * 4 + warp) * 128;
+                    pw[4 * lane] = cs[0];
+                    pw[4 * lane + 1] = cs[1];
+                    pw[4 * lane + 2] = cs[2];
+                    pw[4 * lane + 3] = cs[3];
+                    if (!(ok = csync(88))) break;
+                    // thread c adds column c of each sub-volume (its warps in order)
+                    {
+                        const int col = tid;
+                        if (j * 128 + col < N) {
+                            const float* pp = part + pb * 4 * 128;
+                            for (int s = 0; s < tpu; ++s) {
+                                float acc = 0.f;
+                                for (int w = 0; w < warps_per_tile; ++w) acc += pp[(s * warps_per_tile + w) * 128 + col];
+                                score[(size_t)s * N + j * 128 + col] += acc;
+                            }
+                        }
+                    }
+                    pb ^= 1;
+                }
+            }
+            if (!ok) break;
+            if (!(ok = csync(89))) break;
+            // ------------------------------------------------ Top-K per sub-volume
+            const int k = a.top_k;
+            for (int s = 0; s < tpu && ok; ++s) {
+                const int ti = unit * tpu + s;
+                if (ti >= n_sel) break;
+                const int t_s = a.sel_tiles[ti];
+                const float* sc = score + (size_t)s * N;
+                int32_t* out = a.sel + (size_t)t_s * k;
+                if (k >= N) {
+                    for (int j = tid; j < N; j += NCOMP) out[j] = j;
+                    continue;
+                }
+                uint32_t prefix = 0, pmask = 0;
+                int need = k;
+                for (int shift = 24; shift >= 0 && ok; shift -= 8) {
+                    for (int b = tid; b < 256; b += NCOMP) sh.hist[b] = 0;
+                    if (!(ok = csync(90))) break;
+                    for (int j = tid; j < N; j += NCOMP) {
+                        const uint32_t key = __float_as_uint(sc[j]);
+                        if ((key & pmask) == prefix) atomicAdd(&sh.hist[(key >> shift) & 255], 1);
+                    }
+                    if (!(ok = csync(91))) break;
+                    if (tid == 0) {
+                        int acc = 0, b = 255;
+                        for (; b > 0; --b) {
+                            if (acc + sh.hist[b] >= need) break;
+                            acc += sh.hist[b];
+                        }
+                        sh.red[0] = b;
+                        sh.red[1] = need - acc;
+                    }
+                    if (!(ok = csync(92))) break;
+                    prefix |= (uint32_t)sh.red[0] << shift;
+                    pmask |= 255u << shift;
+                    need = sh.red[1];
+                }
+                if (!ok) break;
+                const uint32_t thr = prefix;
+                const int per = (N + NCOMP - 1) / NCOMP;
+                const int j_lo = tid * per, j_hi = min(N, j_lo + per);
+                int eq = 0;
+                for (int j = j_lo; j < j_hi; ++j) eq += __float_as_uint(sc[j]) == thr;
+                int x = eq;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o) x += y;
+                }
+                if (lane == 31) sh.wsum[warp] = x;
+                if (!(ok = csync(93))) break;
+                int eq_before = x - eq;
+                for (int w = 0; w < warp; ++w) eq_before += sh.wsum[w];
+                if (!(ok = csync(94))) break;
+                int take = 0;
+                {
+                    int e = eq_before;
+                    for (int j = j_lo; j < j_hi; ++j) {
+                        const uint32_t key = __float_as_uint(sc[j]);
+                        take += key > thr || (key == thr && e < need);
+                        e += key == thr;
+                    }
+                }
+                x = take;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o) x += y;
+                }
+                if (lane == 31) sh.wsum[warp] = x;
+                if (!(ok = csync(95))) break;
+                int pos = x - take;
+                for (int w = 0; w < warp; ++w) pos += sh.wsum[w];
+                {
+                    int e = eq_before;
+                    for (int j = j_lo; j < j_hi; ++j) {
+                        const uint32_t key = __float_as_uint(sc[j]);
+                        if (key > thr || (key == thr && e < need)) out[pos++] = j;
+                        e += key == thr;
+                    }
+                }
+                if (!(ok = csync(96))) break;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+static size_t select_tc_smem(int n_probe, int N) {
+    return 1024 + 16384 + (size_t)NS * SLOT + (size_t)(128 / n_probe) * N * 4 + 2 * 4 * 128 * 4;
+}
+
+bool select_tc_supported(int C, int n_probe, int N, vdm_dtype dt) {
+    return dt == VDM_BF16 && (C == 128 || C == 256 || C == 512) && (n_probe == 32 || n_probe == 64 || n_probe == 128) &&
+           select_tc_smem(n_probe, N) <= 227 * 1024;
+}
+
+vdm_status launch_select_tc(const SelectTcLaunch& L, cudaStream_t st) {
+    if (L.T <= 0) return VDM_OK;
+    SelArgs a;
+    a.C = L.C; a.H = L.H; a.N = L.N;
+    a.bq_unused = nullptr;
+    a.bq = L.bq;
+    a.n_sel_max = L.T;
+    a.n_sel = L.n_sel;
+    a.sel_tiles = L.sel_tiles;
+    a.tile_off = L.tile_off;
+    a.plist = L.plist;
+    a.qorder = L.qorder;
+    a.probe_ml = L.probe_ml;
+    a.R = L.R;
+    a.n_probe = L.n_probe;
+    a.tpu = 128 / L.n_probe;
+    a.top_k = L.top_k;
+    a.sel = L.sel;
+    a.err = tc_error_word();
+    if (!a.err) return fail(VDM_ERR_CUDA, "error word lookup failed");
+    a.timeout = 4000000000ll;
+    CUtensorMap m_wq64, m_k;
+    VDM_TRY(make_bf16_map(&m_wq64, L.Wq, L.C, 64, 64));
+    VDM_TRY(make_bf16_map(&m_k, L.K, (int64_t)L.H * L.N, 64, 128));
+    const size_t smem = select_tc_smem(L.n_probe, L.N);
+    if (smem > 227 * 1024) return fail(VDM_ERR_UNSUPPORTED, "selection needs %zu bytes of shared memory", smem);
+    cudaError_t e = cudaFuncSetAttribute(select_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "select_tc smem attribute: %s", cudaGetErrorString(e));
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int max_units = (L.T + a.tpu - 1) / a.tpu;
+    const int grid = max_units < sms ? max_units : sms;
+    prof_begin(kProfSelect, st);
+    select_tc_kernel<<<grid, NT, smem, st>>>(m_wq64, m_k, a);
+    prof_end(kProfSelect, st);
+    return check_launch("select_tc_kernel");
+}
+
+}  // namespace vdm

@@ -99,9 +99,7 @@ __device__ __forceinline__ void reg_fence(float (&v)[32]) {
                    "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]),
                    "+f"(v[14]), "+f"(v[15]), "+f"(v[16]), "+f"(v[17]), "+f"(v[18]), "+f"(v[19]), "+f"(v[20]),
                    "+f"(v[21]), "+f"(v[22]), "+f"(v[23]), "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]),
-                   "+f"(v[28]), "+f"(v[29]), "+f"(v[30]), "+f"(v[31])
-                 :
-                 : "memory");
+                   "+f"(v[28]), "+f"(v[29]), "+f"(v[30]), "+f"(v[31]));
 }
 // load 32 columns and wait for them
 __device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, float (&v)[32]) {
@@ -159,10 +157,43 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
                  : "memory");
 }
 
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// 32 consecutive floats (16-byte aligned) into registers, as eight 16-byte loads
+__device__ __forceinline__ void ldg32(const float* p, float (&v)[32]) {
+    const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float4 t = __ldg(q + i);
+        v[4 * i] = t.x;
+        v[4 * i + 1] = t.y;
+        v[4 * i + 2] = t.z;
+        v[4 * i + 3] = t.w;
+    }
+}
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+// GELU(x) = x Phi(x) with Phi(x) = (1 + erf(x / sqrt 2)) / 2, erf by the rational
+// approximation of Abramowitz & Stegun, formula 7.1.26 (Hastings):
+// erf(z) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2), t = 1 / (1 + p z),
+// z >= 0, |error| <= 1.5e-7; odd extension for z < 0.  Branch free.
+__device__ __forceinline__ float gelu_as(float x) {
+    const float z = fabsf(x) * 0.70710678118654752f;
+    const float t = rcp_approx(fmaf(0.3275911f, z, 1.0f));
+    float q = fmaf(1.061405429f, t, -1.453152027f);
+    q = fmaf(q, t, 1.421413741f);
+    q = fmaf(q, t, -0.284496736f);
+    q = fmaf(q, t, 0.254829592f);
+    q *= t;
+    const float e = ex2(-z * z * 1.4426950408889634f);
+    const float erf_abs = fmaf(-q, e, 1.0f);
+    return 0.5f * x * (1.0f + copysignf(erf_abs, x));
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;

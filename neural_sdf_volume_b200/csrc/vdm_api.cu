@@ -54,7 +54,7 @@ vdm_status check_decoder(const vdm_decoder* d, bool need_query_side) {
         return fail(VDM_ERR_UNSUPPORTED, "F = %d must be a multiple of 64 in [64, 4096]", d->F);
     if (d->query_ln != 0 && d->query_ln != 1)
         return fail(VDM_ERR_INVALID_ARG, "query_ln must be 0 or 1");
-    const size_t al = d->dtype == VDM_F32 ? 16 : 8;
+    const size_t al = 16;
     const void* mats[] = {d->Wq, d->Wk, d->Wv, d->Wo, d->W1, d->W2};
     const char* names[] = {"Wq", "Wk", "Wv", "Wo", "W1", "W2"};
     for (int i = 0; i < 6; ++i) {
@@ -65,8 +65,11 @@ vdm_status check_decoder(const vdm_decoder* d, bool need_query_side) {
     const float* vecs[] = {d->bk, d->bv, d->ln_kv_g, d->ln_kv_b, d->bq, d->bo, d->b1, d->b2,
                            d->ln1_g, d->ln1_b, d->ln2_g, d->ln2_b, d->w_head, d->b_head};
     const int nvec = need_query_side ? 14 : 4;
-    for (int i = 0; i < nvec; ++i)
+    for (int i = 0; i < nvec; ++i) {
         if (!vecs[i]) return fail(VDM_ERR_INVALID_ARG, "decoder vector %d is NULL", i);
+        if (i < 13 && !aligned(vecs[i], 16))
+            return fail(VDM_ERR_INVALID_ARG, "decoder vector %d is not 16-byte aligned", i);
+    }
     return VDM_OK;
 }
 
@@ -92,15 +95,16 @@ struct Plan {
     int R[VDM_MAX_LEVELS];
     size_t off_grid[VDM_MAX_LEVELS];
     size_t off_words, off_word_off, off_tile_ids, off_tile_off, off_counts, off_scan, off_plist,
-        off_qorder, off_sel;
+        off_qorder, off_sel, off_seltiles, off_ml;
     int nw_max;
     int k;
+    size_t ml_bytes;
     size_t total;
 };
 
 size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
 
-vdm_status make_plan(const vdm_hier_params* p, int N, Plan& pl) {
+vdm_status make_plan(const vdm_hier_params* p, int N, int ml_heads, Plan& pl) {
     if (!p) return fail(VDM_ERR_INVALID_ARG, "params is NULL");
     if (p->n_levels < 1 || p->n_levels > VDM_MAX_LEVELS)
         return fail(VDM_ERR_UNSUPPORTED, "n_levels = %d not in [1, %d]", p->n_levels, VDM_MAX_LEVELS);
@@ -138,6 +142,9 @@ vdm_status make_plan(const vdm_hier_params* p, int N, Plan& pl) {
     pl.off_plist = o;     o = align_up(o + (size_t)vox_max * 4);
     pl.off_qorder = o;    o = align_up(o + (p->adaptive ? (size_t)vox_max * 8 * 4 : 0));
     pl.off_sel = o;       o = align_up(o + (p->adaptive ? (size_t)nw_max * pl.k * 4 : 0));
+    pl.off_seltiles = o;  o = align_up(o + (p->adaptive ? (size_t)nw_max * 4 : 0));
+    pl.ml_bytes = p->adaptive ? (size_t)nw_max * p->n_probe * ml_heads * 2 * 4 : 0;
+    pl.off_ml = o;        o = align_up(o + pl.ml_bytes);
     pl.total = o + 256;
     return VDM_OK;
 }
@@ -265,7 +272,7 @@ vdm_status vdm_hierarchical_workspace_size(const vdm_decoder* dec, const vdm_hie
     if (!bytes) return fail(VDM_ERR_INVALID_ARG, "bytes is NULL");
     if (N < 1 || N > kMaxN) return fail(VDM_ERR_UNSUPPORTED, "N = %d not in [1, %d]", N, kMaxN);
     Plan pl;
-    VDM_TRY(make_plan(p, N, pl));
+    VDM_TRY(make_plan(p, N, dec->H, pl));
     *bytes = pl.total;
     return VDM_OK;
 }
@@ -282,7 +289,7 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
     if (an && (!an->spheres || an->n_spheres < 1))
         return fail(VDM_ERR_INVALID_ARG, "analytic term needs spheres and n_spheres >= 1");
     Plan pl;
-    VDM_TRY(make_plan(p, N, pl));
+    VDM_TRY(make_plan(p, N, dec->H, pl));
     if (pl.L > 1 && (!d_ws || ws_bytes < pl.total))
         return fail(VDM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.total, ws_bytes);
     void* ws = d_ws ? reinterpret_cast<void*>(align_up((uintptr_t)d_ws)) : nullptr;
@@ -371,8 +378,11 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
                 continue;
             }
             const uint64_t salt = splitmix64(p->seed ^ ((uint64_t)(l + 1) << 32));
+            int32_t* sel_tiles = at<int32_t>(ws, pl.off_seltiles);
+            float* probe_ml = at<float>(ws, pl.off_ml);
+            const bool sel_tc = select_tc_supported(dec->C, p->n_probe, N, dec->dtype);
             VDM_CUDA_TRY(cudaMemsetAsync(counts + 2, 0, 2 * sizeof(int32_t), st));
-            VDM_TRY(launch_probe_order(tile_off, T, plist, R2, p->n_probe, salt, qorder, counts + 2, st));
+            VDM_TRY(launch_probe_order(tile_off, T, plist, R2, p->n_probe, salt, qorder, counts + 2, sel_tiles, st));
             DecodeArgs a = base;
             a.qmode = kQueryChildren;
             a.R = R2;
@@ -383,10 +393,25 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             a.n_probe = p->n_probe;
             a.grid = grid[l + 1];
             a.dec_grid = decg;
-            // dense pass: probes and small sub-volumes
+            // dense pass: probes and small sub-volumes (exports the probes' softmax statistics)
             a.work = kWorkTileDense;
+            a.probe_ml = sel_tc ? probe_ml : nullptr;
             VDM_TRY(launch_decode(a, dec->dtype, st));
+            a.probe_ml = nullptr;
             // selection
+            if (sel_tc) {
+                SelectTcLaunch L;
+                L.C = dec->C; L.H = dec->H; L.N = N;
+                L.Wq = dec->Wq; L.bq = dec->bq; L.K = K;
+                L.T = T;
+                L.n_sel = counts + 2;
+                L.sel_tiles = sel_tiles;
+                L.tile_off = tile_off; L.plist = plist; L.qorder = qorder;
+                L.probe_ml = probe_ml;
+                L.R = R2; L.n_probe = p->n_probe; L.top_k = pl.k;
+                L.sel = sel;
+                VDM_TRY(launch_select_tc(L, st));
+            } else {
             SelectArgs s;
             memset(&s, 0, sizeof(s));
             s.C = dec->C; s.H = dec->H; s.N = N;
@@ -397,6 +422,7 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             s.top_k = pl.k;
             s.sel = sel;
             VDM_TRY(launch_select(s, dec->dtype, st));
+            }
             // sparse pass: the remaining queries over the selected tokens
             if (p->n_probe < 512) {
                 a.work = kWorkTileSparse;

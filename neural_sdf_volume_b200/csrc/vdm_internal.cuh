@@ -127,6 +127,24 @@ bool tc_supported(const DecodeArgs& a, vdm_dtype dt);
 vdm_status launch_decode_tc(const DecodeArgs& a, cudaStream_t s);
 vdm_status tc_check_error();
 constexpr int kTcTile = 128;
+// tensor-core probe scoring + Top-K (hierarchical adaptive levels)
+struct SelectTcLaunch {
+    int C, H, N;
+    const void* Wq;
+    const float* bq;
+    const void* K;              // [H][N][64] bf16
+    int T;                      // upper bound of the tiles to score
+    const int32_t* n_sel;       // device: tiles to score
+    const int32_t* sel_tiles;   // device: their ids
+    const int32_t* tile_off;
+    const int32_t* plist;
+    const int32_t* qorder;
+    const float* probe_ml;      // [T][n_probe][H][2] from the dense pass
+    int R, n_probe, top_k;
+    int32_t* sel;               // [T][top_k]
+};
+bool select_tc_supported(int C, int n_probe, int N, vdm_dtype dt);
+vdm_status launch_select_tc(const SelectTcLaunch& L, cudaStream_t s);
 // picks the kernel for the decoder's dtype and shape; `slots` of tile modes follow its tile size
 vdm_status launch_decode(DecodeArgs a, vdm_dtype dt, cudaStream_t s);
 
@@ -143,7 +161,7 @@ vdm_status launch_fill(const float* f_coarse, const uint64_t* words, int R, floa
                        cudaStream_t s);
 vdm_status launch_probe_order(const int32_t* tile_off, int n_tiles, const int32_t* plist, int R2,
                               int n_probe, uint64_t salt, int32_t* qorder, int32_t* counters,
-                              cudaStream_t s);
+                              int32_t* sel_tiles, cudaStream_t s);
 
 size_t scan_tmp_ints(int n_words);
 

@@ -254,7 +254,8 @@ __global__ void __launch_bounds__(PO_T) probe_order_kernel(const int32_t* __rest
                                                            const int32_t* __restrict__ plist, int R2,
                                                            int n_probe, uint64_t salt,
                                                            int32_t* __restrict__ qorder,
-                                                           int32_t* __restrict__ counters) {
+                                                           int32_t* __restrict__ counters,
+                                                           int32_t* __restrict__ sel_tiles) {
     __shared__ uint64_t key[PO_MAX];
     __shared__ int64_t vox[PO_MAX];
     __shared__ int wsum[PO_T / 32];
@@ -262,7 +263,10 @@ __global__ void __launch_bounds__(PO_T) probe_order_kernel(const int32_t* __rest
     const int base = 8 * tile_off[t];
     const int cnt = 8 * (tile_off[t + 1] - tile_off[t]);
     if (threadIdx.x == 0) {   // integer counters: [0] sub-volumes with a selection, [1] full-KV queries
-        if (cnt > n_probe) atomicAdd(&counters[0], 1);
+        if (cnt > n_probe) {
+            const int pos = atomicAdd(&counters[0], 1);
+            if (sel_tiles) sel_tiles[pos] = t;   // list order is irrelevant: each entry is scored alone
+        }
         atomicAdd(&counters[1], cnt > n_probe ? n_probe : cnt);
     }
     if (cnt <= n_probe) {
@@ -383,10 +387,10 @@ vdm_status launch_fill(const float* f_coarse, const uint64_t* words, int R, floa
 
 vdm_status launch_probe_order(const int32_t* tile_off, int n_tiles, const int32_t* plist, int R2,
                               int n_probe, uint64_t salt, int32_t* qorder, int32_t* counters,
-                              cudaStream_t s) {
+                              int32_t* sel_tiles, cudaStream_t s) {
     if (n_tiles <= 0) return VDM_OK;
     prof_begin(kProfProbe, s);
-    probe_order_kernel<<<n_tiles, PO_T, 0, s>>>(tile_off, plist, R2, n_probe, salt, qorder, counters);
+    probe_order_kernel<<<n_tiles, PO_T, 0, s>>>(tile_off, plist, R2, n_probe, salt, qorder, counters, sel_tiles);
     prof_end(kProfProbe, s);
     return check_launch("probe_order_kernel");
 }
