@@ -234,6 +234,14 @@ VDM_API vdm_status vdm_decode_hierarchical_noalloc(const vdm_decoder* dec, const
                                                    vdm_hier_stats* stats,
                                                    const vdm_hier_debug* debug, vdm_stream stream);
 
+/* Test hook for failure detection (not needed for decoding).  mode 1 makes
+ * the next tensor-core decode launch withhold one completion signal, so its
+ * warps run into their bounded waits; `timeout_cycles` (> 0) shortens those
+ * waits.  The decode then reports VDM_ERR_TIMEOUT at its next check (the
+ * hierarchical call checks after each level) and the CUDA context stays
+ * usable.  mode 0 restores normal operation.                               */
+VDM_API vdm_status vdm_debug_inject(int32_t mode, int64_t timeout_cycles);
+
 /* Kernel timing for measurement (not needed for decoding).  Between
  * vdm_profile_begin() and vdm_profile_end() the calling thread's launches are
  * bracketed by CUDA events on their stream; vdm_profile_end() waits for those

@@ -158,9 +158,10 @@ __global__ void __launch_bounds__(NT) decode_kernel(DecodeArgs a) {
     const int32_t* sel = nullptr;
     int64_t qbeg = 0;   // first query slot (flat) or qorder position (tiles)
     if (a.work == kWorkFlat) {
+        const int64_t M = a.M_dev ? (int64_t)*a.M_dev : a.M;
         qbeg = (int64_t)blockIdx.x * QT;
-        if (qbeg >= a.M) return;
-        nq = (int)(a.M - qbeg < QT ? a.M - qbeg : QT);
+        if (qbeg >= M) return;
+        nq = (int)(M - qbeg < QT ? M - qbeg : QT);
     } else {
         const int t = blockIdx.x / a.slots, sl = blockIdx.x - t * a.slots;
         if (t >= a.T) return;
@@ -196,7 +197,8 @@ __global__ void __launch_bounds__(NT) decode_kernel(DecodeArgs a) {
                 voxel_point(v, a.R, p);
                 q = (int)slot;
             } else {
-                const int e = a.qorder ? a.qorder[slot] : (int)slot;
+                const int64_t pos = a.qlist ? (int64_t)a.qlist[slot] : slot;
+                const int e = a.qorder ? a.qorder[pos] : (int)pos;
                 v = child_index(a.plist[e >> 3], e & 7, a.R);
                 voxel_point(v, a.R, p);
                 q = (int)slot;

@@ -71,12 +71,13 @@ struct TcArgs {
     int ns;
     int* err;
     long long timeout;   // cycles per bounded wait
+    int inject;          // test hook: withhold the first Q-projection completion signal
 };
 
 struct Shared {
     uint64_t full[MAX_NS], empty[MAX_NS];
     // MMA commits (count 1); bar_hd and bar_w2 are waited on by the MMA warp only
-    uint64_t bar_q, bar_s[2], bar_pv, bar_x, bar_h[2], bar_acc, bar_hd, bar_w2;
+    uint64_t bar_q, bar_s[2], bar_pv, bar_x, bar_h[2], bar_acc, bar_hd, bar_w2, bar_fin;
     // compute-warp arrivals (count 128)
     uint64_t bar_pe, bar_qc, bar_p[2], bar_a, bar_hin, bar_r, bar_g[2], bar_cs;
     uint32_t tmem_base;
@@ -111,6 +112,14 @@ struct Waiter {
     }
 };
 
+// Wind-down wait for our own asynchronous work (loads, MMAs), which always
+// completes; bounded by `cycles` all the same, and not cut short by an abort.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, long long cycles) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity) && clock64() - t0 < cycles) {
+    }
+}
+
 __device__ __forceinline__ uint32_t swz(uint32_t base, int r, int c) {
     return base + r * 128 + ((c ^ (r & 7)) << 4);
 }
@@ -136,8 +145,9 @@ __device__ __forceinline__ Unit unit_of(const DecodeArgs& a, int64_t unit) {
     u.t = -1;
     u.first = 0;
     if (a.work == kWorkFlat) {
+        const int64_t M = a.M_dev ? (int64_t)*a.M_dev : a.M;
         u.qbeg = unit * BM;
-        u.nq = (int)(a.M - u.qbeg < BM ? a.M - u.qbeg : BM);
+        u.nq = u.qbeg < M ? (int)(M - u.qbeg < BM ? M - u.qbeg : BM) : 0;
         return u;
     }
     const int t = (int)(unit / a.slots), sl = (int)(unit - (int64_t)t * a.slots);
@@ -195,7 +205,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             mbar_init(smem_u32(&sh.empty[i]), 1);
         }
         uint64_t* one[] = {&sh.bar_q, &sh.bar_s[0], &sh.bar_s[1], &sh.bar_pv, &sh.bar_x,
-                           &sh.bar_h[0], &sh.bar_h[1], &sh.bar_acc, &sh.bar_hd, &sh.bar_w2};
+                           &sh.bar_h[0], &sh.bar_h[1], &sh.bar_acc, &sh.bar_hd, &sh.bar_w2, &sh.bar_fin};
         for (auto* b : one) mbar_init(smem_u32(b), 1);
         uint64_t* many[] = {&sh.bar_pe, &sh.bar_qc, &sh.bar_p[0], &sh.bar_p[1], &sh.bar_a,
                             &sh.bar_hin, &sh.bar_r, &sh.bar_g[0], &sh.bar_g[1], &sh.bar_cs};
@@ -336,6 +346,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             }
         }
         drain();
+        // every load issued has landed before the CTA may exit (they always
+        // complete; consumed or not, the last use of each slot is awaited)
+        if (lane == 0) {
+            const uint32_t first = ring_head > (uint32_t)NS ? ring_head - NS : 0;
+            for (uint32_t i = first; i < ring_head; ++i) drain_wait(smem_u32(&sh.full[i % NS]), (i / NS) & 1, ta.timeout);
+        }
+        __syncwarp();
     }
     // ==================================================================== MMA issue
     else if (warp == WARP_MMA) {
@@ -369,7 +386,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         for (int kk = 0; kk < 4; ++kk)
                             mma_ss(tmem + T_Q, da + 2 * kk, db + 2 * kk, idesc_bf16(128, 64, false), kk > 0);
                         release(slot);
-                        mma_commit(smem_u32(&sh.bar_q));
+                        if (!(ta.inject && h == 0 && unit == blockIdx.x)) mma_commit(smem_u32(&sh.bar_q));
                     }
                     if (!(ok = W.wait(&sh.bar_qc, ph_qc, 52))) break;
                     tc_fence_after();
@@ -474,6 +491,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     mma_commit(smem_u32(&sh.bar_acc));   // the half's accumulator is complete
                 }
             }
+            // nothing of ours may run on the tensor cores once TMEM is released
+            mma_commit(smem_u32(&sh.bar_fin));
+            drain_wait(smem_u32(&sh.bar_fin), 0, ta.timeout);
         }
     }
     // ==================================================================== compute warps
@@ -503,7 +523,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     vox = slot;
                     voxel_point(vox, a.R, p);
                 } else {
-                    const int e = a.qorder ? a.qorder[slot] : (int)slot;
+                    const int64_t pos = a.qlist ? (int64_t)a.qlist[slot] : slot;
+                    const int e = a.qorder ? a.qorder[pos] : (int)pos;
                     vox = child_index(a.plist[e >> 3], e & 7, a.R);
                     voxel_point(vox, a.R, p);
                 }
@@ -515,9 +536,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             }
             fence_proxy_async();
             arrive(&sh.bar_pe);
-            float* ml_out = (a.probe_ml && a.work == kWorkTileDense && tid < u.nq)
-                                ? a.probe_ml + ((size_t)u.t * a.n_probe + u.first + tid) * H * 2
-                                : nullptr;
+            float* ml_out = nullptr;
+            if (a.probe_ml && tid < u.nq) {
+                if (a.work == kWorkTileDense) ml_out = a.probe_ml + ((size_t)u.t * a.n_probe + u.first + tid) * H * 2;
+                else if (a.ml_slot) ml_out = a.probe_ml + (size_t)a.ml_slot[u.qbeg + tid] * H * 2;
+            }
             // ================================================= attention
             for (int h = 0; h < H && ok; ++h) {
                 if (!(ok = W.wait(&sh.bar_q, ph_q, 60))) break;
@@ -932,7 +955,9 @@ vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
     ta.ns = ns;
     ta.err = tc_error_word();
     if (!ta.err) return fail(VDM_ERR_CUDA, "error word lookup failed");
-    ta.timeout = 4000000000ll;
+    ta.timeout = g_debug.timeout > 0 ? g_debug.timeout : 4000000000ll;
+    ta.inject = g_debug.inject;
+    g_debug.inject = 0;   // one launch only
     cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "decode_tc smem attribute: %s", cudaGetErrorString(e));
     const unsigned grid = (unsigned)(n_units < sms ? n_units : sms);

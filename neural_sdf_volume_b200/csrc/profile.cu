@@ -45,11 +45,20 @@ void prof_end(int cls, cudaStream_t s) {
     cudaEventRecord(g_recs.back().b, s);
 }
 
+DebugHooks g_debug = {0, 0};
+
 }  // namespace vdm
 
 using namespace vdm;
 
 extern "C" {
+
+vdm_status vdm_debug_inject(int32_t mode, int64_t timeout_cycles) {
+    if (mode != 0 && mode != 1) return fail(VDM_ERR_INVALID_ARG, "unknown inject mode %d", mode);
+    g_debug.inject = mode;
+    g_debug.timeout = timeout_cycles > 0 ? timeout_cycles : 0;
+    return VDM_OK;
+}
 
 vdm_status vdm_profile_begin(void) {
     for (auto& r : g_recs) {

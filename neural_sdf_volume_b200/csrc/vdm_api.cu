@@ -95,7 +95,7 @@ struct Plan {
     int R[VDM_MAX_LEVELS];
     size_t off_grid[VDM_MAX_LEVELS];
     size_t off_words, off_word_off, off_tile_ids, off_tile_off, off_counts, off_scan, off_plist,
-        off_qorder, off_sel, off_seltiles, off_ml;
+        off_qorder, off_sel, off_seltiles, off_ml, off_dense, off_dense_ml;
     int nw_max;
     int k;
     size_t ml_bytes;
@@ -145,6 +145,9 @@ vdm_status make_plan(const vdm_hier_params* p, int N, int ml_heads, Plan& pl) {
     pl.off_seltiles = o;  o = align_up(o + (p->adaptive ? (size_t)nw_max * 4 : 0));
     pl.ml_bytes = p->adaptive ? (size_t)nw_max * p->n_probe * ml_heads * 2 * 4 : 0;
     pl.off_ml = o;        o = align_up(o + pl.ml_bytes);
+    const size_t dense_max = p->adaptive ? (size_t)nw_max * (p->n_probe < 512 ? p->n_probe : 512) : 0;
+    pl.off_dense = o;     o = align_up(o + dense_max * 4);
+    pl.off_dense_ml = o;  o = align_up(o + dense_max * 4);
     pl.total = o + 256;
     return VDM_OK;
 }
@@ -382,7 +385,10 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             float* probe_ml = at<float>(ws, pl.off_ml);
             const bool sel_tc = select_tc_supported(dec->C, p->n_probe, N, dec->dtype);
             VDM_CUDA_TRY(cudaMemsetAsync(counts + 2, 0, 2 * sizeof(int32_t), st));
-            VDM_TRY(launch_probe_order(tile_off, T, plist, R2, p->n_probe, salt, qorder, counts + 2, sel_tiles, st));
+            int32_t* dense_q = at<int32_t>(ws, pl.off_dense);
+            int32_t* dense_ml = at<int32_t>(ws, pl.off_dense_ml);
+            VDM_TRY(launch_probe_order(tile_off, T, plist, R2, p->n_probe, salt, qorder, counts + 2, sel_tiles,
+                                       dense_q, dense_ml, st));
             DecodeArgs a = base;
             a.qmode = kQueryChildren;
             a.R = R2;
@@ -393,11 +399,18 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             a.n_probe = p->n_probe;
             a.grid = grid[l + 1];
             a.dec_grid = decg;
-            // dense pass: probes and small sub-volumes (exports the probes' softmax statistics)
-            a.work = kWorkTileDense;
-            a.probe_ml = sel_tc ? probe_ml : nullptr;
-            VDM_TRY(launch_decode(a, dec->dtype, st));
-            a.probe_ml = nullptr;
+            // dense pass: probes and small sub-volumes, packed into one flat list
+            // (exports the probes' softmax statistics for the scoring kernel)
+            {
+                DecodeArgs d = a;
+                d.work = kWorkFlat;
+                d.qlist = dense_q;
+                d.M = std::min<int64_t>(8 * (int64_t)Mp, (int64_t)T * std::min(p->n_probe, 512));
+                d.M_dev = counts + 3;
+                d.probe_ml = sel_tc ? probe_ml : nullptr;
+                d.ml_slot = sel_tc ? dense_ml : nullptr;
+                VDM_TRY(launch_decode(d, dec->dtype, st));
+            }
             // selection
             if (sel_tc) {
                 SelectTcLaunch L;

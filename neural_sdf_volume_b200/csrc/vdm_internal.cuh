@@ -62,7 +62,10 @@ struct DecodeArgs {
     const float* xyz;           // kQueryXyz
     const int32_t* plist;       // kQueryChildren: parent linear indices at R/2
     const int32_t* qorder;      // kQueryChildren: optional permutation of children
-    int64_t M;                  // kWorkFlat: number of queries
+    const int32_t* qlist;       // kWorkFlat + kQueryChildren: optional slot -> qorder position
+    const int32_t* ml_slot;     // with probe_ml in flat work: slot -> probe statistics index
+    int64_t M;                  // kWorkFlat: number of queries (upper bound when M_dev is set)
+    const int32_t* M_dev;       // kWorkFlat: device-side query count (read by the kernel) or NULL
     // tiles (kWorkTile*)
     int work;
     const int32_t* tile_off;    // [T+1] parent offsets per tile
@@ -111,6 +114,13 @@ struct SelectArgs {
     int32_t* sel;               // [T][top_k]
     float* score;               // [T][N] or NULL
 };
+
+// ---------------------------------------------------------------- test hooks
+struct DebugHooks {
+    int inject;              // 1: withhold one MMA completion signal in the next decode launch
+    long long timeout;       // bounded-wait limit in cycles (0: default)
+};
+extern DebugHooks g_debug;
 
 // ---------------------------------------------------------------- profiling
 enum ProfClass : int { kProfKv = 0, kProfDecode = 1, kProfSelect = 2, kProfMark = 3, kProfScan = 4,
@@ -161,7 +171,7 @@ vdm_status launch_fill(const float* f_coarse, const uint64_t* words, int R, floa
                        cudaStream_t s);
 vdm_status launch_probe_order(const int32_t* tile_off, int n_tiles, const int32_t* plist, int R2,
                               int n_probe, uint64_t salt, int32_t* qorder, int32_t* counters,
-                              int32_t* sel_tiles, cudaStream_t s);
+                              int32_t* sel_tiles, int32_t* dense_q, int32_t* dense_ml, cudaStream_t s);
 
 size_t scan_tmp_ints(int n_words);
 

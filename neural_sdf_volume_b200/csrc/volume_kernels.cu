@@ -255,19 +255,32 @@ __global__ void __launch_bounds__(PO_T) probe_order_kernel(const int32_t* __rest
                                                            int n_probe, uint64_t salt,
                                                            int32_t* __restrict__ qorder,
                                                            int32_t* __restrict__ counters,
-                                                           int32_t* __restrict__ sel_tiles) {
+                                                           int32_t* __restrict__ sel_tiles,
+                                                           int32_t* __restrict__ dense_q,
+                                                           int32_t* __restrict__ dense_ml) {
+    __shared__ int dpos;
     __shared__ uint64_t key[PO_MAX];
     __shared__ int64_t vox[PO_MAX];
     __shared__ int wsum[PO_T / 32];
     const int t = blockIdx.x;
     const int base = 8 * tile_off[t];
     const int cnt = 8 * (tile_off[t + 1] - tile_off[t]);
+    const int nd = cnt > n_probe ? n_probe : cnt;   // queries decoded over all tokens
     if (threadIdx.x == 0) {   // integer counters: [0] sub-volumes with a selection, [1] full-KV queries
         if (cnt > n_probe) {
             const int pos = atomicAdd(&counters[0], 1);
             if (sel_tiles) sel_tiles[pos] = t;   // list order is irrelevant: each entry is scored alone
         }
-        atomicAdd(&counters[1], cnt > n_probe ? n_probe : cnt);
+        dpos = atomicAdd(&counters[1], nd);
+    }
+    __syncthreads();
+    if (dense_q) {
+        // packed list of this sub-volume's full-attention queries (order across
+        // sub-volumes is irrelevant: every query is decoded independently)
+        for (int i = threadIdx.x; i < nd; i += PO_T) {
+            dense_q[dpos + i] = base + i;
+            dense_ml[dpos + i] = t * n_probe + i;
+        }
     }
     if (cnt <= n_probe) {
         for (int e = threadIdx.x; e < cnt; e += PO_T) qorder[base + e] = base + e;
@@ -387,10 +400,11 @@ vdm_status launch_fill(const float* f_coarse, const uint64_t* words, int R, floa
 
 vdm_status launch_probe_order(const int32_t* tile_off, int n_tiles, const int32_t* plist, int R2,
                               int n_probe, uint64_t salt, int32_t* qorder, int32_t* counters,
-                              int32_t* sel_tiles, cudaStream_t s) {
+                              int32_t* sel_tiles, int32_t* dense_q, int32_t* dense_ml, cudaStream_t s) {
     if (n_tiles <= 0) return VDM_OK;
     prof_begin(kProfProbe, s);
-    probe_order_kernel<<<n_tiles, PO_T, 0, s>>>(tile_off, plist, R2, n_probe, salt, qorder, counters, sel_tiles);
+    probe_order_kernel<<<n_tiles, PO_T, 0, s>>>(tile_off, plist, R2, n_probe, salt, qorder, counters, sel_tiles,
+                                               dense_q, dense_ml);
     prof_end(kProfProbe, s);
     return check_launch("probe_order_kernel");
 }
