@@ -274,6 +274,44 @@ def run_vdm(args, world, rank, local):
     return res
 
 
+def run_dense(args, world, rank, local):
+    """Dense decoding of ``--dense-queries`` random points with the full-width
+    decoder (N=3072, C=512, 8 heads, F=2048): the fused kernel alone, for
+    profiling and for the dense points/s figure."""
+    import torch
+
+    import neural_sdf_volume_b200 as vdm
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = W.CONFIGS[2]
+    inp = W.make_decoder(cfg.dec, seed=0, key=cfg.seed_key, B=1)
+    dec = vdm.Decoder.from_numpy(inp["weights"], cfg.dec.C, cfg.dec.H, cfg.dec.F, cfg.dec.query_ln,
+                                 cfg.dec.dtype, device=dev)
+    K, V = vdm.vdm_precompute_kv(dec, torch.from_numpy(inp["z"]).to(dev))
+    M = args.dense_queries
+    pts = torch.from_numpy(W.make_points(M, seed=1, key=2)).to(dev)
+    out = torch.empty((1, M), device=dev)
+    for _ in range(args.warmup):
+        vdm.vdm_decode_dense(dec, K, V, xyz=pts, out=out)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        vdm.vdm_decode_dense(dec, K, V, xyz=pts, out=out)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = M * decode_flops_per_query(cfg.dec, cfg.dec.N)
+    peaks = _peaks()
+    return {"metric": "dense decode points/sec (N=3072, C=512)", "value": M / (ms / 1e3), "unit": UNIT,
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"dense decode of {M} uniform points, config 2 decoder"},
+            "tflops": flops / (ms / 1e3) / 1e12,
+            "frac_of_bf16_burst": flops / (ms / 1e3) / 1e12 / peaks["bf16"]}
+
+
 def _oracle_sample_points(cfg, n: int, seed: int = 0) -> np.ndarray:
     """A bounded, seeded sample of the workload's query points: coarse voxels and
     fine voxels near the spheres' surfaces (where the fine levels decode)."""
@@ -346,12 +384,16 @@ def main():
     ap.add_argument("--config", type=int, default=4, choices=[3, 4, 5])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dense-queries", type=int, default=0,
+                    help="time dense decoding of this many points instead (config 2 decoder)")
     args = ap.parse_args()
     world, rank, local = _dist_init()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         res = run_reference(args, world, rank)
+    elif args.dense_queries > 0:
+        res = run_dense(args, world, rank, local)
     else:
         res = run_vdm(args, world, rank, local)
     if rank == 0 and res is not None:

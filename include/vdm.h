@@ -221,8 +221,9 @@ VDM_API vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d
  * own all device memory themselves, and latency-critical code that avoids
  * cudaMalloc/cudaFree because they can synchronise the device.
  *   - Problems whose vdm_hierarchical_workspace_size exceeds 32 MiB return
- *     VDM_ERR_UNSUPPORTED (a 32 -> 64 -> 128 adaptive decode with top_k 1024
- *     needs about 26 MiB; 64 -> 128 -> 256 without adaptive KV about 18 MiB).
+ *     VDM_ERR_UNSUPPORTED (a 32 -> 64 -> 128 adaptive decode with 32 probes and
+ *     top_k 512 needs about 27 MiB, with 64 probes and top_k 1024 about 44 MiB,
+ *     which is rejected; 64 -> 128 -> 256 without adaptive KV about 18 MiB).
  *   - All calls on a device share that scratch: calls that overlap on the GPU
  *     race; issue them one after another on one stream.
  *   - The first call on each device looks up the scratch address (no

@@ -7,13 +7,22 @@
 // One persistent CTA per SM decodes 128-query tiles; nothing but the final
 // SDF value (and, for probe queries, their softmax statistics) leaves the SM.
 //
-// Warp roles (192 threads):
-//   warps 0-3  compute: one thread per query row = TMEM lane; embedding,
-//              softmax, LayerNorms, GELU, SDF head;
-//   warp 4     MMA issue (one lane);
-//   warp 5     producer: TMA loads of weights and of contiguous K/V blocks,
+// Warp roles (320 threads):
+//   warps 0-7  compute: two warpgroups; thread (g, r) owns TMEM lane r and
+//              half g of the row's columns (softmax columns, head dims, hidden
+//              units, LayerNorm columns), so every SM sub-partition runs two
+//              compute warps; the halves exchange a block maximum (bf16, in
+//              smem) per attention block and a few row statistics per tile;
+//   warp 8     MMA issue (one lane);
+//   warp 9     producer: TMA loads of weights and of contiguous K/V blocks,
 //              cp.async gathers of a sub-volume's selected K/V rows;
 // connected only by mbarriers (no CTA-wide barrier inside a tile).
+//
+// Split-packed A operands: Q and the GELU output are produced by the two
+// warpgroups, each packing its half (bf16 pairs) into the start of its own
+// fp32 source columns (so neither overwrites the other's unread source); the
+// k-step q of 16 elements then sits at column  g*W/2 + (16q mod W/2)/2  with
+// g = 16q / (W/2) for a W-wide block.
 //
 // Per tile:
 //   PE (bf16 smem) ; per head h: Q_h = PE Wq_h^T (TMEM) -> bf16 in TMEM;
@@ -30,8 +39,8 @@
 //   MLP, C == 512: the 128 x 512 fp32 residual alone fills TMEM, so the MLP
 //              output is produced in two 256-wide halves (the hidden projection
 //              is recomputed for the second half); while the first half runs,
-//              x1's second half waits in TMEM as bf16 [256,384); hidden chunks
-//              (64 wide) at [384,448) [448,512).
+//              x1's second half (fp32) waits in a per-CTA global parking area
+//              (L2 resident); hidden chunks (128 wide) at [256,384) [384,512).
 //
 // Softmax: logits in log2 units (the 1/8 scale and log2 e folded into Q);
 // the running maximum is only raised when a block exceeds it by more than 8
@@ -56,9 +65,9 @@ namespace {
 using namespace ptx;
 
 constexpr int BM = 128;        // queries per tile (TMEM lanes)
-constexpr int NCOMP = 128;     // compute threads
-constexpr int NT = 192;        // + MMA warp + producer warp
-constexpr int WARP_MMA = 4, WARP_PROD = 5;
+constexpr int NCOMP = 256;     // compute threads (two warpgroups)
+constexpr int NT = 320;        // + MMA warp + producer warp
+constexpr int WARP_MMA = 8, WARP_PROD = 9;
 constexpr int SLOT = 16384;    // ring slot bytes
 constexpr int MAX_NS = 8;
 constexpr int GATHER_LAG = 2;  // gathered items in flight before their barrier is signalled
@@ -66,9 +75,18 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr uint32_t T_S0 = 0, T_S1 = 128, T_P0 = 256, T_P1 = 320, T_O = 384, T_Q = 448;
 
+// ring depth: 16 KB slots in what the 227 KB of shared memory leaves after the
+// activation buffer (C/64 atoms of 16 KB), the embedding tile and alignment
+__host__ __device__ constexpr int ring_slots(int C) {
+    return (int)((227 * 1024 - ((C / 64) * 16384 + 16384 + 1024) - 512) / SLOT) < MAX_NS
+               ? (int)((227 * 1024 - ((C / 64) * 16384 + 16384 + 1024) - 512) / SLOT)
+               : MAX_NS;
+}
+
 struct TcArgs {
     DecodeArgs d;
     int ns;
+    float* park;         // C == 512: per-CTA parking area, 128 x 256 fp32 each
     int* err;
     long long timeout;   // cycles per bounded wait
     int inject;          // test hook: withhold the first Q-projection completion signal
@@ -79,8 +97,9 @@ struct Shared {
     // MMA commits (count 1); bar_hd and bar_w2 are waited on by the MMA warp only
     uint64_t bar_q, bar_s[2], bar_pv, bar_x, bar_h[2], bar_acc, bar_hd, bar_w2, bar_fin;
     // compute-warp arrivals (count 128)
-    uint64_t bar_pe, bar_qc, bar_p[2], bar_a, bar_hin, bar_r, bar_g[2], bar_cs;
+    uint64_t bar_pe, bar_qc, bar_p[2], bar_a, bar_hin, bar_r, bar_g[2], bar_cs, bar_wg;
     uint32_t tmem_base;
+    uint16_t xmax[2][2][128];   // per attention block: [block parity][warpgroup][row] block max (bf16 bits)
     int abort;
     float G, Bc;
 };
@@ -122,6 +141,12 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, long l
 
 __device__ __forceinline__ uint32_t swz(uint32_t base, int r, int c) {
     return base + r * 128 + ((c ^ (r & 7)) << 4);
+}
+
+// TMEM column of k-step q (16 elements) of a W-wide split-packed A operand
+__device__ __forceinline__ uint32_t split_col(int q, int W) {
+    const int half = W / 2, g0 = 16 * q;
+    return (uint32_t)((g0 / half) * half + (g0 % half) / 2);
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t* w) {
@@ -170,6 +195,7 @@ __device__ __forceinline__ Unit unit_of(const DecodeArgs& a, int64_t unit) {
 }
 
 // ---------------------------------------------------------------- the kernel
+template <int CC>
 __global__ void __launch_bounds__(NT, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_wq64,
                  const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_w1,
@@ -180,17 +206,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
     __shared__ Shared sh;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int C = a.C, H = a.H, F = a.F, N = a.N;
-    const int NA = C / 64;
-    const bool halves = C > 256;
-    const int HN = halves ? 64 : 128;
-    const int NS = ta.ns;
-    const int CW = halves ? 256 : C;
-    const int n_half = halves ? 2 : 1;
-    const uint32_t T_H0 = halves ? 384 : 256, T_H1 = halves ? 448 : 384;
+    // the model width fixes the TMEM plan, the ring depth and every MMA shape at compile time
+    constexpr int C = CC;
+    const int H = a.H, F = a.F, N = a.N;
+    constexpr int NA = C / 64;
+    constexpr bool halves = C > 256;
+    constexpr int HN = 128;
+    constexpr int NS = ring_slots(C);
+    constexpr int CW = halves ? 256 : C;
+    constexpr int n_half = halves ? 2 : 1;
+    constexpr uint32_t T_H0 = 256, T_H1 = 384;
     const int n_chunks = F / HN;
-    const int w1_gran = NA;
-    const int w2_gran = (CW / 128) * (HN / 64);
+    constexpr int w1_gran = NA;
+    constexpr int w2_gran = (CW / 128) * (HN / 64);
 
     const uint32_t dyn0 = (smem_u32(dyn_raw) + 1023u) & ~1023u;
     const uint32_t s_abuf = dyn0;
@@ -208,7 +236,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                            &sh.bar_h[0], &sh.bar_h[1], &sh.bar_acc, &sh.bar_hd, &sh.bar_w2, &sh.bar_fin};
         for (auto* b : one) mbar_init(smem_u32(b), 1);
         uint64_t* many[] = {&sh.bar_pe, &sh.bar_qc, &sh.bar_p[0], &sh.bar_p[1], &sh.bar_a,
-                            &sh.bar_hin, &sh.bar_r, &sh.bar_g[0], &sh.bar_g[1], &sh.bar_cs};
+                            &sh.bar_hin, &sh.bar_r, &sh.bar_g[0], &sh.bar_g[1], &sh.bar_cs, &sh.bar_wg};
         for (auto* b : many) mbar_init(smem_u32(b), NCOMP);
         sh.abort = 0;
         fence_mbar_init();
@@ -261,13 +289,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             cp_async_wait<0>();
             while (n_pend > 0) signal_oldest();
         };
+        int p_slot = 0;
+        uint32_t p_ph = 1;   // parity of the empty-phase a reused slot waits for (first pass: none)
         auto take_slot = [&](int& slot) -> bool {
-            slot = ring_head % NS;
+            slot = p_slot;
             if (ring_head >= (uint32_t)NS) {
-                uint32_t ph = ((ring_head / NS) + 1) & 1;
+                uint32_t ph = p_ph;
                 if (!W.wait(&sh.empty[slot], ph, 40)) return false;
             }
             ++ring_head;
+            if (++p_slot == NS) {
+                p_slot = 0;
+                p_ph ^= 1;
+            }
             return true;
         };
         auto push_tma = [&](const CUtensorMap* m, int x, int y, uint32_t bytes) -> bool {
@@ -361,12 +395,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             uint32_t ph_pe = 0, ph_qc = 0, ph_p[2] = {0, 0}, ph_a = 0, ph_hin = 0, ph_r = 0, ph_g[2] = {0, 0};
             uint32_t ph_hd = 0, ph_w2 = 0;
             bool ok = true;
+            int c_slot = 0;
+            uint32_t c_ph = 0;
             auto consume = [&](int& slot) -> bool {
-                slot = ring_tail % NS;
-                uint32_t ph = (ring_tail / NS) & 1;
+                slot = c_slot;
+                uint32_t ph = c_ph;
                 if (!W.wait(&sh.full[slot], ph, 50)) return false;
                 tc_fence_after();
                 ++ring_tail;
+                if (++c_slot == NS) {
+                    c_slot = 0;
+                    c_ph ^= 1;
+                }
                 return true;
             };
             auto release = [&](int slot) { mma_commit(smem_u32(&sh.empty[slot])); };
@@ -383,6 +423,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     if (!(ok = consume(slot))) break;
                     {
                         const uint64_t da = desc_sw128(s_pe), db = desc_sw128(s_ring + slot * SLOT);
+                        #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             mma_ss(tmem + T_Q, da + 2 * kk, db + 2 * kk, idesc_bf16(128, 64, false), kk > 0);
                         release(slot);
@@ -395,8 +436,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         if (!consume(sl)) return false;
                         const uint64_t db = desc_sw128(s_ring + sl * SLOT);
                         const uint32_t sd = tmem + ((j & 1) ? T_S1 : T_S0);
+                        #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_ts(sd, tmem + T_Q + 8 * kk, db + 2 * kk, idesc_bf16(128, 128, false), kk > 0);
+                            mma_ts(sd, tmem + T_Q + split_col(kk, 64), db + 2 * kk, idesc_bf16(128, 128, false), kk > 0);
                         release(sl);
                         mma_commit(smem_u32(&sh.bar_s[j & 1]));
                         return true;
@@ -408,6 +450,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         if (!(ok = consume(slot))) break;
                         const uint32_t pa = tmem + ((j & 1) ? T_P1 : T_P0);
                         const uint64_t dv = desc_sw128(s_ring + slot * SLOT);
+                        #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
                             mma_ts(tmem + T_O, pa + 8 * kk, dv + 128 * kk, idesc_bf16(128, 64, true), (j > 0 || kk > 0));
                         release(slot);
@@ -431,6 +474,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     const int nc = g / KA, ka = g % KA;
                     const uint64_t da = desc_sw128(ka == 0 ? s_pe : s_abuf + (ka - 1) * 16384);
                     const uint64_t db = desc_sw128(s_ring + slot * SLOT);
+                    #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_ss(tmem + nc * 128, da + 2 * kk, db + 2 * kk, idesc_bf16(128, 128, false),
                                (ka > 0 || kk > 0));
@@ -442,10 +486,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 if (!(ok = W.wait(&sh.bar_hin, ph_hin, 56))) break;
                 tc_fence_after();
                 for (int hf = 0; hf < n_half && ok; ++hf) {
-                    if (hf == 1) {
-                        if (!(ok = W.wait(&sh.bar_r, ph_r, 57))) break;
-                        tc_fence_after();
-                    }
                     auto issue_w1 = [&](int c) -> bool {
                         const uint32_t hd = tmem + ((c & 1) ? T_H1 : T_H0);
                         for (int ka = 0; ka < NA; ++ka) {
@@ -453,6 +493,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                             if (!consume(sl)) return false;
                             const uint64_t da = desc_sw128(s_abuf + ka * 16384);
                             const uint64_t db = desc_sw128(s_ring + sl * SLOT);
+                            #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
                                 mma_ss(hd, da + 2 * kk, db + 2 * kk, idesc_bf16(128, HN, false), (ka > 0 || kk > 0));
                             release(sl);
@@ -467,14 +508,20 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                             if (!consume(sl)) return false;
                             const int nc = q / (HN / 64), kh = q % (HN / 64);
                             const uint64_t db = desc_sw128(s_ring + sl * SLOT);
+                            #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
-                                mma_ts(tmem + nc * 128, ha + kh * 32 + 8 * kk, db + 2 * kk,
+                                mma_ts(tmem + nc * 128, ha + split_col(4 * kh + kk, HN), db + 2 * kk,
                                        idesc_bf16(128, 128, false), 1u);
                             release(sl);
                         }
                         return true;
                     };
                     ok = issue_w1(0) && (n_chunks < 2 || issue_w1(1));
+                    if (ok && hf == 1) {
+                        // the first hidden chunks do not touch the accumulator; W2 needs the restored x1
+                        if (!(ok = W.wait(&sh.bar_r, ph_r, 57))) break;
+                        tc_fence_after();
+                    }
                     for (int c = 0; c < n_chunks && ok; ++c) {
                         if (!(ok = W.wait(&sh.bar_g[c & 1], ph_g[c & 1], 58))) break;
                         tc_fence_after();
@@ -498,12 +545,22 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
     }
     // ==================================================================== compute warps
     else {
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const uint32_t trow = tmem + lane_off;
-        uint32_t ph_q = 0, ph_s[2] = {0, 0}, ph_pv = 0, ph_x = 0, ph_h[2] = {0, 0}, ph_acc = 0, ph_cs = 0;
+        const int wg = tid >> 7;             // warpgroup: column half
+        const int row = tid & 127;           // query row = TMEM lane
+        const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        uint32_t ph_q = 0, ph_s[2] = {0, 0}, ph_pv = 0, ph_x = 0, ph_h[2] = {0, 0}, ph_acc = 0, ph_cs = 0,
+                 ph_wg = 0;
         const float qscale = 0.125f * kLog2e;
+        // smem scratch for row statistics after the attention (the embedding tile is free then)
+        float* xs = reinterpret_cast<float*>(dyn_raw + (s_pe - smem_u32(dyn_raw)));
         bool ok = true;
         auto arrive = [&](uint64_t* b) { mbar_arrive(smem_u32(b)); };
+        auto wg_sync = [&](int site) -> bool {
+            arrive(&sh.bar_wg);
+            return W.wait(&sh.bar_wg, ph_wg, site);
+        };
+        const int HALF = HN / 2;             // hidden units per warpgroup
+        float4* park = halves ? reinterpret_cast<float4*>(ta.park) + (size_t)blockIdx.x * (256 / 4) * BM : nullptr;
         for (int64_t unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
             const Unit u = unit_of(a, unit);
             if (u.nq <= 0) continue;
@@ -512,8 +569,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             // ---- this row's query
             float p[3] = {0.f, 0.f, 0.f};
             int64_t vox = -1, qid = -1;
-            if (tid < u.nq) {
-                const int64_t slot = u.qbeg + tid;
+            if (row < u.nq) {
+                const int64_t slot = u.qbeg + row;
                 qid = slot;
                 if (a.qmode == kQueryXyz) {
                     p[0] = a.xyz[slot * 3];
@@ -529,115 +586,106 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     voxel_point(vox, a.R, p);
                 }
             }
-            for (int c = 0; c < 8; ++c) {
+            #pragma unroll
+            for (int c = 4 * wg; c < 4 * wg + 4; ++c) {
                 uint32_t w[4];
+                #pragma unroll
                 for (int v = 0; v < 4; ++v) w[v] = pack_bf16(pe_lane(p, c * 8 + 2 * v), pe_lane(p, c * 8 + 2 * v + 1));
-                st_shared_v4(swz(s_pe, tid, c), w);
+                st_shared_v4(swz(s_pe, row, c), w);
             }
             fence_proxy_async();
             arrive(&sh.bar_pe);
             float* ml_out = nullptr;
-            if (a.probe_ml && tid < u.nq) {
-                if (a.work == kWorkTileDense) ml_out = a.probe_ml + ((size_t)u.t * a.n_probe + u.first + tid) * H * 2;
-                else if (a.ml_slot) ml_out = a.probe_ml + (size_t)a.ml_slot[u.qbeg + tid] * H * 2;
+            if (a.probe_ml && row < u.nq && wg == 0) {
+                if (a.work == kWorkTileDense) ml_out = a.probe_ml + ((size_t)u.t * a.n_probe + u.first + row) * H * 2;
+                else if (a.ml_slot) ml_out = a.probe_ml + (size_t)a.ml_slot[u.qbeg + row] * H * 2;
             }
             // ================================================= attention
             for (int h = 0; h < H && ok; ++h) {
                 if (!(ok = W.wait(&sh.bar_q, ph_q, 60))) break;
                 tc_fence_after();
                 {
-                    float q0[32], q1[32], b0[32], b1v[32];
-                    tmem_ld32(trow + T_Q, q0);
-                    tmem_ld32(trow + T_Q + 32, q1);
-                    ldg32(a.bq + h * 64, b0);
-                    ldg32(a.bq + h * 64 + 32, b1v);
+                    // dims [32 wg, 32 wg + 32): + bq, scale, pack into the first 16 columns of the source
+                    float q[32], b[32];
+                    tmem_ld32(trow + T_Q + 32 * wg, q);
+                    ldg32(a.bq + h * 64 + 32 * wg, b);
                     tmem_wait_ld();
-                    reg_fence(q0);
-                    reg_fence(q1);
-                    uint32_t pk[32];
+                    reg_fence(q);
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int v = 0; v < 16; ++v) {
-                        pk[v] = pack_bf16((q0[2 * v] + b0[2 * v]) * qscale, (q0[2 * v + 1] + b0[2 * v + 1]) * qscale);
-                        pk[16 + v] = pack_bf16((q1[2 * v] + b1v[2 * v]) * qscale, (q1[2 * v + 1] + b1v[2 * v + 1]) * qscale);
-                    }
-                    tmem_st32(trow + T_Q, pk);
+                    for (int v = 0; v < 16; ++v)
+                        pk[v] = pack_bf16((q[2 * v] + b[2 * v]) * qscale, (q[2 * v + 1] + b[2 * v + 1]) * qscale);
+                    tmem_st16(trow + T_Q + 32 * wg, pk);
                     tmem_wait_st();
                 }
                 tc_fence_before();
                 arrive(&sh.bar_qc);
-                float m_ref = -INFINITY, l_run = 0.f;
+                float m_ref = -INFINITY, l_part = 0.f;
                 for (int j = 0; j < nb; ++j) {
                     if (!(ok = W.wait(&sh.bar_s[j & 1], ph_s[j & 1], 61))) break;
                     tc_fence_after();
-                    const uint32_t sbase = trow + ((j & 1) ? T_S1 : T_S0);
-                    float s0[32], s1[32], s2[32], s3[32];
+                    const uint32_t sbase = trow + ((j & 1) ? T_S1 : T_S0) + 64 * wg;
+                    float s0[32], s1[32];
                     tmem_ld32(sbase, s0);
                     tmem_ld32(sbase + 32, s1);
-                    tmem_ld32(sbase + 64, s2);
-                    tmem_ld32(sbase + 96, s3);
                     tmem_wait_ld();
                     reg_fence(s0);
                     reg_fence(s1);
-                    reg_fence(s2);
-                    reg_fence(s3);
-                    const int valid = nk - j * 128;
-                    if (valid < 128) {
+                    const int valid = nk - j * 128 - 64 * wg;   // own columns < valid are real tokens
+                    if (valid < 64) {
 #pragma unroll
                         for (int c = 0; c < 32; ++c) {
                             if (c >= valid) s0[c] = -INFINITY;
                             if (c + 32 >= valid) s1[c] = -INFINITY;
-                            if (c + 64 >= valid) s2[c] = -INFINITY;
-                            if (c + 96 >= valid) s3[c] = -INFINITY;
                         }
                     }
-                    float mb = -INFINITY;
+                    float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) mb = fmaxf(mb, fmaxf(fmaxf(s0[c], s1[c]), fmaxf(s2[c], s3[c])));
+                    for (int c = 0; c < 32; c += 2) {
+                        m0 = fmaxf(m0, s0[c]);
+                        m1 = fmaxf(m1, s0[c + 1]);
+                        m2 = fmaxf(m2, s1[c]);
+                        m3 = fmaxf(m3, s1[c + 1]);
+                    }
+                    // both halves decide on the same (bf16-truncated) block maximum
+                    const uint16_t own = (uint16_t)(__float_as_uint(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3))) >> 16);
+                    sh.xmax[j & 1][wg][row] = own;
+                    if (!(ok = wg_sync(69))) break;
+                    const uint16_t oth = sh.xmax[j & 1][wg ^ 1][row];
+                    const float mb = fmaxf(__uint_as_float((uint32_t)own << 16), __uint_as_float((uint32_t)oth << 16));
                     const bool need = (j == 0) || (mb > m_ref + 8.0f);
                     const float m_new = need ? fmaxf(mb, m_ref) : m_ref;
                     const float f = (j == 0) ? 0.f : ex2(m_ref - m_new);
                     if (need) m_ref = m_new;
-                    float ls = 0.f;
-                    uint32_t pk0[32], pk1[32];
+                    float la = 0.f, lb = 0.f;
+                    uint32_t pk[32];
 #pragma unroll
                     for (int v = 0; v < 16; ++v) {
                         const float e0 = ex2(s0[2 * v] - m_ref), e1 = ex2(s0[2 * v + 1] - m_ref);
                         const float e2 = ex2(s1[2 * v] - m_ref), e3 = ex2(s1[2 * v + 1] - m_ref);
-                        const float e4 = ex2(s2[2 * v] - m_ref), e5 = ex2(s2[2 * v + 1] - m_ref);
-                        const float e6 = ex2(s3[2 * v] - m_ref), e7 = ex2(s3[2 * v + 1] - m_ref);
-                        ls += (e0 + e1) + (e2 + e3) + (e4 + e5) + (e6 + e7);
-                        pk0[v] = pack_bf16(e0, e1);
-                        pk0[16 + v] = pack_bf16(e2, e3);
-                        pk1[v] = pack_bf16(e4, e5);
-                        pk1[16 + v] = pack_bf16(e6, e7);
+                        la += e0 + e1;
+                        lb += e2 + e3;
+                        pk[v] = pack_bf16(e0, e1);
+                        pk[16 + v] = pack_bf16(e2, e3);
                     }
-                    // P_j's buffer was read by PV_{j-2}; O is rescaled below: PV_{j-1} must be done
-                    if (j > 0) {
+                    if (j > 0) {   // PV_{j-1} (hence PV_{j-2}) done: P buffer free, O stable
                         if (!(ok = W.wait(&sh.bar_pv, ph_pv, 62))) break;
                         tc_fence_after();
                     }
-                    if (need && j > 0) l_run *= f;
-                    l_run += ls;
+                    if (need && j > 0) l_part *= f;
+                    l_part += la + lb;
                     if (j > 0 && __any_sync(0xffffffffu, need)) {
-                        float o0[32], o1[32];
-                        tmem_ld32(trow + T_O, o0);
-                        tmem_ld32(trow + T_O + 32, o1);
+                        float o[32];
+                        tmem_ld32(trow + T_O + 32 * wg, o);
                         tmem_wait_ld();
-                        reg_fence(o0);
-                        reg_fence(o1);
+                        reg_fence(o);
                         const float g = need ? f : 1.0f;
-                        uint32_t u0[32], u1[32];
+                        uint32_t uo[32];
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            u0[c] = __float_as_uint(o0[c] * g);
-                            u1[c] = __float_as_uint(o1[c] * g);
-                        }
-                        tmem_st32(trow + T_O, u0);
-                        tmem_st32(trow + T_O + 32, u1);
+                        for (int c = 0; c < 32; ++c) uo[c] = __float_as_uint(o[c] * g);
+                        tmem_st32(trow + T_O + 32 * wg, uo);
                     }
-                    const uint32_t pbase = trow + ((j & 1) ? T_P1 : T_P0);
-                    tmem_st32(pbase, pk0);
-                    tmem_st32(pbase + 32, pk1);
+                    tmem_st32(trow + ((j & 1) ? T_P1 : T_P0) + 32 * wg, pk);
                     tmem_wait_st();
                     tc_fence_before();
                     arrive(&sh.bar_p[j & 1]);
@@ -645,46 +693,56 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 if (!ok) break;
                 if (!(ok = W.wait(&sh.bar_pv, ph_pv, 63))) break;   // PV_{nb-1}
                 tc_fence_after();
+                // row sum: exchange the halves through TMEM (S0 is idle until the next head's S_0)
+                tmem_st1(trow + T_S0 + wg, __float_as_uint(l_part));
+                tmem_wait_st();
+                tc_fence_before();
+                if (!(ok = wg_sync(70))) break;
+                tc_fence_after();
+                uint32_t l_bits = tmem_ld1(trow + T_S0 + (wg ^ 1));
+                tmem_wait_ld();
+                asm volatile("" : "+r"(l_bits));
+                const float l_oth = __uint_as_float(l_bits);
+                const float l_tot = l_part + l_oth;
                 {
-                    float o0[32], o1[32];
-                    tmem_ld32(trow + T_O, o0);
-                    tmem_ld32(trow + T_O + 32, o1);
+                    float o[32];
+                    tmem_ld32(trow + T_O + 32 * wg, o);
                     tmem_wait_ld();
-                    reg_fence(o0);
-                    reg_fence(o1);
-                    const float inv = 1.0f / l_run;
+                    reg_fence(o);
+                    const float inv = 1.0f / l_tot;
                     const uint32_t atom = s_abuf + h * 16384;
-                    for (int c = 0; c < 8; ++c) {
-                        const float* src = c < 4 ? &o0[c * 8] : &o1[(c - 4) * 8];
+                    #pragma unroll
+                    for (int c = 0; c < 4; ++c) {
                         uint32_t w[4];
-                        for (int v = 0; v < 4; ++v) w[v] = pack_bf16(src[2 * v] * inv, src[2 * v + 1] * inv);
-                        st_shared_v4(swz(atom, tid, c), w);
+                        #pragma unroll
+                        for (int v = 0; v < 4; ++v) w[v] = pack_bf16(o[c * 8 + 2 * v] * inv, o[c * 8 + 2 * v + 1] * inv);
+                        st_shared_v4(swz(atom, row, 4 * wg + c), w);
                     }
                 }
                 if (ml_out) {
                     ml_out[h * 2] = m_ref;
-                    ml_out[h * 2 + 1] = l_run;
+                    ml_out[h * 2 + 1] = l_tot;
                 }
             }
             if (!ok) break;
             fence_proxy_async();
             tc_fence_before();
             arrive(&sh.bar_a);
-            // ================================================= LN1
+            // ================================================= LN1 (each half: C/2 columns)
             if (!(ok = W.wait(&sh.bar_x, ph_x, 64))) break;
             tc_fence_after();
+            const int CH = C / 2, c_lo = wg * CH;
             float mean1 = 0.f, rstd1 = 1.f;
             {
-                // x1 = X + bq + bo; statistics in one pass (sums shifted by the row's first value)
                 float shift = 0.f, s1 = 0.f, s2 = 0.f;
-                for (int cc = 0; cc < C; cc += 32) {
+                for (int cc = c_lo; cc < c_lo + CH; cc += 32) {
                     float v[32], bqv[32], bov[32];
                     tmem_ld32(trow + cc, v);
                     ldg32(a.bq + cc, bqv);
                     ldg32(a.bo + cc, bov);
                     tmem_wait_ld();
                     reg_fence(v);
-                    if (cc == 0) shift = v[0] + bqv[0] + bov[0];
+                    if (cc == c_lo) shift = v[0] + bqv[0] + bov[0];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const float d = v[e] + bqv[e] + bov[e] - shift;
@@ -692,23 +750,31 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         s2 = fmaf(d, d, s2);
                     }
                 }
-                const float m_s = s1 / (float)C;
-                mean1 = shift + m_s;
-                if (a.query_ln) rstd1 = rsqrtf(fmaxf(s2 / (float)C - m_s * m_s, 0.f) + kLnEps);
-                for (int cc = 0; cc < C; cc += 32) {
-                    float v[32], bqv[32], bov[32], g[32], be[32];
-                    tmem_ld32(trow + cc, v);
-                    ldg32(a.bq + cc, bqv);
-                    ldg32(a.bo + cc, bov);
+                const float mh = shift + s1 / (float)CH;
+                const float m2h = fmaxf(s2 - s1 * (s1 / (float)CH), 0.f);
+                xs[(wg * 128 + row) * 2] = mh;
+                xs[(wg * 128 + row) * 2 + 1] = m2h;
+                if (!(ok = wg_sync(71))) break;
+                const float mo = xs[((wg ^ 1) * 128 + row) * 2], m2o = xs[((wg ^ 1) * 128 + row) * 2 + 1];
+                const float m_a = wg ? mo : mh, m_b = wg ? mh : mo;   // fixed order: identical in both halves
+                const float d = m_b - m_a;
+                mean1 = 0.5f * (m_a + m_b);
+                const float m2 = (wg ? m2o : m2h) + (wg ? m2h : m2o) + d * d * 0.25f * (float)C;
+                if (a.query_ln) rstd1 = rsqrtf(m2 / (float)C + kLnEps);
+                for (int cc = c_lo; cc < c_lo + CH; cc += 16) {
+                    float v[16], bqv[16], bov[16], g[16], be[16];
+                    tmem_ld16(trow + cc, v);
+                    ldg16(a.bq + cc, bqv);
+                    ldg16(a.bo + cc, bov);
                     if (a.query_ln) {
-                        ldg32(a.ln1_g + cc, g);
-                        ldg32(a.ln1_b + cc, be);
+                        ldg16(a.ln1_g + cc, g);
+                        ldg16(a.ln1_b + cc, be);
                     }
                     tmem_wait_ld();
-                    reg_fence(v);
-                    uint32_t w[16];
+                    reg_fence16(v);
+                    uint32_t w[8];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
+                    for (int e = 0; e < 8; ++e) {
                         float y0 = v[2 * e] + bqv[2 * e] + bov[2 * e];
                         float y1 = v[2 * e + 1] + bqv[2 * e + 1] + bov[2 * e + 1];
                         if (a.query_ln) {
@@ -719,24 +785,23 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     }
                     const uint32_t atom = s_abuf + (cc / 64) * 16384;
                     const int c0 = (cc % 64) / 8;
-                    for (int q = 0; q < 4; ++q) st_shared_v4(swz(atom, tid, c0 + q), &w[4 * q]);
+                    st_shared_v4(swz(atom, row, c0), &w[0]);
+                    st_shared_v4(swz(atom, row, c0 + 1), &w[4]);
                 }
                 if (halves) {
-                    for (int i = 0; i < 4; ++i) {
-                        float v0[32], v1[32];
-                        tmem_ld32(trow + 256 + 64 * i, v0);
-                        tmem_ld32(trow + 256 + 64 * i + 32, v1);
+                    // park x1[:, 256 + 128 wg, +128) (fp32) until the second half: four
+                    // consecutive columns per 16-byte word, the 128 rows of a word group adjacent
+#pragma unroll 1
+                    for (int part = 0; part < 4; ++part) {
+                        float v[32];
+                        tmem_ld32(trow + 256 + 128 * wg + 32 * part, v);
                         tmem_wait_ld();
-                        reg_fence(v0);
-                        reg_fence(v1);
-                        uint32_t w[32];
-                        for (int e = 0; e < 16; ++e) {
-                            w[e] = pack_bf16(v0[2 * e], v0[2 * e + 1]);
-                            w[16 + e] = pack_bf16(v1[2 * e], v1[2 * e + 1]);
-                        }
-                        tmem_st32(trow + 256 + 32 * i, w);
+                        reg_fence(v);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            park[(32 * wg + 8 * part + q) * BM + row] =
+                                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                     }
-                    tmem_wait_st();
                 }
             }
             fence_proxy_async();
@@ -746,20 +811,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             float hs_mean0 = 0.f, hs_m20 = 0.f, hs_dot0 = 0.f, hs_mean1 = 0.f, hs_m21 = 0.f, hs_dot1 = 0.f;
             for (int hf = 0; hf < n_half && ok; ++hf) {
                 if (hf == 1) {
-                    for (int i = 0; i < 4; ++i) {
-                        float pv[32];
-                        tmem_ld32_sync(trow + 256 + 32 * i, pv);
-                        uint32_t w0[32], w1[32];
-                        for (int e = 0; e < 16; ++e) {
-                            const uint32_t x = __float_as_uint(pv[e]);
-                            w0[2 * e] = __float_as_uint(bf16_lo(x));
-                            w0[2 * e + 1] = __float_as_uint(bf16_hi(x));
-                            const uint32_t y = __float_as_uint(pv[16 + e]);
-                            w1[2 * e] = __float_as_uint(bf16_lo(y));
-                            w1[2 * e + 1] = __float_as_uint(bf16_hi(y));
+                    // restore the parked x1[:, 256 + 128 wg, +128) into the accumulator [128 wg, +128)
+#pragma unroll 1
+                    for (int part = 0; part < 4; ++part) {
+                        uint32_t w[32];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 t = park[(32 * wg + 8 * part + q) * BM + row];
+                            w[4 * q] = __float_as_uint(t.x);
+                            w[4 * q + 1] = __float_as_uint(t.y);
+                            w[4 * q + 2] = __float_as_uint(t.z);
+                            w[4 * q + 3] = __float_as_uint(t.w);
                         }
-                        tmem_st32(trow + 64 * i, w0);
-                        tmem_st32(trow + 64 * i + 32, w1);
+                        tmem_st32(trow + 128 * wg + 32 * part, w);
                     }
                     tmem_wait_st();
                     tc_fence_before();
@@ -768,24 +832,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 for (int c = 0; c < n_chunks; ++c) {
                     if (!(ok = W.wait(&sh.bar_h[c & 1], ph_h[c & 1], 65))) break;
                     tc_fence_after();
-                    const uint32_t hb = trow + ((c & 1) ? T_H1 : T_H0);
-                    for (int part = 0; part < HN / 64; ++part) {
-                        float v0[32], v1[32], c0v[32], c1v[32];
-                        const int f0 = c * HN + part * 64;
-                        tmem_ld32(hb + part * 64, v0);
-                        tmem_ld32(hb + part * 64 + 32, v1);
-                        ldg32(a.b1 + f0, c0v);
-                        ldg32(a.b1 + f0 + 32, c1v);
+                    const uint32_t hb = trow + ((c & 1) ? T_H1 : T_H0) + HALF * wg;
+                    const int f0 = c * HN + HALF * wg;
+                    for (int part = 0; part < HALF / 32; ++part) {
+                        float v[32], bb[32];
+                        tmem_ld32(hb + 32 * part, v);
+                        ldg32(a.b1 + f0 + 32 * part, bb);
                         tmem_wait_ld();
-                        reg_fence(v0);
-                        reg_fence(v1);
-                        uint32_t w[32];
+                        reg_fence(v);
+                        uint32_t w[16];
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            w[e] = pack_bf16(gelu_as(v0[2 * e] + c0v[2 * e]), gelu_as(v0[2 * e + 1] + c0v[2 * e + 1]));
-                            w[16 + e] = pack_bf16(gelu_as(v1[2 * e] + c1v[2 * e]), gelu_as(v1[2 * e + 1] + c1v[2 * e + 1]));
-                        }
-                        tmem_st32(hb + part * 32, w);
+                        for (int e = 0; e < 16; ++e)
+                            w[e] = pack_bf16(gelu_as(v[2 * e] + bb[2 * e]), gelu_as(v[2 * e + 1] + bb[2 * e + 1]));
+                        tmem_st16(hb + 16 * part, w);
                     }
                     tmem_wait_st();
                     tc_fence_before();
@@ -794,68 +853,87 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 if (!ok) break;
                 if (!(ok = W.wait(&sh.bar_acc, ph_acc, 67))) break;
                 tc_fence_after();
-                const int cb = hf * 256;
-                // x2 = acc + bq + bo + b2 on this half's columns: shifted sums and the head dot product
+                // x2 = acc + bq + bo + b2 on this warpgroup's half of the half's columns
+                const int CWH = CW / 2, cb = hf * 256 + wg * CWH;
                 float shift = 0.f, s1 = 0.f, s2 = 0.f, dot = 0.f;
-                for (int cc = 0; cc < CW; cc += 32) {
+                for (int cc = 0; cc < CWH; cc += 16) {
                     const int col0 = cb + cc;
-                    float v[32], bqv[32], bov[32], b2v[32], wv[32], gv[32];
-                    tmem_ld32(trow + cc, v);
-                    ldg32(a.bq + col0, bqv);
-                    ldg32(a.bo + col0, bov);
-                    ldg32(a.b2 + col0, b2v);
-                    ldg32(a.w_head + col0, wv);
-                    if (a.query_ln) ldg32(a.ln2_g + col0, gv);
+                    float v[16], bqv[16], bov[16], wv[16];
+                    tmem_ld16(trow + wg * CWH + cc, v);
+                    ldg16(a.bq + col0, bqv);
+                    ldg16(a.bo + col0, bov);
+                    ldg16(a.w_head + col0, wv);
                     tmem_wait_ld();
-                    reg_fence(v);
-                    if (cc == 0) shift = v[0] + bqv[0] + bov[0] + b2v[0];
+                    reg_fence16(v);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float x = v[e] + bqv[e] + bov[e] + b2v[e];
+                    for (int e = 0; e < 16; ++e) bqv[e] += bov[e];
+                    ldg16(a.b2 + col0, bov);
+                    if (a.query_ln) {
+                        float gv[16];
+                        ldg16(a.ln2_g + col0, gv);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) wv[e] *= gv[e];
+                    }
+                    if (cc == 0) shift = v[0] + bqv[0] + bov[0];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float x = v[e] + bqv[e] + bov[e];
                         const float d = x - shift;
                         s1 += d;
                         s2 = fmaf(d, d, s2);
-                        dot = fmaf(x, a.query_ln ? wv[e] * gv[e] : wv[e], dot);
+                        dot = fmaf(x, wv[e], dot);
                     }
                 }
-                const float m_s = s1 / (float)CW;
-                const float mh = shift + m_s;
-                const float m2 = fmaxf(s2 - s1 * m_s, 0.f);   // sum of squared deviations from mh
+                const float mh = shift + s1 / (float)CWH;
+                const float m2h = fmaxf(s2 - s1 * (s1 / (float)CWH), 0.f);
+                float* xh = xs + 512 + hf * 768;
+                xh[(wg * 128 + row) * 3] = mh;
+                xh[(wg * 128 + row) * 3 + 1] = m2h;
+                xh[(wg * 128 + row) * 3 + 2] = dot;
+                if (!(ok = wg_sync(73))) break;
+                const float* ra = xh + row * 3;            // warpgroup 0's values
+                const float* rb = xh + (128 + row) * 3;    // warpgroup 1's values
+                const float d = rb[0] - ra[0];
+                const float mean_h = 0.5f * (ra[0] + rb[0]);
+                const float m2_h = ra[1] + rb[1] + d * d * 0.25f * (float)CW;
+                const float dot_h = ra[2] + rb[2];
                 if (hf == 0) {
-                    hs_mean0 = mh;
-                    hs_m20 = m2;
-                    hs_dot0 = dot;
+                    hs_mean0 = mean_h;
+                    hs_m20 = m2_h;
+                    hs_dot0 = dot_h;
                 } else {
-                    hs_mean1 = mh;
-                    hs_m21 = m2;
-                    hs_dot1 = dot;
+                    hs_mean1 = mean_h;
+                    hs_m21 = m2_h;
+                    hs_dot1 = dot_h;
                 }
             }
             if (!ok) break;
             // ================================================= head + output
-            float dec;
-            if (a.query_ln) {
-                float mean, m2;
-                if (n_half == 1) {
-                    mean = hs_mean0;
-                    m2 = hs_m20;
+            if (wg == 0) {
+                float dec;
+                if (a.query_ln) {
+                    float mean, m2;
+                    if (n_half == 1) {
+                        mean = hs_mean0;
+                        m2 = hs_m20;
+                    } else {
+                        const float d = hs_mean1 - hs_mean0;
+                        mean = 0.5f * (hs_mean0 + hs_mean1);
+                        m2 = hs_m20 + hs_m21 + d * d * 0.25f * (float)C;
+                    }
+                    const float rstd = rsqrtf(m2 / (float)C + kLnEps);
+                    dec = (hs_dot0 + hs_dot1 - mean * sh.G) * rstd + sh.Bc;
                 } else {
-                    const float d = hs_mean1 - hs_mean0;
-                    mean = 0.5f * (hs_mean0 + hs_mean1);
-                    m2 = hs_m20 + hs_m21 + d * d * 0.25f * (float)C;
+                    dec = hs_dot0 + hs_dot1 + sh.Bc;
                 }
-                const float rstd = rsqrtf(m2 / (float)C + kLnEps);
-                dec = (hs_dot0 + hs_dot1 - mean * sh.G) * rstd + sh.Bc;
-            } else {
-                dec = hs_dot0 + hs_dot1 + sh.Bc;
-            }
-            if (tid < u.nq) {
-                float val = dec;
-                if (a.spheres) val = sphere_union(p, a.spheres, a.n_spheres) + a.dec_scale * tanhf(dec);
-                if (a.out) a.out[qid] = val;
-                if (vox >= 0) {
-                    if (a.grid) a.grid[vox] = val;
-                    if (a.dec_grid) a.dec_grid[vox] = dec;
+                if (row < u.nq) {
+                    float val = dec;
+                    if (a.spheres) val = sphere_union(p, a.spheres, a.n_spheres) + a.dec_scale * tanhf(dec);
+                    if (a.out) a.out[qid] = val;
+                    if (vox >= 0) {
+                        if (a.grid) a.grid[vox] = val;
+                        if (a.dec_grid) a.dec_grid[vox] = dec;
+                    }
                 }
             }
             // the next tile's first MMA waits for bar_pe, which these threads
@@ -893,6 +971,10 @@ EncodeTiledFn encode_fn() {
 
 __device__ int g_tc_error = 0;
 
+// parking area for the second half of x1 (C == 512): one 128 x 256 fp32 block per CTA
+constexpr int kParkCtas = 160;
+__device__ float4 g_x1_park[(size_t)kParkCtas * 256 / 4 * BM];
+
 }  // namespace
 
 // 2D bf16 matrix [rows][cols] row-major, box {64 cols, box_rows rows}, 128 B swizzle
@@ -925,9 +1007,7 @@ bool tc_supported(const DecodeArgs& a, vdm_dtype dt) {
 
 size_t tc_smem_bytes(int C, int* ns_out) {
     const size_t fixed = (size_t)(C / 64) * 16384 + 16384 + 1024;
-    const size_t limit = 227 * 1024;
-    int ns = (int)((limit - fixed - 512) / SLOT);
-    if (ns > MAX_NS) ns = MAX_NS;
+    const int ns = ring_slots(C);
     if (ns_out) *ns_out = ns;
     return fixed + (size_t)ns * SLOT;
 }
@@ -939,7 +1019,7 @@ vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
     const size_t smem = tc_smem_bytes(d.C, &ns);
     if (ns < GATHER_LAG + 2) return fail(VDM_ERR_INTERNAL, "not enough shared memory for the ring (%d slots)", ns);
     CUtensorMap m_wq, m_wq64, m_wo, m_w1, m_w2, m_k, m_v;
-    const int HN = d.C > 256 ? 64 : 128;
+    const int HN = 128;
     VDM_TRY(make_bf16_map(&m_wq, d.Wq, d.C, 64, 128));
     VDM_TRY(make_bf16_map(&m_wq64, d.Wq, d.C, 64, 64));
     VDM_TRY(make_bf16_map(&m_wo, d.Wo, d.C, d.C, 128));
@@ -953,16 +1033,21 @@ vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
     TcArgs ta;
     ta.d = d;
     ta.ns = ns;
+    ta.park = nullptr;
+    if (d.C > 256 && cudaGetSymbolAddress((void**)&ta.park, g_x1_park) != cudaSuccess)
+        return fail(VDM_ERR_CUDA, "parking area lookup failed");
     ta.err = tc_error_word();
     if (!ta.err) return fail(VDM_ERR_CUDA, "error word lookup failed");
     ta.timeout = g_debug.timeout > 0 ? g_debug.timeout : 4000000000ll;
     ta.inject = g_debug.inject;
     g_debug.inject = 0;   // one launch only
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = d.C == 128 ? decode_tc_kernel<128> : d.C == 256 ? decode_tc_kernel<256> : decode_tc_kernel<512>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "decode_tc smem attribute: %s", cudaGetErrorString(e));
+    if (sms > kParkCtas) sms = kParkCtas;   // one parking block per CTA
     const unsigned grid = (unsigned)(n_units < sms ? n_units : sms);
     prof_begin(kProfDecode, st);
-    decode_tc_kernel<<<grid, NT, smem, st>>>(m_wq, m_wq64, m_wo, m_w1, m_w2, m_k, m_v, ta);
+    kern<<<grid, NT, smem, st>>>(m_wq, m_wq64, m_wo, m_w1, m_w2, m_k, m_v, ta);
     prof_end(kProfDecode, st);
     return check_launch("decode_tc_kernel");
 }
