@@ -70,7 +70,7 @@ constexpr int NT = 320;        // + MMA warp + producer warp
 constexpr int WARP_MMA = 8, WARP_PROD = 9;
 constexpr int SLOT = 16384;    // ring slot bytes
 constexpr int MAX_NS = 8;
-constexpr int GATHER_LAG = 2;  // gathered items in flight before their barrier is signalled
+constexpr int GATHER_LAG = 3;  // gathered items in flight before their barrier is signalled
 constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr uint32_t T_S0 = 0, T_S1 = 128, T_P0 = 256, T_P1 = 320, T_O = 384, T_Q = 448;
@@ -320,13 +320,20 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             int slot;
             if (!take_slot(slot)) return false;
             const uint32_t dst = s_ring + slot * SLOT;
-            for (int i = 0; i < 32; ++i) {   // 128 rows x 8 chunks, 32 lanes
-                const int idx = i * 32 + lane;
-                const int r = idx >> 3, c = idx & 7;
-                const int tok = j * 128 + r;
-                const bool okr = tok < nk;
-                const int row = okr ? sel[tok] : 0;
-                cp_async16(swz(dst, r, c), src + ((size_t)h * N + row) * 64 + c * 8, okr);
+            // 128 rows x 8 chunks of 16 B: lane l copies chunk l % 8 of rows 4i + l / 8; the
+            // 32 row indices are loaded first (independent loads), then the copies are issued
+            const int c = lane & 7;
+            int rows[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int tok = j * 128 + 4 * i + (lane >> 3);
+                rows[i] = tok < nk ? __ldg(sel + tok) : -1;
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int r = 4 * i + (lane >> 3);
+                const bool okr = rows[i] >= 0;
+                cp_async16(swz(dst, r, c), src + ((size_t)h * N + (okr ? rows[i] : 0)) * 64 + c * 8, okr);
             }
             cp_async_commit();
             pend[n_pend++] = slot;
