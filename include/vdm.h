@@ -243,6 +243,17 @@ VDM_API vdm_status vdm_decode_hierarchical_noalloc(const vdm_decoder* dec, const
  * usable.  mode 0 restores normal operation.                               */
 VDM_API vdm_status vdm_debug_inject(int32_t mode, int64_t timeout_cycles);
 
+/* Tensor-core decoding on CTA pairs: with enable = 1, each 256-query MMA runs
+ * on the two CTAs of a cluster (cta_group::2); each CTA holds 128 query rows
+ * and loads half of every weight and key/value tile, which halves the bytes
+ * each SM streams per query.  enable = 0 (the default) runs one CTA per
+ * 128-query MMA.  Both give the same results up to the order of floating-point
+ * sums.  Measured on B200: pairs are faster when attention is short (128
+ * tokens), slower for 3072-token attention, and about even on the adaptive
+ * hierarchical workload.  Takes effect for the launches that follow; not
+ * thread-safe against concurrent decodes.                                     */
+VDM_API vdm_status vdm_set_cta_pairs(int32_t enable);
+
 /* Kernel timing for measurement (not needed for decoding).  Between
  * vdm_profile_begin() and vdm_profile_end() the calling thread's launches are
  * bracketed by CUDA events on their stream; vdm_profile_end() waits for those

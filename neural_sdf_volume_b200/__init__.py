@@ -35,7 +35,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "workspace", 4: "
 
 EXPORTS = ("vdm_precompute_kv", "vdm_decode_dense", "vdm_select_kv",
            "vdm_hierarchical_workspace_size", "vdm_decode_hierarchical",
-           "vdm_decode_hierarchical_noalloc", "vdm_debug_inject", "vdm_profile_begin", "vdm_profile_end",
+           "vdm_decode_hierarchical_noalloc", "vdm_debug_inject", "vdm_set_cta_pairs",
+           "vdm_profile_begin", "vdm_profile_end",
            "vdm_status_string", "vdm_last_error", "vdm_abi_version")
 PROF_CLASSES = ("kv", "decode", "select", "mark", "scan", "list", "fill", "probe")
 
@@ -99,6 +100,8 @@ _lib.vdm_decode_hierarchical_noalloc.argtypes = [C.POINTER(CDecoder), _vp, _vp, 
                                                  C.POINTER(CHierStats), C.POINTER(CHierDebug), _vp]
 _lib.vdm_debug_inject.argtypes = [_i32, _i64]
 _lib.vdm_debug_inject.restype = C.c_int
+_lib.vdm_set_cta_pairs.argtypes = [_i32]
+_lib.vdm_set_cta_pairs.restype = C.c_int
 _lib.vdm_profile_begin.argtypes = []
 _lib.vdm_profile_end.argtypes = [C.POINTER(CProfile)]
 for _f in ("vdm_precompute_kv", "vdm_decode_dense", "vdm_select_kv",
@@ -302,6 +305,11 @@ def vdm_debug_inject(mode: int, timeout_cycles: int = 0):
     """Test hook: mode 1 withholds one completion signal in the next
     tensor-core decode launch (its bounded waits then report a timeout)."""
     _check(_lib.vdm_debug_inject(mode, timeout_cycles))
+
+
+def vdm_set_cta_pairs(enable: bool):
+    """Run tensor-core decoding on CTA pairs (True) or one CTA per MMA (False, the default)."""
+    _check(_lib.vdm_set_cta_pairs(1 if enable else 0))
 
 
 def vdm_profile_begin():

@@ -69,7 +69,7 @@ constexpr int NCOMP = 256;     // compute threads (two warpgroups)
 constexpr int NT = 320;        // + MMA warp + producer warp
 constexpr int WARP_MMA = 8, WARP_PROD = 9;
 constexpr int SLOT = 16384;    // ring slot bytes
-constexpr int MAX_NS = 8;
+constexpr int MAX_NS = 16;   // ring slots (CTA pairs use twice as many, half as large)
 constexpr int GATHER_LAG = 3;  // gathered items in flight before their barrier is signalled
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -78,9 +78,9 @@ constexpr uint32_t T_S0 = 0, T_S1 = 128, T_P0 = 256, T_P1 = 320, T_O = 384, T_Q 
 // ring depth: 16 KB slots in what the 227 KB of shared memory leaves after the
 // activation buffer (C/64 atoms of 16 KB), the embedding tile and alignment
 __host__ __device__ constexpr int ring_slots(int C) {
-    return (int)((227 * 1024 - ((C / 64) * 16384 + 16384 + 1024) - 512) / SLOT) < MAX_NS
+    return (int)((227 * 1024 - ((C / 64) * 16384 + 16384 + 1024) - 512) / SLOT) < MAX_NS / 2
                ? (int)((227 * 1024 - ((C / 64) * 16384 + 16384 + 1024) - 512) / SLOT)
-               : MAX_NS;
+               : MAX_NS / 2;
 }
 
 struct TcArgs {
@@ -108,26 +108,33 @@ struct Waiter {
     Shared* sh;
     int* err;
     long long timeout;
-    // Wait for the phase with parity `phase` to complete; flips `phase`.
+    uint32_t peer_abort;   // CTA pairs: shared::cluster address of the other CTA's abort flag (else 0)
+    bool cluster_acq;      // acquire at cluster scope (barriers that collect the other CTA's arrivals)
+    // Wait for the phase with parity `phase` to complete; flips `phase`.  Called by
+    // whole warps (every role runs converged); the result is the same in all lanes.
     __device__ bool wait(uint64_t* bar, uint32_t& phase, int site) {
         const uint32_t b = smem_u32(bar);
         long long t0 = 0;
+        bool done = false;
         for (uint32_t it = 0;; ++it) {
-            if (mbar_try_wait(b, phase)) {
+            if (cluster_acq ? mbar_try_wait_cluster(b, phase) : mbar_try_wait(b, phase)) {
                 phase ^= 1;
-                return true;
+                done = true;
+                break;
             }
             if ((it & 63) == 63) {
-                if (*reinterpret_cast<volatile int*>(&sh->abort)) return false;
+                if (*reinterpret_cast<volatile int*>(&sh->abort)) break;
                 const long long t = clock64();
                 if (t0 == 0) t0 = t;
                 else if (t - t0 > timeout) {
                     *reinterpret_cast<volatile int*>(&sh->abort) = 1;
+                    if (peer_abort) st_cluster_u32(peer_abort, 1u);
                     atomicCAS(err, 0, site);
-                    return false;
+                    break;
                 }
             }
         }
+        return __all_sync(0xffffffffu, done);
     }
 };
 
@@ -141,6 +148,10 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, long l
 
 __device__ __forceinline__ uint32_t swz(uint32_t base, int r, int c) {
     return base + r * 128 + ((c ^ (r & 7)) << 4);
+}
+// 64-byte rows, 64 B swizzle: the 16-byte chunk index is XORed with address bits 7-8
+__device__ __forceinline__ uint32_t swz64(uint32_t base, int r, int c) {
+    return base + r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
 }
 
 // TMEM column of k-step q (16 elements) of a W-wide split-packed A operand
@@ -195,7 +206,7 @@ __device__ __forceinline__ Unit unit_of(const DecodeArgs& a, int64_t unit) {
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int CC>
+template <int CC, int CG>
 __global__ void __launch_bounds__(NT, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_wq64,
                  const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_w1,
@@ -212,32 +223,49 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
     constexpr int NA = C / 64;
     constexpr bool halves = C > 256;
     constexpr int HN = 128;
-    constexpr int NS = ring_slots(C);
+    constexpr int NS = ring_slots(C);   // 16 KB slots that fit
     constexpr int CW = halves ? 256 : C;
     constexpr int n_half = halves ? 2 : 1;
     constexpr uint32_t T_H0 = 256, T_H1 = 384;
     const int n_chunks = F / HN;
     constexpr int w1_gran = NA;
     constexpr int w2_gran = (CW / 128) * (HN / 64);
+    // CG == 2: the CTA pair of a cluster runs 256-row MMAs; each CTA loads half of
+    // every B operand (its N/2 rows), the even CTA issues the MMAs, and the odd
+    // CTA forwards the completion of its loads to the even CTA's ring barriers.
+    constexpr bool PAIR = CG == 2;
+    const uint32_t crank = PAIR ? cluster_rank() : 0u;
+    const bool leader = crank == 0;
+    constexpr int BR = PAIR ? 64 : 128;   // weight / key rows of a 128-row B tile held by this CTA
+    // ring items: a CTA of a pair holds half of each weight tile (8 KB), so one 16 KB slot
+    // carries two consecutive 64-wide K atoms (8 MMA k-steps per wait and release)
+    constexpr int RS = SLOT;
+    constexpr int NR = NS;
+    constexpr int AT = PAIR ? 2 : 1;      // K atoms per weight item
+    constexpr int KA = NA + 1;            // output-projection K atoms: embedding + attention
 
     const uint32_t dyn0 = (smem_u32(dyn_raw) + 1023u) & ~1023u;
     const uint32_t s_abuf = dyn0;
     const uint32_t s_pe = s_abuf + NA * 16384;
     const uint32_t s_ring = s_pe + 16384;
 
-    Waiter W{&sh, ta.err, ta.timeout};
+    Waiter W{&sh, ta.err, ta.timeout, PAIR ? mapa(smem_u32(&sh.abort), crank ^ 1u) : 0u, false};
 
     if (tid == 0) {
-        for (int i = 0; i < NS; ++i) {
-            mbar_init(smem_u32(&sh.full[i]), 1);
+        for (int i = 0; i < NR; ++i) {
+            // the even CTA's ring slot is complete when its own load and the odd CTA's forward arrived
+            mbar_init(smem_u32(&sh.full[i]), PAIR && leader ? 2 : 1);
             mbar_init(smem_u32(&sh.empty[i]), 1);
         }
         uint64_t* one[] = {&sh.bar_q, &sh.bar_s[0], &sh.bar_s[1], &sh.bar_pv, &sh.bar_x,
                            &sh.bar_h[0], &sh.bar_h[1], &sh.bar_acc, &sh.bar_hd, &sh.bar_w2, &sh.bar_fin};
         for (auto* b : one) mbar_init(smem_u32(b), 1);
-        uint64_t* many[] = {&sh.bar_pe, &sh.bar_qc, &sh.bar_p[0], &sh.bar_p[1], &sh.bar_a,
-                            &sh.bar_hin, &sh.bar_r, &sh.bar_g[0], &sh.bar_g[1], &sh.bar_cs, &sh.bar_wg};
-        for (auto* b : many) mbar_init(smem_u32(b), NCOMP);
+        // compute -> MMA: one arrival per compute thread, or per compute warp of both CTAs
+        uint64_t* to_mma[] = {&sh.bar_pe, &sh.bar_qc, &sh.bar_p[0], &sh.bar_p[1], &sh.bar_a,
+                              &sh.bar_hin, &sh.bar_r, &sh.bar_g[0], &sh.bar_g[1]};
+        for (auto* b : to_mma) mbar_init(smem_u32(b), PAIR ? 2 * (NCOMP / 32) : NCOMP);
+        mbar_init(smem_u32(&sh.bar_cs), NCOMP);
+        mbar_init(smem_u32(&sh.bar_wg), NCOMP);
         sh.abort = 0;
         fence_mbar_init();
         fence_proxy_async();
@@ -259,15 +287,62 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
         }
     }
     if (warp == 0) {
-        tmem_alloc(smem_u32(&sh.tmem_base), 512);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(smem_u32(&sh.tmem_base), 512);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(&sh.tmem_base), 512);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();   // both CTAs' barriers are initialised before any remote arrival
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
 
+    // Work: units of 128 queries; a CTA pair takes two units that attend to the same keys
+    // (consecutive flat units, or two slots of one sub-volume) and skips a pair only when
+    // both are empty.
     const int64_t n_units = a.work == kWorkFlat ? (a.M + BM - 1) / BM : (int64_t)a.T * a.slots;
+    const int spt = PAIR ? (a.slots + 1) / 2 : a.slots;   // slot pairs per sub-volume
+    const int64_t n_iter = !PAIR ? n_units : a.work == kWorkFlat ? (n_units + 1) / 2 : (int64_t)a.T * spt;
+    const int64_t it0 = PAIR ? blockIdx.x / 2 : blockIdx.x;
+    const int64_t it_step = PAIR ? gridDim.x / 2 : gridDim.x;
+    auto unit_at = [&](int64_t it, uint32_t r) -> Unit {
+        if (!PAIR) return unit_of(a, it);
+        if (a.work == kWorkFlat) return unit_of(a, 2 * it + r);
+        const int64_t t = it / spt;
+        const int sl = 2 * (int)(it - t * spt) + (int)r;
+        if (sl < a.slots) return unit_of(a, t * a.slots + sl);
+        Unit u = unit_of(a, t * a.slots);   // same sub-volume (same keys), no queries
+        u.nq = 0;
+        return u;
+    };
+    auto active = [&](int64_t it) -> bool {
+        if (unit_at(it, crank).nq > 0) return true;
+        return PAIR && unit_at(it, crank ^ 1u).nq > 0;
+    };
+    // barriers of the MMA-issuing CTA, and commits that reach both CTAs
+    auto lead_bar = [&](uint64_t* b) -> uint32_t { return PAIR ? mapa(smem_u32(b), 0u) : smem_u32(b); };
+    // (issued by the whole MMA warp; one elected lane commits)
+    auto commit_both = [&](uint64_t* b) {
+        if (PAIR) {
+            mma_commit_pair_w(mapa(smem_u32(b), 0u));
+            mma_commit_pair_w(mapa(smem_u32(b), 1u));
+        } else {
+            mma_commit_w(smem_u32(b));
+        }
+    };
+    auto commit_own = [&](uint64_t* b) {
+        if (PAIR) mma_commit_pair_w(smem_u32(b));
+        else mma_commit_w(smem_u32(b));
+    };
+    // items a unit pushes through the ring (producer, MMA and forwarder agree on it)
+    auto n_items = [&](int nb) -> int {
+        return H * (1 + 2 * nb) + (C / 128) * ((KA + AT - 1) / AT) +
+               n_half * n_chunks * (w1_gran / AT + w2_gran / AT);
+    };
 
     // ==================================================================== producer
     if (warp == WARP_PROD) {
@@ -293,12 +368,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
         uint32_t p_ph = 1;   // parity of the empty-phase a reused slot waits for (first pass: none)
         auto take_slot = [&](int& slot) -> bool {
             slot = p_slot;
-            if (ring_head >= (uint32_t)NS) {
+            if (ring_head >= (uint32_t)NR) {
                 uint32_t ph = p_ph;
                 if (!W.wait(&sh.empty[slot], ph, 40)) return false;
             }
             ++ring_head;
-            if (++p_slot == NS) {
+            if (++p_slot == NR) {
                 p_slot = 0;
                 p_ph ^= 1;
             }
@@ -311,29 +386,78 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             if (lane == 0) {
                 const uint32_t fb = smem_u32(&sh.full[slot]);
                 mbar_expect_tx(fb, bytes);
-                tma_load_2d(s_ring + slot * SLOT, m, x, y, fb);
+                tma_load_2d(s_ring + slot * RS, m, x, y, fb);
             }
             __syncwarp();
             return true;
         };
-        auto push_gather = [&](const __nv_bfloat16* src, const int32_t* sel, int h, int j, int nk) -> bool {
+        // two boxes of `bytes` each in one slot (the second at offset `bytes`); nbox = 1 or 2
+        auto push_tma2 = [&](const CUtensorMap* m0, int x0, int y0, const CUtensorMap* m1, int x1, int y1,
+                             uint32_t bytes, int nbox) -> bool {
+            drain();
             int slot;
             if (!take_slot(slot)) return false;
-            const uint32_t dst = s_ring + slot * SLOT;
-            // 128 rows x 8 chunks of 16 B: lane l copies chunk l % 8 of rows 4i + l / 8; the
-            // 32 row indices are loaded first (independent loads), then the copies are issued
-            const int c = lane & 7;
-            int rows[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int tok = j * 128 + 4 * i + (lane >> 3);
-                rows[i] = tok < nk ? __ldg(sel + tok) : -1;
+            if (lane == 0) {
+                const uint32_t fb = smem_u32(&sh.full[slot]);
+                mbar_expect_tx(fb, bytes * nbox);
+                tma_load_2d(s_ring + slot * RS, m0, x0, y0, fb);
+                if (nbox > 1) tma_load_2d(s_ring + slot * RS + bytes, m1, x1, y1, fb);
             }
+            __syncwarp();
+            return true;
+        };
+        auto push_gather = [&](bool isv, const __nv_bfloat16* src, const int32_t* sel, int h, int j,
+                               int nk) -> bool {
+            int slot;
+            if (!take_slot(slot)) return false;
+            const uint32_t dst = s_ring + slot * RS;
+            if (!PAIR) {
+                // 128 rows x 8 chunks of 16 B: lane l copies chunk l % 8 of rows 4i + l / 8; the
+                // 32 row indices are loaded first (independent loads), then the copies are issued
+                const int c = lane & 7;
+                int rows[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int r = 4 * i + (lane >> 3);
-                const bool okr = rows[i] >= 0;
-                cp_async16(swz(dst, r, c), src + ((size_t)h * N + (okr ? rows[i] : 0)) * 64 + c * 8, okr);
+                for (int i = 0; i < 32; ++i) {
+                    const int tok = j * 128 + 4 * i + (lane >> 3);
+                    rows[i] = tok < nk ? __ldg(sel + tok) : -1;
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int r = 4 * i + (lane >> 3);
+                    const bool okr = rows[i] >= 0;
+                    cp_async16(swz(dst, r, c), src + ((size_t)h * N + (okr ? rows[i] : 0)) * 64 + c * 8, okr);
+                }
+            } else if (!isv) {
+                // keys: this CTA's 64 tokens of the block, 8 chunks each (128 B swizzle)
+                const int c = lane & 7;
+                int rows[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int tok = j * 128 + 64 * (int)crank + 4 * i + (lane >> 3);
+                    rows[i] = tok < nk ? __ldg(sel + tok) : -1;
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int r = 4 * i + (lane >> 3);
+                    const bool okr = rows[i] >= 0;
+                    cp_async16(swz(dst, r, c), src + ((size_t)h * N + (okr ? rows[i] : 0)) * 64 + c * 8, okr);
+                }
+            } else {
+                // values: all 128 tokens, this CTA's 32 head dimensions = 4 chunks (64 B swizzle)
+                const int c = lane & 3;
+                int rows[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int tok = j * 128 + 8 * i + (lane >> 2);
+                    rows[i] = tok < nk ? __ldg(sel + tok) : -1;
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int r = 8 * i + (lane >> 2);
+                    const bool okr = rows[i] >= 0;
+                    cp_async16(swz64(dst, r, c),
+                               src + ((size_t)h * N + (okr ? rows[i] : 0)) * 64 + 32 * crank + c * 8, okr);
+                }
             }
             cp_async_commit();
             pend[n_pend++] = slot;
@@ -343,17 +467,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             }
             return true;
         };
-        for (int64_t unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
-            const Unit u = unit_of(a, unit);
-            if (u.nq <= 0) continue;
+        const int rb = (int)crank * BR;   // this CTA's row offset inside a 128-row B tile
+        for (int64_t it = it0; it < n_iter && ok; it += it_step) {
+            if (!active(it)) continue;
+            const Unit u = unit_at(it, crank);
             const int nk = u.sel ? a.ksel : N;
             const int nb = (nk + 127) / 128;
             auto push_kv = [&](bool isv, int h, int j) -> bool {
-                if (u.sel) return push_gather(isv ? Vg : Kg, u.sel, h, j, nk);
-                return push_tma(isv ? &tm_v : &tm_k, 0, h * N + j * 128, SLOT);
+                if (u.sel) return push_gather(isv, isv ? Vg : Kg, u.sel, h, j, nk);
+                if (isv) return push_tma(&tm_v, PAIR ? 32 * (int)crank : 0, h * N + j * 128, PAIR ? 8192 : SLOT);
+                return push_tma(&tm_k, 0, h * N + j * 128 + rb, BR * 128);
             };
             for (int h = 0; h < H && ok; ++h) {
-                ok = push_tma(&tm_wq64, 0, h * 64, 64 * 128);
+                ok = push_tma(&tm_wq64, 0, h * 64 + (PAIR ? 32 * (int)crank : 0), PAIR ? 32 * 128 : 64 * 128);
                 ok = ok && push_kv(false, h, 0);
                 if (nb > 1) ok = ok && push_kv(false, h, 1);
                 for (int j = 0; j < nb && ok; ++j) {
@@ -361,21 +487,25 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     if (j + 2 < nb) ok = ok && push_kv(false, h, j + 2);
                 }
             }
-            // X = PE Wq^T + a Wo^T : granule (nc, ka)
-            const int KA = NA + 1;
-            for (int g = 0; g < (C / 128) * KA && ok; ++g) {
-                const int nc = g / KA, ka = g % KA;
-                ok = ka == 0 ? push_tma(&tm_wq, 0, nc * 128, SLOT) : push_tma(&tm_wo, (ka - 1) * 64, nc * 128, SLOT);
-            }
-            // MLP granules in MMA consumption order
+            // X = PE Wq^T + a Wo^T : items of AT K atoms (atom 0: Wq, atom ka > 0: Wo columns ka-1)
+            for (int nc = 0; nc < C / 128 && ok; ++nc)
+                for (int ka = 0; ka < KA && ok; ka += AT) {
+                    const CUtensorMap* m0 = ka == 0 ? &tm_wq : &tm_wo;
+                    const int x0 = ka == 0 ? 0 : (ka - 1) * 64;
+                    ok = push_tma2(m0, x0, nc * 128 + rb, &tm_wo, ka * 64, nc * 128 + rb, BR * 128,
+                                   ka + AT <= KA ? AT : KA - ka);
+                }
+            // MLP items in MMA consumption order
             for (int hf = 0; hf < n_half && ok; ++hf) {
                 auto w1 = [&](int c) {
-                    for (int s = 0; s < w1_gran && ok; ++s) ok = push_tma(&tm_w1, s * 64, c * HN, HN * 128);
+                    for (int s = 0; s < w1_gran && ok; s += AT)
+                        ok = push_tma2(&tm_w1, s * 64, c * HN + rb, &tm_w1, (s + 1) * 64, c * HN + rb, BR * 128, AT);
                 };
                 auto w2 = [&](int c) {
-                    for (int q = 0; q < w2_gran && ok; ++q) {
+                    for (int q = 0; q < w2_gran && ok; q += AT) {
                         const int nc = q / (HN / 64), kh = q % (HN / 64);
-                        ok = push_tma(&tm_w2, c * HN + kh * 64, hf * 256 + nc * 128, SLOT);
+                        ok = push_tma2(&tm_w2, c * HN + kh * 64, hf * 256 + nc * 128 + rb, &tm_w2,
+                                       c * HN + (kh + 1) * 64, hf * 256 + nc * 128 + rb, BR * 128, AT);
                     }
                 };
                 w1(0);
@@ -388,16 +518,44 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
         }
         drain();
         // every load issued has landed before the CTA may exit (they always
-        // complete; consumed or not, the last use of each slot is awaited)
+        // complete; consumed or not, the last use of each slot is awaited;
+        // in the even CTA of a pair that includes the odd CTA's forwarded half)
         if (lane == 0) {
-            const uint32_t first = ring_head > (uint32_t)NS ? ring_head - NS : 0;
-            for (uint32_t i = first; i < ring_head; ++i) drain_wait(smem_u32(&sh.full[i % NS]), (i / NS) & 1, ta.timeout);
+            const uint32_t first = ring_head > (uint32_t)NR ? ring_head - NR : 0;
+            for (uint32_t i = first; i < ring_head; ++i) drain_wait(smem_u32(&sh.full[i % NR]), (i / NR) & 1, ta.timeout);
         }
         __syncwarp();
     }
     // ==================================================================== MMA issue
+    else if (warp == WARP_MMA && PAIR && !leader) {
+        // odd CTA of a pair: forward the completion of each of its ring loads to the
+        // even CTA's ring barrier, item by item in ring order
+        {
+            int f_slot = 0;
+            uint32_t f_ph = 0;
+            bool ok = true;
+            for (int64_t it = it0; it < n_iter && ok; it += it_step) {
+                if (!active(it)) continue;
+                const Unit u = unit_at(it, crank);
+                const int nb = ((u.sel ? a.ksel : N) + 127) / 128;
+                const int items = n_items(nb);
+                for (int i = 0; i < items && ok; ++i) {
+                    uint32_t ph = f_ph;
+                    if (!(ok = W.wait(&sh.full[f_slot], ph, 49))) break;
+                    // the phase has completed (the half tile is in place), so the arrival itself orders nothing
+                    mbar_arrive_cluster_relaxed_w(mapa(smem_u32(&sh.full[f_slot]), 0u));
+                    if (++f_slot == NR) {
+                        f_slot = 0;
+                        f_ph ^= 1;
+                    }
+                }
+            }
+        }
+    }
     else if (warp == WARP_MMA) {
-        if (lane == 0) {
+        {   // the whole warp runs the issue loop; one elected lane issues each instruction
+            // the MMA issuer of a pair waits on barriers that the other CTA arrives at
+            W.cluster_acq = PAIR;
             uint32_t ring_tail = 0;
             uint32_t ph_pe = 0, ph_qc = 0, ph_p[2] = {0, 0}, ph_a = 0, ph_hin = 0, ph_r = 0, ph_g[2] = {0, 0};
             uint32_t ph_hd = 0, ph_w2 = 0;
@@ -410,16 +568,27 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 if (!W.wait(&sh.full[slot], ph, 50)) return false;
                 tc_fence_after();
                 ++ring_tail;
-                if (++c_slot == NS) {
+                if (++c_slot == NR) {
                     c_slot = 0;
                     c_ph ^= 1;
                 }
                 return true;
             };
-            auto release = [&](int slot) { mma_commit(smem_u32(&sh.empty[slot])); };
-            for (int64_t unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
-                const Unit u = unit_of(a, unit);
-                if (u.nq <= 0) continue;
+            auto release = [&](int slot) { commit_both(&sh.empty[slot]); };
+            constexpr int MR = 128 * CG;   // MMA rows
+            auto mma_s = [&](uint32_t d, uint64_t da, uint64_t db, uint32_t id, uint32_t acc) {
+                if (PAIR) mma_ss_pair_w(d, da, db, id, acc);
+                else mma_ss_w(d, da, db, id, acc);
+            };
+            auto mma_t = [&](uint32_t d, uint32_t ta_, uint64_t db, uint32_t id, uint32_t acc) {
+                if (PAIR) mma_ts_pair_w(d, ta_, db, id, acc);
+                else mma_ts_w(d, ta_, db, id, acc);
+            };
+            int64_t n_done = 0;
+            for (int64_t it = it0; it < n_iter && ok; it += it_step) {
+                if (!active(it)) continue;
+                const Unit u = unit_at(it, crank);
+                const bool first_unit = n_done++ == 0;
                 const int nk = u.sel ? a.ksel : N;
                 const int nb = (nk + 127) / 128;
                 if (!(ok = W.wait(&sh.bar_pe, ph_pe, 51))) break;
@@ -429,25 +598,25 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     // Q_h = PE Wq_h^T (M=128, N=64, K=64)
                     if (!(ok = consume(slot))) break;
                     {
-                        const uint64_t da = desc_sw128(s_pe), db = desc_sw128(s_ring + slot * SLOT);
+                        const uint64_t da = desc_sw128(s_pe), db = desc_sw128(s_ring + slot * RS);
                         #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_ss(tmem + T_Q, da + 2 * kk, db + 2 * kk, idesc_bf16(128, 64, false), kk > 0);
+                            mma_s(tmem + T_Q, da + 2 * kk, db + 2 * kk, idesc_bf16(MR, 64, false), kk > 0);
                         release(slot);
-                        if (!(ta.inject && h == 0 && unit == blockIdx.x)) mma_commit(smem_u32(&sh.bar_q));
+                        if (!(ta.inject && h == 0 && first_unit)) commit_both(&sh.bar_q);
                     }
                     if (!(ok = W.wait(&sh.bar_qc, ph_qc, 52))) break;
                     tc_fence_after();
                     auto issue_s = [&](int j) -> bool {
                         int sl;
                         if (!consume(sl)) return false;
-                        const uint64_t db = desc_sw128(s_ring + sl * SLOT);
+                        const uint64_t db = desc_sw128(s_ring + sl * RS);
                         const uint32_t sd = tmem + ((j & 1) ? T_S1 : T_S0);
                         #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_ts(sd, tmem + T_Q + split_col(kk, 64), db + 2 * kk, idesc_bf16(128, 128, false), kk > 0);
+                            mma_t(sd, tmem + T_Q + split_col(kk, 64), db + 2 * kk, idesc_bf16(MR, 128, false), kk > 0);
                         release(sl);
-                        mma_commit(smem_u32(&sh.bar_s[j & 1]));
+                        commit_both(&sh.bar_s[j & 1]);
                         return true;
                     };
                     ok = issue_s(0) && (nb < 2 || issue_s(1));
@@ -456,17 +625,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         tc_fence_after();
                         if (!(ok = consume(slot))) break;
                         const uint32_t pa = tmem + ((j & 1) ? T_P1 : T_P0);
-                        const uint64_t dv = desc_sw128(s_ring + slot * SLOT);
+                        // V is N-major: 16 tokens per k-step = 16 rows of 128 B (64 B per CTA of a pair)
+                        const uint64_t dv = PAIR ? desc_sw64(s_ring + slot * RS) : desc_sw128(s_ring + slot * RS);
+                        constexpr int vstep = PAIR ? 64 : 128;
                         #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            mma_ts(tmem + T_O, pa + 8 * kk, dv + 128 * kk, idesc_bf16(128, 64, true), (j > 0 || kk > 0));
+                            mma_t(tmem + T_O, pa + 8 * kk, dv + vstep * kk, idesc_bf16(MR, 64, true), (j > 0 || kk > 0));
                         release(slot);
-                        mma_commit(smem_u32(&sh.bar_pv));
+                        commit_both(&sh.bar_pv);
                         if (j + 2 < nb) ok = issue_s(j + 2);
                     }
                     if (!ok) break;
                     // the next head's Q projection rewrites T_Q, which this head's S MMAs read
-                    mma_commit(smem_u32(&sh.bar_hd));
+                    commit_own(&sh.bar_hd);
                     if (!(ok = W.wait(&sh.bar_hd, ph_hd, 54))) break;
                     tc_fence_after();
                 }
@@ -474,51 +645,61 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 // ---- X = PE Wq^T + a Wo^T
                 if (!(ok = W.wait(&sh.bar_a, ph_a, 55))) break;
                 tc_fence_after();
-                const int KA = NA + 1;
-                for (int g = 0; g < (C / 128) * KA && ok; ++g) {
-                    int slot;
-                    if (!(ok = consume(slot))) break;
-                    const int nc = g / KA, ka = g % KA;
-                    const uint64_t da = desc_sw128(ka == 0 ? s_pe : s_abuf + (ka - 1) * 16384);
-                    const uint64_t db = desc_sw128(s_ring + slot * SLOT);
-                    #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ss(tmem + nc * 128, da + 2 * kk, db + 2 * kk, idesc_bf16(128, 128, false),
-                               (ka > 0 || kk > 0));
-                    release(slot);
-                }
+                for (int nc = 0; nc < C / 128 && ok; ++nc)
+                    for (int ka0 = 0; ka0 < KA && ok; ka0 += AT) {
+                        int slot;
+                        if (!(ok = consume(slot))) break;
+                        for (int at = 0; at < AT && ka0 + at < KA; ++at) {
+                            const int ka = ka0 + at;
+                            const uint64_t da = desc_sw128(ka == 0 ? s_pe : s_abuf + (ka - 1) * 16384);
+                            const uint64_t db = desc_sw128(s_ring + slot * RS + at * BR * 128);
+                            #pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_s(tmem + nc * 128, da + 2 * kk, db + 2 * kk, idesc_bf16(MR, 128, false),
+                                      (ka > 0 || kk > 0));
+                        }
+                        release(slot);
+                    }
                 if (!ok) break;
-                mma_commit(smem_u32(&sh.bar_x));
+                commit_both(&sh.bar_x);
                 // ---- MLP
                 if (!(ok = W.wait(&sh.bar_hin, ph_hin, 56))) break;
                 tc_fence_after();
                 for (int hf = 0; hf < n_half && ok; ++hf) {
                     auto issue_w1 = [&](int c) -> bool {
                         const uint32_t hd = tmem + ((c & 1) ? T_H1 : T_H0);
-                        for (int ka = 0; ka < NA; ++ka) {
+                        for (int ka0 = 0; ka0 < NA; ka0 += AT) {
                             int sl;
                             if (!consume(sl)) return false;
-                            const uint64_t da = desc_sw128(s_abuf + ka * 16384);
-                            const uint64_t db = desc_sw128(s_ring + sl * SLOT);
                             #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma_ss(hd, da + 2 * kk, db + 2 * kk, idesc_bf16(128, HN, false), (ka > 0 || kk > 0));
+                            for (int at = 0; at < AT; ++at) {
+                                const int ka = ka0 + at;
+                                const uint64_t da = desc_sw128(s_abuf + ka * 16384);
+                                const uint64_t db = desc_sw128(s_ring + sl * RS + at * BR * 128);
+                                #pragma unroll
+                                for (int kk = 0; kk < 4; ++kk)
+                                    mma_s(hd, da + 2 * kk, db + 2 * kk, idesc_bf16(MR, HN, false), (ka > 0 || kk > 0));
+                            }
                             release(sl);
                         }
-                        mma_commit(smem_u32(&sh.bar_h[c & 1]));
+                        commit_both(&sh.bar_h[c & 1]);
                         return true;
                     };
                     auto issue_w2 = [&](int c) -> bool {
                         const uint32_t ha = tmem + ((c & 1) ? T_H1 : T_H0);
-                        for (int q = 0; q < w2_gran; ++q) {
+                        for (int q0 = 0; q0 < w2_gran; q0 += AT) {
                             int sl;
                             if (!consume(sl)) return false;
-                            const int nc = q / (HN / 64), kh = q % (HN / 64);
-                            const uint64_t db = desc_sw128(s_ring + sl * SLOT);
                             #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma_ts(tmem + nc * 128, ha + split_col(4 * kh + kk, HN), db + 2 * kk,
-                                       idesc_bf16(128, 128, false), 1u);
+                            for (int at = 0; at < AT; ++at) {
+                                const int q = q0 + at;
+                                const int nc = q / (HN / 64), kh = q % (HN / 64);
+                                const uint64_t db = desc_sw128(s_ring + sl * RS + at * BR * 128);
+                                #pragma unroll
+                                for (int kk = 0; kk < 4; ++kk)
+                                    mma_t(tmem + nc * 128, ha + split_col(4 * kh + kk, HN), db + 2 * kk,
+                                          idesc_bf16(MR, 128, false), 1u);
+                            }
                             release(sl);
                         }
                         return true;
@@ -535,18 +716,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         if (!(ok = issue_w2(c))) break;
                         if (c + 2 < n_chunks) {
                             // H[c%2] is re-written by W1(c+2): W2(c) must have read it first
-                            mma_commit(smem_u32(&sh.bar_w2));
+                            commit_own(&sh.bar_w2);
                             if (!(ok = W.wait(&sh.bar_w2, ph_w2, 59))) break;
                             tc_fence_after();
                             ok = issue_w1(c + 2);
                         }
                     }
                     if (!ok) break;
-                    mma_commit(smem_u32(&sh.bar_acc));   // the half's accumulator is complete
+                    commit_both(&sh.bar_acc);   // the half's accumulator is complete
                 }
             }
             // nothing of ours may run on the tensor cores once TMEM is released
-            mma_commit(smem_u32(&sh.bar_fin));
+            commit_own(&sh.bar_fin);
             drain_wait(smem_u32(&sh.bar_fin), 0, ta.timeout);
         }
     }
@@ -562,15 +743,25 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
         float* xs = reinterpret_cast<float*>(dyn_raw + (s_pe - smem_u32(dyn_raw)));
         bool ok = true;
         auto arrive = [&](uint64_t* b) { mbar_arrive(smem_u32(b)); };
+        // compute -> MMA signal: per thread, or (CTA pairs) per warp to the even CTA's barrier;
+        // every thread has fenced its own stores before it
+        auto arrive_mma = [&](uint64_t* b) {
+            if (PAIR) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(lead_bar(b));
+            } else {
+                mbar_arrive(smem_u32(b));
+            }
+        };
         auto wg_sync = [&](int site) -> bool {
             arrive(&sh.bar_wg);
             return W.wait(&sh.bar_wg, ph_wg, site);
         };
         const int HALF = HN / 2;             // hidden units per warpgroup
         float4* park = halves ? reinterpret_cast<float4*>(ta.park) + (size_t)blockIdx.x * (256 / 4) * BM : nullptr;
-        for (int64_t unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
-            const Unit u = unit_of(a, unit);
-            if (u.nq <= 0) continue;
+        for (int64_t it = it0; it < n_iter && ok; it += it_step) {
+            if (!active(it)) continue;
+            const Unit u = unit_at(it, crank);
             const int nk = u.sel ? a.ksel : N;
             const int nb = (nk + 127) / 128;
             // ---- this row's query
@@ -601,7 +792,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 st_shared_v4(swz(s_pe, row, c), w);
             }
             fence_proxy_async();
-            arrive(&sh.bar_pe);
+            arrive_mma(&sh.bar_pe);
             float* ml_out = nullptr;
             if (a.probe_ml && row < u.nq && wg == 0) {
                 if (a.work == kWorkTileDense) ml_out = a.probe_ml + ((size_t)u.t * a.n_probe + u.first + row) * H * 2;
@@ -626,7 +817,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     tmem_wait_st();
                 }
                 tc_fence_before();
-                arrive(&sh.bar_qc);
+                arrive_mma(&sh.bar_qc);
                 float m_ref = -INFINITY, l_part = 0.f;
                 for (int j = 0; j < nb; ++j) {
                     if (!(ok = W.wait(&sh.bar_s[j & 1], ph_s[j & 1], 61))) break;
@@ -695,7 +886,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     tmem_st32(trow + ((j & 1) ? T_P1 : T_P0) + 32 * wg, pk);
                     tmem_wait_st();
                     tc_fence_before();
-                    arrive(&sh.bar_p[j & 1]);
+                    arrive_mma(&sh.bar_p[j & 1]);
                 }
                 if (!ok) break;
                 if (!(ok = W.wait(&sh.bar_pv, ph_pv, 63))) break;   // PV_{nb-1}
@@ -734,7 +925,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             if (!ok) break;
             fence_proxy_async();
             tc_fence_before();
-            arrive(&sh.bar_a);
+            arrive_mma(&sh.bar_a);
             // ================================================= LN1 (each half: C/2 columns)
             if (!(ok = W.wait(&sh.bar_x, ph_x, 64))) break;
             tc_fence_after();
@@ -813,7 +1004,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             }
             fence_proxy_async();
             tc_fence_before();
-            arrive(&sh.bar_hin);
+            arrive_mma(&sh.bar_hin);
             // ================================================= MLP
             float hs_mean0 = 0.f, hs_m20 = 0.f, hs_dot0 = 0.f, hs_mean1 = 0.f, hs_m21 = 0.f, hs_dot1 = 0.f;
             for (int hf = 0; hf < n_half && ok; ++hf) {
@@ -834,7 +1025,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     }
                     tmem_wait_st();
                     tc_fence_before();
-                    arrive(&sh.bar_r);
+                    arrive_mma(&sh.bar_r);
                 }
                 for (int c = 0; c < n_chunks; ++c) {
                     if (!(ok = W.wait(&sh.bar_h[c & 1], ph_h[c & 1], 65))) break;
@@ -855,7 +1046,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     }
                     tmem_wait_st();
                     tc_fence_before();
-                    arrive(&sh.bar_g[c & 1]);
+                    arrive_mma(&sh.bar_g[c & 1]);
                 }
                 if (!ok) break;
                 if (!(ok = W.wait(&sh.bar_acc, ph_acc, 67))) break;
@@ -955,8 +1146,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
     cp_async_wait<0>();
     tc_fence_before();
     __syncthreads();
+    // CTA pairs: neither CTA leaves while the other may still reach its shared memory or TMEM
+    if (PAIR) cluster_sync();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (warp == 0) {
+        if (PAIR) tmem_dealloc_pair(tmem, 512);
+        else tmem_dealloc(tmem, 512);
+    }
 }
 
 // ---------------------------------------------------------------- host side
@@ -985,15 +1181,17 @@ __device__ float4 g_x1_park[(size_t)kParkCtas * 256 / 4 * BM];
 }  // namespace
 
 // 2D bf16 matrix [rows][cols] row-major, box {64 cols, box_rows rows}, 128 B swizzle
-vdm_status make_bf16_map(CUtensorMap* m, const void* base, int64_t rows, int cols, int box_rows) {
+vdm_status make_bf16_map(CUtensorMap* m, const void* base, int64_t rows, int cols, int box_rows, int box_cols) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(VDM_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
+    // 64-column boxes use 128-byte rows (128 B swizzle), 32-column boxes 64-byte rows (64 B swizzle)
+    const CUtensorMapSwizzle sw = box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(VDM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return VDM_OK;
@@ -1025,18 +1223,23 @@ vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
     int ns = 0;
     const size_t smem = tc_smem_bytes(d.C, &ns);
     if (ns < GATHER_LAG + 2) return fail(VDM_ERR_INTERNAL, "not enough shared memory for the ring (%d slots)", ns);
-    CUtensorMap m_wq, m_wq64, m_wo, m_w1, m_w2, m_k, m_v;
-    const int HN = 128;
-    VDM_TRY(make_bf16_map(&m_wq, d.Wq, d.C, 64, 128));
-    VDM_TRY(make_bf16_map(&m_wq64, d.Wq, d.C, 64, 64));
-    VDM_TRY(make_bf16_map(&m_wo, d.Wo, d.C, d.C, 128));
-    VDM_TRY(make_bf16_map(&m_w1, d.W1, d.F, d.C, HN));
-    VDM_TRY(make_bf16_map(&m_w2, d.W2, d.C, d.F, 128));
-    VDM_TRY(make_bf16_map(&m_k, d.K, (int64_t)d.H * d.N, 64, 128));
-    VDM_TRY(make_bf16_map(&m_v, d.V, (int64_t)d.H * d.N, 64, 128));
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms > kParkCtas) sms = kParkCtas;   // one parking block per CTA
+    // CTA pairs (256-row MMAs, each CTA loading half of every weight and key tile) when
+    // switched on and at least two SMs
+    const bool pair = g_debug.single_cta == 0 && sms >= 2;
+    const int br = pair ? 64 : 128;   // rows of a 128-row B tile loaded per CTA
+    CUtensorMap m_wq, m_wq64, m_wo, m_w1, m_w2, m_k, m_v;
+    VDM_TRY(make_bf16_map(&m_wq, d.Wq, d.C, 64, br, 64));
+    VDM_TRY(make_bf16_map(&m_wq64, d.Wq, d.C, 64, br / 2, 64));
+    VDM_TRY(make_bf16_map(&m_wo, d.Wo, d.C, d.C, br, 64));
+    VDM_TRY(make_bf16_map(&m_w1, d.W1, d.F, d.C, br, 64));
+    VDM_TRY(make_bf16_map(&m_w2, d.W2, d.C, d.F, br, 64));
+    VDM_TRY(make_bf16_map(&m_k, d.K, (int64_t)d.H * d.N, 64, br, 64));
+    // values are read N-major: a pair splits the 64 head dimensions, 32 per CTA
+    VDM_TRY(make_bf16_map(&m_v, d.V, (int64_t)d.H * d.N, 64, 128, pair ? 32 : 64));
     TcArgs ta;
     ta.d = d;
     ta.ns = ns;
@@ -1048,14 +1251,35 @@ vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
     ta.timeout = g_debug.timeout > 0 ? g_debug.timeout : 4000000000ll;
     ta.inject = g_debug.inject;
     g_debug.inject = 0;   // one launch only
-    auto kern = d.C == 128 ? decode_tc_kernel<128> : d.C == 256 ? decode_tc_kernel<256> : decode_tc_kernel<512>;
+    typedef void (*Kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+                         CUtensorMap, TcArgs);
+    Kern kern;
+    if (pair) kern = d.C == 128 ? decode_tc_kernel<128, 2> : d.C == 256 ? decode_tc_kernel<256, 2> : decode_tc_kernel<512, 2>;
+    else kern = d.C == 128 ? decode_tc_kernel<128, 1> : d.C == 256 ? decode_tc_kernel<256, 1> : decode_tc_kernel<512, 1>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "decode_tc smem attribute: %s", cudaGetErrorString(e));
-    if (sms > kParkCtas) sms = kParkCtas;   // one parking block per CTA
-    const unsigned grid = (unsigned)(n_units < sms ? n_units : sms);
+    // work items: units of 128 queries, or pairs of them
+    const int slots_pairs = pair ? (d.slots + 1) / 2 : d.slots;
+    const int64_t n_iter = !pair ? n_units : d.work == kWorkFlat ? (n_units + 1) / 2 : (int64_t)d.T * slots_pairs;
+    const int per = pair ? 2 : 1;
+    const int64_t groups = sms / per;
+    const unsigned grid = (unsigned)(per * (n_iter < groups ? n_iter : groups));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = per;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     prof_begin(kProfDecode, st);
-    kern<<<grid, NT, smem, st>>>(m_wq, m_wq64, m_wo, m_w1, m_w2, m_k, m_v, ta);
+    e = cudaLaunchKernelEx(&cfg, kern, m_wq, m_wq64, m_wo, m_w1, m_w2, m_k, m_v, ta);
     prof_end(kProfDecode, st);
+    if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "decode_tc_kernel launch: %s", cudaGetErrorString(e));
     return check_launch("decode_tc_kernel");
 }
 

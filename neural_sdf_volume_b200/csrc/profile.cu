@@ -45,7 +45,7 @@ void prof_end(int cls, cudaStream_t s) {
     cudaEventRecord(g_recs.back().b, s);
 }
 
-DebugHooks g_debug = {0, 0};
+DebugHooks g_debug = {0, 0, 1};   // CTA pairs off by default
 
 }  // namespace vdm
 
@@ -57,6 +57,12 @@ vdm_status vdm_debug_inject(int32_t mode, int64_t timeout_cycles) {
     if (mode != 0 && mode != 1) return fail(VDM_ERR_INVALID_ARG, "unknown inject mode %d", mode);
     g_debug.inject = mode;
     g_debug.timeout = timeout_cycles > 0 ? timeout_cycles : 0;
+    return VDM_OK;
+}
+
+vdm_status vdm_set_cta_pairs(int32_t enable) {
+    if (enable != 0 && enable != 1) return fail(VDM_ERR_INVALID_ARG, "enable must be 0 or 1, got %d", enable);
+    g_debug.single_cta = enable ? 0 : 1;
     return VDM_OK;
 }
 

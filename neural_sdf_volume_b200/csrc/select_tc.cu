@@ -25,7 +25,7 @@
 
 namespace vdm {
 
-vdm_status make_bf16_map(CUtensorMap* m, const void* base, int64_t rows, int cols, int box_rows);
+vdm_status make_bf16_map(CUtensorMap* m, const void* base, int64_t rows, int cols, int box_rows, int box_cols);
 int* tc_error_word();
 
 namespace {
@@ -493,8 +493,8 @@ vdm_status launch_select_tc(const SelectTcLaunch& L, cudaStream_t st) {
     if (!a.err) return fail(VDM_ERR_CUDA, "error word lookup failed");
     a.timeout = 4000000000ll;
     CUtensorMap m_wq64, m_k;
-    VDM_TRY(make_bf16_map(&m_wq64, L.Wq, L.C, 64, 64));
-    VDM_TRY(make_bf16_map(&m_k, L.K, (int64_t)L.H * L.N, 64, 128));
+    VDM_TRY(make_bf16_map(&m_wq64, L.Wq, L.C, 64, 64, 64));
+    VDM_TRY(make_bf16_map(&m_k, L.K, (int64_t)L.H * L.N, 64, 128, 64));
     const size_t smem = select_tc_smem(L.n_probe, L.N);
     if (smem > 227 * 1024) return fail(VDM_ERR_UNSUPPORTED, "selection needs %zu bytes of shared memory", smem);
     cudaError_t e = cudaFuncSetAttribute(select_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

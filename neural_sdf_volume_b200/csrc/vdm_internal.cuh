@@ -119,6 +119,7 @@ struct SelectArgs {
 struct DebugHooks {
     int inject;              // 1: withhold one MMA completion signal in the next decode launch
     long long timeout;       // bounded-wait limit in cycles (0: default)
+    int single_cta;          // 1: tensor-core decoding with one CTA per MMA (no CTA pairs)
 };
 extern DebugHooks g_debug;
 
