@@ -275,41 +275,53 @@ def run_vdm(args, world, rank, local):
 
 
 def run_dense(args, world, rank, local):
-    """Dense decoding of ``--dense-queries`` random points with the full-width
-    decoder (N=3072, C=512, 8 heads, F=2048): the fused kernel alone, for
-    profiling and for the dense points/s figure."""
+    """Dense decoding on one GPU: the full grid of a dense workload (``--config 1``:
+    32^3 fp32, ``--config 2``: 128^3 bf16), or ``--dense-queries M`` uniform random
+    points with the workload-2 decoder (N=3072, C=512, 8 heads, F=2048)."""
     import torch
 
     import neural_sdf_volume_b200 as vdm
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    cfg = W.CONFIGS[2]
+    cfg = W.CONFIGS[args.config if args.config in (1, 2) else 2]
     inp = W.make_decoder(cfg.dec, seed=0, key=cfg.seed_key, B=1)
     dec = vdm.Decoder.from_numpy(inp["weights"], cfg.dec.C, cfg.dec.H, cfg.dec.F, cfg.dec.query_ln,
                                  cfg.dec.dtype, device=dev)
     K, V = vdm.vdm_precompute_kv(dec, torch.from_numpy(inp["z"]).to(dev))
-    M = args.dense_queries
-    pts = torch.from_numpy(W.make_points(M, seed=1, key=2)).to(dev)
+    if args.dense_queries > 0:
+        M = args.dense_queries
+        pts = torch.from_numpy(W.make_points(M, seed=1, key=2)).to(dev)
+        call = lambda out: vdm.vdm_decode_dense(dec, K, V, xyz=pts, out=out)
+        workload = f"dense decode of {M} uniform points, config 2 decoder"
+    else:
+        M = cfg.grid_R ** 3
+        pts = None
+        call = lambda out: vdm.vdm_decode_dense(dec, K, V, grid_R=cfg.grid_R, out=out)
+        workload = f"config {cfg.cid}: {cfg.name}"
     out = torch.empty((1, M), device=dev)
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), device=dev, dtype=torch.float32)
     for _ in range(args.warmup):
-        vdm.vdm_decode_dense(dec, K, V, xyz=pts, out=out)
+        call(out)
     torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
+    evs = []
     for _ in range(args.steps):
-        vdm.vdm_decode_dense(dec, K, V, xyz=pts, out=out)
-    e1.record()
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call(out)
+        e1.record()
+        evs.append((e0, e1))
     torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
     flops = M * decode_flops_per_query(cfg.dec, cfg.dec.N)
     peaks = _peaks()
-    return {"metric": "dense decode points/sec (N=3072, C=512)", "value": M / (ms / 1e3), "unit": UNIT,
-            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"dense decode of {M} uniform points, config 2 decoder"},
-            "tflops": flops / (ms / 1e3) / 1e12,
-            "frac_of_bf16_burst": flops / (ms / 1e3) / 1e12 / peaks["bf16"]}
+    tf = flops / (ms / 1e3) / 1e12
+    return {"metric": f"dense decode points/sec ({cfg.dec.dtype}, N={cfg.dec.N}, C={cfg.dec.C})",
+            "value": M / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "dtype": cfg.dec.dtype, "data": "synthetic",
+            "config": {"workload": workload, "queries": M, "l2": "flushed between timed steps"},
+            "tflops": tf, "frac_of_bf16_burst": tf / peaks["bf16"] if cfg.dec.dtype == "bf16" else None}
 
 
 def _oracle_sample_points(cfg, n: int, seed: int = 0) -> np.ndarray:
@@ -317,6 +329,8 @@ def _oracle_sample_points(cfg, n: int, seed: int = 0) -> np.ndarray:
     fine voxels near the spheres' surfaces (where the fine levels decode)."""
     from oracle import decoder as OD
     rng = np.random.default_rng(seed)
+    if cfg.mode != "hier":   # dense workloads: voxels of the grid
+        return OD.grid_points(cfg.grid_R, rng.integers(0, cfg.grid_R ** 3, n))
     half = n // 2
     coarse = OD.grid_points(cfg.r0, rng.integers(0, cfg.r0 ** 3, half))
     sp = W.make_spheres(cfg.n_spheres, 0, cfg.sphere_key, 1)[0]
@@ -381,7 +395,8 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="vdm", choices=["vdm", "reference"])
-    ap.add_argument("--config", type=int, default=4, choices=[3, 4, 5])
+    ap.add_argument("--config", type=int, default=4, choices=[1, 2, 3, 4, 5],
+                    help="3-5: hierarchical workloads (the step of the headline metric); 1-2: dense grids")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dense-queries", type=int, default=0,
@@ -392,7 +407,7 @@ def main():
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         res = run_reference(args, world, rank)
-    elif args.dense_queries > 0:
+    elif args.dense_queries > 0 or args.config in (1, 2):
         res = run_dense(args, world, rank, local)
     else:
         res = run_vdm(args, world, rank, local)

@@ -70,7 +70,7 @@ constexpr int NT = 320;        // + MMA warp + producer warp
 constexpr int WARP_MMA = 8, WARP_PROD = 9;
 constexpr int SLOT = 16384;    // ring slot bytes
 constexpr int MAX_NS = 16;   // ring slots (CTA pairs use twice as many, half as large)
-constexpr int GATHER_LAG = 3;  // gathered items in flight before their barrier is signalled
+constexpr int RING_ARRIVALS = 32;   // arrivals completing a ring slot: one per producer lane
 constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr uint32_t T_S0 = 0, T_S1 = 128, T_P0 = 256, T_P1 = 320, T_O = 384, T_Q = 448;
@@ -253,8 +253,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
 
     if (tid == 0) {
         for (int i = 0; i < NR; ++i) {
-            // the even CTA's ring slot is complete when its own load and the odd CTA's forward arrived
-            mbar_init(smem_u32(&sh.full[i]), PAIR && leader ? 2 : 1);
+            // a slot is complete when the producer warp's 32 lanes arrived (a TMA item: one counted
+            // arrival plus its bytes; a gathered item: each lane once its copies landed) and, in the
+            // even CTA of a pair, the odd CTA's forward
+            mbar_init(smem_u32(&sh.full[i]), RING_ARRIVALS + (PAIR && leader ? 1 : 0));
             mbar_init(smem_u32(&sh.empty[i]), 1);
         }
         uint64_t* one[] = {&sh.bar_q, &sh.bar_s[0], &sh.bar_s[1], &sh.bar_pv, &sh.bar_x,
@@ -347,23 +349,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
     // ==================================================================== producer
     if (warp == WARP_PROD) {
         uint32_t ring_head = 0;
-        int pend[GATHER_LAG + 1];
-        int n_pend = 0;
         const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.K);
         const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.V);
         bool ok = true;
-        auto signal_oldest = [&]() {
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sh.full[pend[0]]));
-            for (int i = 1; i < n_pend; ++i) pend[i - 1] = pend[i];
-            --n_pend;
-        };
-        auto drain = [&]() {
-            if (n_pend == 0) return;
-            cp_async_wait<0>();
-            while (n_pend > 0) signal_oldest();
-        };
         int p_slot = 0;
         uint32_t p_ph = 1;   // parity of the empty-phase a reused slot waits for (first pass: none)
         auto take_slot = [&](int& slot) -> bool {
@@ -380,13 +368,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             return true;
         };
         auto push_tma = [&](const CUtensorMap* m, int x, int y, uint32_t bytes) -> bool {
-            drain();
             int slot;
             if (!take_slot(slot)) return false;
             if (lane == 0) {
                 const uint32_t fb = smem_u32(&sh.full[slot]);
-                mbar_expect_tx(fb, bytes);
+                mbar_expect_tx_only(fb, bytes);
                 tma_load_2d(s_ring + slot * RS, m, x, y, fb);
+                mbar_arrive_n(fb, RING_ARRIVALS);
             }
             __syncwarp();
             return true;
@@ -394,14 +382,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
         // two boxes of `bytes` each in one slot (the second at offset `bytes`); nbox = 1 or 2
         auto push_tma2 = [&](const CUtensorMap* m0, int x0, int y0, const CUtensorMap* m1, int x1, int y1,
                              uint32_t bytes, int nbox) -> bool {
-            drain();
             int slot;
             if (!take_slot(slot)) return false;
             if (lane == 0) {
                 const uint32_t fb = smem_u32(&sh.full[slot]);
-                mbar_expect_tx(fb, bytes * nbox);
+                mbar_expect_tx_only(fb, bytes * nbox);
                 tma_load_2d(s_ring + slot * RS, m0, x0, y0, fb);
                 if (nbox > 1) tma_load_2d(s_ring + slot * RS + bytes, m1, x1, y1, fb);
+                mbar_arrive_n(fb, RING_ARRIVALS);
             }
             __syncwarp();
             return true;
@@ -459,12 +447,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                                src + ((size_t)h * N + (okr ? rows[i] : 0)) * 64 + 32 * crank + c * 8, okr);
                 }
             }
-            cp_async_commit();
-            pend[n_pend++] = slot;
-            if (n_pend > GATHER_LAG) {
-                cp_async_wait<GATHER_LAG>();
-                signal_oldest();
-            }
+            // each lane arrives once its own copies landed: the warp never waits for them
+            cp_async_mbar_arrive_noinc(smem_u32(&sh.full[slot]));
             return true;
         };
         const int rb = (int)crank * BR;   // this CTA's row offset inside a 128-row B tile
@@ -516,7 +500,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 }
             }
         }
-        drain();
         // every load issued has landed before the CTA may exit (they always
         // complete; consumed or not, the last use of each slot is awaited;
         // in the even CTA of a pair that includes the odd CTA's forwarded half)
@@ -542,6 +525,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 for (int i = 0; i < items && ok; ++i) {
                     uint32_t ph = f_ph;
                     if (!(ok = W.wait(&sh.full[f_slot], ph, 49))) break;
+                    fence_proxy_async();   // gathered rows (cp.async) become visible to the async proxy
                     // the phase has completed (the half tile is in place), so the arrival itself orders nothing
                     mbar_arrive_cluster_relaxed_w(mapa(smem_u32(&sh.full[f_slot]), 0u));
                     if (++f_slot == NR) {
@@ -610,6 +594,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     auto issue_s = [&](int j) -> bool {
                         int sl;
                         if (!consume(sl)) return false;
+                        // gathered rows were written by cp.async (generic proxy): order them before the MMA's reads
+                        if (u.sel) fence_proxy_async();
                         const uint64_t db = desc_sw128(s_ring + sl * RS);
                         const uint32_t sd = tmem + ((j & 1) ? T_S1 : T_S0);
                         #pragma unroll
@@ -624,6 +610,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         if (!(ok = W.wait(&sh.bar_p[j & 1], ph_p[j & 1], 53))) break;
                         tc_fence_after();
                         if (!(ok = consume(slot))) break;
+                        if (u.sel) fence_proxy_async();
                         const uint32_t pa = tmem + ((j & 1) ? T_P1 : T_P0);
                         // V is N-major: 16 tokens per k-step = 16 rows of 128 B (64 B per CTA of a pair)
                         const uint64_t dv = PAIR ? desc_sw64(s_ring + slot * RS) : desc_sw128(s_ring + slot * RS);
@@ -1143,6 +1130,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
     }
 
     // ---------------------------------------------------------------- wind down
+    cp_async_commit();   // copies issued without a group, then wait for all of them
     cp_async_wait<0>();
     tc_fence_before();
     __syncthreads();
@@ -1222,7 +1210,7 @@ vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
     if (n_units <= 0) return VDM_OK;
     int ns = 0;
     const size_t smem = tc_smem_bytes(d.C, &ns);
-    if (ns < GATHER_LAG + 2) return fail(VDM_ERR_INTERNAL, "not enough shared memory for the ring (%d slots)", ns);
+    if (ns < 2) return fail(VDM_ERR_INTERNAL, "not enough shared memory for the ring (%d slots)", ns);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
