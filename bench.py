@@ -49,6 +49,12 @@ def _peaks():
                 "src": "fallback"}
 
 
+# dram__bytes_read.sum + dram__bytes_write.sum per decode launch, mean over the five
+# launches of one config-4 shape, captured with ncu on the bench's own launches
+# (profiles/launches_config4_hierarchical_384.md); re-capture when the kernel changes.
+DECODE_DRAM_BYTES_PER_LAUNCH = {4: 39.66e6}
+
+
 def decode_flops_per_query(spec: W.DecoderSpec, n_tokens: int) -> float:
     """Algorithmic FLOPs of one decoded query: 2 x multiply-adds of the Q
     projection (51 embedding lanes), attention (QK^T and PV over n_tokens), output
@@ -251,7 +257,10 @@ def run_vdm(args, world, rank, local):
                 "d2h_bytes_per_step": int(out_host.numel() * 4)},
         "roofline": {"kernel": "decode_tc_kernel", "bound": "tensor", "achieved": achieved_tflops,
                      "peak": tc_peak, "unit": "TFLOP/s", "frac": achieved_tflops / tc_peak,
-                     "traffic": None,
+                     "traffic": DECODE_DRAM_BYTES_PER_LAUNCH.get(cfg.cid),
+                     "traffic_note": "DRAM bytes read + written per decode launch (mean of the step's "
+                                     "launches) from ncu on this workload's own launches; null where "
+                                     "not captured for the current kernel",
                      "peak_note": "measured sustained bf16 matmul peak (MEASURED_PEAKS.json), "
                                   f"{peaks['src']}; algorithmic FLOPs: {dec_flops / 1e12:.2f} TFLOP/step"},
         "select_roofline": {"kernel": "select_tc_kernel", "achieved":
