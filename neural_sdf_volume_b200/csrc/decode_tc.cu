@@ -11,8 +11,9 @@
 //   warps 0-7  compute: two warpgroups; thread (g, r) owns TMEM lane r and
 //              half g of the row's columns (softmax columns, head dims, hidden
 //              units, LayerNorm columns), so every SM sub-partition runs two
-//              compute warps; the halves exchange a block maximum (bf16, in
-//              smem) per attention block and a few row statistics per tile;
+//              compute warps; each warpgroup runs its own online softmax over
+//              its half of every key block (own maximum, sum and O
+//              accumulator), and the halves combine once per head;
 //   warp 8     MMA issue (one lane);
 //   warp 9     producer: TMA loads of weights and of contiguous K/V blocks,
 //              cp.async gathers of a sub-volume's selected K/V rows;
@@ -32,7 +33,7 @@
 //   H_c = LN1(x1) W1_c^T, GELU, X += GELU(H_c) W2_c^T ; LN2 . w_head -> SDF.
 //
 // TMEM (512 columns x 128 lanes):
-//   attention: S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384) O [384,448)
+//   attention: S0 [0,128) S1 [128,256) P [256,320) O0 [320,384) O1 [384,448)
 //              Q accumulator / packed bf16 Q [448,512)
 //   output projection: X [0, C)
 //   MLP, C <= 256: acc [0, C); hidden chunks (128 wide) at [256,384) [384,512)
@@ -73,7 +74,9 @@ constexpr int MAX_NS = 16;   // ring slots (CTA pairs use twice as many, half as
 constexpr int RING_ARRIVALS = 32;   // arrivals completing a ring slot: one per producer lane
 constexpr float kLog2e = 1.4426950408889634f;
 
-constexpr uint32_t T_S0 = 0, T_S1 = 128, T_P0 = 256, T_P1 = 320, T_O = 384, T_Q = 448;
+// attention: S double-buffered; one P buffer (each warpgroup's 64 tokens as bf16 pairs in
+// 32 columns); one O accumulator per warpgroup (its token half, all 64 head dims); Q
+constexpr uint32_t T_S0 = 0, T_S1 = 128, T_P = 256, T_O0 = 320, T_O1 = 384, T_Q = 448;
 
 // ring depth: 16 KB slots in what the 227 KB of shared memory leaves after the
 // activation buffer (C/64 atoms of 16 KB), the embedding tile and alignment
@@ -99,7 +102,6 @@ struct Shared {
     // compute-warp arrivals (count 128)
     uint64_t bar_pe, bar_qc, bar_p[2], bar_a, bar_hin, bar_r, bar_g[2], bar_cs, bar_wg;
     uint32_t tmem_base;
-    uint16_t xmax[2][2][128];   // per attention block: [block parity][warpgroup][row] block max (bf16 bits)
     int abort;
     float G, Bc;
 };
@@ -611,13 +613,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         tc_fence_after();
                         if (!(ok = consume(slot))) break;
                         if (u.sel) fence_proxy_async();
-                        const uint32_t pa = tmem + ((j & 1) ? T_P1 : T_P0);
-                        // V is N-major: 16 tokens per k-step = 16 rows of 128 B (64 B per CTA of a pair)
+                        // O_g += P_g V_g for the two warpgroups' token halves. V is N-major: 16 tokens
+                        // per k-step = 16 rows of 128 B (64 B per CTA of a pair)
                         const uint64_t dv = PAIR ? desc_sw64(s_ring + slot * RS) : desc_sw128(s_ring + slot * RS);
                         constexpr int vstep = PAIR ? 64 : 128;
                         #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            mma_t(tmem + T_O, pa + 8 * kk, dv + vstep * kk, idesc_bf16(MR, 64, true), (j > 0 || kk > 0));
+                        for (int g = 0; g < 2; ++g)
+                            #pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_t(tmem + (g ? T_O1 : T_O0), tmem + T_P + 32 * g + 8 * kk,
+                                      dv + vstep * (4 * g + kk), idesc_bf16(MR, 64, true), (j > 0 || kk > 0));
                         release(slot);
                         commit_both(&sh.bar_pv);
                         if (j + 2 < nb) ok = issue_s(j + 2);
@@ -832,45 +837,46 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         m2 = fmaxf(m2, s1[c]);
                         m3 = fmaxf(m3, s1[c + 1]);
                     }
-                    // both halves decide on the same (bf16-truncated) block maximum
-                    const uint16_t own = (uint16_t)(__float_as_uint(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3))) >> 16);
-                    sh.xmax[j & 1][wg][row] = own;
-                    if (!(ok = wg_sync(69))) break;
-                    const uint16_t oth = sh.xmax[j & 1][wg ^ 1][row];
-                    const float mb = fmaxf(__uint_as_float((uint32_t)own << 16), __uint_as_float((uint32_t)oth << 16));
+                    // this warpgroup's own running maximum over its token half
+                    const float mb = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
                     const bool need = (j == 0) || (mb > m_ref + 8.0f);
                     const float m_new = need ? fmaxf(mb, m_ref) : m_ref;
-                    const float f = (j == 0) ? 0.f : ex2(m_ref - m_new);
+                    const float f = (j == 0 || m_new == -INFINITY) ? 0.f : ex2(m_ref - m_new);
                     if (need) m_ref = m_new;
+                    const float m_use = m_ref == -INFINITY ? 0.f : m_ref;   // no real token yet: P = 0
                     float la = 0.f, lb = 0.f;
                     uint32_t pk[32];
 #pragma unroll
                     for (int v = 0; v < 16; ++v) {
-                        const float e0 = ex2(s0[2 * v] - m_ref), e1 = ex2(s0[2 * v + 1] - m_ref);
-                        const float e2 = ex2(s1[2 * v] - m_ref), e3 = ex2(s1[2 * v + 1] - m_ref);
+                        const float e0 = ex2(s0[2 * v] - m_use), e1 = ex2(s0[2 * v + 1] - m_use);
+                        const float e2 = ex2(s1[2 * v] - m_use), e3 = ex2(s1[2 * v + 1] - m_use);
                         la += e0 + e1;
                         lb += e2 + e3;
                         pk[v] = pack_bf16(e0, e1);
                         pk[16 + v] = pack_bf16(e2, e3);
                     }
-                    if (j > 0) {   // PV_{j-1} (hence PV_{j-2}) done: P buffer free, O stable
+                    if (j > 0) {   // PV_{j-1} done: the P buffer is free and O stable
                         if (!(ok = W.wait(&sh.bar_pv, ph_pv, 62))) break;
                         tc_fence_after();
                     }
+                    tmem_st32(trow + T_P + 32 * wg, pk);
                     if (need && j > 0) l_part *= f;
                     l_part += la + lb;
                     if (j > 0 && __any_sync(0xffffffffu, need)) {
-                        float o[32];
-                        tmem_ld32(trow + T_O + 32 * wg, o);
-                        tmem_wait_ld();
-                        reg_fence(o);
+                        const uint32_t ob = trow + (wg ? T_O1 : T_O0);
                         const float g = need ? f : 1.0f;
-                        uint32_t uo[32];
+                        #pragma unroll 1
+                        for (int hh = 0; hh < 4; ++hh) {
+                            float o[16];
+                            tmem_ld16(ob + 16 * hh, o);
+                            tmem_wait_ld();
+                            reg_fence16(o);
+                            uint32_t uo[16];
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) uo[c] = __float_as_uint(o[c] * g);
-                        tmem_st32(trow + T_O + 32 * wg, uo);
+                            for (int c = 0; c < 16; ++c) uo[c] = __float_as_uint(o[c] * g);
+                            tmem_st16(ob + 16 * hh, uo);
+                        }
                     }
-                    tmem_st32(trow + ((j & 1) ? T_P1 : T_P0) + 32 * wg, pk);
                     tmem_wait_st();
                     tc_fence_before();
                     arrive_mma(&sh.bar_p[j & 1]);
@@ -878,34 +884,49 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 if (!ok) break;
                 if (!(ok = W.wait(&sh.bar_pv, ph_pv, 63))) break;   // PV_{nb-1}
                 tc_fence_after();
-                // row sum: exchange the halves through TMEM (S0 is idle until the next head's S_0)
-                tmem_st1(trow + T_S0 + wg, __float_as_uint(l_part));
+                // combine the halves: exchange (maximum, sum) through TMEM (S0 is idle until the
+                // next head's S_0), then O = (O0 2^(m0-M) + O1 2^(m1-M)) / (l0 2^(m0-M) + l1 2^(m1-M))
+                tmem_st1(trow + T_S0 + 2 * wg, __float_as_uint(m_ref));
+                tmem_st1(trow + T_S0 + 2 * wg + 1, __float_as_uint(l_part));
                 tmem_wait_st();
                 tc_fence_before();
                 if (!(ok = wg_sync(70))) break;
                 tc_fence_after();
-                uint32_t l_bits = tmem_ld1(trow + T_S0 + (wg ^ 1));
+                uint32_t mo_bits = tmem_ld1(trow + T_S0 + 2 * (wg ^ 1));
+                uint32_t lo_bits = tmem_ld1(trow + T_S0 + 2 * (wg ^ 1) + 1);
                 tmem_wait_ld();
-                asm volatile("" : "+r"(l_bits));
-                const float l_oth = __uint_as_float(l_bits);
-                const float l_tot = l_part + l_oth;
+                asm volatile("" : "+r"(mo_bits), "+r"(lo_bits));
+                const float m_oth = __uint_as_float(mo_bits), l_oth = __uint_as_float(lo_bits);
+                const float M = fmaxf(m_ref, m_oth);
+                const float f_own = m_ref == -INFINITY ? 0.f : ex2(m_ref - M);
+                const float f_oth = m_oth == -INFINITY ? 0.f : ex2(m_oth - M);
+                const float l_tot = l_part * f_own + l_oth * f_oth;
                 {
-                    float o[32];
-                    tmem_ld32(trow + T_O + 32 * wg, o);
-                    tmem_wait_ld();
-                    reg_fence(o);
                     const float inv = 1.0f / l_tot;
+                    const float g0 = (wg ? f_oth : f_own) * inv, g1 = (wg ? f_own : f_oth) * inv;
                     const uint32_t atom = s_abuf + h * 16384;
                     #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t w[4];
+                    for (int hh = 0; hh < 2; ++hh) {   // 16 of this warpgroup's 32 head dims at a time
+                        float o0[16], o1[16];
+                        tmem_ld16(trow + T_O0 + 32 * wg + 16 * hh, o0);
+                        tmem_ld16(trow + T_O1 + 32 * wg + 16 * hh, o1);
+                        tmem_wait_ld();
+                        reg_fence16(o0);
+                        reg_fence16(o1);
                         #pragma unroll
-                        for (int v = 0; v < 4; ++v) w[v] = pack_bf16(o[c * 8 + 2 * v] * inv, o[c * 8 + 2 * v + 1] * inv);
-                        st_shared_v4(swz(atom, row, 4 * wg + c), w);
+                        for (int c = 0; c < 2; ++c) {
+                            uint32_t w[4];
+                            #pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                const int d = c * 8 + 2 * v;
+                                w[v] = pack_bf16(fmaf(o0[d], g0, o1[d] * g1), fmaf(o0[d + 1], g0, o1[d + 1] * g1));
+                            }
+                            st_shared_v4(swz(atom, row, 4 * wg + 2 * hh + c), w);
+                        }
                     }
                 }
                 if (ml_out) {
-                    ml_out[h * 2] = m_ref;
+                    ml_out[h * 2] = M;
                     ml_out[h * 2 + 1] = l_tot;
                 }
             }
