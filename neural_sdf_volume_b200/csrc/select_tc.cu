@@ -17,7 +17,9 @@
 // largest scores (ties to the smaller token) per sub-volume, in shared memory.
 //
 // Rows: 128 TMEM lanes hold 128 / n_probe sub-volumes' probes (n_probe in
-// {32, 64, 128}).  Roles: warps 0-3 compute, warp 4 MMA issue, warp 5 TMA.
+// {32, 64, 128}).  Roles: warps 0-7 compute in two warpgroups (thread (g, r)
+// owns row r and the 64 columns of half g of each 128-token block, so every
+// SM sub-partition runs two compute warps), warp 8 MMA issue, warp 9 TMA.
 #include <cuda.h>
 
 #include "tc_ptx.cuh"
@@ -32,8 +34,9 @@ namespace {
 
 using namespace ptx;
 
-constexpr int NT = 192;
-constexpr int NCOMP = 128;
+constexpr int NT = 320;
+constexpr int NCOMP = 256;
+constexpr int WARP_MMA = 8, WARP_PROD = 9;
 constexpr int SLOT = 16384;
 constexpr int NS = 6;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -67,7 +70,7 @@ struct Shared {
     int abort;
     int hist[256];
     int red[4];
-    int wsum[4];
+    int wsum[NCOMP / 32];
 };
 
 struct Waiter {
@@ -98,6 +101,50 @@ struct Waiter {
 
 __device__ __forceinline__ uint32_t swz(uint32_t base, int r, int c) {
     return base + r * 128 + ((c ^ (r & 7)) << 4);
+}
+
+// Sum of v over the 32 lanes for each of 64 columns; lane L returns the sums of
+// columns 2L and 2L+1 (the same recursive halving as below, one round fewer).
+__device__ __forceinline__ void warp_colsum64(const float (&v)[64], int lane, float (&out)[2]) {
+    float a32[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const bool up = lane & 16;
+        const float send = up ? v[i] : v[i + 32];
+        const float keep = up ? v[i + 32] : v[i];
+        a32[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    float a16[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const bool up = lane & 8;
+        const float send = up ? a32[i] : a32[i + 16];
+        const float keep = up ? a32[i + 16] : a32[i];
+        a16[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float a8[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const bool up = lane & 4;
+        const float send = up ? a16[i] : a16[i + 8];
+        const float keep = up ? a16[i + 8] : a16[i];
+        a8[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+    float a4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool up = lane & 2;
+        const float send = up ? a8[i] : a8[i + 4];
+        const float keep = up ? a8[i + 4] : a8[i];
+        a4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const bool up = lane & 1;
+        const float send = up ? a4[i] : a4[i + 2];
+        const float keep = up ? a4[i + 2] : a4[i];
+        out[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    }
 }
 
 // Sum of v over the 32 lanes for each of 128 columns; lane L returns the sums
@@ -157,7 +204,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
     const uint32_t s_pe = dyn0;
     const uint32_t s_ring = s_pe + 16384;
     float* score = reinterpret_cast<float*>(dyn_raw + (dyn0 - smem_u32(dyn_raw)) + 16384 + NS * SLOT);  // [tpu][N]
-    float* part = score + (size_t)tpu * N;    // [2][4 warps][128]
+    float* part = score + (size_t)tpu * N;    // [2][8 warps][64]
     Waiter W{&sh, a.err, a.timeout};
 
     if (tid == 0) {
@@ -189,7 +236,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
     const int n_sel = *a.n_sel < a.n_sel_max ? *a.n_sel : a.n_sel_max;
     const int n_units = (n_sel + tpu - 1) / tpu;
 
-    if (warp == 5) {
+    if (warp == WARP_PROD) {
         // ------------------------------------------------------------ producer
         uint32_t ring_head = 0;
         bool ok = true;
@@ -213,7 +260,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                 ok = push(&tm_wq64, h * 64, 64 * 128);
                 for (int j = 0; j < nb && ok; ++j) ok = push(&tm_k, h * N + j * 128, SLOT);
             }
-    } else if (warp == 4) {
+    } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------ MMA issue
         if (lane == 0) {
             uint32_t ring_tail = 0, ph_pe = 0, ph_qc = 0, ph_p[2] = {0, 0}, ph_hd = 0;
@@ -231,8 +278,10 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                 if (!consume(sl)) return false;
                 const uint64_t db = desc_sw128(s_ring + sl * SLOT);
                 const uint32_t sd = tmem + ((j & 1) ? T_S1 : T_S0);
+                // Q: the warpgroups packed head dims [0,32) into columns [0,16) and [32,64) into [32,48)
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(sd, tmem + T_Q + 8 * kk, db + 2 * kk, idesc_bf16(128, 128, false), kk > 0);
+                    mma_ts(sd, tmem + T_Q + (kk < 2 ? 8 * kk : 32 + 8 * (kk - 2)), db + 2 * kk,
+                           idesc_bf16(128, 128, false), kk > 0);
                 mma_commit(smem_u32(&sh.empty[sl]));
                 mma_commit(smem_u32(&sh.bar_s[j & 1]));
                 return true;
@@ -265,7 +314,8 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
         }
     } else {
         // ------------------------------------------------------------ compute
-        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+        const int wg = tid >> 7, row = tid & 127;
+        const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
         uint32_t ph_q = 0, ph_s[2] = {0, 0}, ph_cs = 0;
         const float qscale = 0.125f * kLog2e;
         bool ok = true;
@@ -274,9 +324,9 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
             arrive(&sh.bar_cs);
             return W.wait(&sh.bar_cs, ph_cs, site);
         };
-        const int my_slot = tid / np;            // sub-volume slot of this row
-        const int my_i = tid % np;               // probe index within it
-        const int warps_per_tile = np >= 32 ? np / 32 : 1;
+        const int my_slot = row / np;            // sub-volume slot of this row
+        const int my_i = row % np;               // probe index within it
+        const int warps_per_tile = np >= 32 ? np / 32 : 1;   // per warpgroup
         for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
             const int t_idx = unit * tpu + my_slot;
             const bool valid = my_slot < tpu && t_idx < n_sel;
@@ -286,10 +336,10 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                 const int e = a.qorder[8 * a.tile_off[t] + my_i];
                 voxel_point(child_index(a.plist[e >> 3], e & 7, a.R), a.R, p);
             }
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 4 * wg; c < 4 * wg + 4; ++c) {
                 uint32_t w[4];
                 for (int v = 0; v < 4; ++v) w[v] = pack_bf16(pe_lane(p, c * 8 + 2 * v), pe_lane(p, c * 8 + 2 * v + 1));
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(swz(s_pe, tid, c)), "r"(w[0]),
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(swz(s_pe, row, c)), "r"(w[0]),
                              "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
             }
             for (int j = tid; j < tpu * N; j += NCOMP) score[j] = 0.f;
@@ -301,19 +351,17 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                 if (!(ok = W.wait(&sh.bar_q, ph_q, 86))) break;
                 tc_fence_after();
                 {
-                    float q0[32], q1[32];
-                    tmem_ld32(trow + T_Q, q0);
-                    tmem_ld32(trow + T_Q + 32, q1);
+                    // head dims [32 wg, 32 wg + 32): + bq, scale, pack into the first 16 columns of the source
+                    float q[32];
+                    tmem_ld32(trow + T_Q + 32 * wg, q);
                     tmem_wait_ld();
-                    reg_fence(q0);
-                    reg_fence(q1);
-                    uint32_t pk[32];
+                    reg_fence(q);
+                    uint32_t pk[16];
                     for (int v = 0; v < 16; ++v) {
-                        const int c0 = h * 64 + 2 * v, c1 = h * 64 + 32 + 2 * v;
-                        pk[v] = pack_bf16((q0[2 * v] + a.bq[c0]) * qscale, (q0[2 * v + 1] + a.bq[c0 + 1]) * qscale);
-                        pk[16 + v] = pack_bf16((q1[2 * v] + a.bq[c1]) * qscale, (q1[2 * v + 1] + a.bq[c1 + 1]) * qscale);
+                        const int c0 = h * 64 + 32 * wg + 2 * v;
+                        pk[v] = pack_bf16((q[2 * v] + a.bq[c0]) * qscale, (q[2 * v + 1] + a.bq[c0 + 1]) * qscale);
                     }
-                    tmem_st32(trow + T_Q, pk);
+                    tmem_st16(trow + T_Q + 32 * wg, pk);
                     tmem_wait_st();
                 }
                 tc_fence_before();
@@ -323,48 +371,39 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                 for (int j = 0; j < nb; ++j) {
                     if (!(ok = W.wait(&sh.bar_s[j & 1], ph_s[j & 1], 87))) break;
                     tc_fence_after();
-                    float v[128];
+                    float v[64];
                     {
-                        const uint32_t sb = trow + ((j & 1) ? T_S1 : T_S0);
-                        float s0[32], s1[32], s2[32], s3[32];
+                        const uint32_t sb = trow + ((j & 1) ? T_S1 : T_S0) + 64 * wg;
+                        float s0[32], s1[32];
                         tmem_ld32(sb, s0);
                         tmem_ld32(sb + 32, s1);
-                        tmem_ld32(sb + 64, s2);
-                        tmem_ld32(sb + 96, s3);
                         tmem_wait_ld();
                         reg_fence(s0);
                         reg_fence(s1);
-                        reg_fence(s2);
-                        reg_fence(s3);
                         tc_fence_before();
-                        arrive(&sh.bar_p[j & 1]);   // S_j consumed
-                        const int vcols = N - j * 128;
+                        arrive(&sh.bar_p[j & 1]);   // this half of S_j consumed
+                        const int vcols = N - j * 128 - 64 * wg;
 #pragma unroll
                         for (int c = 0; c < 32; ++c) {
                             v[c] = (c < vcols) ? ex2(s0[c] - m) * inv_l : 0.f;
                             v[32 + c] = (32 + c < vcols) ? ex2(s1[c] - m) * inv_l : 0.f;
-                            v[64 + c] = (64 + c < vcols) ? ex2(s2[c] - m) * inv_l : 0.f;
-                            v[96 + c] = (96 + c < vcols) ? ex2(s3[c] - m) * inv_l : 0.f;
                         }
                     }
-                    float cs[4];
-                    warp_colsum128(v, lane, cs);
-                    float* pw = part + (pb * 4 + warp) * 128;
-                    pw[4 * lane] = cs[0];
-                    pw[4 * lane + 1] = cs[1];
-                    pw[4 * lane + 2] = cs[2];
-                    pw[4 * lane + 3] = cs[3];
+                    float cs[2];
+                    warp_colsum64(v, lane, cs);
+                    float* pw = part + (pb * 8 + warp) * 64;
+                    pw[2 * lane] = cs[0];
+                    pw[2 * lane + 1] = cs[1];
                     if (!(ok = csync(88))) break;
-                    // thread c adds column c of each sub-volume (its warps in order)
-                    {
-                        const int col = tid;
+                    // column col of sub-volume s: its warps of the column's warpgroup, in order
+                    for (int idx = tid; idx < tpu * 128; idx += NCOMP) {
+                        const int sv = idx >> 7, col = idx & 127;
                         if (j * 128 + col < N) {
-                            const float* pp = part + pb * 4 * 128;
-                            for (int s = 0; s < tpu; ++s) {
-                                float acc = 0.f;
-                                for (int w = 0; w < warps_per_tile; ++w) acc += pp[(s * warps_per_tile + w) * 128 + col];
-                                score[(size_t)s * N + j * 128 + col] += acc;
-                            }
+                            const int g = col >> 6;
+                            const float* pp = part + (pb * 8 + 4 * g + sv * warps_per_tile) * 64 + (col & 63);
+                            float acc = 0.f;
+                            for (int w = 0; w < warps_per_tile; ++w) acc += pp[w * 64];
+                            score[(size_t)sv * N + j * 128 + col] += acc;
                         }
                     }
                     pb ^= 1;
