@@ -139,6 +139,7 @@ def _oracle_adaptive_dec(case, b, R, decoded, idx, dbg, l, n_probe, seed):
     want = np.empty(idx.size)
     idx_tiles = OA.tile_of(idx, R, 8)
     pos = {int(v): n for n, v in enumerate(idx)}
+    checked = [0]
     for t in np.unique(idx_tiles):
         members = np.sort(decoded[tiles == t])
         probe = OA.choose_probes(members, n_probe, seed, l)
@@ -154,6 +155,13 @@ def _oracle_adaptive_dec(case, b, R, decoded, idx, dbg, l, n_probe, seed):
             assert int(t) in row, f"tile {t} has no GPU selection"
             sel = sel_gpu[row[int(t)]]
             assert (sel >= 0).all() and np.all(np.diff(sel) > 0)
+            if checked[0] < 16:   # the selection itself: the oracle's Top-K from the same probes
+                K, _ = case.okv(b)
+                q = OA.query_vectors(OD.grid_points(R, members[probe]), case.w)
+                top = OA.top_k(OA.token_scores(q, K), sel.size)
+                overlap = len(np.intersect1d(sel, top)) / sel.size
+                assert overlap >= 0.9, f"tile {t}: Top-K overlap {overlap}"
+                checked[0] += 1
             v = case.oracle_dec(OD.grid_points(R, sparse_pts), b, sel=sel)
             for p_, x in zip(sparse_pts, v):
                 want[pos[int(p_)]] = x
