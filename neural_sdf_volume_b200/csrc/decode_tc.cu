@@ -14,10 +14,13 @@
 //              compute warps; each warpgroup runs its own online softmax over
 //              its half of every key block (own maximum, sum and O
 //              accumulator), and the halves combine once per head;
-//   warp 8     MMA issue (one lane);
+//   warp 8     MMA issue (the whole warp runs the loop; one elected lane issues);
 //   warp 9     producer: TMA loads of weights and of contiguous K/V blocks,
-//              cp.async gathers of a sub-volume's selected K/V rows;
+//              cp.async gathers of a sub-volume's selected K/V rows (each lane's
+//              copies arrive on the slot's barrier when they land);
 // connected only by mbarriers (no CTA-wide barrier inside a tile).
+// Compiled twice per width: one CTA per 128-row MMA, or (cta_group::2) a CTA
+// pair of a cluster per 256-row MMA, each CTA holding half of every B tile.
 //
 // Split-packed A operands: Q and the GELU output are produced by the two
 // warpgroups, each packing its half (bf16 pairs) into the start of its own
@@ -27,8 +30,9 @@
 //
 // Per tile:
 //   PE (bf16 smem) ; per head h: Q_h = PE Wq_h^T (TMEM) -> bf16 in TMEM;
-//   per 128-token block j: S_j = Q_h K_j^T ; softmax -> P_j (bf16, TMEM) ;
-//   O += P_j V_j ; a[:, h] = O / l (bf16 smem).
+//   per 128-token block j: S_j = Q_h K_j^T ; per warpgroup g: softmax of its
+//   64 tokens -> P_j,g (bf16, TMEM), O_g += P_j,g V_j,g ; end of head: combine
+//   the two (max, sum, O_g) -> a[:, h] (bf16 smem).
 //   X = PE Wq^T + a Wo^T ; LN1 -> bf16 smem ; MLP hidden chunks:
 //   H_c = LN1(x1) W1_c^T, GELU, X += GELU(H_c) W2_c^T ; LN2 . w_head -> SDF.
 //
