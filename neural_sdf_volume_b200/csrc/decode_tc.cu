@@ -30,15 +30,17 @@
 //
 // Per tile:
 //   PE (bf16 smem) ; per head h: Q_h = PE Wq_h^T (TMEM) -> bf16 in TMEM;
-//   per 128-token block j: S_j = Q_h K_j^T ; per warpgroup g: softmax of its
-//   64 tokens -> P_j,g (bf16, TMEM), O_g += P_j,g V_j,g ; end of head: combine
-//   the two (max, sum, O_g) -> a[:, h] (bf16 smem).
+//   Q_h -> bf16 smem (attention-output atom h, free until the head's combine);
+//   per 128-token block j, owned by warpgroup g = j mod 2: S_j = Q_h K_j^T into
+//   S_{j mod 3} ; softmax of the block -> P_j (bf16, in place) ; O_g += P_j V_j ;
+//   end of head: combine the two (max, sum, O_g) -> a[:, h] (bf16 smem).
 //   X = PE Wq^T + a Wo^T ; LN1 -> bf16 smem ; MLP hidden chunks:
 //   H_c = LN1(x1) W1_c^T, GELU, X += GELU(H_c) W2_c^T ; LN2 . w_head -> SDF.
 //
 // TMEM (512 columns x 128 lanes):
-//   attention: S0 [0,128) S1 [128,256) P [256,320) O0 [320,384) O1 [384,448)
-//              Q accumulator / packed bf16 Q [448,512)
+//   attention: S0 [0,128) S1 [128,256) S2 [256,384) (P_j overwrites the first 16 of
+//              each 32 S columns once they are read; the Q accumulator sits in S2
+//              before the head's first block) O0 [384,448) O1 [448,512)
 //   output projection: X [0, C)
 //   MLP, C <= 256: acc [0, C); hidden chunks (128 wide) at [256,384) [384,512)
 //   MLP, C == 512: the 128 x 512 fp32 residual alone fills TMEM, so the MLP
@@ -78,9 +80,14 @@ constexpr int MAX_NS = 16;   // ring slots (CTA pairs use twice as many, half as
 constexpr int RING_ARRIVALS = 32;   // arrivals completing a ring slot: one per producer lane
 constexpr float kLog2e = 1.4426950408889634f;
 
-// attention: S double-buffered; one P buffer (each warpgroup's 64 tokens as bf16 pairs in
-// 32 columns); one O accumulator per warpgroup (its token half, all 64 head dims); Q
-constexpr uint32_t T_S0 = 0, T_S1 = 128, T_P = 256, T_O0 = 320, T_O1 = 384, T_Q = 448;
+// attention: three S buffers in rotation (block j in S_{j mod 3}; its P overwrites the S
+// columns already read), so the next block's scores are ready before a warpgroup needs them;
+// the warpgroups alternate blocks, so one's exponentials overlap the other's loads, maximum
+// and hand-offs; one O accumulator per warpgroup (its blocks, all 64 head dims); the Q
+// projection accumulates in S2 before the head's first block, the packed Q waits in shared
+// memory
+constexpr uint32_t T_S0 = 0, T_O0 = 384, T_O1 = 448, T_QACC = 256;
+constexpr int NSB = 3;   // S buffers
 
 // ring depth: 16 KB slots in what the 227 KB of shared memory leaves after the
 // activation buffer (C/64 atoms of 16 KB), the embedding tile and alignment
@@ -102,7 +109,8 @@ struct TcArgs {
 struct Shared {
     uint64_t full[MAX_NS], empty[MAX_NS];
     // MMA commits (count 1); bar_hd and bar_w2 are waited on by the MMA warp only
-    uint64_t bar_q, bar_s[2], bar_pv, bar_x, bar_h[2], bar_acc, bar_hd, bar_w2, bar_fin;
+    // bar_s[j mod 6]: S_j ready (block j's buffer and owner both follow from j mod 6)
+    uint64_t bar_q, bar_s[6], bar_pvg[2], bar_pvm, bar_pv, bar_x, bar_h[2], bar_acc, bar_hd, bar_w2, bar_fin;
     // compute-warp arrivals (count 128)
     uint64_t bar_pe, bar_qc, bar_p[2], bar_a, bar_hin, bar_r, bar_g[2], bar_cs, bar_wg;
     uint32_t tmem_base;
@@ -265,13 +273,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             mbar_init(smem_u32(&sh.full[i]), RING_ARRIVALS + (PAIR && leader ? 1 : 0));
             mbar_init(smem_u32(&sh.empty[i]), 1);
         }
-        uint64_t* one[] = {&sh.bar_q, &sh.bar_s[0], &sh.bar_s[1], &sh.bar_pv, &sh.bar_x,
+        uint64_t* one[] = {&sh.bar_q, &sh.bar_s[0], &sh.bar_s[1], &sh.bar_s[2], &sh.bar_s[3], &sh.bar_s[4],
+                           &sh.bar_s[5], &sh.bar_pvg[0], &sh.bar_pvg[1], &sh.bar_pvm, &sh.bar_pv, &sh.bar_x,
                            &sh.bar_h[0], &sh.bar_h[1], &sh.bar_acc, &sh.bar_hd, &sh.bar_w2, &sh.bar_fin};
         for (auto* b : one) mbar_init(smem_u32(b), 1);
         // compute -> MMA: one arrival per compute thread, or per compute warp of both CTAs
-        uint64_t* to_mma[] = {&sh.bar_pe, &sh.bar_qc, &sh.bar_p[0], &sh.bar_p[1], &sh.bar_a,
+        uint64_t* to_mma[] = {&sh.bar_pe, &sh.bar_qc, &sh.bar_a,
                               &sh.bar_hin, &sh.bar_r, &sh.bar_g[0], &sh.bar_g[1]};
         for (auto* b : to_mma) mbar_init(smem_u32(b), PAIR ? 2 * (NCOMP / 32) : NCOMP);
+        // P_j comes from one warpgroup (the one that owns block j)
+        for (auto* b : {&sh.bar_p[0], &sh.bar_p[1]}) mbar_init(smem_u32(b), PAIR ? 2 * (BM / 32) : BM);
         mbar_init(smem_u32(&sh.bar_cs), NCOMP);
         mbar_init(smem_u32(&sh.bar_wg), NCOMP);
         sh.abort = 0;
@@ -470,11 +481,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             };
             for (int h = 0; h < H && ok; ++h) {
                 ok = push_tma(&tm_wq64, 0, h * 64 + (PAIR ? 32 * (int)crank : 0), PAIR ? 32 * 128 : 64 * 128);
-                ok = ok && push_kv(false, h, 0);
-                if (nb > 1) ok = ok && push_kv(false, h, 1);
+                for (int j = 0; j < nb && j < NSB && ok; ++j) ok = push_kv(false, h, j);
                 for (int j = 0; j < nb && ok; ++j) {
                     ok = push_kv(true, h, j);
-                    if (j + 2 < nb) ok = ok && push_kv(false, h, j + 2);
+                    if (j + NSB < nb) ok = ok && push_kv(false, h, j + NSB);
                 }
             }
             // X = PE Wq^T + a Wo^T : items of AT K atoms (atom 0: Wq, atom ka > 0: Wo columns ka-1)
@@ -548,7 +558,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             W.cluster_acq = PAIR;
             uint32_t ring_tail = 0;
             uint32_t ph_pe = 0, ph_qc = 0, ph_p[2] = {0, 0}, ph_a = 0, ph_hin = 0, ph_r = 0, ph_g[2] = {0, 0};
-            uint32_t ph_hd = 0, ph_w2 = 0;
+            uint32_t ph_hd = 0, ph_w2 = 0, ph_pvm = 0;
             bool ok = true;
             int c_slot = 0;
             uint32_t c_ph = 0;
@@ -591,7 +601,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         const uint64_t da = desc_sw128(s_pe), db = desc_sw128(s_ring + slot * RS);
                         #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_s(tmem + T_Q, da + 2 * kk, db + 2 * kk, idesc_bf16(MR, 64, false), kk > 0);
+                            mma_s(tmem + T_QACC, da + 2 * kk, db + 2 * kk, idesc_bf16(MR, 64, false), kk > 0);
                         release(slot);
                         if (!(ta.inject && h == 0 && first_unit)) commit_both(&sh.bar_q);
                     }
@@ -602,37 +612,46 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         if (!consume(sl)) return false;
                         // gathered rows were written by cp.async (generic proxy): order them before the MMA's reads
                         if (u.sel) fence_proxy_async();
-                        const uint64_t db = desc_sw128(s_ring + sl * RS);
-                        const uint32_t sd = tmem + ((j & 1) ? T_S1 : T_S0);
+                        const uint64_t da = desc_sw128(s_abuf + h * 16384), db = desc_sw128(s_ring + sl * RS);
+                        const uint32_t sd = tmem + T_S0 + 128 * (j % NSB);
                         #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_t(sd, tmem + T_Q + split_col(kk, 64), db + 2 * kk, idesc_bf16(MR, 128, false), kk > 0);
+                            mma_s(sd, da + 2 * kk, db + 2 * kk, idesc_bf16(MR, 128, false), kk > 0);
                         release(sl);
-                        commit_both(&sh.bar_s[j & 1]);
+                        commit_both(&sh.bar_s[j % 6]);
                         return true;
                     };
-                    ok = issue_s(0) && (nb < 2 || issue_s(1));
+                    for (int j = 0; j < nb && j < NSB && ok; ++j) ok = issue_s(j);
                     for (int j = 0; j < nb && ok; ++j) {
-                        if (!(ok = W.wait(&sh.bar_p[j & 1], ph_p[j & 1], 53))) break;
+                        const int g = j & 1;   // block j belongs to warpgroup j mod 2
+                        if (!(ok = W.wait(&sh.bar_p[g], ph_p[g], 53))) break;
                         tc_fence_after();
                         if (!(ok = consume(slot))) break;
                         if (u.sel) fence_proxy_async();
-                        // O_g += P_g V_g for the two warpgroups' token halves. V is N-major: 16 tokens
-                        // per k-step = 16 rows of 128 B (64 B per CTA of a pair)
+                        // O_g += P_j V_j. P_j is read in place: the bf16 pairs of tokens [32i, 32i+32)
+                        // occupy columns [32i, 32i+16) of its S buffer. V is N-major: 16 tokens per
+                        // k-step = 16 rows of 128 B (64 B per CTA of a pair)
                         const uint64_t dv = PAIR ? desc_sw64(s_ring + slot * RS) : desc_sw128(s_ring + slot * RS);
                         constexpr int vstep = PAIR ? 64 : 128;
+                        const uint32_t pa = tmem + T_S0 + 128 * (j % NSB);
                         #pragma unroll
-                        for (int g = 0; g < 2; ++g)
-                            #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma_t(tmem + (g ? T_O1 : T_O0), tmem + T_P + 32 * g + 8 * kk,
-                                      dv + vstep * (4 * g + kk), idesc_bf16(MR, 64, true), (j > 0 || kk > 0));
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_t(tmem + (g ? T_O1 : T_O0), pa + 32 * (kk >> 1) + 8 * (kk & 1), dv + vstep * kk,
+                                  idesc_bf16(MR, 64, true), (j >= 2 || kk > 0));
                         release(slot);
-                        commit_both(&sh.bar_pv);
-                        if (j + 2 < nb) ok = issue_s(j + 2);
+                        // O_g is final for this block once the PV is done (the owner waits before its next)
+                        if (j + 2 < nb) commit_both(&sh.bar_pvg[g]);
+                        if (j + NSB < nb) {
+                            // S_{j+3} overwrites the columns this PV reads: let the PV finish first
+                            commit_own(&sh.bar_pvm);
+                            if (!(ok = W.wait(&sh.bar_pvm, ph_pvm, 66))) break;
+                            tc_fence_after();
+                            ok = issue_s(j + NSB);
+                        }
                     }
                     if (!ok) break;
-                    // the next head's Q projection rewrites T_Q, which this head's S MMAs read
+                    commit_both(&sh.bar_pv);   // the head's PVs are complete: O0 and O1 final
+                    // the next head's Q projection accumulates in S2, which this head's PVs read
                     commit_own(&sh.bar_hd);
                     if (!(ok = W.wait(&sh.bar_hd, ph_hd, 54))) break;
                     tc_fence_after();
@@ -732,7 +751,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
         const int wg = tid >> 7;             // warpgroup: column half
         const int row = tid & 127;           // query row = TMEM lane
         const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-        uint32_t ph_q = 0, ph_s[2] = {0, 0}, ph_pv = 0, ph_x = 0, ph_h[2] = {0, 0}, ph_acc = 0, ph_cs = 0,
+        uint32_t ph_q = 0, ph_s = 0 /* bit k: phase of bar_s[k] */, ph_pvg[2] = {0, 0}, ph_pv = 0, ph_x = 0, ph_h[2] = {0, 0}, ph_acc = 0, ph_cs = 0,
                  ph_wg = 0;
         const float qscale = 0.125f * kLog2e;
         // smem scratch for row statistics after the attention (the embedding tile is free then)
@@ -799,74 +818,102 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 if (!(ok = W.wait(&sh.bar_q, ph_q, 60))) break;
                 tc_fence_after();
                 {
-                    // dims [32 wg, 32 wg + 32): + bq, scale, pack into the first 16 columns of the source
+                    // dims [32 wg, 32 wg + 32): + bq, scale, bf16 into attention-output atom h (128 B
+                    // swizzle), which the head's combine overwrites once its MMAs are done
                     float q[32], b[32];
-                    tmem_ld32(trow + T_Q + 32 * wg, q);
+                    tmem_ld32(trow + T_QACC + 32 * wg, q);
                     ldg32(a.bq + h * 64 + 32 * wg, b);
                     tmem_wait_ld();
                     reg_fence(q);
-                    uint32_t pk[16];
+                    const uint32_t qa = s_abuf + h * 16384;
 #pragma unroll
-                    for (int v = 0; v < 16; ++v)
-                        pk[v] = pack_bf16((q[2 * v] + b[2 * v]) * qscale, (q[2 * v + 1] + b[2 * v + 1]) * qscale);
-                    tmem_st16(trow + T_Q + 32 * wg, pk);
-                    tmem_wait_st();
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const int d = 8 * c + 2 * v;
+                            w[v] = pack_bf16((q[d] + b[d]) * qscale, (q[d + 1] + b[d + 1]) * qscale);
+                        }
+                        st_shared_v4(swz(qa, row, 4 * wg + c), w);
+                    }
                 }
+                fence_proxy_async();
                 tc_fence_before();
                 arrive_mma(&sh.bar_qc);
                 float m_ref = -INFINITY, l_part = 0.f;
-                for (int j = 0; j < nb; ++j) {
-                    if (!(ok = W.wait(&sh.bar_s[j & 1], ph_s[j & 1], 61))) break;
+                for (int j = wg; j < nb; j += 2) {
+                    {
+                        const int sb = j % 6;
+                        uint32_t ph = (ph_s >> sb) & 1u;
+                        if (!(ok = W.wait(&sh.bar_s[sb], ph, 61))) break;
+                        ph_s ^= 1u << sb;
+                    }
                     tc_fence_after();
-                    const uint32_t sbase = trow + ((j & 1) ? T_S1 : T_S0) + 64 * wg;
-                    float s0[32], s1[32];
-                    tmem_ld32(sbase, s0);
-                    tmem_ld32(sbase + 32, s1);
-                    tmem_wait_ld();
-                    reg_fence(s0);
-                    reg_fence(s1);
-                    const int valid = nk - j * 128 - 64 * wg;   // own columns < valid are real tokens
-                    if (valid < 64) {
+                    const uint32_t sbase = trow + T_S0 + 128 * (j % NSB);
+                    const bool first = j < 2;
+                    const int valid = nk - j * 128;   // columns < valid are real tokens
+                    // block maximum, 64 columns at a time
+                    float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+                    #pragma unroll 1
+                    for (int c0 = 0; c0 < 128; c0 += 64) {
+                        float sa[32], sb[32];
+                        tmem_ld32(sbase + c0, sa);
+                        tmem_ld32(sbase + c0 + 32, sb);
+                        tmem_wait_ld();
+                        reg_fence(sa);
+                        reg_fence(sb);
+                        if (valid < c0 + 64) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            if (c >= valid) s0[c] = -INFINITY;
-                            if (c + 32 >= valid) s1[c] = -INFINITY;
+                            for (int c = 0; c < 32; ++c) {
+                                if (c0 + c >= valid) sa[c] = -INFINITY;
+                                if (c0 + 32 + c >= valid) sb[c] = -INFINITY;
+                            }
+                        }
+#pragma unroll
+                        for (int c = 0; c < 32; c += 2) {
+                            m0 = fmaxf(m0, sa[c]);
+                            m1 = fmaxf(m1, sa[c + 1]);
+                            m2 = fmaxf(m2, sb[c]);
+                            m3 = fmaxf(m3, sb[c + 1]);
                         }
                     }
-                    float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-#pragma unroll
-                    for (int c = 0; c < 32; c += 2) {
-                        m0 = fmaxf(m0, s0[c]);
-                        m1 = fmaxf(m1, s0[c + 1]);
-                        m2 = fmaxf(m2, s1[c]);
-                        m3 = fmaxf(m3, s1[c + 1]);
-                    }
-                    // this warpgroup's own running maximum over its token half
                     const float mb = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-                    const bool need = (j == 0) || (mb > m_ref + 8.0f);
+                    const bool need = first || (mb > m_ref + 8.0f);
                     const float m_new = need ? fmaxf(mb, m_ref) : m_ref;
-                    const float f = (j == 0 || m_new == -INFINITY) ? 0.f : ex2(m_ref - m_new);
+                    const float f = (first || m_new == -INFINITY) ? 0.f : ex2(m_ref - m_new);
                     if (need) m_ref = m_new;
                     const float m_use = m_ref == -INFINITY ? 0.f : m_ref;   // no real token yet: P = 0
+                    // exponentials, 32 columns at a time; P of columns [c0, c0+32) goes to columns
+                    // [c0, c0+16), which are read already
                     float la = 0.f, lb = 0.f;
-                    uint32_t pk[32];
+                    #pragma unroll 1
+                    for (int c0 = 0; c0 < 128; c0 += 32) {
+                        float x[32];
+                        tmem_ld32(sbase + c0, x);
+                        tmem_wait_ld();
+                        reg_fence(x);
+                        if (valid < c0 + 32) {
 #pragma unroll
-                    for (int v = 0; v < 16; ++v) {
-                        const float e0 = ex2(s0[2 * v] - m_use), e1 = ex2(s0[2 * v + 1] - m_use);
-                        const float e2 = ex2(s1[2 * v] - m_use), e3 = ex2(s1[2 * v + 1] - m_use);
-                        la += e0 + e1;
-                        lb += e2 + e3;
-                        pk[v] = pack_bf16(e0, e1);
-                        pk[16 + v] = pack_bf16(e2, e3);
+                            for (int c = 0; c < 32; ++c)
+                                if (c0 + c >= valid) x[c] = -INFINITY;
+                        }
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int v = 0; v < 16; ++v) {
+                            const float e0 = ex2(x[2 * v] - m_use), e1 = ex2(x[2 * v + 1] - m_use);
+                            la += e0;
+                            lb += e1;
+                            pk[v] = pack_bf16(e0, e1);
+                        }
+                        tmem_st16(sbase + c0, pk);
                     }
-                    if (j > 0) {   // PV_{j-1} done: the P buffer is free and O stable
-                        if (!(ok = W.wait(&sh.bar_pv, ph_pv, 62))) break;
+                    if (need && !first) l_part *= f;
+                    l_part += la + lb;
+                    if (!first) {   // the PV of this warpgroup's previous block is done: O_g is stable
+                        if (!(ok = W.wait(&sh.bar_pvg[wg], ph_pvg[wg], 62))) break;
                         tc_fence_after();
                     }
-                    tmem_st32(trow + T_P + 32 * wg, pk);
-                    if (need && j > 0) l_part *= f;
-                    l_part += la + lb;
-                    if (j > 0 && __any_sync(0xffffffffu, need)) {
+                    if (!first && __any_sync(0xffffffffu, need)) {
                         const uint32_t ob = trow + (wg ? T_O1 : T_O0);
                         const float g = need ? f : 1.0f;
                         #pragma unroll 1
@@ -883,7 +930,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     }
                     tmem_wait_st();
                     tc_fence_before();
-                    arrive_mma(&sh.bar_p[j & 1]);
+                    arrive_mma(&sh.bar_p[wg]);
                 }
                 if (!ok) break;
                 if (!(ok = W.wait(&sh.bar_pv, ph_pv, 63))) break;   // PV_{nb-1}
@@ -901,6 +948,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 tmem_wait_ld();
                 asm volatile("" : "+r"(mo_bits), "+r"(lo_bits));
                 const float m_oth = __uint_as_float(mo_bits), l_oth = __uint_as_float(lo_bits);
+                const bool has_o1 = nb > 1;   // with one block, warpgroup 1 owned none: O1 is unwritten
                 const float M = fmaxf(m_ref, m_oth);
                 const float f_own = m_ref == -INFINITY ? 0.f : ex2(m_ref - M);
                 const float f_oth = m_oth == -INFINITY ? 0.f : ex2(m_oth - M);
@@ -923,7 +971,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                             #pragma unroll
                             for (int v = 0; v < 4; ++v) {
                                 const int d = c * 8 + 2 * v;
-                                w[v] = pack_bf16(fmaf(o0[d], g0, o1[d] * g1), fmaf(o0[d + 1], g0, o1[d + 1] * g1));
+                                const float b0 = has_o1 ? o1[d] * g1 : 0.f, b1 = has_o1 ? o1[d + 1] * g1 : 0.f;
+                                w[v] = pack_bf16(fmaf(o0[d], g0, b0), fmaf(o0[d + 1], g0, b1));
                             }
                             st_shared_v4(swz(atom, row, 4 * wg + 2 * hh + c), w);
                         }
