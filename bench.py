@@ -52,7 +52,7 @@ def _peaks():
 # dram__bytes_read.sum + dram__bytes_write.sum per decode launch, mean over the five
 # launches of one config-4 shape, captured with ncu on the bench's own launches
 # (profiles/launches_config4_hierarchical_384.md); re-capture when the kernel changes.
-DECODE_DRAM_BYTES_PER_LAUNCH = {}
+DECODE_DRAM_BYTES_PER_LAUNCH = {4: 40.18e6}
 
 
 def decode_flops_per_query(spec: W.DecoderSpec, n_tokens: int) -> float:
