@@ -10,11 +10,13 @@
 // The probes were already decoded with full attention by the dense pass of the
 // level, which exported each probe's per-head softmax maximum m and sum l (in
 // log2 units, against the same bf16 Q and K).  One pass suffices here:
-// S = Q K^T on the tensor cores (TMEM), P = 2^(S - m) / l in registers, and
-// the column sums over each sub-volume's probe rows by a warp transpose-reduce
-// (5 shuffle rounds; lane L ends with columns 4L..4L+3) plus a fixed-order sum
-// over the sub-volume's warps -- deterministic.  Then a radix select of the k
-// largest scores (ties to the smaller token) per sub-volume, in shared memory.
+// S = Q K^T on the tensor cores (TMEM), P = 2^(S - m) / l in registers, summed
+// over the heads in registers (key blocks outer, heads inner: the packed Q of
+// every head stays in TMEM), then per key block the column sums over each
+// sub-volume's probe rows by a warp transpose-reduce (5 shuffle rounds; lane L
+// ends with columns 2L, 2L+1) plus a fixed-order sum over the sub-volume's warps
+// -- deterministic.  Then a radix select of the k largest scores (ties to the
+// smaller token) per sub-volume, in shared memory.
 //
 // Rows: 128 TMEM lanes hold 128 / n_probe sub-volumes' probes (n_probe in
 // {32, 64, 128}).  Roles: warps 0-7 compute in two warpgroups (thread (g, r)
@@ -40,7 +42,11 @@ constexpr int WARP_MMA = 8, WARP_PROD = 9;
 constexpr int SLOT = 16384;
 constexpr int NS = 6;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t T_S0 = 0, T_S1 = 128, T_Q = 448;
+// TMEM: packed bf16 Q of head h in [32h, 32h+32) (up to 8 heads); the S double buffer in
+// [256, 384) and [384, 512), which first holds the fp32 Q projections of up to 4 heads
+// (64 columns each) while they are packed
+constexpr uint32_t T_QP = 0, T_S0 = 256, T_QA = 256;
+constexpr int QROUND = 4;   // heads projected per round
 
 struct SelArgs {
     int C, H, N;
@@ -64,7 +70,7 @@ struct SelArgs {
 
 struct Shared {
     uint64_t full[NS], empty[NS];
-    uint64_t bar_q, bar_s[2], bar_hd;          // MMA commits
+    uint64_t bar_q, bar_s[2];                  // MMA commits
     uint64_t bar_pe, bar_qc, bar_p[2], bar_cs; // compute arrivals (128)
     uint32_t tmem_base;
     int abort;
@@ -147,51 +153,6 @@ __device__ __forceinline__ void warp_colsum64(const float (&v)[64], int lane, fl
     }
 }
 
-// Sum of v over the 32 lanes for each of 128 columns; lane L returns the sums
-// of columns 4L .. 4L+3 (recursive halving: at offset o a lane keeps the upper
-// half of its current columns if (lane & o), and adds its partner's copy).
-__device__ __forceinline__ void warp_colsum128(const float (&v)[128], int lane, float (&out)[4]) {
-    float a64[64];
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-        const bool up = lane & 16;
-        const float send = up ? v[i] : v[i + 64];
-        const float keep = up ? v[i + 64] : v[i];
-        a64[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-    float a32[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const bool up = lane & 8;
-        const float send = up ? a64[i] : a64[i + 32];
-        const float keep = up ? a64[i + 32] : a64[i];
-        a32[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-    float a16[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const bool up = lane & 4;
-        const float send = up ? a32[i] : a32[i + 16];
-        const float keep = up ? a32[i + 16] : a32[i];
-        a16[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-    float a8[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const bool up = lane & 2;
-        const float send = up ? a16[i] : a16[i + 8];
-        const float keep = up ? a16[i + 8] : a16[i];
-        a8[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const bool up = lane & 1;
-        const float send = up ? a8[i] : a8[i + 4];
-        const float keep = up ? a8[i + 4] : a8[i];
-        out[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-    }
-}
-
 __global__ void __launch_bounds__(NT, 1)
 select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_constant__ CUtensorMap tm_k,
                  const SelArgs a) {
@@ -215,7 +176,6 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
         mbar_init(smem_u32(&sh.bar_q), 1);
         mbar_init(smem_u32(&sh.bar_s[0]), 1);
         mbar_init(smem_u32(&sh.bar_s[1]), 1);
-        mbar_init(smem_u32(&sh.bar_hd), 1);
         mbar_init(smem_u32(&sh.bar_pe), NCOMP);
         mbar_init(smem_u32(&sh.bar_qc), NCOMP);
         mbar_init(smem_u32(&sh.bar_p[0]), NCOMP);
@@ -255,15 +215,15 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
             __syncwarp();
             return true;
         };
-        for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x)
-            for (int h = 0; h < H && ok; ++h) {
-                ok = push(&tm_wq64, h * 64, 64 * 128);
-                for (int j = 0; j < nb && ok; ++j) ok = push(&tm_k, h * N + j * 128, SLOT);
-            }
+        for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+            for (int h = 0; h < H && ok; ++h) ok = push(&tm_wq64, h * 64, 64 * 128);
+            for (int j = 0; j < nb && ok; ++j)
+                for (int h = 0; h < H && ok; ++h) ok = push(&tm_k, h * N + j * 128, SLOT);
+        }
     } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------ MMA issue
         if (lane == 0) {
-            uint32_t ring_tail = 0, ph_pe = 0, ph_qc = 0, ph_p[2] = {0, 0}, ph_hd = 0;
+            uint32_t ring_tail = 0, ph_pe = 0, ph_qc = 0, ph_p[2] = {0, 0};
             bool ok = true;
             auto consume = [&](int& slot) -> bool {
                 slot = ring_tail % NS;
@@ -273,42 +233,52 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                 ++ring_tail;
                 return true;
             };
-            auto issue_s = [&](int j) -> bool {
+            // S_i for i = j H + h (key block j, head h) into buffer i mod 2
+            auto issue_s = [&](int i, int h) -> bool {
                 int sl;
                 if (!consume(sl)) return false;
                 const uint64_t db = desc_sw128(s_ring + sl * SLOT);
-                const uint32_t sd = tmem + ((j & 1) ? T_S1 : T_S0);
-                // Q: the warpgroups packed head dims [0,32) into columns [0,16) and [32,64) into [32,48)
+                const uint32_t sd = tmem + T_S0 + 128 * (i & 1);
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(sd, tmem + T_Q + (kk < 2 ? 8 * kk : 32 + 8 * (kk - 2)), db + 2 * kk,
-                           idesc_bf16(128, 128, false), kk > 0);
+                    mma_ts(sd, tmem + T_QP + 32 * h + 8 * kk, db + 2 * kk, idesc_bf16(128, 128, false), kk > 0);
                 mma_commit(smem_u32(&sh.empty[sl]));
-                mma_commit(smem_u32(&sh.bar_s[j & 1]));
+                mma_commit(smem_u32(&sh.bar_s[i & 1]));
                 return true;
             };
             for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
                 if (!(ok = W.wait(&sh.bar_pe, ph_pe, 82))) break;
                 tc_fence_after();
-                for (int h = 0; h < H && ok; ++h) {
-                    int slot;
-                    if (!(ok = consume(slot))) break;
-                    const uint64_t da = desc_sw128(s_pe), db = desc_sw128(s_ring + slot * SLOT);
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ss(tmem + T_Q, da + 2 * kk, db + 2 * kk, idesc_bf16(128, 64, false), kk > 0);
-                    mma_commit(smem_u32(&sh.empty[slot]));
-                    mma_commit(smem_u32(&sh.bar_q));
-                    if (!(ok = W.wait(&sh.bar_qc, ph_qc, 83))) break;
-                    tc_fence_after();
-                    ok = issue_s(0) && (nb < 2 || issue_s(1));
-                    for (int j = 0; j < nb && ok; ++j) {
-                        if (!(ok = W.wait(&sh.bar_p[j & 1], ph_p[j & 1], 84))) break;
-                        tc_fence_after();
-                        if (j + 2 < nb) ok = issue_s(j + 2);
+                // Q projections, QROUND heads at a time into the S buffers' columns
+                for (int h0 = 0; h0 < H && ok; h0 += QROUND) {
+                    for (int h = h0; h < H && h < h0 + QROUND && ok; ++h) {
+                        int slot;
+                        if (!(ok = consume(slot))) break;
+                        const uint64_t da = desc_sw128(s_pe), db = desc_sw128(s_ring + slot * SLOT);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ss(tmem + T_QA + 64 * (h - h0), da + 2 * kk, db + 2 * kk, idesc_bf16(128, 64, false),
+                                   kk > 0);
+                        mma_commit(smem_u32(&sh.empty[slot]));
                     }
                     if (!ok) break;
-                    mma_commit(smem_u32(&sh.bar_hd));
-                    if (!(ok = W.wait(&sh.bar_hd, ph_hd, 85))) break;
+                    mma_commit(smem_u32(&sh.bar_q));
+                    // packed (and the accumulators read) before the next round or the first S overwrites them
+                    if (!(ok = W.wait(&sh.bar_qc, ph_qc, 83))) break;
                     tc_fence_after();
+                }
+                if (!ok) break;
+                const int n_s = nb * H;
+                int hi = 0;   // head of the next S to issue
+                for (int i = 0; i < n_s && i < 2 && ok; ++i) {
+                    ok = issue_s(i, hi);
+                    if (++hi == H) hi = 0;
+                }
+                for (int i = 0; i < n_s && ok; ++i) {
+                    if (!(ok = W.wait(&sh.bar_p[i & 1], ph_p[i & 1], 84))) break;
+                    tc_fence_after();
+                    if (i + 2 < n_s) {
+                        ok = issue_s(i + 2, hi);
+                        if (++hi == H) hi = 0;
+                    }
                 }
             }
         }
@@ -342,18 +312,17 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                 asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(swz(s_pe, row, c)), "r"(w[0]),
                              "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
             }
-            for (int j = tid; j < tpu * N; j += NCOMP) score[j] = 0.f;
             fence_proxy_async();
             arrive(&sh.bar_pe);
             const float* ml = valid ? a.probe_ml + ((size_t)t * np + my_i) * H * 2 : nullptr;
-            int pb = 0;   // partial-sum buffer
-            for (int h = 0; h < H && ok; ++h) {
+            // Q of every head: + bq, scale, bf16 pairs; warpgroup g packs head dims [32g, 32g+32) into
+            // columns [32h + 16g, 32h + 16g + 16)
+            for (int h0 = 0; h0 < H && ok; h0 += QROUND) {
                 if (!(ok = W.wait(&sh.bar_q, ph_q, 86))) break;
                 tc_fence_after();
-                {
-                    // head dims [32 wg, 32 wg + 32): + bq, scale, pack into the first 16 columns of the source
+                for (int h = h0; h < H && h < h0 + QROUND; ++h) {
                     float q[32];
-                    tmem_ld32(trow + T_Q + 32 * wg, q);
+                    tmem_ld32(trow + T_QA + 64 * (h - h0) + 32 * wg, q);
                     tmem_wait_ld();
                     reg_fence(q);
                     uint32_t pk[16];
@@ -361,53 +330,58 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                         const int c0 = h * 64 + 32 * wg + 2 * v;
                         pk[v] = pack_bf16((q[2 * v] + a.bq[c0]) * qscale, (q[2 * v + 1] + a.bq[c0 + 1]) * qscale);
                     }
-                    tmem_st16(trow + T_Q + 32 * wg, pk);
-                    tmem_wait_st();
+                    tmem_st16(trow + T_QP + 32 * h + 16 * wg, pk);
                 }
+                tmem_wait_st();
                 tc_fence_before();
                 arrive(&sh.bar_qc);
-                const float m = valid ? ml[h * 2] : 0.f;
-                const float inv_l = valid ? 1.0f / ml[h * 2 + 1] : 0.f;
-                for (int j = 0; j < nb; ++j) {
-                    if (!(ok = W.wait(&sh.bar_s[j & 1], ph_s[j & 1], 87))) break;
-                    tc_fence_after();
-                    float v[64];
-                    {
-                        const uint32_t sb = trow + ((j & 1) ? T_S1 : T_S0) + 64 * wg;
-                        float s0[32], s1[32];
-                        tmem_ld32(sb, s0);
-                        tmem_ld32(sb + 32, s1);
-                        tmem_wait_ld();
-                        reg_fence(s0);
-                        reg_fence(s1);
-                        tc_fence_before();
-                        arrive(&sh.bar_p[j & 1]);   // this half of S_j consumed
-                        const int vcols = N - j * 128 - 64 * wg;
+            }
+            int pb = 0;   // partial-sum buffer
+            int i = 0;    // S index: key block j, head h -> i = j H + h
+            for (int j = 0; j < nb && ok; ++j) {
+                const int vcols = N - j * 128 - 64 * wg;   // own columns < vcols are real tokens
+                float acc[64];
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            v[c] = (c < vcols) ? ex2(s0[c] - m) * inv_l : 0.f;
-                            v[32 + c] = (32 + c < vcols) ? ex2(s1[c] - m) * inv_l : 0.f;
-                        }
-                    }
-                    float cs[2];
-                    warp_colsum64(v, lane, cs);
-                    float* pw = part + (pb * 8 + warp) * 64;
-                    pw[2 * lane] = cs[0];
-                    pw[2 * lane + 1] = cs[1];
-                    if (!(ok = csync(88))) break;
-                    // column col of sub-volume s: its warps of the column's warpgroup, in order
-                    for (int idx = tid; idx < tpu * 128; idx += NCOMP) {
-                        const int sv = idx >> 7, col = idx & 127;
-                        if (j * 128 + col < N) {
-                            const int g = col >> 6;
-                            const float* pp = part + (pb * 8 + 4 * g + sv * warps_per_tile) * 64 + (col & 63);
-                            float acc = 0.f;
-                            for (int w = 0; w < warps_per_tile; ++w) acc += pp[w * 64];
-                            score[(size_t)sv * N + j * 128 + col] += acc;
-                        }
-                    }
-                    pb ^= 1;
+                for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+                for (int h = 0; h < H; ++h, ++i) {
+                    if (!(ok = W.wait(&sh.bar_s[i & 1], ph_s[i & 1], 87))) break;
+                    tc_fence_after();
+                    const uint32_t sb = trow + T_S0 + 128 * (i & 1) + 64 * wg;
+                    const float m = valid ? ml[h * 2] : 0.f;
+                    const float inv_l = valid ? 1.0f / ml[h * 2 + 1] : 0.f;
+                    float s0[32];
+                    tmem_ld32(sb, s0);
+                    tmem_wait_ld();
+                    reg_fence(s0);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) acc[c] += (c < vcols) ? ex2(s0[c] - m) * inv_l : 0.f;
+                    tmem_ld32(sb + 32, s0);
+                    tmem_wait_ld();
+                    reg_fence(s0);
+                    tc_fence_before();
+                    arrive(&sh.bar_p[i & 1]);   // this half of S_i consumed
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) acc[32 + c] += (32 + c < vcols) ? ex2(s0[c] - m) * inv_l : 0.f;
                 }
+                if (!ok) break;
+                float cs[2];
+                warp_colsum64(acc, lane, cs);
+                float* pw = part + (pb * 8 + warp) * 64;
+                pw[2 * lane] = cs[0];
+                pw[2 * lane + 1] = cs[1];
+                if (!(ok = csync(88))) break;
+                // column col of sub-volume s: its warps of the column's warpgroup, in order
+                for (int idx = tid; idx < tpu * 128; idx += NCOMP) {
+                    const int sv = idx >> 7, col = idx & 127;
+                    if (j * 128 + col < N) {
+                        const int g = col >> 6;
+                        const float* pp = part + (pb * 8 + 4 * g + sv * warps_per_tile) * 64 + (col & 63);
+                        float sum = 0.f;
+                        for (int w = 0; w < warps_per_tile; ++w) sum += pp[w * 64];
+                        score[(size_t)sv * N + j * 128 + col] = sum;
+                    }
+                }
+                pb ^= 1;
             }
             if (!ok) break;
             if (!(ok = csync(89))) break;
