@@ -347,21 +347,28 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                     if (!(ok = W.wait(&sh.bar_s[i & 1], ph_s[i & 1], 87))) break;
                     tc_fence_after();
                     const uint32_t sb = trow + T_S0 + 128 * (i & 1) + 64 * wg;
-                    const float m = valid ? ml[h * 2] : 0.f;
-                    const float inv_l = valid ? 1.0f / ml[h * 2 + 1] : 0.f;
+                    // P = 2^(S - m) / l = 2^(S - m - log2 l); rows without a probe add 2^-inf = 0
+                    const float mo = valid ? ml[h * 2] + __log2f(ml[h * 2 + 1]) : INFINITY;
+                    auto accum = [&](const float (&x)[32], int c0) {
+                        if (vcols >= c0 + 32) {
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) acc[c0 + c] += ex2(x[c] - mo);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) acc[c0 + c] += c0 + c < vcols ? ex2(x[c] - mo) : 0.f;
+                        }
+                    };
                     float s0[32];
                     tmem_ld32(sb, s0);
                     tmem_wait_ld();
                     reg_fence(s0);
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) acc[c] += (c < vcols) ? ex2(s0[c] - m) * inv_l : 0.f;
+                    accum(s0, 0);
                     tmem_ld32(sb + 32, s0);
                     tmem_wait_ld();
                     reg_fence(s0);
                     tc_fence_before();
                     arrive(&sh.bar_p[i & 1]);   // this half of S_i consumed
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) acc[32 + c] += (32 + c < vcols) ? ex2(s0[c] - m) * inv_l : 0.f;
+                    accum(s0, 32);
                 }
                 if (!ok) break;
                 float cs[2];

@@ -260,7 +260,6 @@ __global__ void __launch_bounds__(PO_T) probe_order_kernel(const int32_t* __rest
                                                            int32_t* __restrict__ dense_ml) {
     __shared__ int dpos;
     __shared__ uint64_t key[PO_MAX];
-    __shared__ int64_t vox[PO_MAX];
     __shared__ int wsum[PO_T / 32];
     const int t = blockIdx.x;
     const int base = 8 * tile_off[t];
@@ -289,26 +288,23 @@ __global__ void __launch_bounds__(PO_T) probe_order_kernel(const int32_t* __rest
     for (int e = threadIdx.x; e < cnt; e += PO_T) {
         const int ge = base + e;
         const int64_t v = child_index(plist[ge >> 3], ge & 7, R2);
-        vox[e] = v;
         key[e] = splitmix64((uint64_t)v ^ salt);
     }
     __syncthreads();
-    // each thread owns two consecutive enumeration slots
-    int nonp[2] = {0, 0};
+    // each thread owns two consecutive enumeration slots. Rank = number of smaller keys:
+    // the keys are distinct (splitmix64 and the xor with the salt are bijections of the
+    // 64-bit words and the voxel indices are distinct), so the rule's tie-break to the
+    // smaller voxel never applies. Slots past cnt get the largest key and no position.
+    const int e0 = 2 * threadIdx.x;
+    const uint64_t k0 = e0 < cnt ? key[e0] : ~0ull, k1 = e0 + 1 < cnt ? key[e0 + 1] : ~0ull;
     int rank[2] = {0, 0};
-    for (int q = 0; q < 2; ++q) {
-        const int e = 2 * threadIdx.x + q;
-        if (e >= cnt) continue;
-        const uint64_t ke = key[e];
-        const int64_t ve = vox[e];
-        int r = 0;
-        for (int f2 = 0; f2 < cnt; ++f2) {
-            const uint64_t kf = key[f2];
-            r += (kf < ke) || (kf == ke && vox[f2] < ve);
-        }
-        rank[q] = r;
-        nonp[q] = r >= n_probe;
+    for (int f2 = 0; f2 < cnt; ++f2) {
+        const uint64_t kf = key[f2];
+        rank[0] += kf < k0;
+        rank[1] += kf < k1;
     }
+    int nonp[2];
+    for (int q = 0; q < 2; ++q) nonp[q] = e0 + q < cnt && rank[q] >= n_probe;
     // exclusive scan of the non-probe flags in enumeration order
     const int local = nonp[0] + nonp[1];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
