@@ -248,8 +248,8 @@ VDM_API vdm_status vdm_debug_inject(int32_t mode, int64_t timeout_cycles);
  * and loads half of every weight and key/value tile, which halves the bytes
  * each SM streams per query.  enable = 0 (the default) runs one CTA per
  * 128-query MMA.  Both give the same results up to the order of floating-point
- * sums.  Measured on B200: pairs are faster when attention is short (128
- * tokens), slower for 3072-token attention, and about even on the adaptive
+ * sums.  Measured on B200: pairs are slightly faster when attention is short
+ * (128 tokens), and slower for 3072-token attention and on the adaptive
  * hierarchical workload.  Takes effect for the launches that follow; not
  * thread-safe against concurrent decodes.                                     */
 VDM_API vdm_status vdm_set_cta_pairs(int32_t enable);
