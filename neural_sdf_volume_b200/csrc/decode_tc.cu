@@ -9,11 +9,11 @@
 //
 // Warp roles (320 threads):
 //   warps 0-7  compute: two warpgroups; thread (g, r) owns TMEM lane r and
-//              half g of the row's columns (softmax columns, head dims, hidden
-//              units, LayerNorm columns), so every SM sub-partition runs two
-//              compute warps; each warpgroup runs its own online softmax over
-//              its half of every key block (own maximum, sum and O
-//              accumulator), and the halves combine once per head;
+//              half g of the row's columns (head dims, hidden units, LayerNorm
+//              columns), so every SM sub-partition runs two compute warps; in
+//              the attention warpgroup g owns the key blocks j = g mod 2 and
+//              runs its own online softmax over them (own maximum, sum and O
+//              accumulator); the two combine once per head;
 //   warp 8     MMA issue (the whole warp runs the loop; one elected lane issues);
 //   warp 9     producer: TMA loads of weights and of contiguous K/V blocks,
 //              cp.async gathers of a sub-volume's selected K/V rows (each lane's
@@ -22,15 +22,16 @@
 // Compiled twice per width: one CTA per 128-row MMA, or (cta_group::2) a CTA
 // pair of a cluster per 256-row MMA, each CTA holding half of every B tile.
 //
-// Split-packed A operands: Q and the GELU output are produced by the two
-// warpgroups, each packing its half (bf16 pairs) into the start of its own
-// fp32 source columns (so neither overwrites the other's unread source); the
-// k-step q of 16 elements then sits at column  g*W/2 + (16q mod W/2)/2  with
-// g = 16q / (W/2) for a W-wide block.
+// Split-packed A operand: the GELU output is produced by the two warpgroups,
+// each packing its half (bf16 pairs) into the start of its own fp32 source
+// columns (so neither overwrites the other's unread source); the k-step q of
+// 16 elements then sits at column  g*W/2 + (16q mod W/2)/2  with g = 16q / (W/2)
+// for a W-wide block.  The softmax probabilities P_j are packed in place, each
+// 32-column chunk's bf16 pairs in the chunk's first 16 columns.
 //
 // Per tile:
-//   PE (bf16 smem) ; per head h: Q_h = PE Wq_h^T (TMEM) -> bf16 in TMEM;
-//   Q_h -> bf16 smem (attention-output atom h, free until the head's combine);
+//   PE (bf16 smem) ; per head h: Q_h = PE Wq_h^T (fp32 in TMEM) -> + bq, scaled,
+//   bf16 in smem (attention-output atom h, free until the head's combine);
 //   per 128-token block j, owned by warpgroup g = j mod 2: S_j = Q_h K_j^T into
 //   S_{j mod 3} ; softmax of the block -> P_j (bf16, in place) ; O_g += P_j V_j ;
 //   end of head: combine the two (max, sum, O_g) -> a[:, h] (bf16 smem).
