@@ -112,12 +112,6 @@ __device__ __forceinline__ void reg_fence(float (&v)[32]) {
                    "+f"(v[21]), "+f"(v[22]), "+f"(v[23]), "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]),
                    "+f"(v[28]), "+f"(v[29]), "+f"(v[30]), "+f"(v[31]));
 }
-// load 32 columns and wait for them
-__device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, float (&v)[32]) {
-    tmem_ld32(taddr, v);
-    tmem_wait_ld();
-    reg_fence(v);
-}
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     asm volatile(
@@ -243,10 +237,6 @@ __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
-// arrival that orders nothing itself: for forwarding a phase that already completed
-__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_bar) {
-    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
-}
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -264,16 +254,6 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// TMA load into this CTA's shared memory whose completion is counted on an
-// mbarrier of either CTA of the pair (no multicast)
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* tm, int x, int y,
-                                                 uint32_t cluster_bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(cluster_bar)
-        : "memory");
-}
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
                  : "memory");
@@ -284,28 +264,8 @@ __device__ __forceinline__ void tmem_relinquish_pair() {
 __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
+// Pair forms, warp-wide (one elected lane issues):
 // D(tmem, both CTAs) (+)= A(smem desc, both CTAs) * B(smem desc, N/2 rows in each CTA)
-__device__ __forceinline__ void mma_ss_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accum));
-}
-// D(tmem, both CTAs) (+)= A(tmem, both CTAs) * B(smem desc, N/2 rows in each CTA)
-__device__ __forceinline__ void mma_ts_pair(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                            uint32_t accum) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum));
-}
-// arrive on an mbarrier (shared::cluster address, either CTA) once the pair's MMAs issued so far completed
-__device__ __forceinline__ void mma_commit_pair(uint32_t cluster_bar) {
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(cluster_bar)
-                 : "memory");
-}
 __device__ __forceinline__ void mma_ss_pair_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum) {
     asm volatile(
         "{\n\t.reg .pred p, e;\n\t"
@@ -314,6 +274,7 @@ __device__ __forceinline__ void mma_ss_pair_w(uint32_t d, uint64_t a, uint64_t b
         "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accum));
 }
+// D(tmem, both CTAs) (+)= A(tmem, both CTAs) * B(smem desc, N/2 rows in each CTA)
 __device__ __forceinline__ void mma_ts_pair_w(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
                                               uint32_t accum) {
     asm volatile(
@@ -323,12 +284,14 @@ __device__ __forceinline__ void mma_ts_pair_w(uint32_t d, uint32_t a_tmem, uint6
         "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
         ::"r"(d), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum));
 }
+// arrive on an mbarrier (shared::cluster address, either CTA) once the pair's MMAs issued so far completed
 __device__ __forceinline__ void mma_commit_pair_w(uint32_t cluster_bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
         "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(cluster_bar)
         : "memory");
 }
+// arrival that orders nothing itself: for forwarding a phase that already completed
 __device__ __forceinline__ void mbar_arrive_cluster_relaxed_w(uint32_t cluster_bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
@@ -397,8 +360,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
-__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
 }  // namespace ptx
 }  // namespace vdm
