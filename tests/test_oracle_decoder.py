@@ -227,3 +227,39 @@ def test_sphere_sdf_closed_forms():
     np.testing.assert_allclose(D.field(p, dec, sp, 0.01), np.array(want) + 0.01 * np.tanh(dec),
                                atol=1e-15)
     assert np.all(D.field(p, dec, None, 0.01) == dec)
+
+
+def test_decoder_query_layernorm_before_mlp_closed_form():
+    # query_ln = True, attention silent (V = 0, Wo = 0): x1 = q = PE(p) on lanes 0..50.
+    # W1 = W2 = I: x2 = x1 + GELU(LN1(x1)), dec = LN2(x2)[0].  At p = (0.5, 0, 0) the
+    # embedding is worked out by hand: lane 0 = 0.5, sin(pi/2) = 1 at lane 3, sin(2^k pi/2)
+    # = 0 for k >= 1, cos(pi/2) = 0 at lane 27, cos(pi) = -1 at lane 28, cos(2^k pi/2) = 1
+    # at lanes 29..34 (k >= 2), and y = z = 0 give sin = 0, cos = 1 at lanes 35..50.
+    C = 64
+    w = _zero_weights(C, 64)
+    w["Wq"][:51, :51] = np.eye(51)
+    w["W1"][:] = np.eye(64); w["W2"][:] = np.eye(64)
+    w["w_head"][0] = 1.0
+    x1 = np.zeros(64)
+    x1[0] = 0.5
+    x1[3] = 1.0
+    x1[28] = -1.0
+    x1[29:35] = 1.0
+    x1[35:51] = 1.0
+    np.testing.assert_allclose(D.fourier_embed(np.array([[0.5, 0.0, 0.0]]))[0], x1, atol=1e-14)
+
+    def ln(v):   # biased variance, eps 1e-5, unit gain, zero shift
+        m = v.mean()
+        return (v - m) / math.sqrt(((v - m) ** 2).mean() + 1e-5)
+
+    def gelu(v):
+        return v * norm.cdf(v)
+
+    want = ln(x1 + gelu(ln(x1)))[0]
+    K = np.zeros((1, 2, 64)); V = np.zeros((1, 2, 64))
+    got = D.decode_points(np.array([[0.5, 0.0, 0.0]]), K, V, w, query_ln=True)[0]
+    assert got == pytest.approx(want, abs=1e-12)
+    # the case separates the plausible slips: LN1 dropped, or the residual taken after LN1
+    # (x2 = LN1(x1) + MLP, post-norm style)
+    for slip in (ln(x1 + gelu(x1)), ln(ln(x1) + gelu(ln(x1)))):
+        assert abs(slip[0] - want) > 1e-2
