@@ -55,3 +55,19 @@ def hierarchical_volume(K, V, w, r0: int, n_levels: int, query_ln: bool, spheres
     for lv, e in extras.items():
         res["levels"][lv].update({k: v for k, v in e.items() if k != "values"})
     return res
+
+
+def compare_volumes(a: np.ndarray, b: np.ndarray) -> Dict:
+    """Counts behind the volume IoU of two fields on the same grid (aipaper.cc
+    summary, section 5 "Evaluation Metrics": V-IoU of the inside sets; Table 3
+    reports it per acceleration).  Inside means ``f < 0``.  ``max_abs_diff`` is
+    computed in the fields' own precision."""
+    a = np.asarray(a).ravel()
+    b = np.asarray(b).ravel()
+    ia, ib = a < 0, b < 0
+    both = int((ia & ib).sum())
+    union = int(ia.sum()) + int(ib.sum()) - both
+    return {"inside_a": int(ia.sum()), "inside_b": int(ib.sum()), "inside_both": both,
+            "same_sign": int((ia == ib).sum()),
+            "v_iou": both / union if union else 1.0,
+            "max_abs_diff": float(np.abs(a - b).max()) if a.size else 0.0}
