@@ -36,12 +36,21 @@
  *   - Pointers named d_* / documented "device" are CUDA device memory owned by
  *     the caller; the library never allocates device memory.  Host pointers
  *     are documented as such.
- *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL =
- *     legacy default stream), except vdm_decode_hierarchical which reads one
- *     small count back per level (documented there).
+ *   - Work is ordered on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  vdm_precompute_kv returns without waiting.  The decode and
+ *     selection calls synchronise `stream` before they return, so that the
+ *     status of their device-side waits reaches the caller who made the call
+ *     (vdm_decode_hierarchical also reads counts back once per level).
  *   - Errors are returned as vdm_status; nothing aborts, throws across the
  *     ABI or traps on the device.  vdm_last_error() gives a thread-local
- *     message for the last failing call.  Launch failures return VDM_ERR_CUDA.
+ *     message for the last failing call.  Launch failures return VDM_ERR_CUDA;
+ *     a tensor-core kernel whose bounded wait expired returns VDM_ERR_TIMEOUT
+ *     from the call that launched it.
+ *   - Shared device state: the device error word and, for C = 512 decoders on
+ *     the tensor cores, a 20 MiB area that holds half of the residual stream
+ *     while the MLP runs, are global to the library on each device.  Decode
+ *     calls that overlap on the GPU (different streams or host threads, same
+ *     device) race on them: issue decodes of one device on one stream.
  *   - Results are bit-identical run to run (no floating-point atomics).
  *   - Limits: head dim 64; C in {64, 128, 256, 512}; F a multiple of 64 and
  *     <= 4096; 1 <= N <= 8192; B >= 1.  Other shapes: VDM_ERR_UNSUPPORTED.
@@ -126,7 +135,8 @@ VDM_API vdm_status vdm_precompute_kv(const vdm_decoder* dec, const float* d_z, i
  *             the grid_R^3 grid in linear order (then M must be grid_R^3)
  *   analytic  host pointer or NULL (raw decoder output)
  *   d_out     [B][M] float32
- * M = 0 is a no-op.  Errors: INVALID_ARG, UNSUPPORTED, CUDA.                */
+ * M = 0 is a no-op.  Returns after the decode has finished on `stream`.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA, TIMEOUT.                          */
 VDM_API vdm_status vdm_decode_dense(const vdm_decoder* dec, const void* d_k, const void* d_v,
                             int32_t B, int32_t N, const float* d_xyz, int64_t M, int32_t grid_R,
                             const vdm_analytic* analytic, float* d_out, vdm_stream stream);
@@ -142,7 +152,8 @@ VDM_API vdm_status vdm_decode_dense(const vdm_decoder* dec, const void* d_k, con
  *   d_sel_out     [T][top_k] int32 (device)
  *   d_score_out   [T][N] float32 or NULL
  * Sub-volumes with no probe select tokens 0..top_k-1.  top_k >= N selects
- * every token.  Errors: INVALID_ARG, UNSUPPORTED (N, top_k > 8192), CUDA.   */
+ * every token.  Returns after the selection has finished on `stream`.
+ * Errors: INVALID_ARG, UNSUPPORTED (N, top_k > 8192), CUDA, TIMEOUT.        */
 VDM_API vdm_status vdm_select_kv(const vdm_decoder* dec, const void* d_k, const void* d_v, int32_t N,
                          const float* d_probe_xyz, const int32_t* d_tile_off, int32_t T,
                          int64_t P_total, int32_t top_k, int32_t* d_sel_out, float* d_score_out,
@@ -174,7 +185,10 @@ typedef struct {
 
 /* Optional per-level copies for testing (all device pointers, nullable; a
  * NULL entry skips that copy).  Shapes are handled one after the other, so
- * each array holds shape b at offset b * (its per-shape size).             */
+ * each array holds shape b at offset b * (its per-shape size).  "Sub-volume i"
+ * below is entry i of tile_ids: the i-th non-empty 8^3 sub-volume of the fine
+ * level in ascending sub-volume order.  Entries for i >= max_tiles are not
+ * written.                                                                  */
 typedef struct {
     float* grid[VDM_MAX_LEVELS];        /* [B][R_l^3] dense field of level l */
     uint64_t* active[VDM_MAX_LEVELS];   /* [B][(R_l/4)^3] refine mask of level
@@ -184,10 +198,28 @@ typedef struct {
     float* dec[VDM_MAX_LEVELS];         /* [B][R_l^3] raw decoder output at the
                                            voxels decoded at level l; other
                                            voxels are left untouched         */
-    int32_t* tile_ids[VDM_MAX_LEVELS];  /* [B][max_tiles] ids of sub-volumes
-                                           with a selection (adaptive)       */
-    int32_t* sel[VDM_MAX_LEVELS];       /* [B][max_tiles][top_k] their tokens */
-    int64_t max_tiles;                  /* capacity of tile_ids / sel        */
+    int32_t* tile_ids[VDM_MAX_LEVELS];  /* [B][max_tiles] sub-volume ids (linear
+                                           index of the 8^3 tile at level l)
+                                           of the non-empty sub-volumes       */
+    int32_t* sel[VDM_MAX_LEVELS];       /* [B][max_tiles][top_k] kept tokens of
+                                           sub-volume i (rows of sub-volumes
+                                           without a selection: untouched)   */
+    int64_t max_tiles;                  /* capacity of the per-sub-volume rows */
+    int32_t* probes[VDM_MAX_LEVELS];    /* [B][max_tiles][n_probe] fine voxel
+                                           indices of the probes of sub-volume
+                                           i in rank order (all its queries if
+                                           it has <= n_probe), -1 padded      */
+    float* scores[VDM_MAX_LEVELS];      /* [B][max_tiles][N] token scores of
+                                           sub-volume i (rows of sub-volumes
+                                           without a selection: untouched)   */
+    float* attn[VDM_MAX_LEVELS];        /* [B][ceil(R_l^3/attn_stride)][C]
+                                           attention output a (heads
+                                           concatenated, before Wo) at every
+                                           decoded voxel v of level l with
+                                           v % attn_stride == 0, in row
+                                           v / attn_stride; other rows are
+                                           left untouched                    */
+    int64_t attn_stride;                /* >= 1 when any attn[l] is set       */
 } vdm_hier_debug;
 
 /* Workspace bytes needed by vdm_decode_hierarchical (host output).         */
@@ -205,7 +237,8 @@ VDM_API vdm_status vdm_hierarchical_workspace_size(const vdm_decoder* dec, const
  *   d_ws/ws_bytes  device workspace >= vdm_hierarchical_workspace_size
  *   stats    host, B entries, nullable;  debug  host, nullable
  * Synchronisation: after each level's marking the call copies two counts to
- * the host and synchronises `stream` (one round trip per level).
+ * the host and synchronises `stream` (one round trip per level), and it
+ * synchronises once more at the end to read the device error status.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA, TIMEOUT.              */
 VDM_API vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, const void* d_v,
                                    int32_t B, int32_t N, const vdm_hier_params* p,
@@ -226,6 +259,8 @@ VDM_API vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d
  *     which is rejected; 64 -> 128 -> 256 without adaptive KV about 18 MiB).
  *   - All calls on a device share that scratch: calls that overlap on the GPU
  *     race; issue them one after another on one stream.
+ *   - Like vdm_decode_hierarchical, the call synchronises `stream` once per
+ *     level and once at the end.
  *   - The first call on each device looks up the scratch address (no
  *     allocation); make that first call before any stream capture.          */
 VDM_API vdm_status vdm_decode_hierarchical_noalloc(const vdm_decoder* dec, const void* d_k,
@@ -235,12 +270,81 @@ VDM_API vdm_status vdm_decode_hierarchical_noalloc(const vdm_decoder* dec, const
                                                    vdm_hier_stats* stats,
                                                    const vdm_hier_debug* debug, vdm_stream stream);
 
-/* Test hook for failure detection (not needed for decoding).  mode 1 makes
- * the next tensor-core decode launch withhold one completion signal, so its
- * warps run into their bounded waits; `timeout_cycles` (> 0) shortens those
- * waits.  The decode then reports VDM_ERR_TIMEOUT at its next check (the
- * hierarchical call checks after each level) and the CUDA context stays
- * usable.  mode 0 restores normal operation.                               */
+/* One level step of hierarchical volume decoding without the decoder
+ * (section 4.1 item 1, steps 2-3, and the inherit fill), for callers that run
+ * their own decoder on the refined voxels:
+ *   mark: voxels with a sign change in their 3x3x3 neighbourhood or
+ *   |f| < float32(4 / R); dilate once (3x3x3); compact the refined voxels;
+ *   fill: every voxel of the (2R)^3 grid takes its parent's value (decoding
+ *   the children of refined voxels then overwrites them).
+ *   d_f        [R^3] float32 (device, 16-byte aligned), R % 4 == 0, R <= 512
+ *   d_f_fine   [(2R)^3] float32 (device, 16-byte aligned) or NULL (no fill)
+ *   d_mask     [(R/4)^3] uint64 blocked refine mask (layout of vdm_hier_debug)
+ *   d_parents  [R^3] int32 or NULL: refined voxels' linear indices, grouped by
+ *              4^3 block in block order, ascending bit order inside a block
+ *   d_counts   [2] int32 (device): refined voxels, non-empty 4^3 blocks
+ *   d_ws/ws_bytes  device workspace >= vdm_refine_workspace_size(R)
+ * Asynchronous on `stream`.  Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+VDM_API vdm_status vdm_refine_workspace_size(int32_t R, size_t* bytes);
+VDM_API vdm_status vdm_refine_level(const float* d_f, int32_t R, float* d_f_fine, uint64_t* d_mask,
+                                    int32_t* d_parents, int32_t* d_counts, void* d_ws, size_t ws_bytes,
+                                    vdm_stream stream);
+
+/* Comparison of two fields sampled on the same grid, for accuracy reports
+ * (aipaper.cc summary, section 5 "Evaluation Metrics": volume IoU of the
+ * inside sets; Table 3 reports it for each acceleration of the decoder).
+ * Inside means f < 0.  One pass over both arrays.
+ *   d_a, d_b  [n] float32 (device)
+ *   d_out     [5] uint64 (device, 8-byte aligned): number of voxels inside
+ *             a, inside b, inside both, with the same sign in a and b, and
+ *             the largest |a - b| as float32 bits in the low 32 bits
+ * V-IoU = d_out[2] / (d_out[0] + d_out[1] - d_out[2]); sign agreement =
+ * d_out[3] / n.  Counts are exact integers; asynchronous on `stream`.
+ * Errors: INVALID_ARG, CUDA.                                                */
+VDM_API vdm_status vdm_compare_volumes(const float* d_a, const float* d_b, int64_t n, uint64_t* d_out,
+                                       vdm_stream stream);
+
+/* Surface extraction (techwalker article, section 1: the pipeline's last
+ * stage after VAE decoding): marching cubes on the samples of a decoded
+ * R^3 volume (voxel centres, as above), visiting only the 8^3-cube blocks
+ * near voxels with a 26-neighbour of the other sign; the mesh equals marching
+ * cubes over every cube of the grid.  Inside is f < 0.
+ *   d_f            [R^3] float32 (device, 16-byte aligned), R % 8 == 0, R <= 1024
+ *   d_vertices     [max_vertices][3] float32 xyz (device)
+ *   d_triangles    [max_triangles][3] int32 vertex indices (device); triangle
+ *                  normals (right-hand rule) point to f > 0
+ *   n_vertices, n_triangles  host outputs: the mesh's sizes (written even when
+ *                  the capacity is too small, which returns VDM_ERR_WORKSPACE and
+ *                  writes nothing else; capacities of 0 query the sizes)
+ *   d_ws/ws_bytes  device workspace >= vdm_surface_workspace_size(R)
+ * Case rules (no memorised table; the 256 cases are generated from them): a
+ * face with two sign changes gets one segment; with four, two segments that
+ * each cut off one inside corner; loops are fanned from their first vertex
+ * (loop order from the smallest edge id) with no fan diagonal inside a face.
+ * Edge e = 4 a + 2 u + v runs along axis a between the corners whose other
+ * two coordinates are (u, v); corner c = 4 ci + 2 cj + ck.  Vertex on the
+ * crossed edge from sample p0 to p0 + e_a: p0 + t h e_a, t = f0 / (f0 - f1),
+ * h = 2 / R.  Order: samples (vertex owners, vertices in axis order) and cubes
+ * (by minimum corner; triangles in loop and fan order) by 8^3 block in linear
+ * block order, then linear order inside the block.
+ * Synchronises `stream` twice (sizes, then the mesh).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA, INTERNAL.              */
+VDM_API vdm_status vdm_surface_workspace_size(int32_t R, size_t* bytes);
+VDM_API vdm_status vdm_extract_surface(const float* d_f, int32_t R, float* d_vertices, int64_t max_vertices,
+                                       int32_t* d_triangles, int64_t max_triangles, int64_t* n_vertices,
+                                       int64_t* n_triangles, void* d_ws, size_t ws_bytes, vdm_stream stream);
+/* The generated case table (host outputs, for inspection and tests):
+ * ntri[256] triangles per sign pattern (bit c = corner c inside) and
+ * tri[256][5][3] their edge ids.                                            */
+VDM_API vdm_status vdm_surface_case_table(uint8_t* ntri, uint8_t* tri);
+
+/* Test hook for failure detection (not needed for decoding).  mode n >= 1
+ * makes the n-th tensor-core decode launch from now on (1 = the next one)
+ * withhold one completion signal, so its warps run into their bounded waits;
+ * `timeout_cycles` (> 0) shortens those waits.  The call that made that
+ * launch returns VDM_ERR_TIMEOUT (a hierarchical call checks after each
+ * level's marking and at its end) and the CUDA context stays usable.  mode 0
+ * restores normal operation.                                                */
 VDM_API vdm_status vdm_debug_inject(int32_t mode, int64_t timeout_cycles);
 
 /* Tensor-core decoding on CTA pairs: with enable = 1, each 256-query MMA runs
@@ -271,7 +375,7 @@ VDM_API vdm_status vdm_profile_end(vdm_profile* out);
 
 VDM_API const char* vdm_status_string(vdm_status s);
 VDM_API const char* vdm_last_error(void);   /* thread-local message of the last error */
-VDM_API int32_t vdm_abi_version(void);      /* 1                                      */
+VDM_API int32_t vdm_abi_version(void);      /* 2                                      */
 
 #ifdef __cplusplus
 }

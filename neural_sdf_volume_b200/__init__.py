@@ -35,7 +35,10 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "workspace", 4: "
 
 EXPORTS = ("vdm_precompute_kv", "vdm_decode_dense", "vdm_select_kv",
            "vdm_hierarchical_workspace_size", "vdm_decode_hierarchical",
-           "vdm_decode_hierarchical_noalloc", "vdm_debug_inject", "vdm_set_cta_pairs",
+           "vdm_decode_hierarchical_noalloc", "vdm_compare_volumes",
+           "vdm_surface_workspace_size", "vdm_extract_surface", "vdm_surface_case_table",
+           "vdm_refine_workspace_size", "vdm_refine_level",
+           "vdm_debug_inject", "vdm_set_cta_pairs",
            "vdm_profile_begin", "vdm_profile_end",
            "vdm_status_string", "vdm_last_error", "vdm_abi_version")
 PROF_CLASSES = ("kv", "decode", "select", "mark", "scan", "list", "fill", "probe")
@@ -77,7 +80,11 @@ class CHierStats(C.Structure):
 class CHierDebug(C.Structure):
     _fields_ = [("grid", C.c_void_p * MAX_LEVELS), ("active", C.c_void_p * MAX_LEVELS),
                 ("dec", C.c_void_p * MAX_LEVELS), ("tile_ids", C.c_void_p * MAX_LEVELS),
-                ("sel", C.c_void_p * MAX_LEVELS), ("max_tiles", C.c_int64)]
+                ("sel", C.c_void_p * MAX_LEVELS), ("max_tiles", C.c_int64),
+                ("probes", C.c_void_p * MAX_LEVELS), ("scores", C.c_void_p * MAX_LEVELS),
+                ("attn", C.c_void_p * MAX_LEVELS), ("attn_stride", C.c_int64)]
+
+DEBUG_ARRAYS = ("grid", "active", "dec", "tile_ids", "sel", "probes", "scores", "attn")
 
 
 class CProfile(C.Structure):
@@ -98,6 +105,13 @@ _lib.vdm_decode_hierarchical.argtypes = [C.POINTER(CDecoder), _vp, _vp, _i32, _i
 _lib.vdm_decode_hierarchical_noalloc.argtypes = [C.POINTER(CDecoder), _vp, _vp, _i32, _i32,
                                                  C.POINTER(CHierParams), C.POINTER(CAnalytic), _vp,
                                                  C.POINTER(CHierStats), C.POINTER(CHierDebug), _vp]
+_lib.vdm_compare_volumes.argtypes = [_vp, _vp, _i64, _vp, _vp]
+_lib.vdm_surface_workspace_size.argtypes = [_i32, C.POINTER(C.c_size_t)]
+_lib.vdm_extract_surface.argtypes = [_vp, _i32, _vp, _i64, _vp, _i64, C.POINTER(C.c_int64),
+                                     C.POINTER(C.c_int64), _vp, C.c_size_t, _vp]
+_lib.vdm_surface_case_table.argtypes = [_vp, _vp]
+_lib.vdm_refine_workspace_size.argtypes = [_i32, C.POINTER(C.c_size_t)]
+_lib.vdm_refine_level.argtypes = [_vp, _i32, _vp, _vp, _vp, _vp, _vp, C.c_size_t, _vp]
 _lib.vdm_debug_inject.argtypes = [_i32, _i64]
 _lib.vdm_debug_inject.restype = C.c_int
 _lib.vdm_set_cta_pairs.argtypes = [_i32]
@@ -106,7 +120,9 @@ _lib.vdm_profile_begin.argtypes = []
 _lib.vdm_profile_end.argtypes = [C.POINTER(CProfile)]
 for _f in ("vdm_precompute_kv", "vdm_decode_dense", "vdm_select_kv",
            "vdm_hierarchical_workspace_size", "vdm_decode_hierarchical",
-           "vdm_decode_hierarchical_noalloc", "vdm_profile_begin", "vdm_profile_end"):
+           "vdm_decode_hierarchical_noalloc", "vdm_compare_volumes", "vdm_profile_begin",
+           "vdm_profile_end", "vdm_surface_workspace_size", "vdm_extract_surface",
+           "vdm_surface_case_table", "vdm_refine_workspace_size", "vdm_refine_level"):
     getattr(_lib, _f).restype = C.c_int
 _lib.vdm_status_string.argtypes = [C.c_int]
 _lib.vdm_status_string.restype = C.c_char_p
@@ -251,8 +267,8 @@ def vdm_decode_hierarchical(dec: Decoder, K, V, params: CHierParams, spheres=Non
     """Coarse-to-fine decoding of B shapes -> (grid ``[B,Rf,Rf,Rf]``, per-shape stats).
 
     ``debug`` is an optional dict of device tensors keyed like ``vdm_hier_debug``
-    (``grid``, ``active``, ``dec``, ``tile_ids``, ``sel``: lists indexed by level,
-    plus ``max_tiles``)."""
+    (``grid``, ``active``, ``dec``, ``tile_ids``, ``sel``, ``probes``, ``scores``,
+    ``attn``: lists indexed by level, plus ``max_tiles`` and ``attn_stride``)."""
     torch = _torch()
     B, H, N, _ = K.shape
     Rf = params.r0 << (params.n_levels - 1)
@@ -265,11 +281,12 @@ def vdm_decode_hierarchical(dec: Decoder, K, V, params: CHierParams, spheres=Non
     dbg = None
     if debug is not None:
         dbg = CHierDebug()
-        for key in ("grid", "active", "dec", "tile_ids", "sel"):
+        for key in DEBUG_ARRAYS:
             arr = getattr(dbg, key)
             for l, t in enumerate(debug.get(key, [])):
                 arr[l] = _ptr(t) or 0
         dbg.max_tiles = int(debug.get("max_tiles", 0))
+        dbg.attn_stride = int(debug.get("attn_stride", 0))
     cd = dec.cstruct()
     an = _analytic(spheres, dec_scale)
     _check(_lib.vdm_decode_hierarchical(C.byref(cd), K.data_ptr(), V.data_ptr(), B, N,
@@ -299,6 +316,85 @@ def vdm_decode_hierarchical_noalloc(dec: Decoder, K, V, params: CHierParams, sph
                                                 C.byref(params), C.byref(an) if an else None,
                                                 out.data_ptr(), stats, None, _stream(stream)))
     return out
+
+
+def vdm_compare_volumes(a, b, stream=None) -> Dict[str, float]:
+    """Counts of two same-shaped float32 device volumes: inside each (f < 0),
+    inside both, same sign, and the largest |a - b|; plus V-IoU and sign
+    agreement derived from them."""
+    torch = _torch()
+    assert a.shape == b.shape and a.dtype == torch.float32 and b.dtype == torch.float32
+    a = a.contiguous()
+    b = b.contiguous()
+    out = torch.empty((5,), device=a.device, dtype=torch.int64)
+    _check(_lib.vdm_compare_volumes(a.data_ptr(), b.data_ptr(), a.numel(), out.data_ptr(),
+                                    _stream(stream)))
+    c = out.cpu().numpy().astype(np.uint64)
+    n = int(a.numel())
+    in_a, in_b, both, same = (int(x) for x in c[:4])
+    union = in_a + in_b - both
+    dmax = float(np.array([int(c[4]) & 0xFFFFFFFF], np.uint32).view(np.float32)[0])
+    return {"n": n, "inside_a": in_a, "inside_b": in_b, "inside_both": both, "same_sign": same,
+            "v_iou": both / union if union else 1.0, "sign_agreement": same / n if n else 1.0,
+            "max_abs_diff": dmax}
+
+
+def vdm_refine_workspace_size(R: int) -> int:
+    n = C.c_size_t(0)
+    _check(_lib.vdm_refine_workspace_size(R, C.byref(n)))
+    return int(n.value)
+
+
+def vdm_refine_level(f, fine=None, parents=None, workspace=None, stream=None):
+    """One level step without the decoder: ``f[R,R,R]`` -> (refine mask words
+    ``[(R/4)^3]`` int64 view of uint64, device counts ``[2]``); fills ``fine``
+    ``[2R,2R,2R]`` with parent values and ``parents`` ``[R^3]`` when given."""
+    torch = _torch()
+    R = int(f.shape[-1])
+    if workspace is None:
+        workspace = torch.empty((vdm_refine_workspace_size(R),), device=f.device, dtype=torch.uint8)
+    mask = torch.empty(((R // 4) ** 3,), device=f.device, dtype=torch.int64)
+    counts = torch.zeros((2,), device=f.device, dtype=torch.int32)
+    _check(_lib.vdm_refine_level(f.data_ptr(), R, _ptr(fine), mask.data_ptr(), _ptr(parents),
+                                 counts.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                 _stream(stream)))
+    return mask, counts
+
+
+def vdm_surface_workspace_size(R: int) -> int:
+    n = C.c_size_t(0)
+    _check(_lib.vdm_surface_workspace_size(R, C.byref(n)))
+    return int(n.value)
+
+
+def vdm_extract_surface(f, workspace=None, stream=None):
+    """Marching-cubes mesh of a float32 device volume ``f[R,R,R]``:
+    ``(vertices [V,3] float32, triangles [T,3] int32)`` on the device."""
+    torch = _torch()
+    R = int(f.shape[-1])
+    f = f.contiguous()
+    if workspace is None:
+        workspace = torch.empty((vdm_surface_workspace_size(R),), device=f.device, dtype=torch.uint8)
+    nv, nt = C.c_int64(0), C.c_int64(0)
+    st = _lib.vdm_extract_surface(f.data_ptr(), R, None, 0, None, 0, C.byref(nv), C.byref(nt),
+                                  workspace.data_ptr(), workspace.numel(), _stream(stream))
+    if st not in (0, 3):
+        _check(st)
+    verts = torch.empty((nv.value, 3), device=f.device, dtype=torch.float32)
+    tris = torch.empty((nt.value, 3), device=f.device, dtype=torch.int32)
+    if nv.value or nt.value:
+        _check(_lib.vdm_extract_surface(f.data_ptr(), R, verts.data_ptr(), nv.value, tris.data_ptr(),
+                                        nt.value, C.byref(nv), C.byref(nt), workspace.data_ptr(),
+                                        workspace.numel(), _stream(stream)))
+    return verts, tris
+
+
+def vdm_surface_case_table():
+    """The library's generated marching-cubes case table: ``(ntri[256], tri[256,5,3])``."""
+    ntri = np.zeros(256, np.uint8)
+    tri = np.zeros((256, 5, 3), np.uint8)
+    _check(_lib.vdm_surface_case_table(ntri.ctypes.data, tri.ctypes.data))
+    return ntri, tri
 
 
 def vdm_debug_inject(mode: int, timeout_cycles: int = 0):

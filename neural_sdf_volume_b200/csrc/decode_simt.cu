@@ -311,6 +311,14 @@ __global__ void __launch_bounds__(NT) decode_kernel(DecodeArgs a) {
         for (int d = 0; d < 8; ++d) s.buf[r8 * ldc + h * kHeadDim + j8 * 8 + d] = o[d] * inv;
     }
     __syncthreads();
+    if (a.attn_out) {   // debug export of the attention output at sampled voxels
+        for (int i = tid; i < QT * C; i += NT) {
+            const int r = i / C, c = i - r * C;
+            const int64_t v = s.vox[r];
+            if (r < nq && v >= 0 && v % a.attn_stride == 0)
+                a.attn_out[(size_t)(v / a.attn_stride) * C + c] = s.buf[r * ldc + c];
+        }
+    }
 
     // ---------------- x1 = q + Wo a + bo
     for (int c0 = tid; c0 < C; c0 += NT) {

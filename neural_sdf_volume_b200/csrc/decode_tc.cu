@@ -15,9 +15,10 @@
 //              runs its own online softmax over them (own maximum, sum and O
 //              accumulator); the two combine once per head;
 //   warp 8     MMA issue (the whole warp runs the loop; one elected lane issues);
-//   warp 9     producer: TMA loads of weights and of contiguous K/V blocks,
-//              cp.async gathers of a sub-volume's selected K/V rows (each lane's
-//              copies arrive on the slot's barrier when they land);
+//   warp 9     producer: TMA loads of weights and of contiguous K/V blocks;
+//              a sub-volume's selected K/V rows come by TMA tile::gather4, each
+//              lane bringing 4 rows of a 128-row block (CTA pairs: cp.async
+//              gathers, each lane's copies arriving on the slot's barrier);
 // connected only by mbarriers (no CTA-wide barrier inside a tile).
 // Compiled twice per width: one CTA per 128-row MMA, or (cta_group::2) a CTA
 // pair of a cluster per 256-row MMA, each CTA holding half of every B tile.
@@ -226,7 +227,8 @@ __global__ void __launch_bounds__(NT, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_wq64,
                  const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_w1,
                  const __grid_constant__ CUtensorMap tm_w2, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const TcArgs ta) {
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kr,
+                 const __grid_constant__ CUtensorMap tm_vr, const TcArgs ta) {
     const DecodeArgs& a = ta.d;
     extern __shared__ uint8_t dyn_raw[];
     __shared__ Shared sh;
@@ -418,21 +420,27 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             if (!take_slot(slot)) return false;
             const uint32_t dst = s_ring + slot * RS;
             if (!PAIR) {
-                // 128 rows x 8 chunks of 16 B: lane l copies chunk l % 8 of rows 4i + l / 8; the
-                // 32 row indices are loaded first (independent loads), then the copies are issued
-                const int c = lane & 7;
-                int rows[32];
+                // TMA gathers: lane l brings rows 4l..4l+3 of the block (one-row boxes, the slot's
+                // 128 B swizzle applied by the copy engine).  Tokens past the selection read token 0
+                // of the head: their scores are masked, so their probabilities are exactly 0.
+                const int t0 = j * 128 + 4 * lane;
+                int r[4];
+                if (t0 + 3 < nk && (nk & 3) == 0) {   // 16-byte aligned index loads
+                    const int4 q = __ldg(reinterpret_cast<const int4*>(sel + t0));
+                    r[0] = q.x; r[1] = q.y; r[2] = q.z; r[3] = q.w;
+                } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int tok = j * 128 + 4 * i + (lane >> 3);
-                    rows[i] = tok < nk ? __ldg(sel + tok) : -1;
+                    for (int i = 0; i < 4; ++i) r[i] = t0 + i < nk ? __ldg(sel + t0 + i) : 0;
                 }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int r = 4 * i + (lane >> 3);
-                    const bool okr = rows[i] >= 0;
-                    cp_async16(swz(dst, r, c), src + ((size_t)h * N + (okr ? rows[i] : 0)) * 64 + c * 8, okr);
-                }
+                const uint32_t fb = smem_u32(&sh.full[slot]);
+                if (lane == 0) mbar_expect_tx_only(fb, SLOT);
+                __syncwarp();
+                const int base = h * N;
+                tma_gather4(dst + 512 * lane, isv ? &tm_vr : &tm_kr, 0, base + r[0], base + r[1], base + r[2],
+                            base + r[3], fb);
+                __syncwarp();
+                if (lane == 0) mbar_arrive_n(fb, RING_ARRIVALS);
+                return true;
             } else if (!isv) {
                 // keys: this CTA's 64 tokens of the block, 8 chunks each (128 B swizzle)
                 const int c = lane & 7;
@@ -611,8 +619,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     auto issue_s = [&](int j) -> bool {
                         int sl;
                         if (!consume(sl)) return false;
-                        // gathered rows were written by cp.async (generic proxy): order them before the MMA's reads
-                        if (u.sel) fence_proxy_async();
+                        // CTA pairs gather rows with cp.async (generic proxy): order them before the MMA's reads
+                        if (PAIR && u.sel) fence_proxy_async();
                         const uint64_t da = desc_sw128(s_abuf + h * 16384), db = desc_sw128(s_ring + sl * RS);
                         const uint32_t sd = tmem + T_S0 + 128 * (j % NSB);
                         #pragma unroll
@@ -628,7 +636,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         if (!(ok = W.wait(&sh.bar_p[g], ph_p[g], 53))) break;
                         tc_fence_after();
                         if (!(ok = consume(slot))) break;
-                        if (u.sel) fence_proxy_async();
+                        if (PAIR && u.sel) fence_proxy_async();
                         // O_g += P_j V_j. P_j is read in place: the bf16 pairs of tokens [32i, 32i+32)
                         // occupy columns [32i, 32i+16) of its S buffer. V is N-major: 16 tokens per
                         // k-step = 16 rows of 128 B (64 B per CTA of a pair)
@@ -958,6 +966,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     const float inv = 1.0f / l_tot;
                     const float g0 = (wg ? f_oth : f_own) * inv, g1 = (wg ? f_own : f_oth) * inv;
                     const uint32_t atom = s_abuf + h * 16384;
+                    // debug export of the attention output at sampled voxels (fp32, before rounding)
+                    float* arow = (a.attn_out && vox >= 0 && vox % a.attn_stride == 0)
+                                      ? a.attn_out + (size_t)(vox / a.attn_stride) * C + h * 64 + 32 * wg
+                                      : nullptr;
                     #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {   // 16 of this warpgroup's 32 head dims at a time
                         float o0[16], o1[16];
@@ -973,7 +985,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                             for (int v = 0; v < 4; ++v) {
                                 const int d = c * 8 + 2 * v;
                                 const float b0 = has_o1 ? o1[d] * g1 : 0.f, b1 = has_o1 ? o1[d + 1] * g1 : 0.f;
-                                w[v] = pack_bf16(fmaf(o0[d], g0, b0), fmaf(o0[d + 1], g0, b1));
+                                const float x0 = fmaf(o0[d], g0, b0), x1 = fmaf(o0[d + 1], g0, b1);
+                                w[v] = pack_bf16(x0, x1);
+                                if (arow) {
+                                    arow[16 * hh + d] = x0;
+                                    arow[16 * hh + d + 1] = x1;
+                                }
                             }
                             st_shared_v4(swz(atom, row, 4 * wg + 2 * hh + c), w);
                         }
@@ -1303,6 +1320,10 @@ vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
     VDM_TRY(make_bf16_map(&m_k, d.K, (int64_t)d.H * d.N, 64, br, 64));
     // values are read N-major: a pair splits the 64 head dimensions, 32 per CTA
     VDM_TRY(make_bf16_map(&m_v, d.V, (int64_t)d.H * d.N, 64, 128, pair ? 32 : 64));
+    // one-row boxes for the gathers of selected K / V rows (tile::gather4)
+    CUtensorMap m_kr, m_vr;
+    VDM_TRY(make_bf16_map(&m_kr, d.K, (int64_t)d.H * d.N, 64, 1, 64));
+    VDM_TRY(make_bf16_map(&m_vr, d.V, (int64_t)d.H * d.N, 64, 1, 64));
     TcArgs ta;
     ta.d = d;
     ta.ns = ns;
@@ -1312,10 +1333,11 @@ vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
     ta.err = tc_error_word();
     if (!ta.err) return fail(VDM_ERR_CUDA, "error word lookup failed");
     ta.timeout = g_debug.timeout > 0 ? g_debug.timeout : 4000000000ll;
-    ta.inject = g_debug.inject;
-    g_debug.inject = 0;   // one launch only
+    // test hook: the g_debug.inject-th launch from the hook's call withholds one signal
+    ta.inject = g_debug.inject == 1;
+    if (g_debug.inject > 0) --g_debug.inject;
     typedef void (*Kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
-                         CUtensorMap, TcArgs);
+                         CUtensorMap, CUtensorMap, CUtensorMap, TcArgs);
     Kern kern;
     if (pair) kern = d.C == 128 ? decode_tc_kernel<128, 2> : d.C == 256 ? decode_tc_kernel<256, 2> : decode_tc_kernel<512, 2>;
     else kern = d.C == 128 ? decode_tc_kernel<128, 1> : d.C == 256 ? decode_tc_kernel<256, 1> : decode_tc_kernel<512, 1>;
@@ -1340,7 +1362,7 @@ vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     prof_begin(kProfDecode, st);
-    e = cudaLaunchKernelEx(&cfg, kern, m_wq, m_wq64, m_wo, m_w1, m_w2, m_k, m_v, ta);
+    e = cudaLaunchKernelEx(&cfg, kern, m_wq, m_wq64, m_wo, m_w1, m_w2, m_k, m_v, m_kr, m_vr, ta);
     prof_end(kProfDecode, st);
     if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "decode_tc_kernel launch: %s", cudaGetErrorString(e));
     return check_launch("decode_tc_kernel");

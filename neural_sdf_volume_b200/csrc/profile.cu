@@ -54,7 +54,7 @@ using namespace vdm;
 extern "C" {
 
 vdm_status vdm_debug_inject(int32_t mode, int64_t timeout_cycles) {
-    if (mode != 0 && mode != 1) return fail(VDM_ERR_INVALID_ARG, "unknown inject mode %d", mode);
+    if (mode < 0) return fail(VDM_ERR_INVALID_ARG, "inject mode must be >= 0, got %d", mode);
     g_debug.inject = mode;
     g_debug.timeout = timeout_cycles > 0 ? timeout_cycles : 0;
     return VDM_OK;

@@ -64,6 +64,8 @@ struct SelArgs {
     int tpu;                       // sub-volumes per unit = 128 / n_probe
     int top_k;
     int32_t* sel;                  // [T][top_k]
+    float* score_out;              // debug: [score_rows][N] scores by tile id, or NULL
+    int score_rows;
     int* err;
     long long timeout;
 };
@@ -386,6 +388,10 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                         float sum = 0.f;
                         for (int w = 0; w < warps_per_tile; ++w) sum += pp[w * 64];
                         score[(size_t)sv * N + j * 128 + col] = sum;
+                        if (a.score_out && unit * tpu + sv < n_sel) {
+                            const int ts = a.sel_tiles[unit * tpu + sv];
+                            if (ts < a.score_rows) a.score_out[(size_t)ts * N + j * 128 + col] = sum;
+                        }
                     }
                 }
                 pb ^= 1;
@@ -509,6 +515,8 @@ vdm_status launch_select_tc(const SelectTcLaunch& L, cudaStream_t st) {
     a.tpu = 128 / L.n_probe;
     a.top_k = L.top_k;
     a.sel = L.sel;
+    a.score_out = L.score_out;
+    a.score_rows = L.score_rows;
     a.err = tc_error_word();
     if (!a.err) return fail(VDM_ERR_CUDA, "error word lookup failed");
     a.timeout = 4000000000ll;

@@ -94,7 +94,7 @@ struct Plan {
     int L;
     int R[VDM_MAX_LEVELS];
     size_t off_grid[VDM_MAX_LEVELS];
-    size_t off_words, off_word_off, off_tile_ids, off_tile_off, off_counts, off_scan, off_plist,
+    size_t off_words, off_bits, off_word_off, off_tile_ids, off_tile_off, off_counts, off_scan, off_plist,
         off_qorder, off_sel, off_seltiles, off_ml, off_dense, off_dense_ml;
     int nw_max;
     int k;
@@ -134,11 +134,12 @@ vdm_status make_plan(const vdm_hier_params* p, int N, int ml_heads, Plan& pl) {
     }
     pl.nw_max = nw_max;
     pl.off_words = o;     o = align_up(o + (size_t)nw_max * 8);
+    pl.off_bits = o;      o = align_up(o + (size_t)nw_max * 2 * 8);
     pl.off_word_off = o;  o = align_up(o + (size_t)(nw_max + 1) * 4);
     pl.off_tile_ids = o;  o = align_up(o + (size_t)nw_max * 4);
     pl.off_tile_off = o;  o = align_up(o + (size_t)(nw_max + 1) * 4);
     pl.off_counts = o;    o = align_up(o + 4 * 4 * VDM_MAX_LEVELS);
-    pl.off_scan = o;      o = align_up(o + scan_tmp_ints(nw_max) * 4);
+    pl.off_scan = o;      o = align_up(o + compact_tmp_ints(nw_max) * 4);
     pl.off_plist = o;     o = align_up(o + (size_t)vox_max * 4);
     pl.off_qorder = o;    o = align_up(o + (p->adaptive ? (size_t)vox_max * 8 * 4 : 0));
     pl.off_sel = o;       o = align_up(o + (p->adaptive ? (size_t)nw_max * pl.k * 4 : 0));
@@ -163,7 +164,7 @@ using namespace vdm;
 
 extern "C" {
 
-int32_t vdm_abi_version(void) { return 1; }
+int32_t vdm_abi_version(void) { return 2; }
 
 const char* vdm_last_error(void) { return g_err; }
 
@@ -241,7 +242,9 @@ vdm_status vdm_decode_dense(const vdm_decoder* dec, const void* d_k, const void*
         }
         VDM_TRY(launch_decode(a, dec->dtype, st));
     }
-    return VDM_OK;
+    // the status of the kernels' bounded waits reaches the caller who made this call
+    VDM_CUDA_TRY(cudaStreamSynchronize(st));
+    return tc_check_error();
 }
 
 vdm_status vdm_select_kv(const vdm_decoder* dec, const void* d_k, const void* d_v, int32_t N,
@@ -266,7 +269,51 @@ vdm_status vdm_select_kv(const vdm_decoder* dec, const void* d_k, const void* d_
     a.top_k = top_k;
     a.sel = d_sel_out;
     a.score = d_score_out;
-    return launch_select(a, dec->dtype, reinterpret_cast<cudaStream_t>(stream));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    VDM_TRY(launch_select(a, dec->dtype, st));
+    VDM_CUDA_TRY(cudaStreamSynchronize(st));
+    return tc_check_error();
+}
+
+static size_t refine_ws_bytes(int R, size_t* off) {
+    const size_t nw = (size_t)(R / 4) * (R / 4) * (R / 4);
+    size_t o = 0;
+    off[0] = o; o = align_up(o + mark_bits_words(R) * 8);         // sign / near words
+    off[1] = o; o = align_up(o + (nw + 1) * 4);                   // word offsets
+    off[2] = o; o = align_up(o + nw * 4);                         // non-empty word ids
+    off[3] = o; o = align_up(o + (nw + 1) * 4);                   // their parent offsets
+    off[4] = o; o = align_up(o + compact_tmp_ints((int)nw) * 4);  // chunk sums
+    return o + 256;
+}
+
+vdm_status vdm_refine_workspace_size(int32_t R, size_t* bytes) {
+    if (!bytes) return fail(VDM_ERR_INVALID_ARG, "bytes is NULL");
+    if (R < 4 || R % 4 || R > 512) return fail(VDM_ERR_UNSUPPORTED, "R = %d must be a multiple of 4 in [4, 512]", R);
+    size_t off[5];
+    *bytes = refine_ws_bytes(R, off);
+    return VDM_OK;
+}
+
+vdm_status vdm_refine_level(const float* d_f, int32_t R, float* d_f_fine, uint64_t* d_mask, int32_t* d_parents,
+                            int32_t* d_counts, void* d_ws, size_t ws_bytes, vdm_stream stream) {
+    size_t need = 0;
+    VDM_TRY(vdm_refine_workspace_size(R, &need));
+    if (!d_f || !d_mask || !d_counts) return fail(VDM_ERR_INVALID_ARG, "null f / mask / counts");
+    if ((uintptr_t)d_f % 16 || (d_f_fine && (uintptr_t)d_f_fine % 16))
+        return fail(VDM_ERR_INVALID_ARG, "grids must be 16-byte aligned");
+    if (!d_ws || ws_bytes < need) return fail(VDM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+    void* ws = reinterpret_cast<void*>(align_up((uintptr_t)d_ws));
+    if ((uintptr_t)ws - (uintptr_t)d_ws + need - 256 > ws_bytes)
+        return fail(VDM_ERR_WORKSPACE, "workspace too small after alignment");
+    size_t off[5];
+    refine_ws_bytes(R, off);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int nw = (R / 4) * (R / 4) * (R / 4);
+    VDM_TRY(launch_mark_dilate(d_f, R, d_mask, at<uint64_t>(ws, off[0]), st));
+    VDM_TRY(launch_compact(d_mask, nw, R, at<int32_t>(ws, off[1]), at<int32_t>(ws, off[2]), at<int32_t>(ws, off[3]),
+                           d_parents, d_counts, at<int32_t>(ws, off[4]), st));
+    if (d_f_fine) VDM_TRY(launch_fill(d_f, R, d_f_fine, st));
+    return VDM_OK;
 }
 
 vdm_status vdm_hierarchical_workspace_size(const vdm_decoder* dec, const vdm_hier_params* p, int32_t N,
@@ -293,6 +340,12 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
         return fail(VDM_ERR_INVALID_ARG, "analytic term needs spheres and n_spheres >= 1");
     Plan pl;
     VDM_TRY(make_plan(p, N, dec->H, pl));
+    if (dbg) {
+        bool any_attn = false;
+        for (int l = 0; l < VDM_MAX_LEVELS; ++l) any_attn |= dbg->attn[l] != nullptr;
+        if (any_attn && dbg->attn_stride < 1)
+            return fail(VDM_ERR_INVALID_ARG, "debug attn needs attn_stride >= 1");
+    }
     if (pl.L > 1 && (!d_ws || ws_bytes < pl.total))
         return fail(VDM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.total, ws_bytes);
     void* ws = d_ws ? reinterpret_cast<void*>(align_up((uintptr_t)d_ws)) : nullptr;
@@ -320,6 +373,14 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
         auto dbg_ptr = [&](float* const* arr, int l, int64_t per) -> float* {
             return (dbg && arr[l]) ? arr[l] + (size_t)b * per : nullptr;
         };
+        // attention-output rows of level l: one per attn_stride voxels
+        auto attn_ptr = [&](int l) -> float* {
+            if (!dbg || !dbg->attn[l]) return nullptr;
+            const int64_t R = pl.R[l];
+            const int64_t rows = (R * R * R + dbg->attn_stride - 1) / dbg->attn_stride;
+            return dbg->attn[l] + (size_t)b * rows * dec->C;
+        };
+        const int64_t astride = dbg ? dbg->attn_stride : 0;
         // ---- level 0: dense
         {
             const int R = pl.R[0];
@@ -330,6 +391,8 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             a.M = (int64_t)R * R * R;
             a.grid = grid[0];
             a.dec_grid = dbg_ptr(dbg ? dbg->dec : nullptr, 0, a.M);
+            a.attn_out = attn_ptr(0);
+            a.attn_stride = astride;
             VDM_TRY(launch_decode(a, dec->dtype, st));
             if (sb) { sb->resolution[0] = R; sb->decoded[0] = a.M; }
         }
@@ -346,8 +409,10 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             int32_t* plist = at<int32_t>(ws, pl.off_plist);
             int32_t* qorder = at<int32_t>(ws, pl.off_qorder);
             int32_t* sel = at<int32_t>(ws, pl.off_sel);
-            VDM_TRY(launch_mark_dilate(grid[l], R, words, st));
-            VDM_TRY(launch_word_scan(words, nw, word_off, tile_ids, counts, scan_tmp, st));
+            VDM_TRY(launch_mark_dilate(grid[l], R, words, at<uint64_t>(ws, pl.off_bits), st));
+            VDM_TRY(launch_compact(words, nw, R, word_off, tile_ids, tile_off, plist, counts, scan_tmp, st));
+            // the inherit fill needs no count: it runs while the counts travel to the host
+            VDM_TRY(launch_fill(grid[l], R, grid[l + 1], st));
             int32_t hc[2] = {0, 0};
             VDM_CUDA_TRY(cudaMemcpyAsync(hc, counts, sizeof(hc), cudaMemcpyDeviceToHost, st));
             VDM_CUDA_TRY(cudaStreamSynchronize(st));
@@ -356,9 +421,6 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             if (dbg && dbg->active[l])
                 VDM_CUDA_TRY(cudaMemcpyAsync(dbg->active[l] + (size_t)b * nw, words, (size_t)nw * 8,
                                              cudaMemcpyDeviceToDevice, st));
-            VDM_TRY(launch_parent_list(words, word_off, nw, R, plist, st));
-            VDM_TRY(launch_tile_offsets(word_off, tile_ids, T, nw, tile_off, st));
-            VDM_TRY(launch_fill(grid[l], words, R, grid[l + 1], st));
             const int64_t vox2 = (int64_t)R2 * R2 * R2;
             float* decg = dbg_ptr(dbg ? dbg->dec : nullptr, l + 1, vox2);
             if (sb) {
@@ -376,6 +438,8 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
                 a.M = 8 * (int64_t)Mp;
                 a.grid = grid[l + 1];
                 a.dec_grid = decg;
+                a.attn_out = attn_ptr(l + 1);
+                a.attn_stride = astride;
                 VDM_TRY(launch_decode(a, dec->dtype, st));
                 if (sb) sb->decoded[l + 1] = a.M;
                 continue;
@@ -389,6 +453,14 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             int32_t* dense_ml = at<int32_t>(ws, pl.off_dense_ml);
             VDM_TRY(launch_probe_order(tile_off, T, plist, R2, p->n_probe, salt, qorder, counts + 2, sel_tiles,
                                        dense_q, dense_ml, st));
+            const int dbg_rows = dbg ? (int)std::min<int64_t>(T, dbg->max_tiles) : 0;
+            if (dbg && dbg->probes[l + 1] && dbg_rows > 0)
+                VDM_TRY(launch_probe_export(tile_off, dbg_rows, plist, qorder, R2, p->n_probe,
+                                            dbg->probes[l + 1] + (size_t)b * dbg->max_tiles * p->n_probe,
+                                            st));
+            float* score_dbg = (dbg && dbg->scores[l + 1] && dbg_rows > 0)
+                                   ? dbg->scores[l + 1] + (size_t)b * dbg->max_tiles * N
+                                   : nullptr;
             DecodeArgs a = base;
             a.qmode = kQueryChildren;
             a.R = R2;
@@ -399,6 +471,8 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             a.n_probe = p->n_probe;
             a.grid = grid[l + 1];
             a.dec_grid = decg;
+            a.attn_out = attn_ptr(l + 1);
+            a.attn_stride = astride;
             // dense pass: probes and small sub-volumes, packed into one flat list
             // (exports the probes' softmax statistics for the scoring kernel)
             {
@@ -423,6 +497,8 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
                 L.probe_ml = probe_ml;
                 L.R = R2; L.n_probe = p->n_probe; L.top_k = pl.k;
                 L.sel = sel;
+                L.score_out = score_dbg;
+                L.score_rows = dbg_rows;
                 VDM_TRY(launch_select_tc(L, st));
             } else {
             SelectArgs s;
@@ -434,6 +510,8 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             s.n_probe = p->n_probe;
             s.top_k = pl.k;
             s.sel = sel;
+            // the CUDA-core selection writes a score row for every sub-volume it scores
+            s.score = (score_dbg && T <= dbg_rows) ? score_dbg : nullptr;
             VDM_TRY(launch_select(s, dec->dtype, st));
             }
             // sparse pass: the remaining queries over the selected tokens
@@ -473,7 +551,9 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             }
         }
     }
-    return VDM_OK;
+    // the last level's kernels: their bounded-wait status reaches this caller too
+    VDM_CUDA_TRY(cudaStreamSynchronize(st));
+    return tc_check_error();
 }
 
 }  // extern "C"

@@ -79,6 +79,8 @@ struct DecodeArgs {
     float* out;                 // out[q] (flat work only) or NULL
     float* grid;                // scatter field at voxel linear index or NULL
     float* dec_grid;            // debug: raw decoder output at voxel index or NULL
+    float* attn_out;            // debug: attention output a[v / attn_stride][C] at voxels v with
+    int64_t attn_stride;        //   v % attn_stride == 0 (grid and children modes) or NULL
     // analytic field
     const float* spheres;       // [S][4] or NULL
     int n_spheres;
@@ -117,7 +119,7 @@ struct SelectArgs {
 
 // ---------------------------------------------------------------- test hooks
 struct DebugHooks {
-    int inject;              // 1: withhold one MMA completion signal in the next decode launch
+    int inject;              // n >= 1: the n-th tensor-core decode launch from now withholds one signal
     long long timeout;       // bounded-wait limit in cycles (0: default)
     int single_cta;          // 1: tensor-core decoding with one CTA per MMA (no CTA pairs)
 };
@@ -153,6 +155,8 @@ struct SelectTcLaunch {
     const float* probe_ml;      // [T][n_probe][H][2] from the dense pass
     int R, n_probe, top_k;
     int32_t* sel;               // [T][top_k]
+    float* score_out;           // debug: [score_rows][N] scores of tiles t < score_rows, or NULL
+    int score_rows;
 };
 bool select_tc_supported(int C, int n_probe, int N, vdm_dtype dt);
 vdm_status launch_select_tc(const SelectTcLaunch& L, cudaStream_t s);
@@ -160,21 +164,29 @@ vdm_status launch_select_tc(const SelectTcLaunch& L, cudaStream_t s);
 vdm_status launch_decode(DecodeArgs a, vdm_dtype dt, cudaStream_t s);
 
 // volume kernels
-vdm_status launch_mark_dilate(const float* f, int R, uint64_t* words, cudaStream_t s);
-vdm_status launch_word_scan(const uint64_t* words, int n_words, int32_t* word_off,
-                            int32_t* tile_ids, int32_t* counts, int32_t* block_tmp,
-                            cudaStream_t s);
-vdm_status launch_parent_list(const uint64_t* words, const int32_t* word_off, int n_words, int R,
-                              int32_t* plist, cudaStream_t s);
-vdm_status launch_tile_offsets(const int32_t* word_off, const int32_t* tile_ids, int n_tiles,
-                               int n_words, int32_t* tile_off, cudaStream_t s);
-vdm_status launch_fill(const float* f_coarse, const uint64_t* words, int R, float* f_fine,
-                       cudaStream_t s);
+// boundary mark + dilation of a level grid -> blocked refine mask; `bits` is scratch of
+// mark_bits_words(R) words
+size_t mark_bits_words(int R);
+vdm_status launch_mark_dilate(const float* f, int R, uint64_t* words, uint64_t* bits, cudaStream_t s);
+// voxels with a 26-neighbour of the other sign (no band, no dilation), blocked words
+vdm_status launch_sign_change(const float* f, int R, uint64_t* words, uint64_t* bits, cudaStream_t s);
+// compaction of the refine mask: word offsets, non-empty word ids (sub-volumes) and
+// their parent offsets, parent list, counts[0..1] = refined voxels, sub-volumes;
+// `chunk_tmp` is scratch of compact_tmp_ints(n_words) ints
+size_t compact_tmp_ints(int n_words);
+vdm_status launch_compact(const uint64_t* words, int n_words, int R, int32_t* word_off, int32_t* tile_ids,
+                          int32_t* tile_off, int32_t* plist, int32_t* counts, int32_t* chunk_tmp,
+                          cudaStream_t s);
+// every voxel of the (2R)^3 grid takes its parent's value
+vdm_status launch_fill(const float* f_coarse, int R, float* f_fine, cudaStream_t s);
+// debug: fine voxel indices of each tile's first min(n_probe, count) queries of qorder
+vdm_status launch_probe_export(const int32_t* tile_off, int n_tiles, const int32_t* plist,
+                               const int32_t* qorder, int R2, int n_probe, int32_t* out,
+                               cudaStream_t s);
 vdm_status launch_probe_order(const int32_t* tile_off, int n_tiles, const int32_t* plist, int R2,
                               int n_probe, uint64_t salt, int32_t* qorder, int32_t* counters,
                               int32_t* sel_tiles, int32_t* dense_q, int32_t* dense_ml, cudaStream_t s);
 
-size_t scan_tmp_ints(int n_words);
 
 // ---------------------------------------------------------------- device helpers
 __device__ __forceinline__ float to_f(float x) { return x; }

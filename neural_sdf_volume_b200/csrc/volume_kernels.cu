@@ -17,83 +17,161 @@
 namespace vdm {
 namespace {
 
-// ------------------------------------------------------------------ mark + dilate
-// One CTA covers an 8^3 region (2^3 words).  f is staged with a halo of 2,
-// the mark is evaluated on the 10^3 region (halo 1), the dilation on the core.
-constexpr int MD_T = 256;
-constexpr int MD_E = 12;   // staged edge
-constexpr int MM_E = 10;   // mark edge
+// ------------------------------------------------------------------ pack
+// Sign and near-surface bits of every voxel, packed into the blocked layout:
+// S[w] bit b = f(v) < 0, Nr[w] bit b = |f(v)| < thr.  One CTA per (bi, bj): its
+// 16 warps read the 16 rows (4 bi + di, 4 bj + dj) of the block row with 16-byte
+// loads (all of a lane's loads in flight at once), each lane turns a float4 into
+// the 4-bit nibble (di, dj) of block bk, and the nibbles are gathered into words
+// through shared memory.  One read of f, 1/16 of it written.
+constexpr int PK_T = 512;          // one warp per row (di, dj)
+constexpr int PK_MAXV = 8;         // float4 per lane: R <= 1024
 
-__global__ void __launch_bounds__(MD_T) mark_dilate_kernel(const float* __restrict__ f, int R,
-                                                           float thr, uint64_t* __restrict__ words) {
-    __shared__ float fs[MD_E * MD_E * MD_E];
-    __shared__ unsigned char ms[MM_E * MM_E * MM_E];
-    __shared__ uint32_t half[16];
+__global__ void __launch_bounds__(PK_T) pack_kernel(const float* __restrict__ f, int R, float thr,
+                                                    uint64_t* __restrict__ S, uint64_t* __restrict__ Nr) {
+    __shared__ __align__(16) uint8_t ns[256][16];   // [bk][row] sign nibbles
+    __shared__ __align__(16) uint8_t nn[256][16];   // [bk][row] near nibbles
     const int nb = R >> 2;
-    const int ncta = (nb + 1) >> 1;
+    const int bi = blockIdx.x / nb, bj = blockIdx.x - bi * nb;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int di = warp >> 2, dj = warp & 3;
+    const float4* row = reinterpret_cast<const float4*>(f + ((size_t)(4 * bi + di) * R + (4 * bj + dj)) * R);
+    float4 v[PK_MAXV];
+#pragma unroll
+    for (int u = 0; u < PK_MAXV; ++u)
+        if (lane + 32 * u < nb) v[u] = __ldcs(row + lane + 32 * u);
+#pragma unroll
+    for (int u = 0; u < PK_MAXV; ++u) {
+        const int bk = lane + 32 * u;
+        if (bk < nb) {
+            const float4 x = v[u];
+            ns[bk][warp] = (uint8_t)((x.x < 0.f) | ((x.y < 0.f) << 1) | ((x.z < 0.f) << 2) | ((x.w < 0.f) << 3));
+            nn[bk][warp] = (uint8_t)((fabsf(x.x) < thr) | ((fabsf(x.y) < thr) << 1) | ((fabsf(x.z) < thr) << 2) |
+                                     ((fabsf(x.w) < thr) << 3));
+        }
+    }
+    __syncthreads();
+    // thread t < nb: word (bi, bj, t) from its 16 sign nibbles; thread 256 + t: near word
+    const int t = threadIdx.x & 255;
+    if (t < nb) {
+        const uint4 q = *reinterpret_cast<const uint4*>(threadIdx.x < 256 ? ns[t] : nn[t]);
+        const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+        uint64_t w = 0;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {   // bytes (rows 4h..4h+3, one nibble each) -> 16 bits
+            uint32_t x = qq[h];
+            x = (x | (x >> 4)) & 0x00FF00FFu;
+            x = (x | (x >> 8)) & 0x0000FFFFu;
+            w |= (uint64_t)x << (16 * h);
+        }
+        const size_t wi = ((size_t)bi * nb + bj) * nb + t;
+        if (threadIdx.x < 256) S[wi] = w;
+        else Nr[wi] = w;
+    }
+}
+
+// ------------------------------------------------------------------ mark + dilate on words
+// mark = near | (D(inside) & D(outside)), act = D(mark), where D is the 3x3x3 dilation
+// clipped at the grid border (a voxel's own sign is in its cube, so "some neighbour has
+// the other sign" is "the cube holds both signs").  D = D_i o D_j o D_k, and along one
+// axis a word's dilation is its shifted copies plus the facing bit planes of its two
+// neighbour words.  One CTA computes the act words of an 8^3-word core from the sign
+// and near words of the core plus a 2-word halo (12^3 words in shared memory).
+constexpr int MW_T = 512;
+constexpr int MW_C = 8;                 // core edge (words)
+constexpr int MW_E = MW_C + 4;          // staged edge
+constexpr int MW_N = MW_E * MW_E * MW_E;
+constexpr uint64_t K0 = 0x1111111111111111ull, K3 = 0x8888888888888888ull;   // dk = 0 / 3
+constexpr uint64_t J0 = 0x000F000F000F000Full, J3 = 0xF000F000F000F000ull;   // dj = 0 / 3
+
+// one axis of the dilation over the staged region; words whose neighbour along the
+// axis lies outside the region take it as empty (they are never used as valid)
+template <int AXIS>
+__device__ __forceinline__ void dilate_axis(const uint64_t* __restrict__ src, uint64_t* __restrict__ dst) {
+    constexpr int step = AXIS == 0 ? MW_E * MW_E : AXIS == 1 ? MW_E : 1;
+    for (int r = threadIdx.x; r < MW_N; r += MW_T) {
+        const int c = AXIS == 0 ? r / (MW_E * MW_E) : AXIS == 1 ? (r / MW_E) % MW_E : r % MW_E;
+        const uint64_t x = src[r];
+        const uint64_t xp = c > 0 ? src[r - step] : 0ull, xn = c < MW_E - 1 ? src[r + step] : 0ull;
+        uint64_t y;
+        if (AXIS == 2)
+            y = x | ((x >> 1) & ~K3) | ((x << 1) & ~K0) | ((xn & K0) << 3) | ((xp & K3) >> 3);
+        else if (AXIS == 1)
+            y = x | ((x >> 4) & ~J3) | ((x << 4) & ~J0) | ((xn & J0) << 12) | ((xp & J3) >> 12);
+        else
+            y = x | (x >> 16) | (x << 16) | ((xn & 0xFFFFull) << 48) | (xp >> 48);
+        dst[r] = y;
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ void dilate3(uint64_t* a, uint64_t* tmp) {   // a <- D(a)
+    dilate_axis<2>(a, tmp);
+    dilate_axis<1>(tmp, a);
+    dilate_axis<0>(a, tmp);
+    for (int r = threadIdx.x; r < MW_N; r += MW_T) a[r] = tmp[r];
+    __syncthreads();
+}
+
+// DILATE = false: the sign-change words D(inside) & D(outside) | near, undilated.
+template <bool DILATE>
+__global__ void __launch_bounds__(MW_T) mark_words_kernel(const uint64_t* __restrict__ S,
+                                                          const uint64_t* __restrict__ Nr, int nb,
+                                                          uint64_t* __restrict__ act) {
+    extern __shared__ uint64_t mw_smem[];
+    uint64_t* in = mw_smem;              // inside words, then D(inside)
+    uint64_t* out = in + MW_N;           // outside words, then D(outside)
+    uint64_t* near = out + MW_N;         // near words, then mark, then D(mark)
+    uint64_t* tmp = near + MW_N;
+    const int ncta = (nb + MW_C - 1) / MW_C;
     int c = blockIdx.x;
     const int ck = c % ncta; c /= ncta;
     const int cj = c % ncta; c /= ncta;
     const int ci = c;
-    const int i0 = ci * 8, j0 = cj * 8, k0 = ck * 8;
-    for (int t = threadIdx.x; t < MD_E * MD_E * MD_E; t += MD_T) {
-        const int a = t / (MD_E * MD_E), b = (t / MD_E) % MD_E, e = t % MD_E;
-        const int i = i0 - 2 + a, j = j0 - 2 + b, k = k0 - 2 + e;
-        float v = 0.f;
-        if (i >= 0 && i < R && j >= 0 && j < R && k >= 0 && k < R)
-            v = f[((size_t)i * R + j) * R + k];
-        fs[t] = v;
-    }
-    __syncthreads();
-    for (int t = threadIdx.x; t < MM_E * MM_E * MM_E; t += MD_T) {
-        const int a = t / (MM_E * MM_E), b = (t / MM_E) % MM_E, e = t % MM_E;
-        const int i = i0 - 1 + a, j = j0 - 1 + b, k = k0 - 1 + e;
-        unsigned char m = 0;
-        if (i >= 0 && i < R && j >= 0 && j < R && k >= 0 && k < R) {
-            const float fv = fs[((a + 1) * MD_E + (b + 1)) * MD_E + (e + 1)];
-            const bool in = fv < 0.f;
-            bool hit = fabsf(fv) < thr;
-            for (int da = -1; da <= 1; ++da)
-                for (int db = -1; db <= 1; ++db)
-                    for (int de = -1; de <= 1; ++de) {
-                        const int ni = i + da, nj = j + db, nk = k + de;
-                        if (ni < 0 || ni >= R || nj < 0 || nj >= R || nk < 0 || nk >= R) continue;
-                        const float fu = fs[((a + 1 + da) * MD_E + (b + 1 + db)) * MD_E + (e + 1 + de)];
-                        hit |= ((fu < 0.f) != in);
-                    }
-            m = hit;
+    const int i0 = ci * MW_C - 2, j0 = cj * MW_C - 2, k0 = ck * MW_C - 2;
+    for (int r = threadIdx.x; r < MW_N; r += MW_T) {
+        const int a = r / (MW_E * MW_E), b = (r / MW_E) % MW_E, e = r % MW_E;
+        const int bi = i0 + a, bj = j0 + b, bk = k0 + e;
+        uint64_t s = 0, o = 0, n = 0;
+        if (bi >= 0 && bi < nb && bj >= 0 && bj < nb && bk >= 0 && bk < nb) {
+            const size_t w = ((size_t)bi * nb + bj) * nb + bk;
+            s = S[w];
+            o = ~s;
+            n = Nr[w];
         }
-        ms[t] = m;
+        in[r] = s;
+        out[r] = o;
+        near[r] = n;
     }
     __syncthreads();
-    // 512 core voxels = 8 words x 64 bits; item -> (word, bit)
-    for (int item = threadIdx.x; item < 512; item += MD_T) {
-        const int wl = item >> 6, bit = item & 63;
-        const int wi = wl >> 2, wj = (wl >> 1) & 1, wk = wl & 1;
-        const int di = bit >> 4, dj = (bit >> 2) & 3, dk = bit & 3;
-        const int a = wi * 4 + di, b = wj * 4 + dj, e = wk * 4 + dk;   // core coords
-        bool act = false;
-        for (int da = 0; da < 3; ++da)
-            for (int db = 0; db < 3; ++db)
-                for (int de = 0; de < 3; ++de)
-                    act |= ms[((a + da) * MM_E + (b + db)) * MM_E + (e + de)] != 0;
-        const unsigned bal = __ballot_sync(0xffffffffu, act);
-        if ((threadIdx.x & 31) == 0) half[item >> 5] = bal;
+    dilate3(in, tmp);
+    dilate3(out, tmp);
+    // mark; words off the grid stay empty (their dilated sign words are not)
+    for (int r = threadIdx.x; r < MW_N; r += MW_T) {
+        const int a = r / (MW_E * MW_E), b = (r / MW_E) % MW_E, e = r % MW_E;
+        const int bi = i0 + a, bj = j0 + b, bk = k0 + e;
+        const bool on = bi >= 0 && bi < nb && bj >= 0 && bj < nb && bk >= 0 && bk < nb;
+        near[r] = on ? (near[r] | (in[r] & out[r])) : 0ull;
     }
     __syncthreads();
-    if (threadIdx.x < 8) {
-        const int wl = threadIdx.x;
-        const int bi = ci * 2 + (wl >> 2), bj = cj * 2 + ((wl >> 1) & 1), bk = ck * 2 + (wl & 1);
+    if (DILATE) dilate3(near, tmp);
+    for (int r = threadIdx.x; r < MW_C * MW_C * MW_C; r += MW_T) {
+        const int a = r / (MW_C * MW_C), b = (r / MW_C) % MW_C, e = r % MW_C;
+        const int bi = ci * MW_C + a, bj = cj * MW_C + b, bk = ck * MW_C + e;
         if (bi < nb && bj < nb && bk < nb)
-            words[((size_t)bi * nb + bj) * nb + bk] =
-                (uint64_t)half[2 * wl] | ((uint64_t)half[2 * wl + 1] << 32);
+            act[((size_t)bi * nb + bj) * nb + bk] = near[((a + 2) * MW_E + (b + 2)) * MW_E + (e + 2)];
     }
 }
 
-// ------------------------------------------------------------------ scan of word popcounts
-constexpr int SC_T = 256;
-constexpr int SC_PER = 4;
-constexpr int SC_BLK = SC_T * SC_PER;   // words per scan block
+// ------------------------------------------------------------------ compaction
+// Chunks of 1024 words in linear word order.  chunk_sum_kernel: per chunk, the number
+// of refined voxels and of non-empty words.  compact_kernel: per chunk, the prefix of
+// the earlier chunks' sums (each CTA adds them itself: no inter-CTA waiting), then the
+// word offsets, the ids and parent offsets of the non-empty words (sub-volumes) and the
+// parent list (each word's set bits in ascending bit order, written warp-cooperatively).
+constexpr int CP_T = 256;
+constexpr int CP_PER = 4;
+constexpr int CP_CHUNK = CP_T * CP_PER;
 
 // Block-wide exclusive scan of (a, b) pairs held one per thread; returns totals.
 __device__ __forceinline__ int2 block_scan2(int2 v, int2* tmp, int2& total) {
@@ -107,137 +185,149 @@ __device__ __forceinline__ int2 block_scan2(int2 v, int2* tmp, int2& total) {
     if (lane == 31) tmp[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int2 w = lane < SC_T / 32 ? tmp[lane] : make_int2(0, 0);
+        int2 w = lane < CP_T / 32 ? tmp[lane] : make_int2(0, 0);
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             int ya = __shfl_up_sync(0xffffffffu, w.x, o), yb = __shfl_up_sync(0xffffffffu, w.y, o);
             if (lane >= o) { w.x += ya; w.y += yb; }
         }
-        if (lane < SC_T / 32) tmp[lane] = w;
+        if (lane < CP_T / 32) tmp[lane] = w;
     }
     __syncthreads();
     int2 base = warp ? tmp[warp - 1] : make_int2(0, 0);
-    total = tmp[SC_T / 32 - 1];
+    total = tmp[CP_T / 32 - 1];
     __syncthreads();
     return make_int2(base.x + x.x - v.x, base.y + x.y - v.y);
 }
 
-__global__ void __launch_bounds__(SC_T) scan_reduce_kernel(const uint64_t* __restrict__ words, int n,
-                                                           int2* __restrict__ bsum) {
-    __shared__ int2 tmp[SC_T / 32];
+__device__ __forceinline__ int2 block_sum2(int2 v, int2* tmp) {
+    int2 tot;
+    block_scan2(v, tmp, tot);
+    return tot;
+}
+
+__global__ void __launch_bounds__(CP_T) chunk_sum_kernel(const uint64_t* __restrict__ words, int n,
+                                                         int2* __restrict__ csum) {
+    __shared__ int2 tmp[CP_T / 32];
     int2 v = make_int2(0, 0);
-    const int base = blockIdx.x * SC_BLK + threadIdx.x * SC_PER;
-    for (int q = 0; q < SC_PER; ++q) {
-        const int w = base + q;
+    const int base = blockIdx.x * CP_CHUNK;
+    for (int q = 0; q < CP_PER; ++q) {
+        const int w = base + q * CP_T + threadIdx.x;   // coalesced: consecutive threads, consecutive words
         if (w < n) {
             const int pc = __popcll(words[w]);
             v.x += pc;
             v.y += pc > 0;
         }
     }
-    int2 tot;
-    block_scan2(v, tmp, tot);
-    if (threadIdx.x == 0) bsum[blockIdx.x] = tot;
+    const int2 tot = block_sum2(v, tmp);
+    if (threadIdx.x == 0) csum[blockIdx.x] = tot;
 }
 
-__global__ void __launch_bounds__(SC_T) scan_blocks_kernel(int2* __restrict__ bsum, int nblk,
-                                                           int32_t* __restrict__ counts) {
-    __shared__ int2 tmp[SC_T / 32];
-    int2 carry = make_int2(0, 0);
-    for (int b0 = 0; b0 < nblk; b0 += SC_T) {
-        const int b = b0 + threadIdx.x;
-        int2 v = b < nblk ? bsum[b] : make_int2(0, 0);
-        int2 tot;
-        int2 ex = block_scan2(v, tmp, tot);
-        if (b < nblk) bsum[b] = make_int2(carry.x + ex.x, carry.y + ex.y);
-        carry.x += tot.x;
-        carry.y += tot.y;
+__global__ void __launch_bounds__(CP_T) compact_kernel(const uint64_t* __restrict__ words, int n, int R,
+                                                       const int2* __restrict__ csum,
+                                                       int32_t* __restrict__ word_off,
+                                                       int32_t* __restrict__ tile_ids,
+                                                       int32_t* __restrict__ tile_off,
+                                                       int32_t* __restrict__ plist,
+                                                       int32_t* __restrict__ counts) {
+    __shared__ int2 tmp[CP_T / 32];
+    __shared__ uint64_t sw[CP_CHUNK];
+    __shared__ int so[CP_CHUNK];
+    const int chunk = blockIdx.x;
+    // prefix of the earlier chunks
+    int2 pre = make_int2(0, 0);
+    for (int c = threadIdx.x; c < chunk; c += CP_T) {
+        const int2 x = csum[c];
+        pre.x += x.x;
+        pre.y += x.y;
     }
-    if (threadIdx.x == 0) {
-        counts[0] = carry.x;   // active parents
-        counts[1] = carry.y;   // non-empty words (sub-volumes)
-    }
-}
-
-__global__ void __launch_bounds__(SC_T) scan_write_kernel(const uint64_t* __restrict__ words, int n,
-                                                          const int2* __restrict__ bsum,
-                                                          int32_t* __restrict__ word_off,
-                                                          int32_t* __restrict__ tile_ids,
-                                                          const int32_t* __restrict__ counts) {
-    __shared__ int2 tmp[SC_T / 32];
-    int pc[SC_PER];
+    pre = block_sum2(pre, tmp);
+    // this thread's CP_PER consecutive words of the chunk
+    const int base = chunk * CP_CHUNK;
+    const int w0 = base + threadIdx.x * CP_PER;
+    uint64_t m[CP_PER];
     int2 v = make_int2(0, 0);
-    const int base = blockIdx.x * SC_BLK + threadIdx.x * SC_PER;
-    for (int q = 0; q < SC_PER; ++q) {
-        const int w = base + q;
-        pc[q] = w < n ? __popcll(words[w]) : 0;
-        v.x += pc[q];
-        v.y += pc[q] > 0;
+#pragma unroll
+    for (int q = 0; q < CP_PER; ++q) {
+        m[q] = w0 + q < n ? words[w0 + q] : 0ull;
+        const int pc = __popcll(m[q]);
+        v.x += pc;
+        v.y += pc > 0;
     }
     int2 tot;
-    int2 ex = block_scan2(v, tmp, tot);
-    const int2 bo = bsum[blockIdx.x];
-    int run = bo.x + ex.x, nt = bo.y + ex.y;
-    for (int q = 0; q < SC_PER; ++q) {
-        const int w = base + q;
+    const int2 ex = block_scan2(v, tmp, tot);
+    int run = pre.x + ex.x, nt = pre.y + ex.y;
+#pragma unroll
+    for (int q = 0; q < CP_PER; ++q) {
+        const int w = w0 + q;
+        const int l = threadIdx.x * CP_PER + q;
+        sw[l] = m[q];
+        so[l] = run;
         if (w < n) {
             word_off[w] = run;
-            if (pc[q] > 0) tile_ids[nt++] = w;
-            run += pc[q];
+            if (m[q]) {
+                tile_ids[nt] = w;
+                tile_off[nt] = run;
+                ++nt;
+            }
+            run += __popcll(m[q]);
         }
     }
-    if (blockIdx.x == 0 && threadIdx.x == 0) word_off[n] = counts[0];
-}
-
-// ------------------------------------------------------------------ parent list
-__global__ void parent_list_kernel(const uint64_t* __restrict__ words, const int32_t* __restrict__ word_off,
-                                   int n, int R, int32_t* __restrict__ plist) {
-    const int w = blockIdx.x * blockDim.x + threadIdx.x;
-    if (w >= n) return;
-    uint64_t m = words[w];
-    if (!m) return;
-    const int nb = R >> 2;
-    const int bi = w / (nb * nb), bj = (w / nb) % nb, bk = w % nb;
-    int o = word_off[w];
-    while (m) {
-        const int bit = __ffsll((long long)m) - 1;
-        m &= m - 1;
-        const int i = bi * 4 + (bit >> 4), j = bj * 4 + ((bit >> 2) & 3), k = bk * 4 + (bit & 3);
-        plist[o++] = (i * R + j) * R + k;
+    if (base + CP_CHUNK >= n && threadIdx.x == 0) {   // last chunk: totals
+        const int total = pre.x + tot.x, T = pre.y + tot.y;
+        word_off[n] = total;
+        tile_off[T] = total;
+        counts[0] = total;   // refined voxels (active parents)
+        counts[1] = T;       // non-empty words (sub-volumes)
     }
-}
-
-__global__ void tile_off_kernel(const int32_t* __restrict__ word_off, const int32_t* __restrict__ tile_ids,
-                                int n_tiles, int n_words, int32_t* __restrict__ tile_off) {
-    const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if (t < n_tiles) tile_off[t] = word_off[tile_ids[t]];
-    if (t == n_tiles) tile_off[t] = word_off[n_words];
+    __syncthreads();
+    if (!plist) return;
+    // parent list: one warp per word, lane L places bits L and L + 32
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nbw = R >> 2;
+    const uint32_t below = (1u << lane) - 1u;
+    for (int l = warp; l < CP_CHUNK && base + l < n; l += CP_T / 32) {
+        const uint64_t x = sw[l];
+        if (!x) continue;
+        const int w = base + l;
+        const int bi = w / (nbw * nbw), bj = (w / nbw) % nbw, bk = w % nbw;
+        const uint32_t lo = (uint32_t)x, hi = (uint32_t)(x >> 32);
+        const int o = so[l];
+        if ((lo >> lane) & 1u) {
+            const int bit = lane;
+            const int i = 4 * bi + (bit >> 4), j = 4 * bj + ((bit >> 2) & 3), k = 4 * bk + (bit & 3);
+            plist[o + __popc(lo & below)] = (i * R + j) * R + k;
+        }
+        if ((hi >> lane) & 1u) {
+            const int bit = lane + 32;
+            const int i = 4 * bi + (bit >> 4), j = 4 * bj + ((bit >> 2) & 3), k = 4 * bk + (bit & 3);
+            plist[o + __popc(lo) + __popc(hi & below)] = (i * R + j) * R + k;
+        }
+    }
 }
 
 // ------------------------------------------------------------------ inherit fill
-// Fine voxels (i, j, 4q..4q+3) at R2 = 2R; parents (i/2, j/2, 2q..2q+1).
-__global__ void fill_kernel(const float* __restrict__ fc, const uint64_t* __restrict__ words, int R,
-                            float* __restrict__ ff) {
+// Every voxel of the fine grid takes its parent's value (the decode that follows
+// overwrites the children of refined parents): 8 fine voxels along k per thread from
+// 4 parents (one 16-byte load), two 16-byte stores; no partial-sector writes.
+template <bool STREAM>
+__global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ fc, int R, float* __restrict__ ff) {
     const int R2 = 2 * R;
-    const int Q = R2 >> 2;
+    const int Q = R2 >> 3;   // groups of 8 fine voxels per row
     const size_t n = (size_t)R2 * R2 * Q;
-    const int nb = R >> 2;
     for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < n; t += (size_t)gridDim.x * blockDim.x) {
         const int q = (int)(t % Q);
         const size_t ij = t / Q;
         const int j = (int)(ij % R2), i = (int)(ij / R2);
-        const int pi = i >> 1, pj = j >> 1, pk = 2 * q;
-        const size_t pbase = ((size_t)pi * R + pj) * R + pk;
-        const float2 pv = *reinterpret_cast<const float2*>(fc + pbase);
-        const uint64_t wd = words[((size_t)(pi >> 2) * nb + (pj >> 2)) * nb + (pk >> 2)];
-        const int b0 = ((pi & 3) * 4 + (pj & 3)) * 4 + (pk & 3);
-        const bool a0 = (wd >> b0) & 1, a1 = (wd >> (b0 + 1)) & 1;
-        float* dst = ff + ((size_t)i * R2 + j) * R2 + 4 * q;
-        if (!a0 && !a1) {
-            *reinterpret_cast<float4*>(dst) = make_float4(pv.x, pv.x, pv.y, pv.y);
+        const float4 p = *reinterpret_cast<const float4*>(fc + ((size_t)(i >> 1) * R + (j >> 1)) * R + 4 * q);
+        float4* dst = reinterpret_cast<float4*>(ff + ((size_t)i * R2 + j) * R2 + 8 * q);
+        const float4 a = make_float4(p.x, p.x, p.y, p.y), b = make_float4(p.z, p.z, p.w, p.w);
+        if (STREAM) {
+            __stcs(dst, a);
+            __stcs(dst + 1, b);
         } else {
-            if (!a0) { dst[0] = pv.x; dst[1] = pv.x; }
-            if (!a1) { dst[2] = pv.y; dst[3] = pv.y; }
+            dst[0] = a;
+            dst[1] = b;
         }
     }
 }
@@ -331,65 +421,101 @@ __global__ void __launch_bounds__(PO_T) probe_order_kernel(const int32_t* __rest
     }
 }
 
+// debug export: fine voxel index of each of a tile's first min(n_probe, count) queries in
+// the level's query order (its probes, in rank order), -1 after them
+__global__ void probe_export_kernel(const int32_t* __restrict__ tile_off, const int32_t* __restrict__ plist,
+                                    const int32_t* __restrict__ qorder, int R2, int n_probe,
+                                    int32_t* __restrict__ out) {
+    const int t = blockIdx.x;
+    const int base = 8 * tile_off[t];
+    const int cnt = 8 * (tile_off[t + 1] - tile_off[t]);
+    const int nd = cnt < n_probe ? cnt : n_probe;
+    for (int i = threadIdx.x; i < n_probe; i += blockDim.x) {
+        int32_t v = -1;
+        if (i < nd) {
+            const int e = qorder[base + i];
+            v = (int32_t)child_index(plist[e >> 3], e & 7, R2);
+        }
+        out[(size_t)t * n_probe + i] = v;
+    }
+}
+
 }  // namespace
 
-vdm_status launch_mark_dilate(const float* f, int R, uint64_t* words, cudaStream_t s) {
-    const int nb = R >> 2, ncta = (nb + 1) >> 1;
+vdm_status launch_probe_export(const int32_t* tile_off, int n_tiles, const int32_t* plist,
+                               const int32_t* qorder, int R2, int n_probe, int32_t* out, cudaStream_t s) {
+    if (n_tiles <= 0) return VDM_OK;
+    probe_export_kernel<<<n_tiles, 128, 0, s>>>(tile_off, plist, qorder, R2, n_probe, out);
+    return check_launch("probe_export_kernel");
+}
+
+size_t mark_bits_words(int R) {
+    const size_t nb = (size_t)(R >> 2);
+    return 2 * nb * nb * nb;
+}
+
+vdm_status launch_mark_dilate(const float* f, int R, uint64_t* words, uint64_t* bits, cudaStream_t s) {
+    if (R % 4 || R < 4 || R > 1024) return fail(VDM_ERR_UNSUPPORTED, "mark: R = %d", R);
+    const int nb = R >> 2;
+    const size_t nw = (size_t)nb * nb * nb;
     const float thr = (float)(4.0 / (double)R);
+    const int smem = 4 * MW_N * (int)sizeof(uint64_t);   // 55 KB: set for the current device
+    cudaError_t e = cudaFuncSetAttribute(mark_words_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "mark_words smem attribute: %s", cudaGetErrorString(e));
+    const int ncta = (nb + MW_C - 1) / MW_C;
     prof_begin(kProfMark, s);
-    mark_dilate_kernel<<<ncta * ncta * ncta, MD_T, 0, s>>>(f, R, thr, words);
+    pack_kernel<<<nb * nb, PK_T, 0, s>>>(f, R, thr, bits, bits + nw);
+    mark_words_kernel<true><<<ncta * ncta * ncta, MW_T, smem, s>>>(bits, bits + nw, nb, words);
     prof_end(kProfMark, s);
-    return check_launch("mark_dilate_kernel");
+    return check_launch("mark kernels");
 }
 
-size_t scan_tmp_ints(int n_words) {
-    const int nblk = (n_words + SC_BLK - 1) / SC_BLK;
-    return (size_t)2 * nblk + 8;
+vdm_status launch_sign_change(const float* f, int R, uint64_t* words, uint64_t* bits, cudaStream_t s) {
+    if (R % 4 || R < 4 || R > 1024) return fail(VDM_ERR_UNSUPPORTED, "sign change: R = %d", R);
+    const int nb = R >> 2;
+    const size_t nw = (size_t)nb * nb * nb;
+    const int smem = 4 * MW_N * (int)sizeof(uint64_t);
+    cudaError_t e = cudaFuncSetAttribute(mark_words_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "mark_words smem attribute: %s", cudaGetErrorString(e));
+    const int ncta = (nb + MW_C - 1) / MW_C;
+    // threshold 0: no near-surface bits, only voxels with a neighbour of the other sign
+    pack_kernel<<<nb * nb, PK_T, 0, s>>>(f, R, 0.0f, bits, bits + nw);
+    mark_words_kernel<false><<<ncta * ncta * ncta, MW_T, smem, s>>>(bits, bits + nw, nb, words);
+    return check_launch("sign change kernels");
 }
 
-vdm_status launch_word_scan(const uint64_t* words, int n_words, int32_t* word_off, int32_t* tile_ids,
-                            int32_t* counts, int32_t* block_tmp, cudaStream_t s) {
-    const int nblk = (n_words + SC_BLK - 1) / SC_BLK;
-    int2* bsum = reinterpret_cast<int2*>(block_tmp);
-    prof_begin(kProfScan, s);
-    scan_reduce_kernel<<<nblk, SC_T, 0, s>>>(words, n_words, bsum);
-    prof_end(kProfScan, s);
-    VDM_TRY(check_launch("scan_reduce_kernel"));
-    prof_begin(kProfScan, s);
-    scan_blocks_kernel<<<1, SC_T, 0, s>>>(bsum, nblk, counts);
-    prof_end(kProfScan, s);
-    VDM_TRY(check_launch("scan_blocks_kernel"));
-    prof_begin(kProfScan, s);
-    scan_write_kernel<<<nblk, SC_T, 0, s>>>(words, n_words, bsum, word_off, tile_ids, counts);
-    prof_end(kProfScan, s);
-    return check_launch("scan_write_kernel");
+size_t compact_tmp_ints(int n_words) {
+    const int nchunk = (n_words + CP_CHUNK - 1) / CP_CHUNK;
+    return (size_t)2 * nchunk + 8;
 }
 
-vdm_status launch_parent_list(const uint64_t* words, const int32_t* word_off, int n_words, int R,
-                              int32_t* plist, cudaStream_t s) {
+vdm_status launch_compact(const uint64_t* words, int n_words, int R, int32_t* word_off, int32_t* tile_ids,
+                          int32_t* tile_off, int32_t* plist, int32_t* counts, int32_t* chunk_tmp,
+                          cudaStream_t s) {
+    const int nchunk = (n_words + CP_CHUNK - 1) / CP_CHUNK;
+    int2* csum = reinterpret_cast<int2*>(chunk_tmp);
+    prof_begin(kProfScan, s);
+    chunk_sum_kernel<<<nchunk, CP_T, 0, s>>>(words, n_words, csum);
+    prof_end(kProfScan, s);
+    VDM_TRY(check_launch("chunk_sum_kernel"));
     prof_begin(kProfList, s);
-    parent_list_kernel<<<(n_words + 255) / 256, 256, 0, s>>>(words, word_off, n_words, R, plist);
+    compact_kernel<<<nchunk, CP_T, 0, s>>>(words, n_words, R, csum, word_off, tile_ids, tile_off, plist, counts);
     prof_end(kProfList, s);
-    return check_launch("parent_list_kernel");
+    return check_launch("compact_kernel");
 }
 
-vdm_status launch_tile_offsets(const int32_t* word_off, const int32_t* tile_ids, int n_tiles,
-                               int n_words, int32_t* tile_off, cudaStream_t s) {
-    prof_begin(kProfList, s);
-    tile_off_kernel<<<(n_tiles + 1 + 255) / 256, 256, 0, s>>>(word_off, tile_ids, n_tiles, n_words, tile_off);
-    prof_end(kProfList, s);
-    return check_launch("tile_off_kernel");
-}
-
-vdm_status launch_fill(const float* f_coarse, const uint64_t* words, int R, float* f_fine, cudaStream_t s) {
-    const size_t n = (size_t)(2 * R) * (2 * R) * ((2 * R) >> 2);
+vdm_status launch_fill(const float* f_coarse, int R, float* f_fine, cudaStream_t s) {
+    const size_t n = (size_t)(2 * R) * (2 * R) * ((2 * R) >> 3);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const size_t want = (n + 255) / 256;
-    const int grid = (int)(want < (size_t)sms * 16 ? want : (size_t)sms * 16);
+    const int grid = (int)(want < (size_t)sms * 8 ? want : (size_t)sms * 8);
+    // a fine grid much larger than L2 is written with streaming stores
+    const bool stream = n * 32 > ((size_t)64 << 20);
     prof_begin(kProfFill, s);
-    fill_kernel<<<grid, 256, 0, s>>>(f_coarse, words, R, f_fine);
+    if (stream) fill_kernel<true><<<grid, 256, 0, s>>>(f_coarse, R, f_fine);
+    else fill_kernel<false><<<grid, 256, 0, s>>>(f_coarse, R, f_fine);
     prof_end(kProfFill, s);
     return check_launch("fill_kernel");
 }

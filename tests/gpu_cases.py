@@ -35,9 +35,9 @@ class Case:
             self._okv[b] = OD.precompute_kv(self.z[b], self.w)
         return self._okv[b]
 
-    def oracle_dec(self, p: np.ndarray, b: int = 0, sel=None) -> np.ndarray:
+    def oracle_dec(self, p: np.ndarray, b: int = 0, sel=None, want_attn: bool = False):
         K, V = self.okv(b)
-        return OD.decode_points(p, K, V, self.w, self.spec.query_ln, sel=sel)
+        return OD.decode_points(p, K, V, self.w, self.spec.query_ln, sel=sel, return_attn=want_attn)
 
     def sp(self, b: int = 0):
         return None if self.spheres_np is None else self.spheres_np[b]
@@ -52,9 +52,13 @@ def unpack_words(words: np.ndarray, R: int) -> np.ndarray:
     return bits.transpose(0, 3, 1, 4, 2, 5).reshape(R, R, R)
 
 
-def debug_buffers(B: int, r0: int, L: int, adaptive: bool, k: int, max_tiles: int):
+def debug_buffers(B: int, r0: int, L: int, adaptive: bool, k: int, max_tiles: int,
+                  n_probe: int = 0, N: int = 0, C: int = 0, attn_stride: int = 0):
+    """Device buffers for ``vdm_hier_debug``; unwritten entries keep a sentinel
+    (NaN, -1 or -2) so that a missing write shows."""
     import torch
-    dbg = {"grid": [], "active": [], "dec": [], "tile_ids": [], "sel": [], "max_tiles": max_tiles}
+    dbg = {"grid": [], "active": [], "dec": [], "tile_ids": [], "sel": [], "probes": [], "scores": [],
+           "attn": [], "max_tiles": max_tiles, "attn_stride": attn_stride}
     for l in range(L):
         R = r0 << l
         dbg["grid"].append(torch.empty((B, R ** 3), device="cuda", dtype=torch.float32))
@@ -64,21 +68,38 @@ def debug_buffers(B: int, r0: int, L: int, adaptive: bool, k: int, max_tiles: in
         if adaptive and l > 0:
             dbg["tile_ids"].append(torch.full((B, max_tiles), -1, device="cuda", dtype=torch.int32))
             dbg["sel"].append(torch.full((B, max_tiles, k), -1, device="cuda", dtype=torch.int32))
+            dbg["probes"].append(torch.full((B, max_tiles, n_probe), -2, device="cuda", dtype=torch.int32)
+                                 if n_probe else None)
+            dbg["scores"].append(torch.full((B, max_tiles, N), float("nan"), device="cuda",
+                                            dtype=torch.float32) if N else None)
         else:
-            dbg["tile_ids"].append(None)
-            dbg["sel"].append(None)
+            for key in ("tile_ids", "sel", "probes", "scores"):
+                dbg[key].append(None)
+        if attn_stride:
+            rows = -(-R ** 3 // attn_stride)
+            dbg["attn"].append(torch.full((B, rows, C), float("nan"), device="cuda", dtype=torch.float32))
+        else:
+            dbg["attn"].append(None)
     return dbg
 
 
 def check_levels(case: Case, b: int, r0: int, L: int, dbg, dec_scale: float, adaptive: bool,
-                 n_probe: int, seed: int, sample: int = 0, rng=None, report=None):
+                 n_probe: int, seed: int, sample: int = 0, rng=None, report=None,
+                 score_tiles: int = 16, attn_rows: int = 256):
     """Level-by-level parity of one shape's hierarchical decode.
 
     * refine masks bit-exact vs the oracle's mark+dilate of the GPU's own grid;
     * inherited voxels equal their parent's value exactly;
     * decoded voxels: raw decoder output within tolerance of the oracle at the
       same points (adaptive non-probes attend over the GPU's selection), and the
-      stored field equals sphere SDF + scale tanh(dec) of the GPU's own dec.
+      stored field equals sphere SDF + scale tanh(dec) of the GPU's own dec;
+    * adaptive levels (when the debug buffers hold them): the sub-volume list,
+      every sub-volume's probe set and rank order exactly the oracle's
+      (``choose_probes``), every selection exactly the oracle's Top-K rule on
+      the GPU's own scores, and the scores of ``score_tiles`` sub-volumes within
+      2e-2 * max of the oracle's ``token_scores``;
+    * attention output (when exported): up to ``attn_rows`` sampled voxels per
+      level within 2e-2 * max|a| of the oracle's.
     ``sample`` > 0 compares a random subset of the decoded voxels only.
     """
     tol = TOL[case.spec.dtype]
@@ -86,6 +107,7 @@ def check_levels(case: Case, b: int, r0: int, L: int, dbg, dec_scale: float, ada
     report = report if report is not None else {}
     grids = [dbg["grid"][l][b].cpu().numpy() for l in range(L)]
     decs = [dbg["dec"][l][b].cpu().numpy() for l in range(L)]
+    stride = int(dbg.get("attn_stride", 0) or 0)
     worst = 0.0
     for l in range(L):
         R = r0 << l
@@ -115,8 +137,14 @@ def check_levels(case: Case, b: int, r0: int, L: int, dbg, dec_scale: float, ada
         assert np.abs(g.ravel()[decoded] - fld).max() < 1e-5
         idx = decoded if not sample or decoded.size <= sample else \
             np.sort(rng.choice(decoded, sample, replace=False))
+        ad = None
         if l > 0 and adaptive:
-            want = _oracle_adaptive_dec(case, b, R, decoded, idx, dbg, l, n_probe, seed)
+            ad = AdaptiveLevel(case, b, R, decoded, dbg, l, n_probe, seed)
+            if dbg.get("probes") and dbg["probes"][l] is not None:
+                report[f"probe_tiles_{l}"] = ad.check_probes()
+            if dbg.get("scores") and dbg["scores"][l] is not None:
+                report[f"topk_tiles_{l}"], report[f"score_err_{l}"] = ad.check_selection(score_tiles, rng)
+            want = ad.oracle(idx)[0]
         else:
             want = case.oracle_dec(OD.grid_points(R, idx), b)
         got = decs[l][idx].astype(np.float64)
@@ -124,45 +152,130 @@ def check_levels(case: Case, b: int, r0: int, L: int, dbg, dec_scale: float, ada
         worst = max(worst, err)
         report[f"err_{l}"] = err
         assert err <= tol, f"level {l}: max abs dec error {err} > {tol}"
+        if stride and dbg["attn"][l] is not None:
+            cand = decoded[decoded % stride == 0]
+            if cand.size > attn_rows:
+                cand = np.sort(rng.choice(cand, attn_rows, replace=False))
+            if cand.size:
+                a_gpu = dbg["attn"][l][b].cpu().numpy()[cand // stride].astype(np.float64)
+                assert np.isfinite(a_gpu).all(), f"level {l}: attention rows not written"
+                if ad is not None:
+                    a_ref = ad.oracle(cand, want_attn=True)[1]
+                else:
+                    a_ref = case.oracle_dec(OD.grid_points(R, cand), b, want_attn=True)[1]
+                aerr = float(np.abs(a_gpu - a_ref).max())
+                scale = float(np.abs(a_ref).max())
+                report[f"attn_err_{l}"] = aerr / scale
+                assert aerr <= 2e-2 * scale, f"level {l}: attention error {aerr} > 2e-2 * {scale}"
     report["worst"] = worst
     return report
 
 
-def _oracle_adaptive_dec(case, b, R, decoded, idx, dbg, l, n_probe, seed):
-    """Oracle raw decoder output at voxels ``idx`` of adaptive level ``l``:
-    probes / small sub-volumes with full attention, the others over the GPU's
-    Top-K subset of their sub-volume."""
-    tiles = OA.tile_of(decoded, R, 8)
-    tid_gpu = dbg["tile_ids"][l][b].cpu().numpy()
-    sel_gpu = dbg["sel"][l][b].cpu().numpy()
-    row = {int(t): n for n, t in enumerate(tid_gpu) if t >= 0}
-    want = np.empty(idx.size)
-    idx_tiles = OA.tile_of(idx, R, 8)
-    pos = {int(v): n for n, v in enumerate(idx)}
-    checked = [0]
-    for t in np.unique(idx_tiles):
-        members = np.sort(decoded[tiles == t])
-        probe = OA.choose_probes(members, n_probe, seed, l)
-        mine = idx[idx_tiles == t]
-        is_probe = probe[np.searchsorted(members, mine)]
-        dense_pts = mine[is_probe]
-        if dense_pts.size:
-            v = case.oracle_dec(OD.grid_points(R, dense_pts), b)
-            for p_, x in zip(dense_pts, v):
-                want[pos[int(p_)]] = x
-        sparse_pts = mine[~is_probe]
-        if sparse_pts.size:
-            assert int(t) in row, f"tile {t} has no GPU selection"
-            sel = sel_gpu[row[int(t)]]
-            assert (sel >= 0).all() and np.all(np.diff(sel) > 0)
-            if checked[0] < 16:   # the selection itself: the oracle's Top-K from the same probes
-                K, _ = case.okv(b)
-                q = OA.query_vectors(OD.grid_points(R, members[probe]), case.w)
-                top = OA.top_k(OA.token_scores(q, K), sel.size)
-                overlap = len(np.intersect1d(sel, top)) / sel.size
-                assert overlap >= 0.9, f"tile {t}: Top-K overlap {overlap}"
-                checked[0] += 1
-            v = case.oracle_dec(OD.grid_points(R, sparse_pts), b, sel=sel)
-            for p_, x in zip(sparse_pts, v):
-                want[pos[int(p_)]] = x
-    return want
+class AdaptiveLevel:
+    """Oracle view of one adaptive level, built from the GPU's decoded set and
+    debug exports: sub-volumes, probes (``choose_probes``), scores, Top-K."""
+
+    def __init__(self, case, b, R, decoded, dbg, l, n_probe, seed):
+        self.case, self.b, self.R, self.l = case, b, R, l
+        self.n_probe, self.seed = n_probe, seed
+        self.dbg = dbg
+        self.tiles = OA.tile_of(decoded, R, 8)
+        self.decoded = decoded
+        self.tid_gpu = dbg["tile_ids"][l][b].cpu().numpy()
+        self.sel_gpu = dbg["sel"][l][b].cpu().numpy()
+        self.row = {int(t): n for n, t in enumerate(self.tid_gpu) if t >= 0}
+        order = np.argsort(self.tiles, kind="stable")
+        self._members = {}
+        ts = self.tiles[order]
+        bounds = np.flatnonzero(np.diff(ts)) + 1
+        for grp in np.split(order, bounds):
+            if grp.size:
+                self._members[int(self.tiles[grp[0]])] = np.sort(decoded[grp])
+        self._probe = {}
+
+    def members(self, t):
+        return self._members[int(t)]
+
+    def probe_mask(self, t):
+        if t not in self._probe:
+            self._probe[t] = OA.choose_probes(self.members(t), self.n_probe, self.seed, self.l)
+        return self._probe[t]
+
+    def check_probes(self):
+        """The sub-volume list and every probe set (in rank order) exactly the oracle's."""
+        uniq = np.array(sorted(self._members))
+        mt = self.tid_gpu.size
+        assert np.array_equal(self.tid_gpu[:min(mt, uniq.size)], uniq[:mt]), \
+            f"level {self.l}: sub-volume list differs"
+        pr = self.dbg["probes"][self.l][self.b].cpu().numpy()
+        n = min(mt, uniq.size)
+        for i in range(n):
+            t = int(uniq[i])
+            mem = self.members(t)
+            nd = min(mem.size, self.n_probe)
+            got = pr[i, :nd]
+            assert np.all(pr[i, nd:] == -1), f"level {self.l} sub-volume {t}: probe padding"
+            if mem.size <= self.n_probe:
+                assert np.array_equal(np.sort(got), mem), f"level {self.l} sub-volume {t}: dense set"
+            else:
+                key = OA.probe_key(self.seed, self.l, mem)
+                want = mem[np.lexsort((mem, key))[:self.n_probe]]
+                assert np.array_equal(got, want), f"level {self.l} sub-volume {t}: probes differ"
+        return n
+
+    def check_selection(self, score_tiles, rng):
+        """Every selection = Top-K rule on the GPU's scores; sampled scores vs oracle."""
+        sc = self.dbg["scores"][self.l][self.b].cpu().numpy()
+        K, _ = self.case.okv(self.b)
+        H = K.shape[0]
+        sel_rows = [i for i, t in enumerate(self.tid_gpu) if t >= 0 and
+                    self.members(int(t)).size > self.n_probe]
+        k = self.sel_gpu.shape[1]
+        for i in sel_rows:
+            s = sc[i].astype(np.float64)
+            assert np.isfinite(s).all(), f"level {self.l} row {i}: scores not written"
+            assert np.array_equal(self.sel_gpu[i], OA.top_k(s, k)), \
+                f"level {self.l} sub-volume {self.tid_gpu[i]}: selection is not the Top-K of its scores"
+            assert abs(s.sum() - self.n_probe * H) <= 2e-3 * self.n_probe * H
+        pick = sel_rows if len(sel_rows) <= score_tiles else \
+            sorted(rng.choice(sel_rows, score_tiles, replace=False))
+        worst = 0.0
+        for i in pick:
+            t = int(self.tid_gpu[i])
+            mem = self.members(t)
+            q = OA.query_vectors(OD.grid_points(self.R, mem[self.probe_mask(t)]), self.case.w)
+            want = OA.token_scores(q, K)
+            err = float(np.abs(sc[i] - want).max())
+            worst = max(worst, err / max(1.0, want.max()))
+            assert err <= 2e-2 * max(1.0, want.max()), \
+                f"level {self.l} sub-volume {t}: score error {err}"
+        return len(sel_rows), worst
+
+    def oracle(self, idx, want_attn=False):
+        """Oracle raw decoder output (and attention output) at voxels ``idx``:
+        probes / small sub-volumes with full attention, the others over the
+        GPU's Top-K subset of their sub-volume."""
+        C = self.case.spec.C
+        want = np.empty(idx.size)
+        attn = np.empty((idx.size, C)) if want_attn else None
+        idx_tiles = OA.tile_of(idx, self.R, 8)
+        for t in np.unique(idx_tiles):
+            mem = self.members(t)
+            probe = self.probe_mask(int(t))
+            here = np.flatnonzero(idx_tiles == t)
+            mine = idx[here]
+            is_probe = probe[np.searchsorted(mem, mine)]
+            for sub, sel in ((here[is_probe], None), (here[~is_probe], "gpu")):
+                if sub.size == 0:
+                    continue
+                if sel == "gpu":
+                    assert int(t) in self.row, f"tile {t} has no GPU selection"
+                    sel = self.sel_gpu[self.row[int(t)]]
+                    assert (sel >= 0).all() and np.all(np.diff(sel) > 0)
+                r = self.case.oracle_dec(OD.grid_points(self.R, idx[sub]), self.b, sel=sel,
+                                         want_attn=want_attn)
+                if want_attn:
+                    want[sub], attn[sub] = r
+                else:
+                    want[sub] = r
+        return want, attn

@@ -19,14 +19,14 @@ def _header_functions():
 
 def test_every_declared_function_is_exported():
     names = _header_functions()
-    assert len(names) == 13, names
+    assert len(names) == len(vdm.EXPORTS), names
     for n in names:
         assert hasattr(vdm._lib, n), n
     assert set(names) == set(vdm.EXPORTS)
 
 
 def test_status_strings_and_version():
-    assert vdm.abi_version() == 1
+    assert vdm.abi_version() == 2
     assert vdm._lib.vdm_status_string(0) == b"ok"
     assert vdm._lib.vdm_status_string(3) == b"workspace too small"
 
@@ -95,3 +95,32 @@ def test_workspace_sizes_and_too_small_workspace(cid):
     st = vdm._lib.vdm_decode_hierarchical(C.byref(d), 0x1000, 0x2000, 1, cfg.dec.N, C.byref(p), None,
                                           0x3000, 0x4000, n - 1024, stats, None, None)
     assert st == 3 and b"workspace" in vdm._lib.vdm_last_error()
+
+
+def test_compare_volumes_argument_errors():
+    lib = vdm._lib
+    assert lib.vdm_compare_volumes(None, None, -1, 0x1000, None) == 1        # negative size
+    assert lib.vdm_compare_volumes(None, None, 10, 0x1000, None) == 1        # null inputs
+    assert lib.vdm_compare_volumes(0x1000, 0x2000, 10, 0x1004, None) == 1    # misaligned out
+
+
+def test_surface_case_table_equals_the_oracle_rules():
+    """Host logic, no GPU: the library generates its marching-cubes table from the
+    stated face and fan rules; every one of the 256 sign patterns gives exactly
+    the oracle's triangles (edge ids, order)."""
+    from oracle import surface as OS
+    ntri, tri = vdm.vdm_surface_case_table()
+    for cfg in range(256):
+        want = OS.cube_triangles(cfg)
+        assert ntri[cfg] == len(want), cfg
+        assert [tuple(int(x) for x in t) for t in tri[cfg, :ntri[cfg]]] == [tuple(t) for t in want], cfg
+
+
+def test_surface_workspace_and_argument_errors():
+    n = C.c_size_t(0)
+    assert vdm._lib.vdm_surface_workspace_size(12, C.byref(n)) == 2       # R % 8
+    assert vdm._lib.vdm_surface_workspace_size(2048, C.byref(n)) == 2     # too large
+    assert vdm._lib.vdm_surface_workspace_size(64, C.byref(n)) == 0 and n.value > 64 ** 3
+    nv, nt = C.c_int64(0), C.c_int64(0)
+    assert vdm._lib.vdm_extract_surface(None, 64, None, 0, None, 0, C.byref(nv), C.byref(nt),
+                                        0x1000, n.value, None) == 1

@@ -48,3 +48,31 @@ def test_reference_arm_prints_on_rank_zero_only():
               "--warmup", "3")
     assert p0.returncode == 0, p0.stderr
     assert _line(p0.stdout)["n_gpus"] == 2
+
+
+def test_peak_choice_follows_the_sampled_clock():
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = {"bf16": 1700.0, "bf16_sust": 1390.0, "sm_max_mhz": 1965.0}
+    at_max = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    capped = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    slow = {"sm_mhz": 1300.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.pick_tc_peak(peaks, at_max) == (1700.0, "burst")
+    assert bench.pick_tc_peak(peaks, capped) == (1390.0, "sustained")
+    assert bench.pick_tc_peak(peaks, slow) == (1390.0, "sustained")
+    assert bench.pick_tc_peak(peaks, {"sm_mhz": None, "reasons": []}) == (1390.0, "sustained")
+
+
+def test_level_kernel_bytes_by_hand():
+    # one level step 8 -> 16 with 10 refined parents: mark reads 4*512 and writes 64 bytes;
+    # scan/list read the 64-byte mask twice, write 12*(2^3) and 4*10; the fill reads 4*512 + 64
+    # and writes 4*(8*512 - 80)
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    cfg = W.CONFIGS[3].with_(r0=8, n_levels=2)
+    st = [{"active_parents": [0, 10]}]
+    b = bench.level_kernel_bytes(cfg, st)
+    assert b["mark"] == 2048 + 64
+    assert b["scan_list"] == 128 + 96 + 40
+    assert b["fill"] == 2048 + 64 + 4 * (4096 - 80)

@@ -17,27 +17,52 @@ from gpu_cases import TOL, Case, check_levels, debug_buffers
 pytestmark = pytest.mark.gpu
 
 
-def _run(case, B, r0, L, adaptive, n_probe=64, top_k=1024, seed=0, dec_scale=0.01, max_tiles=0):
+def _run(case, B, r0, L, adaptive, n_probe=64, top_k=1024, seed=0, dec_scale=0.01, max_tiles=0,
+         attn_stride=0, exports=True):
     import neural_sdf_volume_b200 as vdm
     p = vdm.hier_params(r0, L, adaptive, 8, n_probe, top_k, seed)
     k = min(top_k, case.spec.N)
     mt = max_tiles or (r0 << (L - 1)) // 8
     mt = mt ** 3 if not max_tiles else max_tiles
-    dbg = debug_buffers(B, r0, L, adaptive, k, mt)
+    dbg = debug_buffers(B, r0, L, adaptive, k, mt, n_probe=n_probe if exports else 0,
+                        N=case.spec.N if exports else 0, C=case.spec.C, attn_stride=attn_stride)
     grid, stats = vdm.vdm_decode_hierarchical(case.dec, case.K, case.V, p, case.spheres, dec_scale,
                                               debug=dbg)
     return grid, stats, dbg
 
 
-@pytest.mark.parametrize("adaptive,n_probe", [(False, 16), (True, 16), (True, 32)])
-def test_small_hierarchical_matches_full_oracle(adaptive, n_probe):
+def _analytic_sign_agreement(grid, spheres, Rf, margin=0.011, chunk=1 << 20):
+    """Share of the voxels with |sphere SDF| > margin whose final value has the
+    sphere SDF's sign: there field = sphere SDF + 0.01 tanh(dec) cannot change
+    sign, whatever the decoder says.  Returns (agreeing, counted)."""
+    g = grid.reshape(-1)
+    agree = counted = 0
+    for s0 in range(0, Rf ** 3, chunk):
+        idx = np.arange(s0, min(s0 + chunk, Rf ** 3))
+        sd = OD.sphere_sdf(OD.grid_points(Rf, idx), spheres)
+        m = np.abs(sd) > margin
+        agree += int(((g[idx][m] < 0) == (sd[m] < 0)).sum())
+        counted += int(m.sum())
+    return agree, counted
+
+
+@pytest.mark.parametrize("stress", [False, True])
+@pytest.mark.parametrize("adaptive,n_probe", [(False, 16), (True, 16), (True, 32), (True, 64)])
+def test_small_hierarchical_matches_full_oracle(adaptive, n_probe, stress):
     """12 -> 24 -> 48 with the full-width bf16 decoder (N=256, C=512): every
-    level checked, then the final sign compared with the oracle's own run.
-    16 probes per sub-volume score on CUDA cores, 32 on the tensor cores."""
+    level checked (probe sets and Top-K exact, attention output at sampled
+    voxels), then the final sign compared with the oracle's own run.  16 probes
+    per sub-volume score on CUDA cores, 32 and 64 on the tensor cores.  The
+    stress weights give attention logits of order 5 and a value bias, so a
+    wrong gathered row or a wrong softmax shows in the output."""
     spec = W.DecoderSpec(C=512, H=8, F=2048, N=256, query_ln=True, dtype="bf16")
-    case = Case(spec, key=2, n_spheres=5, sphere_key=3)
-    grid, stats, dbg = _run(case, 1, 12, 3, adaptive, n_probe=n_probe, top_k=64)
-    rep = check_levels(case, 0, 12, 3, dbg, 0.01, adaptive, n_probe, 0)
+    case = Case(spec, key=2, n_spheres=5, sphere_key=3, stress=stress)
+    grid, stats, dbg = _run(case, 1, 12, 3, adaptive, n_probe=n_probe, top_k=64, attn_stride=7)
+    rep = check_levels(case, 0, 12, 3, dbg, 0.01, adaptive, n_probe, 0, score_tiles=64,
+                       attn_rows=400)
+    if adaptive:   # the exact checks ran on some sub-volumes
+        assert rep["probe_tiles_1"] > 0 and rep["probe_tiles_2"] > 0
+        assert rep["topk_tiles_1"] + rep["topk_tiles_2"] > 0
     assert stats[0]["decoded"][0] == 12 ** 3
     assert stats[0]["decoded"][1] == rep["decoded_1"] and stats[0]["decoded"][2] == rep["decoded_2"]
     K, V = case.okv()
@@ -81,27 +106,37 @@ def test_adaptive_k_equal_n_is_dense_decode():
 
 @pytest.mark.parametrize("cid", [3, 4])
 def test_full_size_96_to_384(cid):
+    """Full workloads 3 and 4: masks bit-exact, sampled decoded voxels and
+    attention rows within tolerance, (4) every sub-volume's probes and Top-K
+    exact and 32 sub-volumes' scores within tolerance per level, and the final
+    sign equal to the analytic sign on >= 99.99 % of the voxels whose sign the
+    decoder term cannot change."""
     cfg = W.CONFIGS[cid]
     case = Case(cfg.dec, key=cfg.seed_key, n_spheres=cfg.n_spheres, sphere_key=cfg.sphere_key)
     grid, stats, dbg = _run(case, 1, cfg.r0, cfg.n_levels, cfg.adaptive, cfg.n_probe, cfg.top_k,
-                            dec_scale=cfg.dec_scale)
+                            dec_scale=cfg.dec_scale, max_tiles=16384, attn_stride=4099)
     rep = check_levels(case, 0, cfg.r0, cfg.n_levels, dbg, cfg.dec_scale, cfg.adaptive,
-                       cfg.n_probe, 0, sample=256)
+                       cfg.n_probe, 0, sample=256, score_tiles=32, attn_rows=64)
     n_dec = sum(stats[0]["decoded"][:3])
     saved = 1.0 - n_dec / 384 ** 3
-    print(f"config {cid}: decoded per level {stats[0]['decoded'][:3]}, queries saved {saved:.3f}, {rep}")
+    agree, counted = _analytic_sign_agreement(grid[0].cpu().numpy(), case.sp(), 384)
+    print(f"config {cid}: decoded per level {stats[0]['decoded'][:3]}, queries saved {saved:.3f}, "
+          f"sign agreement {agree}/{counted}, {rep}")
     assert saved > 0.8
+    assert agree >= 0.9999 * counted
 
 
 def test_full_size_batched_slim_adaptive():
     cfg = W.CONFIGS[5]
     case = Case(cfg.dec, key=cfg.seed_key, B=cfg.B, n_spheres=cfg.n_spheres, sphere_key=cfg.sphere_key)
     grid, stats, dbg = _run(case, cfg.B, cfg.r0, cfg.n_levels, True, cfg.n_probe, cfg.top_k,
-                            dec_scale=cfg.dec_scale, max_tiles=40000)
+                            dec_scale=cfg.dec_scale, max_tiles=40000, attn_stride=8191)
     for b in (0, 3):
         assert stats[b]["tiles"][2] <= 40000
         check_levels(case, b, cfg.r0, cfg.n_levels, dbg, cfg.dec_scale, True, cfg.n_probe, 0,
-                     sample=128, rng=np.random.default_rng(b))
+                     sample=128, rng=np.random.default_rng(b), score_tiles=16, attn_rows=64)
+        agree, counted = _analytic_sign_agreement(grid[b].cpu().numpy(), case.sp(b), 512)
+        assert agree >= 0.9999 * counted, (b, agree, counted)
 
 
 def test_select_kv_scores_and_topk_given_the_same_scores():

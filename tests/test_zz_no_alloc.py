@@ -14,7 +14,7 @@ import pytest
 
 import workloads as W
 
-from gpu_cases import TOL, Case
+from gpu_cases import Case
 
 pytestmark = pytest.mark.gpu
 
@@ -48,8 +48,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         assert st == 0, vdm._lib.vdm_last_error()
         got = out.cpu().numpy()
         assert np.isfinite(got).all(), f"call {call}: voxels left unwritten"
-        err = float(np.abs(got - ref).max())
-        assert err <= TOL["bf16"], f"call {call}: max abs difference {err}"
+        # same kernels on the same inputs: the library's results are bit-identical run to run
+        assert np.array_equal(got, ref), f"call {call}: max abs difference {np.abs(got - ref).max()}"
         for b in range(B):
             assert list(stats[b].decoded) == ref_stats[b]["decoded"]
 

@@ -84,6 +84,9 @@ class Config:
 _DEC_TINY = DecoderSpec(C=64, H=1, F=256, N=256, query_ln=True, dtype="f32")
 _DEC_FULL = DecoderSpec(C=512, H=8, F=2048, N=3072, query_ln=True, dtype="bf16")
 _DEC_SLIM = DecoderSpec(C=256, H=4, F=512, N=4096, query_ln=False, dtype="bf16")
+# the efficient decoder at a quarter of the full width: narrower, smaller MLP ratio, no
+# query-side LayerNorm (techwalker article, section 5; aipaper.cc summary, section 4.1 item 3)
+_DEC_QUARTER = DecoderSpec(C=128, H=2, F=256, N=3072, query_ln=False, dtype="bf16")
 
 CONFIGS: Dict[int, Config] = {
     1: Config(1, "tiny dense fp32, 32^3", _DEC_TINY, grid_R=32, seed_key=1),
@@ -96,6 +99,9 @@ CONFIGS: Dict[int, Config] = {
     5: Config(5, "batched slim decoder, 4 shapes, 128->256->512, adaptive KV",
               _DEC_SLIM, B=4, mode="hier", r0=128, n_levels=3, adaptive=True,
               n_spheres=24, dec_scale=0.01, seed_key=5, sphere_key=5),
+    6: Config(6, "quarter-width efficient decoder, hierarchical + adaptive KV bf16, 96->192->384",
+              _DEC_QUARTER, mode="hier", r0=96, n_levels=3, adaptive=True, n_spheres=16,
+              dec_scale=0.01, seed_key=6, sphere_key=3),
 }
 
 
