@@ -105,19 +105,23 @@ def adaptive_level(level: int, R: int, kids: np.ndarray, K: np.ndarray, V: np.nd
                    w: Dict[str, np.ndarray], query_ln: bool, spheres: Optional[np.ndarray],
                    dec_scale: float, seed: int, tile: int = 8, n_probe: int = 64,
                    k: int = 1024, sel_override: Optional[Dict[int, np.ndarray]] = None,
-                   keep_tiles: bool = False) -> Dict:
+                   keep_tiles: bool = False, tsdf_trunc: Optional[float] = None) -> Dict:
     """Field values of fine level ``level`` at the active voxels ``kids``.
 
     ``sel_override`` maps tile id -> token subset and replaces the oracle's
     own selection for that tile (used to compare a decode given the same
     selection).  Returns ``values`` (aligned with ``kids``), ``dec`` (raw
     decoder outputs) and, with ``keep_tiles``, per-tile probes/scores/subsets.
+    With ``tsdf_trunc`` the tSDF head is decoded too (same attention) and
+    ``tsdf`` holds ``decoder.tsdf_field`` at ``kids``.
     """
     if R % tile:
         raise ValueError("fine resolution must be a multiple of the tile edge")
     kids = np.asarray(kids, np.int64)
     vals = np.empty(kids.size, np.float64)
     decs = np.empty(kids.size, np.float64)
+    tsdf = np.empty(kids.size, np.float64) if tsdf_trunc is not None else None
+    want_t = tsdf is not None
     tiles = {}
     tid = tile_of(kids, R, tile)
     order = np.lexsort((kids, tid))
@@ -130,20 +134,33 @@ def adaptive_level(level: int, R: int, kids: np.ndarray, K: np.ndarray, V: np.nd
         pts = D.grid_points(R, idx)
         probe = choose_probes(idx, n_probe, seed, level)
         dec = np.empty(idx.size, np.float64)
-        dec[probe] = D.decode_points(pts[probe], K, V, w, query_ln)
+        traw = np.empty(idx.size, np.float64)
+        r = D.decode_points(pts[probe], K, V, w, query_ln, return_tsdf=want_t)
+        if want_t:
+            dec[probe], traw[probe] = r
+        else:
+            dec[probe] = r
         info = {"idx": idx, "probe": probe}
         if (~probe).any():
             score = token_scores(query_vectors(pts[probe], w), K)
             sel = top_k(score, k)
             if sel_override is not None and t in sel_override:
                 sel = np.asarray(sel_override[t], np.int64)
-            dec[~probe] = D.decode_points(pts[~probe], K, V, w, query_ln, sel=sel)
+            r = D.decode_points(pts[~probe], K, V, w, query_ln, sel=sel, return_tsdf=want_t)
+            if want_t:
+                dec[~probe], traw[~probe] = r
+            else:
+                dec[~probe] = r
             info.update(score=score, sel=sel)
         decs[grp] = dec
         vals[grp] = D.field(pts, dec, spheres, dec_scale)
+        if want_t:
+            tsdf[grp] = D.tsdf_field(pts, traw, spheres, dec_scale, tsdf_trunc)
         if keep_tiles:
             tiles[t] = info
     out = {"values": vals, "dec": decs}
+    if want_t:
+        out["tsdf"] = tsdf
     if keep_tiles:
         out["tiles"] = tiles
     return out

@@ -133,17 +133,22 @@ def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray,
 
 def decode_points(p: np.ndarray, K: np.ndarray, V: np.ndarray, w: Dict[str, np.ndarray],
                   query_ln: bool = True, sel: Optional[np.ndarray] = None,
-                  chunk: int = 512, return_attn: bool = False):
+                  chunk: int = 512, return_attn: bool = False, return_tsdf: bool = False):
     """Raw decoder output ``dec`` at points ``p[M,3]`` (float64 ``[M]``).
 
     ``sel`` restricts attention to a subset of token indices (adaptive KV
     selection, section 4.1 item 2 step 5).  With ``return_attn`` the
-    attention output ``a[M,C]`` is returned too.
+    attention output ``a[M,C]`` is returned too.  With ``return_tsdf`` the
+    raw truncated-SDF head is returned too: a second linear head on the same
+    final features, ``t = w_tsdf . LN2(x2) + b_tsdf`` (the pages' VAE is
+    trained to output a tSDF beside the SDF, aipaper.cc summary section 4.1
+    item 1, "key details" 1).
     """
     p = np.asarray(p, np.float64).reshape(-1, 3)
     M = p.shape[0]
     out = np.empty(M, np.float64)
     attn = np.empty((M, K.shape[0] * HEAD_DIM)) if return_attn else None
+    tsdf = np.empty(M, np.float64) if return_tsdf else None
     for s in range(0, M, chunk):
         pe = fourier_embed(p[s:s + chunk])
         q = linear(pe, w["Wq"], w["bq"])
@@ -155,7 +160,10 @@ def decode_points(p: np.ndarray, K: np.ndarray, V: np.ndarray, w: Dict[str, np.n
         x2 = x1 + linear(gelu(linear(h_in, w["W1"], w["b1"])), w["W2"], w["b2"])
         y = layer_norm(x2, w["ln2_g"], w["ln2_b"]) if query_ln else x2
         out[s:s + chunk] = y @ np.asarray(w["w_head"], np.float64) + float(w["b_head"][0])
-    return (out, attn) if return_attn else out
+        if return_tsdf:
+            tsdf[s:s + chunk] = y @ np.asarray(w["w_tsdf"], np.float64) + float(w["b_tsdf"][0])
+    res = (out,) + ((attn,) if return_attn else ()) + ((tsdf,) if return_tsdf else ())
+    return res if len(res) > 1 else out
 
 
 def sphere_sdf(p: np.ndarray, spheres: np.ndarray) -> np.ndarray:
@@ -165,6 +173,18 @@ def sphere_sdf(p: np.ndarray, spheres: np.ndarray) -> np.ndarray:
     sp = np.asarray(spheres, np.float64)
     d = np.sqrt(((p[:, None, :] - sp[None, :, :3]) ** 2).sum(axis=2)) - sp[None, :, 3]
     return d.min(axis=1)
+
+
+def tsdf_field(p: np.ndarray, t: np.ndarray, spheres: Optional[np.ndarray], dec_scale: float,
+               trunc: float) -> np.ndarray:
+    """Synthetic truncated SDF: ``clip((sphere SDF + dec_scale tanh(t)) / trunc,
+    -1, 1)`` with ``t`` the raw tSDF head; the raw head itself without
+    spheres.  (A tSDF saturates at +-1 beyond the truncation distance and
+    measures closeness to the surface inside it.)"""
+    t = np.asarray(t, np.float64)
+    if spheres is None:
+        return t
+    return np.clip((sphere_sdf(p, spheres) + float(dec_scale) * np.tanh(t)) / float(trunc), -1.0, 1.0)
 
 
 def field(p: np.ndarray, dec: np.ndarray, spheres: Optional[np.ndarray],

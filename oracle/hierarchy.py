@@ -50,10 +50,13 @@ def _shift_views(a: np.ndarray, pad_value):
         yield p[1 + di:1 + di + R, 1 + dj:1 + dj + R, 1 + dk:1 + dk + R]
 
 
-def mark(f: np.ndarray, thr) -> np.ndarray:
+def mark(f: np.ndarray, thr, near: Optional[np.ndarray] = None) -> np.ndarray:
     """Boundary mark of a dense level grid ``f[R,R,R]``.
 
-    ``mark(v) = (exists in-grid u in cube(v): (f_u < 0) != (f_v < 0)) or |f_v| < thr``
+    ``mark(v) = (exists in-grid u in cube(v): (f_u < 0) != (f_v < 0)) or near(v)``
+    with ``near(v) = |f_v| < thr``, or the given ``near`` mask (the tSDF rule:
+    ``|tsdf_v| < threshold``, section 4.1 item 1 "key details" 1; 0.95 on the
+    techwalker article, section 5).
     """
     f = np.asarray(f)
     inside = f < 0
@@ -66,7 +69,7 @@ def mark(f: np.ndarray, thr) -> np.ndarray:
     for di, dj, dk in _OFFSETS:
         nb = p[1 + di:1 + di + R, 1 + dj:1 + dj + R, 1 + dk:1 + dk + R]
         change |= (nb >= 0) & (nb != inside)
-    return change | (np.abs(f) < thr)
+    return change | ((np.abs(f) < thr) if near is None else np.asarray(near, bool))
 
 
 def dilate(m: np.ndarray) -> np.ndarray:
@@ -119,31 +122,48 @@ def fill(f_coarse: np.ndarray, child_idx: np.ndarray, child_val: np.ndarray) -> 
 
 def hierarchical(decode_level: Callable[[int, int, np.ndarray], np.ndarray],
                  r0: int, n_levels: int, dilation: int = 1,
-                 dtype=np.float64, coarse: Optional[np.ndarray] = None) -> Dict:
+                 dtype=np.float64, coarse: Optional[np.ndarray] = None,
+                 tsdf_threshold: Optional[float] = None) -> Dict:
     """Coarse-to-fine decoding.
 
     ``decode_level(level, R, idx)`` returns field values at the voxels
-    ``idx`` (linear, resolution R) of level ``level`` (0 = coarse).
+    ``idx`` (linear, resolution R) of level ``level`` (0 = coarse); with
+    ``tsdf_threshold`` it returns ``(field, tsdf)`` and the near-surface rule
+    is ``|tsdf| < tsdf_threshold`` (compared in float32), the tSDF grid being
+    decoded and inherited like the field.
     ``coarse`` optionally supplies the level-0 grid instead of decoding it.
     Returns the final dense grid and, per level, the masks, active parents,
     decoded children and their values.
     """
     R = r0
+    use_t = tsdf_threshold is not None
+    tg = None
     if coarse is None:
-        f = decode_level(0, R, np.arange(R ** 3, dtype=np.int64)).astype(dtype).reshape(R, R, R)
+        r = decode_level(0, R, np.arange(R ** 3, dtype=np.int64))
+        if use_t:
+            r, t0 = r
+            tg = np.asarray(t0, dtype).reshape(R, R, R)
+        f = np.asarray(r).astype(dtype).reshape(R, R, R)
     else:
         f = np.asarray(coarse, dtype).reshape(R, R, R)
-    levels: List[Dict] = [{"R": R, "grid": f}]
+    levels: List[Dict] = [{"R": R, "grid": f, "tsdf": tg}]
     for lv in range(1, n_levels):
-        m = mark(f, near_threshold(R))
+        near = None
+        if use_t:
+            near = np.abs(tg.astype(np.float32)) < np.float32(tsdf_threshold)
+        m = mark(f, near_threshold(R), near=near)
         act = m
         for _ in range(dilation):
             act = dilate(act)
         parents = compact(act)
         kids = children(parents, R)
-        vals = decode_level(lv, 2 * R, kids).astype(dtype)
+        r = decode_level(lv, 2 * R, kids)
+        if use_t:
+            r, tv = r
+            tg = fill(tg, kids, np.asarray(tv).astype(dtype))
+        vals = np.asarray(r).astype(dtype)
         f = fill(f, kids, vals)
         levels[-1].update(mark=m, active=act, parents=parents)
         R *= 2
-        levels.append({"R": R, "grid": f, "children": kids, "values": vals})
+        levels.append({"R": R, "grid": f, "children": kids, "values": vals, "tsdf": tg})
     return {"grid": f, "levels": levels}

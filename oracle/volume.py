@@ -34,26 +34,34 @@ def dense_grid(K, V, w, R: int, query_ln: bool, spheres=None, dec_scale: float =
 def hierarchical_volume(K, V, w, r0: int, n_levels: int, query_ln: bool, spheres=None,
                         dec_scale: float = 0.0, adaptive: bool = False, seed: int = 0,
                         tile: int = 8, n_probe: int = 64, top_k: int = 1024,
-                        coarse: Optional[np.ndarray] = None, keep_tiles: bool = False) -> Dict:
+                        coarse: Optional[np.ndarray] = None, keep_tiles: bool = False,
+                        tsdf_trunc: Optional[float] = None, tsdf_threshold: float = 0.95) -> Dict:
     """Hierarchical decoding of one shape, optionally with adaptive KV on the
     fine levels.  Returns ``hierarchy.hierarchical``'s dict plus, per fine
-    level, the raw decoder outputs (``dec``) and adaptive tile records."""
+    level, the raw decoder outputs (``dec``) and adaptive tile records.  With
+    ``tsdf_trunc`` the decoder's tSDF head drives the near-surface rule
+    (``|tsdf| < tsdf_threshold``) instead of ``|f| < 2h``."""
     extras = {}
+    want_t = tsdf_trunc is not None
 
-    def decode_level(level: int, R: int, idx: np.ndarray) -> np.ndarray:
+    def decode_level(level: int, R: int, idx: np.ndarray):
         p = D.grid_points(R, idx)
         if level == 0 or not adaptive:
-            dec = D.decode_points(p, K, V, w, query_ln)
+            r = D.decode_points(p, K, V, w, query_ln, return_tsdf=want_t)
+            dec = r[0] if want_t else r
             extras[level] = {"dec": dec}
-            return D.field(p, dec, spheres, dec_scale)
+            f = D.field(p, dec, spheres, dec_scale)
+            return (f, D.tsdf_field(p, r[1], spheres, dec_scale, tsdf_trunc)) if want_t else f
         out = A.adaptive_level(level, R, idx, K, V, w, query_ln, spheres, dec_scale, seed,
-                               tile=tile, n_probe=n_probe, k=top_k, keep_tiles=keep_tiles)
+                               tile=tile, n_probe=n_probe, k=top_k, keep_tiles=keep_tiles,
+                               tsdf_trunc=tsdf_trunc)
         extras[level] = out
-        return out["values"]
+        return (out["values"], out["tsdf"]) if want_t else out["values"]
 
-    res = HV.hierarchical(decode_level, r0, n_levels, coarse=coarse)
+    res = HV.hierarchical(decode_level, r0, n_levels, coarse=coarse,
+                          tsdf_threshold=tsdf_threshold if want_t else None)
     for lv, e in extras.items():
-        res["levels"][lv].update({k: v for k, v in e.items() if k != "values"})
+        res["levels"][lv].update({k: v for k, v in e.items() if k not in ("values", "tsdf")})
     return res
 
 

@@ -263,3 +263,31 @@ def test_decoder_query_layernorm_before_mlp_closed_form():
     # (x2 = LN1(x1) + MLP, post-norm style)
     for slip in (ln(x1 + gelu(x1)), ln(ln(x1) + gelu(ln(x1)))):
         assert abs(slip[0] - want) > 1e-2
+
+
+def test_tsdf_head_reads_the_same_final_features():
+    # the tSDF head is a second linear head on LN2(x2): at the origin (C = 64, q = PE on
+    # 51 lanes, 24 ones at the cos lanes) a unit weight on lane 27 reads (1 - 3/8) / sigma
+    C = 64
+    w = _zero_weights(C, 64)
+    w["Wq"][:51, :51] = np.eye(51)
+    w["w_head"][0] = 1.0
+    w["w_tsdf"] = np.zeros(C); w["w_tsdf"][27] = 1.0
+    w["b_tsdf"] = np.array([0.125])
+    K = np.zeros((1, 3, 64)); V = np.zeros((1, 3, 64))
+    mean, var = 24 / 64, 24 / 64 * (1 - 24 / 64)
+    dec, t = D.decode_points(np.zeros((1, 3)), K, V, w, query_ln=True, return_tsdf=True)
+    assert dec[0] == pytest.approx((0 - mean) / math.sqrt(var + 1e-5), abs=1e-13)
+    assert t[0] == pytest.approx((1 - mean) / math.sqrt(var + 1e-5) + 0.125, abs=1e-13)
+
+
+def test_tsdf_field_truncates_the_distance():
+    sp = np.array([[0.0, 0.0, 0.0, 0.5]])
+    p = np.array([[0.0, 0.0, 0.52], [0.0, 0.45, 0.0], [0.9, 0.0, 0.0], [0.0, 0.0, 0.0]])
+    got = D.tsdf_field(p, np.zeros(4), sp, 0.01, trunc=0.1)
+    np.testing.assert_allclose(got, [0.2, -0.5, 1.0, -1.0], atol=1e-14)
+    t = np.array([0.0, 0.0, 0.0, 0.0]) + 3.0
+    np.testing.assert_allclose(D.tsdf_field(p, t, sp, 0.01, trunc=0.1),
+                               np.clip((np.array([0.02, -0.05, 0.4, -0.5]) + 0.01 * np.tanh(3.0)) / 0.1, -1, 1),
+                               atol=1e-14)
+    assert np.array_equal(D.tsdf_field(p, t, None, 0.01, 0.1), t)

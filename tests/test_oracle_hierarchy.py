@@ -115,3 +115,33 @@ def test_hierarchical_exact_sdf_lipschitz_guarantee():
     # fewer queries than dense decoding
     n_q = r0 ** 3 + sum(lv["children"].size for lv in res["levels"][1:])
     assert n_q < 0.6 * Rf ** 3
+
+
+def test_tsdf_rule_equals_a_distance_band_for_an_exact_field():
+    # dec_scale = 0: tsdf = clip(sdf / trunc), so |tsdf| < 0.95 marks exactly the voxels with
+    # |sdf| < 0.95 trunc (grid chosen so that no voxel sits on the band edge)
+    from oracle import decoder as D
+    R, trunc = 24, 0.2
+    sp = np.array([[0.1, -0.05, 0.02, 0.437]])
+    p = D.grid_points(R)
+    f = D.sphere_sdf(p, sp).reshape(R, R, R)
+    t = D.tsdf_field(p, np.zeros(p.shape[0]), sp, 0.0, trunc).reshape(R, R, R)
+    assert np.abs(np.abs(f) - 0.95 * trunc).min() > 1e-4
+    near = np.abs(t.astype(np.float32)) < np.float32(0.95)
+    assert np.array_equal(HV.mark(f, 0.0, near=near), HV.mark(f, 0.95 * trunc))
+    assert near.sum() > (np.abs(f) < HV.near_threshold(R)).sum()     # a wider band than 2 h
+
+
+def test_hierarchical_carries_the_tsdf_grid():
+    # decode_level returning (field, tsdf): the tsdf grid is inherited like the field and its
+    # band decides the refinement; with a zero tsdf everywhere every voxel is near: all refined
+    from oracle import decoder as D
+    sp = np.array([[0.0, 0.0, 0.0, 0.5]])
+
+    def dl(level, R, idx):
+        p = D.grid_points(R, idx)
+        return D.sphere_sdf(p, sp), np.zeros(idx.size)
+
+    out = HV.hierarchical(dl, 4, 3, tsdf_threshold=0.95)
+    assert out["levels"][0]["active"].all() and out["levels"][1]["active"].all()
+    assert out["levels"][2]["tsdf"].shape == (16, 16, 16) and not out["levels"][2]["tsdf"].any()

@@ -38,6 +38,7 @@ N_FREQ = 8
 _A_Z, _A_WQ, _A_WK, _A_WV, _A_WO, _A_W1, _A_W2, _A_WH = range(8)
 _A_CENTRE, _A_RADIUS, _A_POINTS = 8, 9, 10
 _A_STRESS = 20
+_A_WT = 21
 
 
 @dataclass(frozen=True)
@@ -118,7 +119,7 @@ def round_bf16(a: np.ndarray) -> np.ndarray:
 
 
 def make_decoder(spec: DecoderSpec, seed: int = 0, key: int = 0, B: int = 1,
-                 stress: bool = False) -> Dict[str, np.ndarray]:
+                 stress: bool = False, tsdf: bool = False) -> Dict[str, np.ndarray]:
     """Latents ``z[B,N,C]`` (float32) and decoder parameters (float32 arrays).
 
     Matrices follow the ``y = x W^T + b`` convention with ``W[out][in]``.
@@ -126,7 +127,9 @@ def make_decoder(spec: DecoderSpec, seed: int = 0, key: int = 0, B: int = 1,
     embedding and are zero.  With ``stress`` the query/key projections get
     std 0.2 (attention logits of order 5 instead of nearly uniform weights)
     and biases, LayerNorm affines and a non-zero-mean value bias are drawn
-    too, so that an error in any of them shows in the output.
+    too, so that an error in any of them shows in the output.  With ``tsdf``
+    a second head ``w_tsdf`` (N(0, 0.02^2), stress: 0.2) and ``b_tsdf`` (0)
+    are drawn for the truncated-SDF output channel.
     """
     C, F, N = spec.C, spec.F, spec.N
     std = 0.02
@@ -165,6 +168,9 @@ def make_decoder(spec: DecoderSpec, seed: int = 0, key: int = 0, B: int = 1,
             w[k] = (r.standard_normal(C) * 0.1).astype(np.float32)
         w["b_head"] = np.array([0.05], np.float32)
 
+    if tsdf:
+        w["w_tsdf"] = mat(_A_WT, (C,), 0.2 if stress else std)
+        w["b_tsdf"] = np.zeros((1,), np.float32)
     z = _rng(seed, key, _A_Z).standard_normal((B, N, C)).astype(np.float32)
     return {"z": z, "weights": w}
 
