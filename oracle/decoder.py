@@ -133,7 +133,8 @@ def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray,
 
 def decode_points(p: np.ndarray, K: np.ndarray, V: np.ndarray, w: Dict[str, np.ndarray],
                   query_ln: bool = True, sel: Optional[np.ndarray] = None,
-                  chunk: int = 512, return_attn: bool = False, return_tsdf: bool = False):
+                  chunk: int = 512, return_attn: bool = False, return_tsdf: bool = False,
+                  return_features: bool = False):
     """Raw decoder output ``dec`` at points ``p[M,3]`` (float64 ``[M]``).
 
     ``sel`` restricts attention to a subset of token indices (adaptive KV
@@ -142,13 +143,15 @@ def decode_points(p: np.ndarray, K: np.ndarray, V: np.ndarray, w: Dict[str, np.n
     raw truncated-SDF head is returned too: a second linear head on the same
     final features, ``t = w_tsdf . LN2(x2) + b_tsdf`` (the pages' VAE is
     trained to output a tSDF beside the SDF, aipaper.cc summary section 4.1
-    item 1, "key details" 1).
+    item 1, "key details" 1).  With ``return_features`` the block output
+    ``x2[M,C]`` (before the head's LayerNorm) is returned last.
     """
     p = np.asarray(p, np.float64).reshape(-1, 3)
     M = p.shape[0]
     out = np.empty(M, np.float64)
     attn = np.empty((M, K.shape[0] * HEAD_DIM)) if return_attn else None
     tsdf = np.empty(M, np.float64) if return_tsdf else None
+    feats = np.empty((M, K.shape[0] * HEAD_DIM)) if return_features else None
     for s in range(0, M, chunk):
         pe = fourier_embed(p[s:s + chunk])
         q = linear(pe, w["Wq"], w["bq"])
@@ -158,11 +161,14 @@ def decode_points(p: np.ndarray, K: np.ndarray, V: np.ndarray, w: Dict[str, np.n
         x1 = q + linear(a, w["Wo"], w["bo"])
         h_in = layer_norm(x1, w["ln1_g"], w["ln1_b"]) if query_ln else x1
         x2 = x1 + linear(gelu(linear(h_in, w["W1"], w["b1"])), w["W2"], w["b2"])
+        if return_features:
+            feats[s:s + chunk] = x2
         y = layer_norm(x2, w["ln2_g"], w["ln2_b"]) if query_ln else x2
         out[s:s + chunk] = y @ np.asarray(w["w_head"], np.float64) + float(w["b_head"][0])
         if return_tsdf:
             tsdf[s:s + chunk] = y @ np.asarray(w["w_tsdf"], np.float64) + float(w["b_tsdf"][0])
-    res = (out,) + ((attn,) if return_attn else ()) + ((tsdf,) if return_tsdf else ())
+    res = (out,) + ((attn,) if return_attn else ()) + ((tsdf,) if return_tsdf else ()) + \
+        ((feats,) if return_features else ())
     return res if len(res) > 1 else out
 
 

@@ -37,6 +37,7 @@ N_FREQ = 8
 # array ids for the per-array seed sequences
 _A_Z, _A_WQ, _A_WK, _A_WV, _A_WO, _A_W1, _A_W2, _A_WH = range(8)
 _A_CENTRE, _A_RADIUS, _A_POINTS = 8, 9, 10
+_A_CLOUD, _A_QUERY, _A_WIN = 11, 12, 13
 _A_STRESS = 20
 _A_WT = 21
 
@@ -185,6 +186,43 @@ def make_spheres(n_spheres: int, seed: int = 0, key: int = 0, B: int = 1) -> np.
 def make_points(M: int, seed: int = 0, key: int = 0, B: int = 1) -> np.ndarray:
     """``[B, M, 3]`` float32 query points uniform in [-1, 1]^3."""
     return _rng(seed, key, _A_POINTS).uniform(-1.0, 1.0, (B, M, 3)).astype(np.float32)
+
+
+def make_point_cloud(spheres: np.ndarray, n_points: int, n_queries: int, seed: int = 0,
+                     key: int = 0) -> Dict[str, np.ndarray]:
+    """A point cloud on the surface of a union of spheres ``[S,4]`` and the
+    encoder's latent query points, a uniform random subset of it.
+
+    Points are drawn on the spheres in proportion to their areas (uniform
+    directions); points inside another sphere are not on the union's surface
+    and are drawn again.  Returns ``points [n_points, 3]`` and
+    ``queries [n_queries, 3]`` (float32)."""
+    rng = _rng(seed, key, _A_CLOUD)
+    sp = np.asarray(spheres, np.float64)
+    area = sp[:, 3] ** 2
+    out = []
+    while sum(len(x) for x in out) < n_points:
+        s_idx = rng.choice(len(sp), n_points, p=area / area.sum())
+        d = rng.standard_normal((n_points, 3))
+        d /= np.linalg.norm(d, axis=1, keepdims=True)
+        pts = sp[s_idx, :3] + d * sp[s_idx, 3:4]
+        dist = np.sqrt(((pts[:, None, :] - sp[None, :, :3]) ** 2).sum(axis=2)) - sp[None, :, 3]
+        inside_other = (dist < -1e-6).any(axis=1)
+        out.append(pts[~inside_other])
+    pts = np.concatenate(out)[:n_points].astype(np.float32)
+    q = _rng(seed, key, _A_QUERY).permutation(n_points)[:n_queries]
+    return {"points": pts, "queries": pts[np.sort(q)]}
+
+
+def make_encoder_input_proj(C: int, seed: int = 0, key: int = 0, dtype: str = "bf16") -> Dict[str, np.ndarray]:
+    """The encoder's point-feature projection ``W_in [C,64]`` (columns 51..63
+    face the zero pad lanes) ~ N(0, 0.02^2), rounded to bf16 for bf16 blocks,
+    and ``b_in = 0``."""
+    w = np.zeros((C, PE_PAD), np.float32)
+    w[:, :PE_DIM] = (_rng(seed, key, _A_WIN).standard_normal((C, PE_DIM)) * 0.02).astype(np.float32)
+    if dtype == "bf16":
+        w = round_bf16(w)
+    return {"W_in": w, "b_in": np.zeros((C,), np.float32)}
 
 
 def make_inputs(cfg: Config, seed: int = 0, stress: bool = False) -> Dict[str, np.ndarray]:
