@@ -38,6 +38,7 @@ N_FREQ = 8
 _A_Z, _A_WQ, _A_WK, _A_WV, _A_WO, _A_W1, _A_W2, _A_WH = range(8)
 _A_CENTRE, _A_RADIUS, _A_POINTS = 8, 9, 10
 _A_CLOUD, _A_QUERY, _A_WIN = 11, 12, 13
+_A_LOCAL = 30
 _A_STRESS = 20
 _A_WT = 21
 
@@ -223,6 +224,34 @@ def make_encoder_input_proj(C: int, seed: int = 0, key: int = 0, dtype: str = "b
     if dtype == "bf16":
         w = round_bf16(w)
     return {"W_in": w, "b_in": np.zeros((C,), np.float32)}
+
+
+def make_local_decoder(spheres: np.ndarray, n_anchors=(4096, 16384), channels=(64, 32), hidden: int = 16,
+                       fuse_hidden: int = 64, seed: int = 0, key: int = 0) -> Dict:
+    """A two-scale latent hierarchy for the local (MSVS-style) decoder query and
+    its weights: per scale s, anchors on the surface of a union of spheres
+    (``n_anchors[s]`` points, as point-shuffle upsampling would place them near
+    the surface), features ``~ N(0, 1)`` with ``channels[s]`` channels (halving
+    from scale to scale), dynamic-weight MLP ``W1 [hidden,3] ~ N(0, 4^2)``
+    (relative offsets are a few hundredths), ``b1 ~ N(0, 0.5^2)``,
+    ``W2 [C,hidden] ~ N(0, 0.25^2)``, ``b2 = 0``; fusion ``Wf [fuse_hidden, sum C]
+    ~ N(0, 0.1^2)``, ``bf = 0``, ``wo ~ N(0, 0.1^2)``, ``bo = 0`` (float32)."""
+    out = {"anchors": [], "feats": [], "scales": []}
+    for s, (n, C) in enumerate(zip(n_anchors, channels)):
+        out["anchors"].append(make_point_cloud(spheres, n, 1, seed, key * 16 + s)["points"])
+        r = _rng(seed, key * 16 + s, _A_LOCAL)
+        out["feats"].append(r.standard_normal((n, C)).astype(np.float32))
+        out["scales"].append({"W1": (r.standard_normal((hidden, 3)) * 4.0).astype(np.float32),
+                              "b1": (r.standard_normal(hidden) * 0.5).astype(np.float32),
+                              "W2": (r.standard_normal((C, hidden)) * 0.25).astype(np.float32),
+                              "b2": np.zeros(C, np.float32)})
+    r = _rng(seed, key, _A_LOCAL + 1)
+    cs = int(sum(channels))
+    out["fuse"] = {"Wf": (r.standard_normal((fuse_hidden, cs)) * 0.1).astype(np.float32),
+                   "bf": np.zeros(fuse_hidden, np.float32),
+                   "wo": (r.standard_normal(fuse_hidden) * 0.1).astype(np.float32),
+                   "bo": np.zeros(1, np.float32)}
+    return out
 
 
 def make_inputs(cfg: Config, seed: int = 0, stress: bool = False) -> Dict[str, np.ndarray]:
