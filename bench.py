@@ -52,7 +52,7 @@ def _peaks():
 # dram__bytes_read.sum + dram__bytes_write.sum per decode launch of one shape of a
 # workload (mean over the shape's decode launches), from ncu's one-pass DRAM counters on
 # this script's own launches; None until captured for the current decoder kernel.
-DECODE_DRAM_BYTES_PER_LAUNCH = {}
+DECODE_DRAM_BYTES_PER_LAUNCH = {4: 39.66e6}
 
 
 def decode_flops_per_query(spec: W.DecoderSpec, n_tokens: int) -> float:
@@ -292,7 +292,7 @@ def run_sweep(args, local):
     return None
 
 
-def level_kernels_large(vdm, cfg, dev, flush, steps, peaks):
+def level_kernels_large(vdm, cfg, dev, flush, steps, peaks, sizes=(384, 512)):
     """The level kernels (vdm_refine_level: mark + dilation, compaction, inherit
     fill) timed alone on level grids larger than the 126 MB L2 (L2 flushed
     before every call): a union of the workload's spheres sampled at R^3, the
@@ -300,7 +300,7 @@ def level_kernels_large(vdm, cfg, dev, flush, steps, peaks):
     import torch
     sp = torch.from_numpy(W.make_spheres(cfg.n_spheres, 0, cfg.sphere_key, 1)[0]).to(dev).double()
     out = {}
-    for R in (384, 512):
+    for R in sizes:
         x = -1.0 + (2.0 * torch.arange(R, device=dev, dtype=torch.float64) + 1.0) / R
         f = torch.empty((R, R, R), device=dev, dtype=torch.float32)
         for i in range(R):   # one slab at a time keeps the temporaries small
@@ -533,6 +533,32 @@ def run_vdm(args, world, rank, local):
                 "flops_per_query_vs_full_width": decode_flops_per_query(c6.dec, c6.dec.N) /
                 decode_flops_per_query(cfg.dec, cfg.dec.N),
                 "decoder_tflop_per_shape": f6 / 1e12}
+        if cfg.cid == 4:   # vecset encoding of a surface point cloud with a full-width block
+            M_pts, N_tok = 8192, cfg.dec.N
+            cloud = W.make_point_cloud(sp_np[0], M_pts, N_tok, seed=0, key=7)
+            proj = W.make_encoder_input_proj(cfg.dec.C, seed=0, key=7)
+            blk_w = W.make_decoder(cfg.dec, seed=0, key=7)["weights"]
+            blk = vdm.Decoder.from_numpy(blk_w, cfg.dec.C, cfg.dec.H, cfg.dec.F, cfg.dec.query_ln, cfg.dec.dtype,
+                                         device=dev)
+            W_in = torch.from_numpy(proj["W_in"]).to(dev).bfloat16()
+            b_in = torch.from_numpy(proj["b_in"]).to(dev)
+            pts = torch.from_numpy(cloud["points"][None]).to(dev)
+            qs = torch.from_numpy(cloud["queries"][None]).to(dev)
+            tenc = _timed(lambda: vdm.vdm_encode(blk, W_in, b_in, pts, qs), args.steps, 3, stream, flush)
+            C_, H_, F_ = cfg.dec.C, cfg.dec.H, cfg.dec.F
+            enc_flops = 2.0 * (M_pts * (51 * C_ + 2 * C_ * C_) +
+                               N_tok * (51 * C_ + 2 * H_ * M_pts * 64 + C_ * C_ + 2 * C_ * F_))
+            res["vecset_encoder"] = {"workload": f"{M_pts}-point surface cloud -> {N_tok} tokens, C={C_}",
+                                     "ms_per_shape": tenc, "TFLOP/s": enc_flops / (tenc / 1e3) / 1e12}
+        if cfg.cid == 4:   # the local (MSVS-style) decoder query at the MSVS page's 200K-query batch
+            ldw = W.make_local_decoder(sp_np[0], seed=0, key=9)
+            ld = vdm.LocalDecoder.from_numpy(ldw, 8, device=dev)
+            q200 = torch.from_numpy(W.make_points(200_000, seed=0, key=9)[0]).to(dev)
+            tloc = _timed(lambda: vdm.vdm_decode_local(ld, q200), args.steps, 3, stream, flush)
+            res["local_decoder_200k"] = {
+                "workload": "200,000 uniform queries, 2 scales (4096 + 16384 surface anchors, C 64 + 32), K = 8",
+                "ms": tloc, "points_per_s": 200_000 / (tloc / 1e3),
+                "context": "MSVS page, 3.3: 213 ms (MSVS) vs 3068 ms (Lattice) for 200K queries, hardware not stated"}
         if cfg.adaptive:
             res["accuracy_vs_dense"] = accuracy_vs_dense(vdm, dec, K, V, cfg, spheres, params, ws, out)
             res["accuracy_vs_dense"].pop("_vol_d", None)
@@ -675,6 +701,8 @@ def main():
     ap.add_argument("--impl", default="vdm", choices=["vdm", "reference"])
     ap.add_argument("--config", type=int, default=4, choices=[1, 2, 3, 4, 5, 6],
                     help="3-6: hierarchical workloads (the step of the headline metric); 1-2: dense grids")
+    ap.add_argument("--level-only", type=int, default=0, metavar="R",
+                    help="only time the level kernels (vdm_refine_level) on an R^3 grid of the workload's spheres")
     ap.add_argument("--sweep", action="store_true",
                     help="adaptive-KV settings (probes, kept tokens) against time and error, one line each")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -691,6 +719,15 @@ def main():
         res = run_reference(args, world, rank)
     elif args.sweep:
         res = run_sweep(args, local)
+    elif args.level_only:
+        import torch
+
+        import neural_sdf_volume_b200 as vdm
+        torch.cuda.set_device(local)
+        dev = torch.device("cuda", local)
+        flush = torch.empty((L2_FLUSH_BYTES // 4,), device=dev, dtype=torch.float32)
+        res = {"level_kernels": level_kernels_large(vdm, W.CONFIGS[args.config], dev, flush, args.steps, _peaks(),
+                                                    sizes=(args.level_only,))}
     elif args.dense_queries > 0 or args.config in (1, 2):
         res = run_dense(args, world, rank, local)
     else:

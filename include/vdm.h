@@ -110,6 +110,13 @@ typedef struct {
     const float *ln1_g, *ln1_b, *ln2_g, *ln2_b;          /* [C]              */
     const float* w_head;                                 /* [C]              */
     const float* b_head;                                 /* [1]              */
+    /* Optional truncated-SDF head (NULL: none): t = w_tsdf . LN2(x2) + b_tsdf,
+     * a second linear output on the same final features (the pages' VAE is
+     * trained to output a tSDF beside the SDF: aipaper.cc summary, section
+     * 4.1 item 1, "key details" 1).  With it, hierarchical decoding takes
+     * |tSDF| < vdm_hier_params.tsdf_threshold as its near-surface rule.      */
+    const float* w_tsdf;                                 /* [C] or NULL      */
+    const float* b_tsdf;                                 /* [1]              */
 } vdm_decoder;
 
 /* Analytic term of the synthetic field (optional).                         */
@@ -117,6 +124,8 @@ typedef struct {
     const float* spheres;  /* device [B][n_spheres][4] = (cx, cy, cz, r)     */
     int32_t n_spheres;     /* >= 1                                           */
     float dec_scale;       /* field = sphere SDF + dec_scale * tanh(dec)     */
+    float tsdf_trunc;      /* with a tSDF head: tSDF = clip((sphere SDF +
+                              dec_scale * tanh(t)) / tsdf_trunc, -1, 1); > 0 */
 } vdm_analytic;
 
 /* K/V projection of B vecsets (section 3: the vecset feeds the decoder's
@@ -168,6 +177,10 @@ typedef struct {
     int32_t n_probe;     /* probes per sub-volume, 1..512                    */
     int32_t top_k;       /* kept tokens per sub-volume                       */
     uint64_t seed;       /* probe sampler seed                               */
+    float tsdf_threshold;/* with a tSDF head: near-surface voxels are those
+                            with |tSDF| < tsdf_threshold (0.95 on the pages:
+                            techwalker article, section 5), compared in
+                            float32; without one: |f| < float32(4 / R)      */
 } vdm_hier_params;
 
 /* Per-shape, per-level counts written by vdm_decode_hierarchical (host).   */
@@ -220,6 +233,9 @@ typedef struct {
                                            v / attn_stride; other rows are
                                            left untouched                    */
     int64_t attn_stride;                /* >= 1 when any attn[l] is set       */
+    float* tsdf[VDM_MAX_LEVELS];        /* [B][R_l^3] tSDF grid of level l
+                                           (decoded or inherited), decoders
+                                           with a tSDF head only             */
 } vdm_hier_debug;
 
 /* Workspace bytes needed by vdm_decode_hierarchical (host output).         */
@@ -230,7 +246,8 @@ VDM_API vdm_status vdm_hierarchical_workspace_size(const vdm_decoder* dec, const
  * on the fine levels when p->adaptive):
  *   level 0: dense decode of the r0^3 grid;
  *   level l -> l+1: mark voxels with a sign change in their 3x3x3
- *   neighbourhood or |f| < 2h (h = 2/R_l, threshold float32(4/R_l)), dilate
+ *   neighbourhood or |f| < 2h (h = 2/R_l, threshold float32(4/R_l); with a
+ *   tSDF head: |tSDF| < p->tsdf_threshold instead), dilate
  *   once (3x3x3), decode the 8 children of every marked voxel at 2R_l, and let
  *   the other fine voxels inherit their parent's value.
  *   d_grid_out [B][Rf^3] float32 final field, Rf = r0 * 2^(n_levels-1)
@@ -289,6 +306,70 @@ VDM_API vdm_status vdm_refine_workspace_size(int32_t R, size_t* bytes);
 VDM_API vdm_status vdm_refine_level(const float* d_f, int32_t R, float* d_f_fine, uint64_t* d_mask,
                                     int32_t* d_parents, int32_t* d_counts, void* d_ws, size_t ws_bytes,
                                     vdm_stream stream);
+
+/* Vecset encoding: a point cloud -> a vecset of N latent tokens by
+ * cross-attention (aipaper.cc summary, section 3 "Foundational Concepts:
+ * encoder").  The tokens sit at N query points (normally a subset of the
+ * cloud); every point of the cloud is embedded with the decoder's Fourier
+ * features and projected, u = W_in pe(p) + b_in; the block's LayerNorm and K/V
+ * projections make keys and values of u (as vdm_precompute_kv does of
+ * latents); each token runs the block from its query point (q = Wq pe(x) + bq,
+ * attention over the cloud, x1 = q + Wo a + bo, x2 = x1 + MLP(LN1 x1)) and is
+ * its block output x2.  The block uses the vdm_decoder layout; its head and
+ * LN2 are not used.
+ *   blk         block parameters (any supported C; dtype of W_in as well)
+ *   d_W_in      [C][64] in blk->dtype (columns 51..63 meet zero lanes); d_b_in [C]
+ *   d_points    [B][M][3] float32, 1 <= M <= 8192;  d_queries [B][N][3] float32
+ *   d_z_out     [B][N][C] float32 vecsets (a decoder's vdm_precompute_kv input)
+ *   d_ws/ws_bytes  device workspace >= vdm_encode_workspace_size(blk, M)
+ * Returns after the encoding has finished on `stream`.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA, TIMEOUT.               */
+VDM_API vdm_status vdm_encode_workspace_size(const vdm_decoder* blk, int32_t M, size_t* bytes);
+VDM_API vdm_status vdm_encode(const vdm_decoder* blk, const void* d_W_in, const float* d_b_in,
+                              const float* d_points, int32_t B, int32_t M, const float* d_queries,
+                              int32_t N, float* d_z_out, void* d_ws, size_t ws_bytes, vdm_stream stream);
+
+/* Local (MSVS-style) decoder query on a multi-scale latent hierarchy (kwkr.cn
+ * MSVS-VAE article, section 1.1 "AVS-Conv" and section 1.3 "multi-scale query
+ * decoding"): per scale s the K anchors nearest to the query (squared
+ * distances in float32, summed x, y then z, no fused multiply-adds; ties to
+ * the smaller anchor index) are aggregated with per-channel dynamic weights
+ * from a small MLP of the relative offsets plus a mean-pooling residual,
+ *   f_s(x) = (1/K) sum_j (W2_s GELU(W1_s (a_j - x) + b1_s) + b2_s + 1) * F_j,
+ * and the scales are fused into the SDF: wo . GELU(Wf [f_0, f_1, ...] + bf) + bo.
+ * All arrays are float32 device memory; anchors anywhere (those outside
+ * [-1, 1]^3 only make the neighbour search visit more cells).             */
+#define VDM_LOCAL_MAX_SCALES 4
+typedef struct {
+    int32_t n_scales;                          /* 1..4                          */
+    int32_t K;                                 /* neighbours per scale, 1..16   */
+    int32_t hidden;                            /* dynamic-weight width, 1..32   */
+    int32_t fuse_hidden;                       /* fusion width, 1..64           */
+    int32_t n_anchors[VDM_LOCAL_MAX_SCALES];   /* host values, K..2^20          */
+    int32_t channels[VDM_LOCAL_MAX_SCALES];    /* C_s, multiple of 4, <= 64;
+                                                  sum over scales <= 128        */
+    const float* anchors[VDM_LOCAL_MAX_SCALES];/* [n_s][3]                      */
+    const float* feats[VDM_LOCAL_MAX_SCALES];  /* [n_s][C_s], 16-byte aligned   */
+    const float* W1[VDM_LOCAL_MAX_SCALES];     /* [hidden][3]                   */
+    const float* b1[VDM_LOCAL_MAX_SCALES];     /* [hidden]                      */
+    const float* W2[VDM_LOCAL_MAX_SCALES];     /* [C_s][hidden]                 */
+    const float* b2[VDM_LOCAL_MAX_SCALES];     /* [C_s]                         */
+    const float* Wf;                           /* [fuse_hidden][sum C_s]        */
+    const float* bf;                           /* [fuse_hidden]                 */
+    const float* wo;                           /* [fuse_hidden]                 */
+    const float* bo;                           /* [1]                           */
+} vdm_local_decoder;
+
+/* SDF of the local decoder at M points.
+ *   d_xyz      [M][3] float32;  d_out [M] float32
+ *   d_knn_out  [M][n_scales][K] int32 neighbour indices (nearest first) or NULL
+ *   d_ws/ws_bytes  device workspace >= vdm_local_workspace_size (the anchors'
+ *              grid binning, rebuilt at every call)
+ * M = 0 is a no-op.  Returns after the decode has finished on `stream`.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.                        */
+VDM_API vdm_status vdm_local_workspace_size(const vdm_local_decoder* dec, size_t* bytes);
+VDM_API vdm_status vdm_decode_local(const vdm_local_decoder* dec, const float* d_xyz, int64_t M, float* d_out,
+                                    int32_t* d_knn_out, void* d_ws, size_t ws_bytes, vdm_stream stream);
 
 /* Comparison of two fields sampled on the same grid, for accuracy reports
  * (aipaper.cc summary, section 5 "Evaluation Metrics": volume IoU of the

@@ -38,6 +38,7 @@ EXPORTS = ("vdm_precompute_kv", "vdm_decode_dense", "vdm_select_kv",
            "vdm_decode_hierarchical_noalloc", "vdm_compare_volumes",
            "vdm_surface_workspace_size", "vdm_extract_surface", "vdm_surface_case_table",
            "vdm_refine_workspace_size", "vdm_refine_level",
+           "vdm_encode_workspace_size", "vdm_encode", "vdm_local_workspace_size", "vdm_decode_local",
            "vdm_debug_inject", "vdm_set_cta_pairs",
            "vdm_profile_begin", "vdm_profile_end",
            "vdm_status_string", "vdm_last_error", "vdm_abi_version")
@@ -59,17 +60,19 @@ class CDecoder(C.Structure):
                 ("b1", C.c_void_p), ("b2", C.c_void_p),
                 ("ln_kv_g", C.c_void_p), ("ln_kv_b", C.c_void_p),
                 ("ln1_g", C.c_void_p), ("ln1_b", C.c_void_p), ("ln2_g", C.c_void_p), ("ln2_b", C.c_void_p),
-                ("w_head", C.c_void_p), ("b_head", C.c_void_p)]
+                ("w_head", C.c_void_p), ("b_head", C.c_void_p),
+                ("w_tsdf", C.c_void_p), ("b_tsdf", C.c_void_p)]
 
 
 class CAnalytic(C.Structure):
-    _fields_ = [("spheres", C.c_void_p), ("n_spheres", C.c_int32), ("dec_scale", C.c_float)]
+    _fields_ = [("spheres", C.c_void_p), ("n_spheres", C.c_int32), ("dec_scale", C.c_float),
+                ("tsdf_trunc", C.c_float)]
 
 
 class CHierParams(C.Structure):
     _fields_ = [("r0", C.c_int32), ("n_levels", C.c_int32), ("adaptive", C.c_int32),
                 ("tile", C.c_int32), ("n_probe", C.c_int32), ("top_k", C.c_int32),
-                ("seed", C.c_uint64)]
+                ("seed", C.c_uint64), ("tsdf_threshold", C.c_float)]
 
 
 class CHierStats(C.Structure):
@@ -82,9 +85,20 @@ class CHierDebug(C.Structure):
                 ("dec", C.c_void_p * MAX_LEVELS), ("tile_ids", C.c_void_p * MAX_LEVELS),
                 ("sel", C.c_void_p * MAX_LEVELS), ("max_tiles", C.c_int64),
                 ("probes", C.c_void_p * MAX_LEVELS), ("scores", C.c_void_p * MAX_LEVELS),
-                ("attn", C.c_void_p * MAX_LEVELS), ("attn_stride", C.c_int64)]
+                ("attn", C.c_void_p * MAX_LEVELS), ("attn_stride", C.c_int64),
+                ("tsdf", C.c_void_p * MAX_LEVELS)]
 
-DEBUG_ARRAYS = ("grid", "active", "dec", "tile_ids", "sel", "probes", "scores", "attn")
+DEBUG_ARRAYS = ("grid", "active", "dec", "tile_ids", "sel", "probes", "scores", "attn", "tsdf")
+
+
+LOCAL_MAX_SCALES = 4
+
+
+class CLocalDecoder(C.Structure):
+    _fields_ = [("n_scales", C.c_int32), ("K", C.c_int32), ("hidden", C.c_int32), ("fuse_hidden", C.c_int32),
+                ("n_anchors", C.c_int32 * LOCAL_MAX_SCALES), ("channels", C.c_int32 * LOCAL_MAX_SCALES)] + \
+        [(n, C.c_void_p * LOCAL_MAX_SCALES) for n in ("anchors", "feats", "W1", "b1", "W2", "b2")] + \
+        [(n, C.c_void_p) for n in ("Wf", "bf", "wo", "bo")]
 
 
 class CProfile(C.Structure):
@@ -112,6 +126,10 @@ _lib.vdm_extract_surface.argtypes = [_vp, _i32, _vp, _i64, _vp, _i64, C.POINTER(
 _lib.vdm_surface_case_table.argtypes = [_vp, _vp]
 _lib.vdm_refine_workspace_size.argtypes = [_i32, C.POINTER(C.c_size_t)]
 _lib.vdm_refine_level.argtypes = [_vp, _i32, _vp, _vp, _vp, _vp, _vp, C.c_size_t, _vp]
+_lib.vdm_encode_workspace_size.argtypes = [C.POINTER(CDecoder), _i32, C.POINTER(C.c_size_t)]
+_lib.vdm_local_workspace_size.argtypes = [C.POINTER(CLocalDecoder), C.POINTER(C.c_size_t)]
+_lib.vdm_decode_local.argtypes = [C.POINTER(CLocalDecoder), _vp, _i64, _vp, _vp, _vp, C.c_size_t, _vp]
+_lib.vdm_encode.argtypes = [C.POINTER(CDecoder), _vp, _vp, _vp, _i32, _i32, _vp, _i32, _vp, _vp, C.c_size_t, _vp]
 _lib.vdm_debug_inject.argtypes = [_i32, _i64]
 _lib.vdm_debug_inject.restype = C.c_int
 _lib.vdm_set_cta_pairs.argtypes = [_i32]
@@ -122,7 +140,8 @@ for _f in ("vdm_precompute_kv", "vdm_decode_dense", "vdm_select_kv",
            "vdm_hierarchical_workspace_size", "vdm_decode_hierarchical",
            "vdm_decode_hierarchical_noalloc", "vdm_compare_volumes", "vdm_profile_begin",
            "vdm_profile_end", "vdm_surface_workspace_size", "vdm_extract_surface",
-           "vdm_surface_case_table", "vdm_refine_workspace_size", "vdm_refine_level"):
+           "vdm_surface_case_table", "vdm_refine_workspace_size", "vdm_refine_level",
+           "vdm_encode_workspace_size", "vdm_encode", "vdm_local_workspace_size", "vdm_decode_local"):
     getattr(_lib, _f).restype = C.c_int
 _lib.vdm_status_string.argtypes = [C.c_int]
 _lib.vdm_status_string.restype = C.c_char_p
@@ -174,7 +193,7 @@ class Decoder:
         t = {}
         for k in _MATS:
             t[k] = torch.from_numpy(np.ascontiguousarray(weights[k], np.float32)).to(device=device, dtype=tdt)
-        for k in _VECS:
+        for k in _VECS + (("w_tsdf", "b_tsdf") if "w_tsdf" in weights else ()):
             t[k] = torch.from_numpy(np.ascontiguousarray(weights[k], np.float32).reshape(-1)).to(device)
         return Decoder(C, H, F, bool(query_ln), dtype, t)
 
@@ -189,16 +208,20 @@ class Decoder:
         d.dtype = VDM_F32 if self.dtype == "f32" else VDM_BF16
         for k in _MATS + _VECS:
             setattr(d, k, self.tensors[k].data_ptr())
+        if "w_tsdf" in self.tensors:   # optional truncated-SDF head
+            d.w_tsdf = self.tensors["w_tsdf"].data_ptr()
+            d.b_tsdf = self.tensors["b_tsdf"].data_ptr()
         return d
 
 
-def _analytic(spheres, dec_scale: float):
+def _analytic(spheres, dec_scale: float, tsdf_trunc: float = 0.0):
     if spheres is None:
         return None
     a = CAnalytic()
     a.spheres = spheres.data_ptr()
     a.n_spheres = int(spheres.shape[1])
     a.dec_scale = float(dec_scale)
+    a.tsdf_trunc = float(tsdf_trunc)
     return a
 
 
@@ -247,10 +270,11 @@ def vdm_select_kv(dec: Decoder, K, V, probe_xyz, tile_off, top_k: int, want_scor
 
 
 def hier_params(r0: int, n_levels: int, adaptive: bool = False, tile: int = 8, n_probe: int = 64,
-                top_k: int = 1024, seed: int = 0) -> CHierParams:
+                top_k: int = 1024, seed: int = 0, tsdf_threshold: float = 0.95) -> CHierParams:
     p = CHierParams()
     p.r0, p.n_levels, p.adaptive, p.tile = r0, n_levels, int(adaptive), tile
     p.n_probe, p.top_k, p.seed = n_probe, top_k, seed
+    p.tsdf_threshold = tsdf_threshold
     return p
 
 
@@ -263,7 +287,7 @@ def vdm_hierarchical_workspace_size(dec: Decoder, params: CHierParams, N: int) -
 
 def vdm_decode_hierarchical(dec: Decoder, K, V, params: CHierParams, spheres=None,
                             dec_scale: float = 0.0, workspace=None, out=None, debug=None,
-                            stream=None):
+                            stream=None, tsdf_trunc: float = 0.0):
     """Coarse-to-fine decoding of B shapes -> (grid ``[B,Rf,Rf,Rf]``, per-shape stats).
 
     ``debug`` is an optional dict of device tensors keyed like ``vdm_hier_debug``
@@ -288,7 +312,7 @@ def vdm_decode_hierarchical(dec: Decoder, K, V, params: CHierParams, spheres=Non
         dbg.max_tiles = int(debug.get("max_tiles", 0))
         dbg.attn_stride = int(debug.get("attn_stride", 0))
     cd = dec.cstruct()
-    an = _analytic(spheres, dec_scale)
+    an = _analytic(spheres, dec_scale, tsdf_trunc)
     _check(_lib.vdm_decode_hierarchical(C.byref(cd), K.data_ptr(), V.data_ptr(), B, N,
                                         C.byref(params), C.byref(an) if an else None,
                                         out.data_ptr(), workspace.data_ptr(), workspace.numel(),
@@ -337,6 +361,78 @@ def vdm_compare_volumes(a, b, stream=None) -> Dict[str, float]:
     return {"n": n, "inside_a": in_a, "inside_b": in_b, "inside_both": both, "same_sign": same,
             "v_iou": both / union if union else 1.0, "sign_agreement": same / n if n else 1.0,
             "max_abs_diff": dmax}
+
+
+def vdm_encode(block: Decoder, W_in, b_in, points, queries, stream=None):
+    """Vecsets ``[B, N, C]`` (float32) of point clouds ``points[B, M, 3]`` with
+    latent tokens at ``queries[B, N, 3]``; ``block`` holds the cross-attention
+    block (decoder layout), ``W_in [C, 64]`` (block dtype) and ``b_in [C]`` the
+    point-feature projection."""
+    torch = _torch()
+    B, M, _ = points.shape
+    N = queries.shape[1]
+    cd = block.cstruct()
+    n = C.c_size_t(0)
+    _check(_lib.vdm_encode_workspace_size(C.byref(cd), M, C.byref(n)))
+    ws = torch.empty((n.value,), device=points.device, dtype=torch.uint8)
+    z = torch.empty((B, N, block.C), device=points.device, dtype=torch.float32)
+    _check(_lib.vdm_encode(C.byref(cd), W_in.data_ptr(), b_in.data_ptr(), points.contiguous().data_ptr(), B, M,
+                           queries.contiguous().data_ptr(), N, z.data_ptr(), ws.data_ptr(), ws.numel(),
+                           _stream(stream)))
+    return z
+
+
+@dataclass
+class LocalDecoder:
+    """Device-resident multi-scale anchors and weights of the local decoder."""
+    K: int
+    tensors: Dict[str, "object"]
+    cs: "object" = None
+
+    @staticmethod
+    def from_numpy(d: Dict, K: int, device="cuda") -> "LocalDecoder":
+        torch = _torch()
+        t = {}
+        for s, (a, f, w) in enumerate(zip(d["anchors"], d["feats"], d["scales"])):
+            t[f"anchors{s}"] = torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
+            t[f"feats{s}"] = torch.from_numpy(np.ascontiguousarray(f, np.float32)).to(device)
+            for k in ("W1", "b1", "W2", "b2"):
+                t[f"{k}{s}"] = torch.from_numpy(np.ascontiguousarray(w[k], np.float32)).to(device)
+        for k in ("Wf", "bf", "wo", "bo"):
+            t[k] = torch.from_numpy(np.ascontiguousarray(d["fuse"][k], np.float32)).to(device)
+        ld = LocalDecoder(K, t)
+        c = CLocalDecoder()
+        c.n_scales = len(d["anchors"])
+        c.K = K
+        c.hidden = int(d["scales"][0]["W1"].shape[0])
+        c.fuse_hidden = int(d["fuse"]["Wf"].shape[0])
+        for s in range(c.n_scales):
+            c.n_anchors[s] = int(d["anchors"][s].shape[0])
+            c.channels[s] = int(d["feats"][s].shape[1])
+            c.anchors[s] = t[f"anchors{s}"].data_ptr()
+            c.feats[s] = t[f"feats{s}"].data_ptr()
+            for k in ("W1", "b1", "W2", "b2"):
+                getattr(c, k)[s] = t[f"{k}{s}"].data_ptr()
+        for k in ("Wf", "bf", "wo", "bo"):
+            setattr(c, k, t[k].data_ptr())
+        ld.cs = c
+        return ld
+
+
+def vdm_decode_local(ld: LocalDecoder, xyz, want_knn: bool = False, workspace=None, stream=None):
+    """SDF of the local decoder at ``xyz[M, 3]`` (float32, device); with
+    ``want_knn`` also the neighbour indices ``[M, n_scales, K]``."""
+    torch = _torch()
+    M = int(xyz.shape[0])
+    out = torch.empty((M,), device=xyz.device, dtype=torch.float32)
+    knn = (torch.empty((M, ld.cs.n_scales, ld.K), device=xyz.device, dtype=torch.int32) if want_knn else None)
+    if workspace is None:
+        n = C.c_size_t(0)
+        _check(_lib.vdm_local_workspace_size(C.byref(ld.cs), C.byref(n)))
+        workspace = torch.empty((n.value,), device=xyz.device, dtype=torch.uint8)
+    _check(_lib.vdm_decode_local(C.byref(ld.cs), xyz.contiguous().data_ptr(), M, out.data_ptr(), _ptr(knn),
+                                 workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return (out, knn) if want_knn else out
 
 
 def vdm_refine_workspace_size(R: int) -> int:

@@ -363,35 +363,88 @@ __global__ void __launch_bounds__(NT) decode_kernel(DecodeArgs a) {
         s.xq[r * ldc + c] += a.b2[c];
     }
     __syncthreads();
+    if (a.feat_out) {   // the block output itself (vecset encoding)
+        for (int i = tid; i < nq * C; i += NT) {
+            const int r = i / C, c = i - r * C;
+            a.feat_out[(size_t)s.qid[r] * C + c] = s.xq[r * ldc + c];
+        }
+    }
     // ---------------- LN2 + head
     layer_norm_rows(s.xq, s.buf, ldc, QT, C, a.ln2_g, a.ln2_b, !a.query_ln);
     __syncthreads();
     {
         const int warp = tid >> 5, lane = tid & 31;
         for (int r = warp; r < nq; r += NT / 32) {
-            float acc = 0.f;
-            for (int c = lane; c < C; c += 32) acc = fmaf(s.buf[r * ldc + c], a.w_head[c], acc);
+            float acc = 0.f, acc_t = 0.f;
+            for (int c = lane; c < C; c += 32) {
+                acc = fmaf(s.buf[r * ldc + c], a.w_head[c], acc);
+                if (a.w_tsdf) acc_t = fmaf(s.buf[r * ldc + c], a.w_tsdf[c], acc_t);
+            }
 #pragma unroll
-            for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            for (int o = 16; o; o >>= 1) {
+                acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                acc_t += __shfl_xor_sync(0xffffffffu, acc_t, o);
+            }
             if (lane == 0) {
                 const float dec = acc + a.b_head[0];
-                float val = dec;
+                float val = dec, sph = 0.f;
                 if (a.spheres) {
                     float p[3] = {s.pts[r * 4], s.pts[r * 4 + 1], s.pts[r * 4 + 2]};
-                    val = sphere_union(p, a.spheres, a.n_spheres) + a.dec_scale * tanhf(dec);
+                    sph = sphere_union(p, a.spheres, a.n_spheres);
+                    val = sph + a.dec_scale * tanhf(dec);
                 }
                 if (a.out) a.out[s.qid[r]] = val;
                 const int64_t v = s.vox[r];
                 if (v >= 0) {
                     if (a.grid) a.grid[v] = val;
                     if (a.dec_grid) a.dec_grid[v] = dec;
+                    if (a.tsdf_grid) a.tsdf_grid[v] = tsdf_value(acc_t + a.b_tsdf[0], sph, a);
                 }
             }
         }
     }
 }
 
+// ------------------------------------------------------------------ point features (encoder)
+// u[m][c] = sum_l W_in[c][l] pe_l(p_m) + b_in[c]: 16 points per CTA, embedding in shared memory
+template <typename T>
+__global__ void __launch_bounds__(NT) point_feature_kernel(const float* __restrict__ pts, int M, int C,
+                                                           const T* __restrict__ W, const float* __restrict__ b,
+                                                           float* __restrict__ u) {
+    __shared__ __align__(16) float pe[KV_ROWS * 68];
+    const int m0 = blockIdx.x * KV_ROWS;
+    const int n = min(KV_ROWS, M - m0);
+    for (int i = threadIdx.x; i < KV_ROWS * 64; i += NT) {
+        const int r = i >> 6, l = i & 63;
+        float p[3] = {0.f, 0.f, 0.f};
+        if (r < n) {
+            p[0] = pts[(size_t)(m0 + r) * 3];
+            p[1] = pts[(size_t)(m0 + r) * 3 + 1];
+            p[2] = pts[(size_t)(m0 + r) * 3 + 2];
+        }
+        pe[r * 68 + l] = pe_lane(p, l);
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += NT) {
+        int cols[1] = {c};
+        float acc[1][KV_ROWS] = {};
+        rows_x_cols<1, KV_ROWS>(pe, 68, W, kPeLanes, cols, kPeLanes, acc);
+        for (int r = 0; r < n; ++r) u[(size_t)(m0 + r) * C + c] = acc[0][r] + b[c];
+    }
+}
+
 }  // namespace
+
+vdm_status launch_point_features(const float* points, int M, int C, const void* W_in, const float* b_in, float* u,
+                                 vdm_dtype dt, cudaStream_t st) {
+    const dim3 grid((M + KV_ROWS - 1) / KV_ROWS);
+    if (dt == VDM_F32)
+        point_feature_kernel<float><<<grid, NT, 0, st>>>(points, M, C, static_cast<const float*>(W_in), b_in, u);
+    else
+        point_feature_kernel<__nv_bfloat16><<<grid, NT, 0, st>>>(points, M, C,
+                                                                 static_cast<const __nv_bfloat16*>(W_in), b_in, u);
+    return check_launch("point_feature_kernel");
+}
 
 vdm_status launch_precompute_kv(const KvArgs& a, vdm_dtype dt, cudaStream_t st) {
     const size_t sm = (size_t)KV_ROWS * (a.C + 4) * 4;

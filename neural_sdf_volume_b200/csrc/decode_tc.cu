@@ -15,10 +15,9 @@
 //              runs its own online softmax over them (own maximum, sum and O
 //              accumulator); the two combine once per head;
 //   warp 8     MMA issue (the whole warp runs the loop; one elected lane issues);
-//   warp 9     producer: TMA loads of weights and of contiguous K/V blocks;
-//              a sub-volume's selected K/V rows come by TMA tile::gather4, each
-//              lane bringing 4 rows of a 128-row block (CTA pairs: cp.async
-//              gathers, each lane's copies arriving on the slot's barrier);
+//   warp 9     producer: TMA loads of weights and of contiguous K/V blocks,
+//              cp.async gathers of a sub-volume's selected K/V rows (each lane's
+//              copies arrive on the slot's barrier when they land);
 // connected only by mbarriers (no CTA-wide barrier inside a tile).
 // Compiled twice per width: one CTA per 128-row MMA, or (cta_group::2) a CTA
 // pair of a cluster per 256-row MMA, each CTA holding half of every B tile.
@@ -117,7 +116,8 @@ struct Shared {
     uint64_t bar_pe, bar_qc, bar_p[2], bar_a, bar_hin, bar_r, bar_g[2], bar_cs, bar_wg;
     uint32_t tmem_base;
     int abort;
-    float G, Bc;
+    float G, Bc;     // SDF head folded with LN2's affine: sum w g, sum w b + b_head
+    float Gt, Bt;    // the same for the tSDF head
 };
 
 struct Waiter {
@@ -227,8 +227,7 @@ __global__ void __launch_bounds__(NT, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_wq64,
                  const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_w1,
                  const __grid_constant__ CUtensorMap tm_w2, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kr,
-                 const __grid_constant__ CUtensorMap tm_vr, const TcArgs ta) {
+                 const __grid_constant__ CUtensorMap tm_v, const TcArgs ta) {
     const DecodeArgs& a = ta.d;
     extern __shared__ uint8_t dyn_raw[];
     __shared__ Shared sh;
@@ -293,19 +292,28 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
         fence_proxy_async();
     }
     if (warp == 1) {
-        float g = 0.f, bc = 0.f;
+        float g = 0.f, bc = 0.f, gt = 0.f, bt = 0.f;
         for (int c = lane; c < C; c += 32) {
             const float w = a.w_head[c];
             g += a.query_ln ? w * a.ln2_g[c] : w;
             bc += a.query_ln ? w * a.ln2_b[c] : 0.f;
+            if (a.w_tsdf) {
+                const float wt = a.w_tsdf[c];
+                gt += a.query_ln ? wt * a.ln2_g[c] : wt;
+                bt += a.query_ln ? wt * a.ln2_b[c] : 0.f;
+            }
         }
         for (int o = 16; o; o >>= 1) {
             g += __shfl_xor_sync(0xffffffffu, g, o);
             bc += __shfl_xor_sync(0xffffffffu, bc, o);
+            gt += __shfl_xor_sync(0xffffffffu, gt, o);
+            bt += __shfl_xor_sync(0xffffffffu, bt, o);
         }
         if (lane == 0) {
             sh.G = g;
             sh.Bc = bc + a.b_head[0];
+            sh.Gt = gt;
+            sh.Bt = a.w_tsdf ? bt + a.b_tsdf[0] : 0.f;
         }
     }
     if (warp == 0) {
@@ -420,27 +428,21 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             if (!take_slot(slot)) return false;
             const uint32_t dst = s_ring + slot * RS;
             if (!PAIR) {
-                // TMA gathers: lane l brings rows 4l..4l+3 of the block (one-row boxes, the slot's
-                // 128 B swizzle applied by the copy engine).  Tokens past the selection read token 0
-                // of the head: their scores are masked, so their probabilities are exactly 0.
-                const int t0 = j * 128 + 4 * lane;
-                int r[4];
-                if (t0 + 3 < nk && (nk & 3) == 0) {   // 16-byte aligned index loads
-                    const int4 q = __ldg(reinterpret_cast<const int4*>(sel + t0));
-                    r[0] = q.x; r[1] = q.y; r[2] = q.z; r[3] = q.w;
-                } else {
+                // 128 rows x 8 chunks of 16 B: lane l copies chunk l % 8 of rows 4i + l / 8; the
+                // 32 row indices are loaded first (independent loads), then the copies are issued
+                const int c = lane & 7;
+                int rows[32];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) r[i] = t0 + i < nk ? __ldg(sel + t0 + i) : 0;
+                for (int i = 0; i < 32; ++i) {
+                    const int tok = j * 128 + 4 * i + (lane >> 3);
+                    rows[i] = tok < nk ? __ldg(sel + tok) : -1;
                 }
-                const uint32_t fb = smem_u32(&sh.full[slot]);
-                if (lane == 0) mbar_expect_tx_only(fb, SLOT);
-                __syncwarp();
-                const int base = h * N;
-                tma_gather4(dst + 512 * lane, isv ? &tm_vr : &tm_kr, 0, base + r[0], base + r[1], base + r[2],
-                            base + r[3], fb);
-                __syncwarp();
-                if (lane == 0) mbar_arrive_n(fb, RING_ARRIVALS);
-                return true;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int r = 4 * i + (lane >> 3);
+                    const bool okr = rows[i] >= 0;
+                    cp_async16(swz(dst, r, c), src + ((size_t)h * N + (okr ? rows[i] : 0)) * 64 + c * 8, okr);
+                }
             } else if (!isv) {
                 // keys: this CTA's 64 tokens of the block, 8 chunks each (128 B swizzle)
                 const int c = lane & 7;
@@ -619,8 +621,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     auto issue_s = [&](int j) -> bool {
                         int sl;
                         if (!consume(sl)) return false;
-                        // CTA pairs gather rows with cp.async (generic proxy): order them before the MMA's reads
-                        if (PAIR && u.sel) fence_proxy_async();
+                        // gathered rows were written by cp.async (generic proxy): order them before the MMA's reads
+                        if (u.sel) fence_proxy_async();
                         const uint64_t da = desc_sw128(s_abuf + h * 16384), db = desc_sw128(s_ring + sl * RS);
                         const uint32_t sd = tmem + T_S0 + 128 * (j % NSB);
                         #pragma unroll
@@ -636,7 +638,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         if (!(ok = W.wait(&sh.bar_p[g], ph_p[g], 53))) break;
                         tc_fence_after();
                         if (!(ok = consume(slot))) break;
-                        if (PAIR && u.sel) fence_proxy_async();
+                        if (u.sel) fence_proxy_async();
                         // O_g += P_j V_j. P_j is read in place: the bf16 pairs of tokens [32i, 32i+32)
                         // occupy columns [32i, 32i+16) of its S buffer. V is N-major: 16 tokens per
                         // k-step = 16 rows of 128 B (64 B per CTA of a pair)
@@ -1086,6 +1088,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             arrive_mma(&sh.bar_hin);
             // ================================================= MLP
             float hs_mean0 = 0.f, hs_m20 = 0.f, hs_dot0 = 0.f, hs_mean1 = 0.f, hs_m21 = 0.f, hs_dot1 = 0.f;
+            float hs_dt0 = 0.f, hs_dt1 = 0.f;   // tSDF head dot products
             for (int hf = 0; hf < n_half && ok; ++hf) {
                 if (hf == 1) {
                     // restore the parked x1[:, 256 + 128 wg, +128) into the accumulator [128 wg, +128)
@@ -1132,7 +1135,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 tc_fence_after();
                 // x2 = acc + bq + bo + b2 on this warpgroup's half of the half's columns
                 const int CWH = CW / 2, cb = hf * 256 + wg * CWH;
-                float shift = 0.f, s1 = 0.f, s2 = 0.f, dot = 0.f;
+                float shift = 0.f, s1 = 0.f, s2 = 0.f, dot = 0.f, dot_t = 0.f;
                 for (int cc = 0; cc < CWH; cc += 16) {
                     const int col0 = cb + cc;
                     float v[16], bqv[16], bov[16], wv[16];
@@ -1160,16 +1163,36 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         s2 = fmaf(d, d, s2);
                         dot = fmaf(x, wv[e], dot);
                     }
+                    if (a.feat_out && row < u.nq) {   // the block output itself (vecset encoding)
+                        float4* fo = reinterpret_cast<float4*>(a.feat_out + (size_t)qid * C + col0);
+#pragma unroll
+                        for (int e = 0; e < 16; e += 4)
+                            fo[e / 4] = make_float4(v[e] + bqv[e] + bov[e], v[e + 1] + bqv[e + 1] + bov[e + 1],
+                                                    v[e + 2] + bqv[e + 2] + bov[e + 2], v[e + 3] + bqv[e + 3] + bov[e + 3]);
+                    }
+                    if (a.w_tsdf) {   // second head on the same features (weights folded with LN2's gain)
+                        float wt[16];
+                        ldg16(a.w_tsdf + col0, wt);
+                        if (a.query_ln) {
+                            float gv[16];
+                            ldg16(a.ln2_g + col0, gv);
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) wt[e] *= gv[e];
+                        }
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) dot_t = fmaf(v[e] + bqv[e] + bov[e], wt[e], dot_t);
+                    }
                 }
                 const float mh = shift + s1 / (float)CWH;
                 const float m2h = fmaxf(s2 - s1 * (s1 / (float)CWH), 0.f);
-                float* xh = xs + 512 + hf * 768;
-                xh[(wg * 128 + row) * 3] = mh;
-                xh[(wg * 128 + row) * 3 + 1] = m2h;
-                xh[(wg * 128 + row) * 3 + 2] = dot;
+                float* xh = xs + 512 + hf * 1024;
+                xh[(wg * 128 + row) * 4] = mh;
+                xh[(wg * 128 + row) * 4 + 1] = m2h;
+                xh[(wg * 128 + row) * 4 + 2] = dot;
+                xh[(wg * 128 + row) * 4 + 3] = dot_t;
                 if (!(ok = wg_sync(73))) break;
-                const float* ra = xh + row * 3;            // warpgroup 0's values
-                const float* rb = xh + (128 + row) * 3;    // warpgroup 1's values
+                const float* ra = xh + row * 4;            // warpgroup 0's values
+                const float* rb = xh + (128 + row) * 4;    // warpgroup 1's values
                 const float d = rb[0] - ra[0];
                 const float mean_h = 0.5f * (ra[0] + rb[0]);
                 const float m2_h = ra[1] + rb[1] + d * d * 0.25f * (float)CW;
@@ -1178,16 +1201,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     hs_mean0 = mean_h;
                     hs_m20 = m2_h;
                     hs_dot0 = dot_h;
+                    hs_dt0 = ra[3] + rb[3];
                 } else {
                     hs_mean1 = mean_h;
                     hs_m21 = m2_h;
                     hs_dot1 = dot_h;
+                    hs_dt1 = ra[3] + rb[3];
                 }
             }
             if (!ok) break;
             // ================================================= head + output
             if (wg == 0) {
-                float dec;
+                float dec, traw;
                 if (a.query_ln) {
                     float mean, m2;
                     if (n_half == 1) {
@@ -1200,16 +1225,22 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     }
                     const float rstd = rsqrtf(m2 / (float)C + kLnEps);
                     dec = (hs_dot0 + hs_dot1 - mean * sh.G) * rstd + sh.Bc;
+                    traw = (hs_dt0 + hs_dt1 - mean * sh.Gt) * rstd + sh.Bt;
                 } else {
                     dec = hs_dot0 + hs_dot1 + sh.Bc;
+                    traw = hs_dt0 + hs_dt1 + sh.Bt;
                 }
                 if (row < u.nq) {
-                    float val = dec;
-                    if (a.spheres) val = sphere_union(p, a.spheres, a.n_spheres) + a.dec_scale * tanhf(dec);
+                    float val = dec, sph = 0.f;
+                    if (a.spheres) {
+                        sph = sphere_union(p, a.spheres, a.n_spheres);
+                        val = sph + a.dec_scale * tanhf(dec);
+                    }
                     if (a.out) a.out[qid] = val;
                     if (vox >= 0) {
                         if (a.grid) a.grid[vox] = val;
                         if (a.dec_grid) a.dec_grid[vox] = dec;
+                        if (a.tsdf_grid) a.tsdf_grid[vox] = tsdf_value(traw, sph, a);
                     }
                 }
             }
@@ -1320,10 +1351,6 @@ vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
     VDM_TRY(make_bf16_map(&m_k, d.K, (int64_t)d.H * d.N, 64, br, 64));
     // values are read N-major: a pair splits the 64 head dimensions, 32 per CTA
     VDM_TRY(make_bf16_map(&m_v, d.V, (int64_t)d.H * d.N, 64, 128, pair ? 32 : 64));
-    // one-row boxes for the gathers of selected K / V rows (tile::gather4)
-    CUtensorMap m_kr, m_vr;
-    VDM_TRY(make_bf16_map(&m_kr, d.K, (int64_t)d.H * d.N, 64, 1, 64));
-    VDM_TRY(make_bf16_map(&m_vr, d.V, (int64_t)d.H * d.N, 64, 1, 64));
     TcArgs ta;
     ta.d = d;
     ta.ns = ns;
@@ -1337,7 +1364,7 @@ vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
     ta.inject = g_debug.inject == 1;
     if (g_debug.inject > 0) --g_debug.inject;
     typedef void (*Kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
-                         CUtensorMap, CUtensorMap, CUtensorMap, TcArgs);
+                         CUtensorMap, TcArgs);
     Kern kern;
     if (pair) kern = d.C == 128 ? decode_tc_kernel<128, 2> : d.C == 256 ? decode_tc_kernel<256, 2> : decode_tc_kernel<512, 2>;
     else kern = d.C == 128 ? decode_tc_kernel<128, 1> : d.C == 256 ? decode_tc_kernel<256, 1> : decode_tc_kernel<512, 1>;
@@ -1362,7 +1389,7 @@ vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     prof_begin(kProfDecode, st);
-    e = cudaLaunchKernelEx(&cfg, kern, m_wq, m_wq64, m_wo, m_w1, m_w2, m_k, m_v, m_kr, m_vr, ta);
+    e = cudaLaunchKernelEx(&cfg, kern, m_wq, m_wq64, m_wo, m_w1, m_w2, m_k, m_v, ta);
     prof_end(kProfDecode, st);
     if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "decode_tc_kernel launch: %s", cudaGetErrorString(e));
     return check_launch("decode_tc_kernel");

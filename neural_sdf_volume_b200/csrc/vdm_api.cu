@@ -70,6 +70,19 @@ vdm_status check_decoder(const vdm_decoder* d, bool need_query_side) {
         if (i < 13 && !aligned(vecs[i], 16))
             return fail(VDM_ERR_INVALID_ARG, "decoder vector %d is not 16-byte aligned", i);
     }
+    if (need_query_side && d->w_tsdf) {
+        if (!d->b_tsdf) return fail(VDM_ERR_INVALID_ARG, "tSDF head: b_tsdf is NULL");
+        if (!aligned(d->w_tsdf, 16)) return fail(VDM_ERR_INVALID_ARG, "w_tsdf is not 16-byte aligned");
+    }
+    return VDM_OK;
+}
+
+vdm_status check_analytic(const vdm_decoder* d, const vdm_analytic* an) {
+    if (!an) return VDM_OK;
+    if (!an->spheres || an->n_spheres < 1)
+        return fail(VDM_ERR_INVALID_ARG, "analytic term needs spheres and n_spheres >= 1");
+    if (d->w_tsdf && !(an->tsdf_trunc > 0.f))
+        return fail(VDM_ERR_INVALID_ARG, "a tSDF head with an analytic term needs tsdf_trunc > 0");
     return VDM_OK;
 }
 
@@ -81,6 +94,7 @@ DecodeArgs base_args(const vdm_decoder* d, const void* K, const void* V, int N) 
     a.bq = d->bq; a.bo = d->bo; a.b1 = d->b1; a.b2 = d->b2;
     a.ln1_g = d->ln1_g; a.ln1_b = d->ln1_b; a.ln2_g = d->ln2_g; a.ln2_b = d->ln2_b;
     a.w_head = d->w_head; a.b_head = d->b_head;
+    a.w_tsdf = d->w_tsdf; a.b_tsdf = d->b_tsdf;
     a.K = K; a.V = V; a.N = N;
     return a;
 }
@@ -94,6 +108,7 @@ struct Plan {
     int L;
     int R[VDM_MAX_LEVELS];
     size_t off_grid[VDM_MAX_LEVELS];
+    size_t off_tgrid[VDM_MAX_LEVELS];   // tSDF grids of levels 0 .. L-2 (decoders with a tSDF head)
     size_t off_words, off_bits, off_word_off, off_tile_ids, off_tile_off, off_counts, off_scan, off_plist,
         off_qorder, off_sel, off_seltiles, off_ml, off_dense, off_dense_ml;
     int nw_max;
@@ -104,7 +119,7 @@ struct Plan {
 
 size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
 
-vdm_status make_plan(const vdm_hier_params* p, int N, int ml_heads, Plan& pl) {
+vdm_status make_plan(const vdm_hier_params* p, int N, int ml_heads, bool tsdf, Plan& pl) {
     if (!p) return fail(VDM_ERR_INVALID_ARG, "params is NULL");
     if (p->n_levels < 1 || p->n_levels > VDM_MAX_LEVELS)
         return fail(VDM_ERR_UNSUPPORTED, "n_levels = %d not in [1, %d]", p->n_levels, VDM_MAX_LEVELS);
@@ -116,6 +131,8 @@ vdm_status make_plan(const vdm_hier_params* p, int N, int ml_heads, Plan& pl) {
         if (p->n_probe < 1 || p->n_probe > 512) return fail(VDM_ERR_UNSUPPORTED, "n_probe must be in [1, 512]");
         if (p->top_k < 1) return fail(VDM_ERR_INVALID_ARG, "top_k must be >= 1");
     }
+    if (tsdf && !(p->tsdf_threshold > 0.f))
+        return fail(VDM_ERR_INVALID_ARG, "a tSDF head needs tsdf_threshold > 0");
     pl.L = p->n_levels;
     pl.k = p->adaptive ? (p->top_k < N ? p->top_k : N) : 0;
     size_t o = 0;
@@ -126,6 +143,8 @@ vdm_status make_plan(const vdm_hier_params* p, int N, int ml_heads, Plan& pl) {
         if (l < pl.L - 1) {
             pl.off_grid[l] = o;
             o = align_up(o + (size_t)pl.R[l] * pl.R[l] * pl.R[l] * 4);
+            pl.off_tgrid[l] = o;
+            if (tsdf) o = align_up(o + (size_t)pl.R[l] * pl.R[l] * pl.R[l] * 4);
             const int nb = pl.R[l] / 4;
             if (nb * nb * nb > nw_max) nw_max = nb * nb * nb;
             const int64_t v = (int64_t)pl.R[l] * pl.R[l] * pl.R[l];
@@ -218,8 +237,7 @@ vdm_status vdm_decode_dense(const vdm_decoder* dec, const void* d_k, const void*
                         (long long)M, grid_R);
     }
     if (M > ((int64_t)1 << 31) - 1) return fail(VDM_ERR_UNSUPPORTED, "M too large");
-    if (an && (!an->spheres || an->n_spheres < 1))
-        return fail(VDM_ERR_INVALID_ARG, "analytic term needs spheres and n_spheres >= 1");
+    VDM_TRY(check_analytic(dec, an));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const size_t kvb = kv_shape_bytes(dec, N);
     for (int b = 0; b < B; ++b) {
@@ -239,6 +257,7 @@ vdm_status vdm_decode_dense(const vdm_decoder* dec, const void* d_k, const void*
             a.spheres = an->spheres + (size_t)b * an->n_spheres * 4;
             a.n_spheres = an->n_spheres;
             a.dec_scale = an->dec_scale;
+            a.tsdf_trunc = an->tsdf_trunc;
         }
         VDM_TRY(launch_decode(a, dec->dtype, st));
     }
@@ -271,6 +290,68 @@ vdm_status vdm_select_kv(const vdm_decoder* dec, const void* d_k, const void* d_
     a.score = d_score_out;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     VDM_TRY(launch_select(a, dec->dtype, st));
+    VDM_CUDA_TRY(cudaStreamSynchronize(st));
+    return tc_check_error();
+}
+
+// encoder workspace: point features u [M][C] fp32, keys and values [H][M][64] in the block's dtype
+static size_t encode_ws_bytes(const vdm_decoder* blk, int M, size_t* off) {
+    size_t o = 0;
+    off[0] = o; o = align_up(o + (size_t)M * blk->C * 4);
+    off[1] = o; o = align_up(o + kv_shape_bytes(blk, M));
+    off[2] = o; o = align_up(o + kv_shape_bytes(blk, M));
+    return o + 256;
+}
+
+vdm_status vdm_encode_workspace_size(const vdm_decoder* blk, int32_t M, size_t* bytes) {
+    VDM_TRY(check_decoder(blk, true));
+    if (!bytes) return fail(VDM_ERR_INVALID_ARG, "bytes is NULL");
+    if (M < 1 || M > kMaxN) return fail(VDM_ERR_UNSUPPORTED, "M = %d not in [1, %d]", M, kMaxN);
+    size_t off[3];
+    *bytes = encode_ws_bytes(blk, M, off);
+    return VDM_OK;
+}
+
+vdm_status vdm_encode(const vdm_decoder* blk, const void* d_W_in, const float* d_b_in, const float* d_points,
+                      int32_t B, int32_t M, const float* d_queries, int32_t N, float* d_z_out, void* d_ws,
+                      size_t ws_bytes, vdm_stream stream) {
+    size_t need = 0;
+    VDM_TRY(vdm_encode_workspace_size(blk, M, &need));
+    if (B < 1 || N < 1) return fail(VDM_ERR_INVALID_ARG, "B and N must be >= 1");
+    if (!d_W_in || !d_b_in || !d_points || !d_queries || !d_z_out)
+        return fail(VDM_ERR_INVALID_ARG, "null W_in / b_in / points / queries / z_out");
+    if (!aligned(d_W_in, 16) || !aligned(d_b_in, 16) || !aligned(d_z_out, 16))
+        return fail(VDM_ERR_INVALID_ARG, "W_in, b_in and z_out must be 16-byte aligned");
+    if (!d_ws || ws_bytes < need) return fail(VDM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+    void* ws = reinterpret_cast<void*>(align_up((uintptr_t)d_ws));
+    if ((uintptr_t)ws - (uintptr_t)d_ws + need - 256 > ws_bytes)
+        return fail(VDM_ERR_WORKSPACE, "workspace too small after alignment");
+    size_t off[3];
+    encode_ws_bytes(blk, M, off);
+    float* u = at<float>(ws, off[0]);
+    void* K = at<char>(ws, off[1]);
+    void* V = at<char>(ws, off[2]);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    for (int b = 0; b < B; ++b) {
+        // keys and values from the cloud: embedded, projected, LayerNormed points
+        VDM_TRY(launch_point_features(d_points + (size_t)b * M * 3, M, blk->C, d_W_in, d_b_in, u, blk->dtype, st));
+        KvArgs k;
+        k.C = blk->C; k.H = blk->H; k.N = M;
+        k.z = u;
+        k.Wk = blk->Wk; k.Wv = blk->Wv; k.bk = blk->bk; k.bv = blk->bv;
+        k.g = blk->ln_kv_g; k.b = blk->ln_kv_b;
+        k.K = K; k.V = V;
+        VDM_TRY(launch_precompute_kv(k, blk->dtype, st));
+        // the latent tokens run the block from their query points; the output is the block's x2
+        DecodeArgs a = base_args(blk, K, V, M);
+        a.w_tsdf = nullptr;
+        a.work = kWorkFlat;
+        a.qmode = kQueryXyz;
+        a.xyz = d_queries + (size_t)b * N * 3;
+        a.M = N;
+        a.feat_out = d_z_out + (size_t)b * N * blk->C;
+        VDM_TRY(launch_decode(a, blk->dtype, st));
+    }
     VDM_CUDA_TRY(cudaStreamSynchronize(st));
     return tc_check_error();
 }
@@ -309,7 +390,7 @@ vdm_status vdm_refine_level(const float* d_f, int32_t R, float* d_f_fine, uint64
     refine_ws_bytes(R, off);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int nw = (R / 4) * (R / 4) * (R / 4);
-    VDM_TRY(launch_mark_dilate(d_f, R, d_mask, at<uint64_t>(ws, off[0]), st));
+    VDM_TRY(launch_mark_dilate(d_f, d_f, R, (float)(4.0 / (double)R), d_mask, at<uint64_t>(ws, off[0]), st));
     VDM_TRY(launch_compact(d_mask, nw, R, at<int32_t>(ws, off[1]), at<int32_t>(ws, off[2]), at<int32_t>(ws, off[3]),
                            d_parents, d_counts, at<int32_t>(ws, off[4]), st));
     if (d_f_fine) VDM_TRY(launch_fill(d_f, R, d_f_fine, st));
@@ -322,7 +403,7 @@ vdm_status vdm_hierarchical_workspace_size(const vdm_decoder* dec, const vdm_hie
     if (!bytes) return fail(VDM_ERR_INVALID_ARG, "bytes is NULL");
     if (N < 1 || N > kMaxN) return fail(VDM_ERR_UNSUPPORTED, "N = %d not in [1, %d]", N, kMaxN);
     Plan pl;
-    VDM_TRY(make_plan(p, N, dec->H, pl));
+    VDM_TRY(make_plan(p, N, dec->H, dec->w_tsdf != nullptr, pl));
     *bytes = pl.total;
     return VDM_OK;
 }
@@ -336,10 +417,10 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
     if (B < 1 || N < 1) return fail(VDM_ERR_INVALID_ARG, "B and N must be >= 1");
     if (N > kMaxN) return fail(VDM_ERR_UNSUPPORTED, "N = %d > %d", N, kMaxN);
     if (!d_k || !d_v || !d_grid_out) return fail(VDM_ERR_INVALID_ARG, "null k / v / grid_out");
-    if (an && (!an->spheres || an->n_spheres < 1))
-        return fail(VDM_ERR_INVALID_ARG, "analytic term needs spheres and n_spheres >= 1");
+    VDM_TRY(check_analytic(dec, an));
+    const bool tsdf = dec->w_tsdf != nullptr;
     Plan pl;
-    VDM_TRY(make_plan(p, N, dec->H, pl));
+    VDM_TRY(make_plan(p, N, dec->H, tsdf, pl));
     if (dbg) {
         bool any_attn = false;
         for (int l = 0; l < VDM_MAX_LEVELS; ++l) any_attn |= dbg->attn[l] != nullptr;
@@ -362,11 +443,18 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
         float* grid[VDM_MAX_LEVELS];
         for (int l = 0; l < L - 1; ++l) grid[l] = at<float>(ws, pl.off_grid[l]);
         grid[L - 1] = d_grid_out + (size_t)b * Rf * Rf * Rf;
+        // tSDF grids: workspace for the marked levels, the caller's debug array (if any) at the last
+        float* tgrid[VDM_MAX_LEVELS] = {};
+        if (tsdf) {
+            for (int l = 0; l < L - 1; ++l) tgrid[l] = at<float>(ws, pl.off_tgrid[l]);
+            if (dbg && dbg->tsdf[L - 1]) tgrid[L - 1] = dbg->tsdf[L - 1] + (size_t)b * Rf * Rf * Rf;
+        }
         DecodeArgs base = base_args(dec, K, V, N);
         if (an) {
             base.spheres = an->spheres + (size_t)b * an->n_spheres * 4;
             base.n_spheres = an->n_spheres;
             base.dec_scale = an->dec_scale;
+            base.tsdf_trunc = an->tsdf_trunc;
         }
         vdm_hier_stats* sb = stats ? stats + b : nullptr;
         if (sb) memset(sb, 0, sizeof(*sb));
@@ -390,6 +478,7 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             a.R = R;
             a.M = (int64_t)R * R * R;
             a.grid = grid[0];
+            a.tsdf_grid = tgrid[0];
             a.dec_grid = dbg_ptr(dbg ? dbg->dec : nullptr, 0, a.M);
             a.attn_out = attn_ptr(0);
             a.attn_stride = astride;
@@ -409,10 +498,14 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             int32_t* plist = at<int32_t>(ws, pl.off_plist);
             int32_t* qorder = at<int32_t>(ws, pl.off_qorder);
             int32_t* sel = at<int32_t>(ws, pl.off_sel);
-            VDM_TRY(launch_mark_dilate(grid[l], R, words, at<uint64_t>(ws, pl.off_bits), st));
+            // near-surface rule: |tSDF| < threshold with a tSDF head, else |f| < float32(4 / R)
+            VDM_TRY(launch_mark_dilate(grid[l], tsdf ? tgrid[l] : grid[l], R,
+                                       tsdf ? p->tsdf_threshold : (float)(4.0 / (double)R), words,
+                                       at<uint64_t>(ws, pl.off_bits), st));
             VDM_TRY(launch_compact(words, nw, R, word_off, tile_ids, tile_off, plist, counts, scan_tmp, st));
             // the inherit fill needs no count: it runs while the counts travel to the host
             VDM_TRY(launch_fill(grid[l], R, grid[l + 1], st));
+            if (tgrid[l + 1]) VDM_TRY(launch_fill(tgrid[l], R, tgrid[l + 1], st));
             int32_t hc[2] = {0, 0};
             VDM_CUDA_TRY(cudaMemcpyAsync(hc, counts, sizeof(hc), cudaMemcpyDeviceToHost, st));
             VDM_CUDA_TRY(cudaStreamSynchronize(st));
@@ -437,6 +530,7 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
                 a.plist = plist;
                 a.M = 8 * (int64_t)Mp;
                 a.grid = grid[l + 1];
+                a.tsdf_grid = tgrid[l + 1];
                 a.dec_grid = decg;
                 a.attn_out = attn_ptr(l + 1);
                 a.attn_stride = astride;
@@ -470,6 +564,7 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             a.T = T;
             a.n_probe = p->n_probe;
             a.grid = grid[l + 1];
+            a.tsdf_grid = tgrid[l + 1];
             a.dec_grid = decg;
             a.attn_out = attn_ptr(l + 1);
             a.attn_stride = astride;
@@ -544,10 +639,13 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
         }
         if (dbg) {
             for (int l = 0; l < L; ++l) {
-                if (!dbg->grid[l]) continue;
                 const size_t v = (size_t)pl.R[l] * pl.R[l] * pl.R[l];
-                VDM_CUDA_TRY(cudaMemcpyAsync(dbg->grid[l] + (size_t)b * v, grid[l], v * 4,
-                                             cudaMemcpyDeviceToDevice, st));
+                if (dbg->grid[l])
+                    VDM_CUDA_TRY(cudaMemcpyAsync(dbg->grid[l] + (size_t)b * v, grid[l], v * 4,
+                                                 cudaMemcpyDeviceToDevice, st));
+                if (tsdf && l < L - 1 && dbg->tsdf[l])
+                    VDM_CUDA_TRY(cudaMemcpyAsync(dbg->tsdf[l] + (size_t)b * v, tgrid[l], v * 4,
+                                                 cudaMemcpyDeviceToDevice, st));
             }
         }
     }

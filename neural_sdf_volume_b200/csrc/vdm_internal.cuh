@@ -53,6 +53,7 @@ struct DecodeArgs {
     int C, H, F, query_ln;
     const void *Wq, *Wo, *W1, *W2;
     const float *bq, *bo, *b1, *b2, *ln1_g, *ln1_b, *ln2_g, *ln2_b, *w_head, *b_head;
+    const float *w_tsdf, *b_tsdf;   // optional tSDF head (NULL: none)
     // keys / values of this shape: [H][N][64]
     const void *K, *V;
     int N;
@@ -79,13 +80,22 @@ struct DecodeArgs {
     float* out;                 // out[q] (flat work only) or NULL
     float* grid;                // scatter field at voxel linear index or NULL
     float* dec_grid;            // debug: raw decoder output at voxel index or NULL
+    float* tsdf_grid;           // tSDF value at voxel linear index or NULL (needs w_tsdf)
+    float* feat_out;            // block output x2[q][C] (fp32) of flat work, or NULL (vecset encoding)
     float* attn_out;            // debug: attention output a[v / attn_stride][C] at voxels v with
     int64_t attn_stride;        //   v % attn_stride == 0 (grid and children modes) or NULL
     // analytic field
     const float* spheres;       // [S][4] or NULL
     int n_spheres;
     float dec_scale;
+    float tsdf_trunc;           // tSDF = clip((sphere SDF + dec_scale tanh(t)) / tsdf_trunc, -1, 1)
 };
+
+// tSDF value of a query from its raw head output t (analytic term when spheres are given)
+__device__ __forceinline__ float tsdf_value(float t, float sphere, const DecodeArgs& a) {
+    if (!a.spheres) return t;
+    return fminf(1.0f, fmaxf(-1.0f, (sphere + a.dec_scale * tanhf(t)) / a.tsdf_trunc));
+}
 
 struct KvArgs {
     int C, H, N;
@@ -133,6 +143,9 @@ void prof_end(int cls, cudaStream_t s);
 
 // ---------------------------------------------------------------- launchers
 vdm_status launch_precompute_kv(const KvArgs& a, vdm_dtype dt, cudaStream_t s);
+// u[m][C] = W_in pe(points[m]) + b_in (fp32 out; W_in [C][64] in dt)
+vdm_status launch_point_features(const float* points, int M, int C, const void* W_in, const float* b_in, float* u,
+                                 vdm_dtype dt, cudaStream_t s);
 vdm_status launch_decode_simt(const DecodeArgs& a, vdm_dtype dt, int n_ctas_hint, cudaStream_t s);
 vdm_status launch_select(const SelectArgs& a, vdm_dtype dt, cudaStream_t s);
 // tensor-core decoder (bf16, C in {128, 256, 512}, F % 128 == 0)
@@ -167,7 +180,9 @@ vdm_status launch_decode(DecodeArgs a, vdm_dtype dt, cudaStream_t s);
 // boundary mark + dilation of a level grid -> blocked refine mask; `bits` is scratch of
 // mark_bits_words(R) words
 size_t mark_bits_words(int R);
-vdm_status launch_mark_dilate(const float* f, int R, uint64_t* words, uint64_t* bits, cudaStream_t s);
+// near-surface bits from |fn| < thr (fn = f for the |f| < 2h rule, the tSDF grid for the tSDF rule)
+vdm_status launch_mark_dilate(const float* f, const float* fn, int R, float thr, uint64_t* words, uint64_t* bits,
+                              cudaStream_t s);
 // voxels with a 26-neighbour of the other sign (no band, no dilation), blocked words
 vdm_status launch_sign_change(const float* f, int R, uint64_t* words, uint64_t* bits, cudaStream_t s);
 // compaction of the refine mask: word offsets, non-empty word ids (sub-volumes) and

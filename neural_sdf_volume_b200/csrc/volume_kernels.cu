@@ -25,29 +25,35 @@ namespace {
 // the 4-bit nibble (di, dj) of block bk, and the nibbles are gathered into words
 // through shared memory.  One read of f, 1/16 of it written.
 constexpr int PK_T = 512;          // one warp per row (di, dj)
-constexpr int PK_MAXV = 8;         // float4 per lane: R <= 1024
 
-__global__ void __launch_bounds__(PK_T) pack_kernel(const float* __restrict__ f, int R, float thr,
-                                                    uint64_t* __restrict__ S, uint64_t* __restrict__ Nr) {
+// MAXV float4 per lane cover rows of up to 128 MAXV voxels; few registers for small
+// MAXV keep four CTAs (2048 threads, all loads in flight) on every SM
+template <int MAXV>
+__global__ void __launch_bounds__(PK_T, MAXV <= 4 ? 4 : 2) pack_kernel(const float* __restrict__ f,
+                                                                      const float* __restrict__ fn, int R,
+                                                                      float thr, uint64_t* __restrict__ S,
+                                                                      uint64_t* __restrict__ Nr) {
     __shared__ __align__(16) uint8_t ns[256][16];   // [bk][row] sign nibbles
     __shared__ __align__(16) uint8_t nn[256][16];   // [bk][row] near nibbles
     const int nb = R >> 2;
     const int bi = blockIdx.x / nb, bj = blockIdx.x - bi * nb;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int di = warp >> 2, dj = warp & 3;
-    const float4* row = reinterpret_cast<const float4*>(f + ((size_t)(4 * bi + di) * R + (4 * bj + dj)) * R);
-    float4 v[PK_MAXV];
+    const size_t roff = ((size_t)(4 * bi + di) * R + (4 * bj + dj)) * R;
+    const float4* row = reinterpret_cast<const float4*>(f + roff);
+    float4 v[MAXV];
 #pragma unroll
-    for (int u = 0; u < PK_MAXV; ++u)
+    for (int u = 0; u < MAXV; ++u)
         if (lane + 32 * u < nb) v[u] = __ldcs(row + lane + 32 * u);
 #pragma unroll
-    for (int u = 0; u < PK_MAXV; ++u) {
+    for (int u = 0; u < MAXV; ++u) {
         const int bk = lane + 32 * u;
         if (bk < nb) {
             const float4 x = v[u];
             ns[bk][warp] = (uint8_t)((x.x < 0.f) | ((x.y < 0.f) << 1) | ((x.z < 0.f) << 2) | ((x.w < 0.f) << 3));
-            nn[bk][warp] = (uint8_t)((fabsf(x.x) < thr) | ((fabsf(x.y) < thr) << 1) | ((fabsf(x.z) < thr) << 2) |
-                                     ((fabsf(x.w) < thr) << 3));
+            const float4 y = fn == f ? x : __ldcs(reinterpret_cast<const float4*>(fn + roff) + bk);
+            nn[bk][warp] = (uint8_t)((fabsf(y.x) < thr) | ((fabsf(y.y) < thr) << 1) | ((fabsf(y.z) < thr) << 2) |
+                                     ((fabsf(y.w) < thr) << 3));
         }
     }
     __syncthreads();
@@ -84,82 +90,91 @@ constexpr int MW_N = MW_E * MW_E * MW_E;
 constexpr uint64_t K0 = 0x1111111111111111ull, K3 = 0x8888888888888888ull;   // dk = 0 / 3
 constexpr uint64_t J0 = 0x000F000F000F000Full, J3 = 0xF000F000F000F000ull;   // dj = 0 / 3
 
-// one axis of the dilation over the staged region; words whose neighbour along the
-// axis lies outside the region take it as empty (they are never used as valid)
+// one step of the dilation along an axis: x with its shifted copies and the facing bit
+// planes of its neighbours xp (minus side) and xn (plus side) along that axis
 template <int AXIS>
-__device__ __forceinline__ void dilate_axis(const uint64_t* __restrict__ src, uint64_t* __restrict__ dst) {
+__device__ __forceinline__ uint64_t dil(uint64_t x, uint64_t xp, uint64_t xn) {
+    if (AXIS == 2) return x | ((x >> 1) & ~K3) | ((x << 1) & ~K0) | ((xn & K0) << 3) | ((xp & K3) >> 3);
+    if (AXIS == 1) return x | ((x >> 4) & ~J3) | ((x << 4) & ~J0) | ((xn & J0) << 12) | ((xp & J3) >> 12);
+    return x | (x >> 16) | (x << 16) | ((xn & 0xFFFFull) << 48) | (xp >> 48);
+}
+
+// the same step over staged words; neighbours outside the staged region count as empty
+// (such words are never used as valid)
+template <int AXIS>
+__device__ __forceinline__ uint64_t dil_at(const uint64_t* __restrict__ src, int r) {
     constexpr int step = AXIS == 0 ? MW_E * MW_E : AXIS == 1 ? MW_E : 1;
-    for (int r = threadIdx.x; r < MW_N; r += MW_T) {
-        const int c = AXIS == 0 ? r / (MW_E * MW_E) : AXIS == 1 ? (r / MW_E) % MW_E : r % MW_E;
-        const uint64_t x = src[r];
-        const uint64_t xp = c > 0 ? src[r - step] : 0ull, xn = c < MW_E - 1 ? src[r + step] : 0ull;
-        uint64_t y;
-        if (AXIS == 2)
-            y = x | ((x >> 1) & ~K3) | ((x << 1) & ~K0) | ((xn & K0) << 3) | ((xp & K3) >> 3);
-        else if (AXIS == 1)
-            y = x | ((x >> 4) & ~J3) | ((x << 4) & ~J0) | ((xn & J0) << 12) | ((xp & J3) >> 12);
-        else
-            y = x | (x >> 16) | (x << 16) | ((xn & 0xFFFFull) << 48) | (xp >> 48);
-        dst[r] = y;
-    }
-    __syncthreads();
+    const int c = AXIS == 0 ? r / (MW_E * MW_E) : AXIS == 1 ? (r / MW_E) % MW_E : r % MW_E;
+    return dil<AXIS>(src[r], c > 0 ? src[r - step] : 0ull, c < MW_E - 1 ? src[r + step] : 0ull);
 }
 
-__device__ __forceinline__ void dilate3(uint64_t* a, uint64_t* tmp) {   // a <- D(a)
-    dilate_axis<2>(a, tmp);
-    dilate_axis<1>(tmp, a);
-    dilate_axis<0>(a, tmp);
-    for (int r = threadIdx.x; r < MW_N; r += MW_T) a[r] = tmp[r];
-    __syncthreads();
-}
-
-// DILATE = false: the sign-change words D(inside) & D(outside) | near, undilated.
+// Six passes: (1) load with the k step done on the fly from the words' global k
+// neighbours (adjacent in memory), for the inside and the outside words; (2) j step;
+// (3) i step and mark = near | (D(inside) & D(outside)); then, when dilating, (4) k,
+// (5) j and (6) i steps of the mark, the last written straight to the core's words.
+// Valid region after each pass: all, b in [1,10], a and b in [1,10], then e in [1,10],
+// b in [2,9], a in [2,9]: the 8^3 core at offset 2.
 template <bool DILATE>
 __global__ void __launch_bounds__(MW_T) mark_words_kernel(const uint64_t* __restrict__ S,
                                                           const uint64_t* __restrict__ Nr, int nb,
                                                           uint64_t* __restrict__ act) {
     extern __shared__ uint64_t mw_smem[];
-    uint64_t* in = mw_smem;              // inside words, then D(inside)
-    uint64_t* out = in + MW_N;           // outside words, then D(outside)
-    uint64_t* near = out + MW_N;         // near words, then mark, then D(mark)
-    uint64_t* tmp = near + MW_N;
+    uint64_t* A = mw_smem;          // D_k(inside), then the mark
+    uint64_t* B = A + MW_N;         // D_k(outside), then D_k(mark)
+    uint64_t* Nw = B + MW_N;        // near words
+    uint64_t* X = Nw + MW_N;        // D_jk(inside), then D_jk(mark)
+    uint64_t* Y = X + MW_N;         // D_jk(outside)
     const int ncta = (nb + MW_C - 1) / MW_C;
     int c = blockIdx.x;
     const int ck = c % ncta; c /= ncta;
     const int cj = c % ncta; c /= ncta;
     const int ci = c;
     const int i0 = ci * MW_C - 2, j0 = cj * MW_C - 2, k0 = ck * MW_C - 2;
-    for (int r = threadIdx.x; r < MW_N; r += MW_T) {
+    auto on_grid = [&](int r, size_t& w) -> bool {
         const int a = r / (MW_E * MW_E), b = (r / MW_E) % MW_E, e = r % MW_E;
         const int bi = i0 + a, bj = j0 + b, bk = k0 + e;
-        uint64_t s = 0, o = 0, n = 0;
-        if (bi >= 0 && bi < nb && bj >= 0 && bj < nb && bk >= 0 && bk < nb) {
-            const size_t w = ((size_t)bi * nb + bj) * nb + bk;
-            s = S[w];
-            o = ~s;
+        w = ((size_t)bi * nb + bj) * nb + bk;
+        return bi >= 0 && bi < nb && bj >= 0 && bj < nb && bk >= 0 && bk < nb;
+    };
+    for (int r = threadIdx.x; r < MW_N; r += MW_T) {
+        size_t w;
+        uint64_t din = 0, dout = 0, n = 0;
+        if (on_grid(r, w)) {
+            const int bk = k0 + r % MW_E;
+            const uint64_t s = S[w];
+            const bool hp = bk > 0, hn = bk + 1 < nb;
+            const uint64_t sp = hp ? S[w - 1] : 0ull, sn = hn ? S[w + 1] : 0ull;
+            din = dil<2>(s, sp, sn);
+            dout = dil<2>(~s, hp ? ~sp : 0ull, hn ? ~sn : 0ull);   // outside words: in-grid only
             n = Nr[w];
         }
-        in[r] = s;
-        out[r] = o;
-        near[r] = n;
+        A[r] = din;
+        B[r] = dout;
+        Nw[r] = n;
     }
     __syncthreads();
-    dilate3(in, tmp);
-    dilate3(out, tmp);
-    // mark; words off the grid stay empty (their dilated sign words are not)
     for (int r = threadIdx.x; r < MW_N; r += MW_T) {
-        const int a = r / (MW_E * MW_E), b = (r / MW_E) % MW_E, e = r % MW_E;
-        const int bi = i0 + a, bj = j0 + b, bk = k0 + e;
-        const bool on = bi >= 0 && bi < nb && bj >= 0 && bj < nb && bk >= 0 && bk < nb;
-        near[r] = on ? (near[r] | (in[r] & out[r])) : 0ull;
+        X[r] = dil_at<1>(A, r);
+        Y[r] = dil_at<1>(B, r);
     }
     __syncthreads();
-    if (DILATE) dilate3(near, tmp);
+    for (int r = threadIdx.x; r < MW_N; r += MW_T) {
+        size_t w;
+        A[r] = on_grid(r, w) ? (Nw[r] | (dil_at<0>(X, r) & dil_at<0>(Y, r))) : 0ull;   // mark, 0 off the grid
+    }
+    __syncthreads();
+    if (DILATE) {
+        for (int r = threadIdx.x; r < MW_N; r += MW_T) B[r] = dil_at<2>(A, r);
+        __syncthreads();
+        for (int r = threadIdx.x; r < MW_N; r += MW_T) X[r] = dil_at<1>(B, r);
+        __syncthreads();
+    }
     for (int r = threadIdx.x; r < MW_C * MW_C * MW_C; r += MW_T) {
         const int a = r / (MW_C * MW_C), b = (r / MW_C) % MW_C, e = r % MW_C;
         const int bi = ci * MW_C + a, bj = cj * MW_C + b, bk = ck * MW_C + e;
+        const int rr = ((a + 2) * MW_E + (b + 2)) * MW_E + (e + 2);
         if (bi < nb && bj < nb && bk < nb)
-            act[((size_t)bi * nb + bj) * nb + bk] = near[((a + 2) * MW_E + (b + 2)) * MW_E + (e + 2)];
+            act[((size_t)bi * nb + bj) * nb + bk] = DILATE ? dil_at<0>(X, rr) : A[rr];
     }
 }
 
@@ -282,26 +297,37 @@ __global__ void __launch_bounds__(CP_T) compact_kernel(const uint64_t* __restric
     }
     __syncthreads();
     if (!plist) return;
-    // parent list: one warp per word, lane L places bits L and L + 32
+    // parent list: each warp takes groups of 32 consecutive words (lane l holds word l of the
+    // group, its coordinates and offset); the group's non-empty words are visited by ballot, and
+    // for each of them lane L places bits L and L + 32
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nbw = R >> 2;
     const uint32_t below = (1u << lane) - 1u;
-    for (int l = warp; l < CP_CHUNK && base + l < n; l += CP_T / 32) {
-        const uint64_t x = sw[l];
-        if (!x) continue;
+    for (int g = warp; g < CP_CHUNK / 32; g += CP_T / 32) {
+        const int l = g * 32 + lane;
         const int w = base + l;
+        const uint64_t x = w < n ? sw[l] : 0ull;
+        uint32_t todo = __ballot_sync(0xffffffffu, x != 0ull);
+        if (!todo) continue;
         const int bi = w / (nbw * nbw), bj = (w / nbw) % nbw, bk = w % nbw;
-        const uint32_t lo = (uint32_t)x, hi = (uint32_t)(x >> 32);
+        const int corner = ((4 * bi) * R + 4 * bj) * R + 4 * bk;   // linear index of the block's first voxel
         const int o = so[l];
-        if ((lo >> lane) & 1u) {
-            const int bit = lane;
-            const int i = 4 * bi + (bit >> 4), j = 4 * bj + ((bit >> 2) & 3), k = 4 * bk + (bit & 3);
-            plist[o + __popc(lo & below)] = (i * R + j) * R + k;
-        }
-        if ((hi >> lane) & 1u) {
-            const int bit = lane + 32;
-            const int i = 4 * bi + (bit >> 4), j = 4 * bj + ((bit >> 2) & 3), k = 4 * bk + (bit & 3);
-            plist[o + __popc(lo) + __popc(hi & below)] = (i * R + j) * R + k;
+        while (todo) {
+            const int src = __ffs(todo) - 1;
+            todo &= todo - 1;
+            const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)x, src);
+            const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(x >> 32), src);
+            const int c0 = __shfl_sync(0xffffffffu, corner, src);
+            const int o0 = __shfl_sync(0xffffffffu, o, src);
+            // bit b = (di * 4 + dj) * 4 + dk -> voxel corner + (di R + dj) R + dk
+            if ((lo >> lane) & 1u) {
+                const int b = lane;
+                plist[o0 + __popc(lo & below)] = c0 + ((b >> 4) * R + ((b >> 2) & 3)) * R + (b & 3);
+            }
+            if ((hi >> lane) & 1u) {
+                const int b = lane + 32;
+                plist[o0 + __popc(lo) + __popc(hi & below)] = c0 + ((b >> 4) * R + ((b >> 2) & 3)) * R + (b & 3);
+            }
         }
     }
 }
@@ -311,25 +337,35 @@ __global__ void __launch_bounds__(CP_T) compact_kernel(const uint64_t* __restric
 // overwrites the children of refined parents): 8 fine voxels along k per thread from
 // 4 parents (one 16-byte load), two 16-byte stores; no partial-sector writes.
 template <bool STREAM>
-__global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ fc, int R, float* __restrict__ ff) {
+__device__ __forceinline__ void fill_group(const float* __restrict__ fc, int R, float* __restrict__ ff, size_t t) {
     const int R2 = 2 * R;
     const int Q = R2 >> 3;   // groups of 8 fine voxels per row
-    const size_t n = (size_t)R2 * R2 * Q;
-    for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < n; t += (size_t)gridDim.x * blockDim.x) {
-        const int q = (int)(t % Q);
-        const size_t ij = t / Q;
-        const int j = (int)(ij % R2), i = (int)(ij / R2);
-        const float4 p = *reinterpret_cast<const float4*>(fc + ((size_t)(i >> 1) * R + (j >> 1)) * R + 4 * q);
-        float4* dst = reinterpret_cast<float4*>(ff + ((size_t)i * R2 + j) * R2 + 8 * q);
-        const float4 a = make_float4(p.x, p.x, p.y, p.y), b = make_float4(p.z, p.z, p.w, p.w);
-        if (STREAM) {
-            __stcs(dst, a);
-            __stcs(dst + 1, b);
-        } else {
-            dst[0] = a;
-            dst[1] = b;
-        }
+    const int q = (int)(t % Q);
+    const size_t ij = t / Q;
+    const int j = (int)(ij % R2), i = (int)(ij / R2);
+    const float4 p = *reinterpret_cast<const float4*>(fc + ((size_t)(i >> 1) * R + (j >> 1)) * R + 4 * q);
+    float4* dst = reinterpret_cast<float4*>(ff + ((size_t)i * R2 + j) * R2 + 8 * q);
+    const float4 a = make_float4(p.x, p.x, p.y, p.y), b = make_float4(p.z, p.z, p.w, p.w);
+    if (STREAM) {
+        __stcs(dst, a);
+        __stcs(dst + 1, b);
+    } else {
+        dst[0] = a;
+        dst[1] = b;
     }
+}
+
+// two groups per thread and iteration (a grid-stride apart): more loads and stores in flight
+template <bool STREAM>
+__global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ fc, int R, float* __restrict__ ff) {
+    const size_t n = (size_t)(2 * R) * (2 * R) * ((2 * R) >> 3);
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+    for (; t + stride < n; t += 2 * stride) {
+        fill_group<STREAM>(fc, R, ff, t);
+        fill_group<STREAM>(fc, R, ff, t + stride);
+    }
+    if (t < n) fill_group<STREAM>(fc, R, ff, t);
 }
 
 // ------------------------------------------------------------------ probe order
@@ -449,22 +485,31 @@ vdm_status launch_probe_export(const int32_t* tile_off, int n_tiles, const int32
     return check_launch("probe_export_kernel");
 }
 
+vdm_status launch_pack(const float* f, const float* fn, int R, float thr, uint64_t* S, uint64_t* Nr,
+                       cudaStream_t s) {
+    const int nb = R >> 2;
+    if (nb <= 64) pack_kernel<2><<<nb * nb, PK_T, 0, s>>>(f, fn, R, thr, S, Nr);
+    else if (nb <= 128) pack_kernel<4><<<nb * nb, PK_T, 0, s>>>(f, fn, R, thr, S, Nr);
+    else pack_kernel<8><<<nb * nb, PK_T, 0, s>>>(f, fn, R, thr, S, Nr);
+    return check_launch("pack_kernel");
+}
+
 size_t mark_bits_words(int R) {
     const size_t nb = (size_t)(R >> 2);
     return 2 * nb * nb * nb;
 }
 
-vdm_status launch_mark_dilate(const float* f, int R, uint64_t* words, uint64_t* bits, cudaStream_t s) {
+vdm_status launch_mark_dilate(const float* f, const float* fn, int R, float thr, uint64_t* words, uint64_t* bits,
+                              cudaStream_t s) {
     if (R % 4 || R < 4 || R > 1024) return fail(VDM_ERR_UNSUPPORTED, "mark: R = %d", R);
     const int nb = R >> 2;
     const size_t nw = (size_t)nb * nb * nb;
-    const float thr = (float)(4.0 / (double)R);
-    const int smem = 4 * MW_N * (int)sizeof(uint64_t);   // 55 KB: set for the current device
+    const int smem = 5 * MW_N * (int)sizeof(uint64_t);   // 69 KB: set for the current device
     cudaError_t e = cudaFuncSetAttribute(mark_words_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "mark_words smem attribute: %s", cudaGetErrorString(e));
     const int ncta = (nb + MW_C - 1) / MW_C;
     prof_begin(kProfMark, s);
-    pack_kernel<<<nb * nb, PK_T, 0, s>>>(f, R, thr, bits, bits + nw);
+    VDM_TRY(launch_pack(f, fn, R, thr, bits, bits + nw, s));
     mark_words_kernel<true><<<ncta * ncta * ncta, MW_T, smem, s>>>(bits, bits + nw, nb, words);
     prof_end(kProfMark, s);
     return check_launch("mark kernels");
@@ -474,12 +519,12 @@ vdm_status launch_sign_change(const float* f, int R, uint64_t* words, uint64_t* 
     if (R % 4 || R < 4 || R > 1024) return fail(VDM_ERR_UNSUPPORTED, "sign change: R = %d", R);
     const int nb = R >> 2;
     const size_t nw = (size_t)nb * nb * nb;
-    const int smem = 4 * MW_N * (int)sizeof(uint64_t);
+    const int smem = 5 * MW_N * (int)sizeof(uint64_t);
     cudaError_t e = cudaFuncSetAttribute(mark_words_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "mark_words smem attribute: %s", cudaGetErrorString(e));
     const int ncta = (nb + MW_C - 1) / MW_C;
     // threshold 0: no near-surface bits, only voxels with a neighbour of the other sign
-    pack_kernel<<<nb * nb, PK_T, 0, s>>>(f, R, 0.0f, bits, bits + nw);
+    VDM_TRY(launch_pack(f, f, R, 0.0f, bits, bits + nw, s));
     mark_words_kernel<false><<<ncta * ncta * ncta, MW_T, smem, s>>>(bits, bits + nw, nb, words);
     return check_launch("sign change kernels");
 }
