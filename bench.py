@@ -551,14 +551,7 @@ def run_vdm(args, world, rank, local):
             res["vecset_encoder"] = {"workload": f"{M_pts}-point surface cloud -> {N_tok} tokens, C={C_}",
                                      "ms_per_shape": tenc, "TFLOP/s": enc_flops / (tenc / 1e3) / 1e12}
         if cfg.cid == 4:   # the local (MSVS-style) decoder query at the MSVS page's 200K-query batch
-            ldw = W.make_local_decoder(sp_np[0], seed=0, key=9)
-            ld = vdm.LocalDecoder.from_numpy(ldw, 8, device=dev)
-            q200 = torch.from_numpy(W.make_points(200_000, seed=0, key=9)[0]).to(dev)
-            tloc = _timed(lambda: vdm.vdm_decode_local(ld, q200), args.steps, 3, stream, flush)
-            res["local_decoder_200k"] = {
-                "workload": "200,000 uniform queries, 2 scales (4096 + 16384 surface anchors, C 64 + 32), K = 8",
-                "ms": tloc, "points_per_s": 200_000 / (tloc / 1e3),
-                "context": "MSVS page, 3.3: 213 ms (MSVS) vs 3068 ms (Lattice) for 200K queries, hardware not stated"}
+            res["local_decoder_200k"] = local_decoder_200k(vdm, sp_np[0], dev, args.steps, stream, flush)
         if cfg.adaptive:
             res["accuracy_vs_dense"] = accuracy_vs_dense(vdm, dec, K, V, cfg, spheres, params, ws, out)
             res["accuracy_vs_dense"].pop("_vol_d", None)
@@ -693,6 +686,18 @@ def run_reference(args, world, rank):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def local_decoder_200k(vdm, spheres, dev, steps, stream, flush):
+    """The local (MSVS-style) decoder query on the MSVS page's 200K-query batch."""
+    import torch
+    ldw = W.make_local_decoder(spheres, seed=0, key=9)
+    ld = vdm.LocalDecoder.from_numpy(ldw, 8, device=dev)
+    q200 = torch.from_numpy(W.make_points(200_000, seed=0, key=9)[0]).to(dev)
+    tloc = _timed(lambda: vdm.vdm_decode_local(ld, q200), steps, 3, stream, flush)
+    return {"workload": "200,000 uniform queries, 2 scales (4096 + 16384 surface anchors, C 64 + 32), K = 8",
+            "ms": tloc, "points_per_s": 200_000 / (tloc / 1e3),
+            "context": "MSVS page, 3.3: 213 ms (MSVS) vs 3068 ms (Lattice) for 200K queries, hardware not stated"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -703,6 +708,8 @@ def main():
                     help="3-6: hierarchical workloads (the step of the headline metric); 1-2: dense grids")
     ap.add_argument("--level-only", type=int, default=0, metavar="R",
                     help="only time the level kernels (vdm_refine_level) on an R^3 grid of the workload's spheres")
+    ap.add_argument("--local-only", action="store_true",
+                    help="only time the local (MSVS-style) decoder query on 200,000 points")
     ap.add_argument("--sweep", action="store_true",
                     help="adaptive-KV settings (probes, kept tokens) against time and error, one line each")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -728,6 +735,16 @@ def main():
         flush = torch.empty((L2_FLUSH_BYTES // 4,), device=dev, dtype=torch.float32)
         res = {"level_kernels": level_kernels_large(vdm, W.CONFIGS[args.config], dev, flush, args.steps, _peaks(),
                                                     sizes=(args.level_only,))}
+    elif args.local_only:
+        import torch
+
+        import neural_sdf_volume_b200 as vdm
+        torch.cuda.set_device(local)
+        dev = torch.device("cuda", local)
+        flush = torch.empty((L2_FLUSH_BYTES // 4,), device=dev, dtype=torch.float32)
+        sp = W.make_spheres(W.CONFIGS[args.config].n_spheres, seed=0, key=W.CONFIGS[args.config].sphere_key)[0]
+        res = {"local_decoder_200k": local_decoder_200k(vdm, sp, dev, args.steps, torch.cuda.current_stream(dev),
+                                                        flush)}
     elif args.dense_queries > 0 or args.config in (1, 2):
         res = run_dense(args, world, rank, local)
     else:

@@ -161,8 +161,20 @@ VDM_API vdm_status vdm_decode_dense(const vdm_decoder* dec, const void* d_k, con
  *   d_sel_out     [T][top_k] int32 (device)
  *   d_score_out   [T][N] float32 or NULL
  * Sub-volumes with no probe select tokens 0..top_k-1.  top_k >= N selects
- * every token.  Returns after the selection has finished on `stream`.
- * Errors: INVALID_ARG, UNSUPPORTED (N, top_k > 8192), CUDA, TIMEOUT.        */
+ * every token.
+ * Kernels: with a bf16 decoder of width 128, 256 or 512 and at most 128
+ * probes per sub-volume, the tensor-core kernels of vdm_decode_hierarchical's
+ * adaptive levels (the probes are decoded with full attention, which gives
+ * their per-head softmax maximum and sum, then scored and ranked in one
+ * pass), so for the same probes, in the same order, the scores and the
+ * selection are bit-identical to that path's; otherwise a CUDA-core kernel
+ * (any dtype, width and probe count).  The tensor-core route takes a
+ * stream-ordered temporary allocation (cudaMallocAsync / cudaFreeAsync on
+ * `stream`) of about T * 128 * H * 8 + 4 P bytes.
+ * Synchronisation: d_tile_off is copied to the host and checked first (one
+ * round trip on `stream`); the call returns after the selection has finished.
+ * Errors: INVALID_ARG (offsets not starting at 0, decreasing or not ending at
+ * P_total), UNSUPPORTED (N, top_k > 8192), CUDA, TIMEOUT.                   */
 VDM_API vdm_status vdm_select_kv(const vdm_decoder* dec, const void* d_k, const void* d_v, int32_t N,
                          const float* d_probe_xyz, const int32_t* d_tile_off, int32_t T,
                          int64_t P_total, int32_t top_k, int32_t* d_sel_out, float* d_score_out,

@@ -22,10 +22,16 @@
 // the query to every cell not yet visited (with a relative margin, so rounding
 // can only search one ring more), which makes the result exact.
 //
-// One thread per query: its kNN in registers, the dynamic-weight hidden layer
-// in registers, the scale's channel accumulators in registers, the scale
-// outputs in its row of shared memory, then the fusion MLP from shared memory.
-// All weights are staged in shared memory once per CTA.
+// Two kernels per chunk of queries.  local_knn_kernel: one thread per query,
+// the neighbour list sorted in registers (fixed capacity, static indices); the
+// cells are scanned through per-row occupancy words (bit k of row (i, j): cell
+// (i, j, k) holds an anchor) staged in shared memory, so empty cells cost a
+// few bit operations and only occupied cells are read from global memory --
+// a query far from every anchor scans many rings of cells.  local_conv_kernel:
+// one thread per query, the dynamic-weight hidden layer and the scale's
+// channel accumulators in registers, the scale outputs in its row of shared
+// memory, then the fusion MLP from shared memory; all weights are staged in
+// shared memory once per CTA.
 #include <mutex>
 #include <string.h>
 
@@ -34,28 +40,35 @@
 namespace vdm {
 namespace {
 
-constexpr int LQ_T = 64;          // queries per CTA
+constexpr int LQ_T = 64;          // queries per CTA (AVS-Conv and fusion)
+constexpr int LK_T = 128;         // queries per CTA (neighbour search)
+constexpr int L_CHUNK = 1 << 16;  // queries per chunk (neighbour ids kept in the workspace)
 constexpr int L_MAXS = VDM_LOCAL_MAX_SCALES;
 constexpr int L_MAXK = 16, L_MAXH = 32, L_MAXC = 64, L_MAXSUMC = 128, L_MAXF = 64;
 
 struct ScaleGrid {
-    int G;                 // cells per axis
+    int G;                 // cells per axis (<= 64)
     const int32_t* start;  // [G^3 + 1]
     const int32_t* ids;    // [n] anchor ids sorted by cell
+    const uint64_t* rows;  // [G^2] occupancy of the cells of row (i, j): bit k = cell (i, j, k)
+    int row_off;           // offset of the rows in the search kernel's shared memory (words)
 };
 
 struct LocalArgs {
     int n_scales, K, hidden, fuse_hidden;
     int C[L_MAXS], coff[L_MAXS], sumC;
+    int woff[L_MAXS + 1];  // staged weights: scale s's W1, b1, W2, b2 from woff[s]; the fusion weights at woff[n_scales]
     const float* anchors[L_MAXS];
     const float* feats[L_MAXS];
     const float *W1[L_MAXS], *b1[L_MAXS], *W2[L_MAXS], *b2[L_MAXS];
     const float *Wf, *bf, *wo, *bo;
     ScaleGrid grid[L_MAXS];
     const float* xyz;
-    int64_t M;
+    int64_t q0, q1;        // this chunk's queries [q0, q1)
     float* out;
-    int32_t* knn_out;      // [M][n_scales][K] or NULL
+    int32_t* nbr;          // neighbour ids of query q at nbr[(q - nbr_q0) * n_scales * K]
+    int64_t nbr_q0;
+    int row_words;         // total occupancy words of all scales
 };
 
 __device__ __forceinline__ int cell_of(float v, int G) {
@@ -118,82 +131,94 @@ __global__ void bin_place_kernel(const int32_t* __restrict__ cell, int n, int32_
     ids[atomicAdd(&cursor[cell[i]], 1)] = i;
 }
 
+// occupancy word of each row of cells
+__global__ void row_mask_kernel(const int32_t* __restrict__ cnt, int G, uint64_t* __restrict__ rows) {
+    const int r = blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= G * G) return;
+    uint64_t m = 0;
+    for (int k = 0; k < G; ++k) m |= (uint64_t)(cnt[r * G + k] > 0) << k;
+    rows[r] = m;
+}
+
 // ---------------------------------------------------------------- query
 __device__ __forceinline__ float d2_rn(float ax, float ay, float az, float x, float y, float z) {
     const float dx = __fsub_rn(ax, x), dy = __fsub_rn(ay, y), dz = __fsub_rn(az, z);
     return __fadd_rn(__fadd_rn(__fmul_rn(dx, dx), __fmul_rn(dy, dy)), __fmul_rn(dz, dz));
 }
 
-// insert (d, id) into the sorted list (d2 ascending, ties by id) of length cnt <= K
-__device__ __forceinline__ void knn_insert(float (&bd)[L_MAXK], int (&bi)[L_MAXK], int& cnt, int K, float d,
-                                           int id) {
-    if (cnt == K && (d > bd[K - 1] || (d == bd[K - 1] && id > bi[K - 1]))) return;
-    int p = cnt < K ? cnt : K - 1;
-    while (p > 0 && (bd[p - 1] > d || (bd[p - 1] == d && bi[p - 1] > id))) {
-        bd[p] = bd[p - 1];
-        bi[p] = bi[p - 1];
-        --p;
-    }
-    bd[p] = d;
-    bi[p] = id;
-    if (cnt < K) ++cnt;
+// (d, id) orders before (e, jd): smaller squared distance, ties to the smaller index
+__device__ __forceinline__ bool nb_less(float d, int id, float e, int jd) {
+    return d < e || (d == e && id < jd);
 }
 
-__global__ void __launch_bounds__(LQ_T) local_query_kernel(const LocalArgs a) {
-    extern __shared__ float lsm[];
-    // staged weights: per scale W1, b1, W2, b2; then Wf, bf, wo; then the per-thread feature rows
-    float* w1s[L_MAXS];
-    float* b1s[L_MAXS];
-    float* w2s[L_MAXS];
-    float* b2s[L_MAXS];
-    float* p = lsm;
-    for (int s = 0; s < a.n_scales; ++s) {
-        w1s[s] = p; p += a.hidden * 3;
-        b1s[s] = p; p += a.hidden;
-        w2s[s] = p; p += a.C[s] * a.hidden;
-        b2s[s] = p; p += a.C[s];
+// insert (d, id) into the sorted list of the KC best (padded with (+inf, INT_MAX));
+// every index is static, so the list stays in registers
+template <int KC>
+__device__ __forceinline__ void knn_insert(float (&bd)[KC], int (&bi)[KC], float d, int id) {
+    if (!nb_less(d, id, bd[KC - 1], bi[KC - 1])) return;
+#pragma unroll
+    for (int p = KC - 1; p > 0; --p) {
+        const bool shift = nb_less(d, id, bd[p - 1], bi[p - 1]);
+        const bool here = !shift && nb_less(d, id, bd[p], bi[p]);
+        bd[p] = shift ? bd[p - 1] : here ? d : bd[p];
+        bi[p] = shift ? bi[p - 1] : here ? id : bi[p];
     }
-    float* wfs = p; p += a.fuse_hidden * a.sumC;
-    float* bfs = p; p += a.fuse_hidden;
-    float* wos = p; p += a.fuse_hidden;
-    float* frow = p + threadIdx.x * (a.sumC + 1);   // odd row stride: rows in different banks
-    for (int s = 0; s < a.n_scales; ++s) {
-        for (int i = threadIdx.x; i < a.hidden * 3; i += LQ_T) w1s[s][i] = a.W1[s][i];
-        for (int i = threadIdx.x; i < a.hidden; i += LQ_T) b1s[s][i] = a.b1[s][i];
-        for (int i = threadIdx.x; i < a.C[s] * a.hidden; i += LQ_T) w2s[s][i] = a.W2[s][i];
-        for (int i = threadIdx.x; i < a.C[s]; i += LQ_T) b2s[s][i] = a.b2[s][i];
+    if (nb_less(d, id, bd[0], bi[0])) {
+        bd[0] = d;
+        bi[0] = id;
     }
-    for (int i = threadIdx.x; i < a.fuse_hidden * a.sumC; i += LQ_T) wfs[i] = a.Wf[i];
-    for (int i = threadIdx.x; i < a.fuse_hidden; i += LQ_T) {
-        bfs[i] = a.bf[i];
-        wos[i] = a.wo[i];
+}
+
+template <int KC>
+__global__ void __launch_bounds__(LK_T) local_knn_kernel(const LocalArgs a) {
+    extern __shared__ uint64_t lrows[];
+    for (int s = 0; s < a.n_scales; ++s) {
+        const int G = a.grid[s].G;
+        for (int i = threadIdx.x; i < G * G; i += LK_T) lrows[a.grid[s].row_off + i] = a.grid[s].rows[i];
     }
     __syncthreads();
-    const int64_t q = (int64_t)blockIdx.x * LQ_T + threadIdx.x;
-    if (q >= a.M) return;
+    const int64_t q = a.q0 + (int64_t)blockIdx.x * LK_T + threadIdx.x;
+    if (q >= a.q1) return;
     const float x = a.xyz[3 * q], y = a.xyz[3 * q + 1], z = a.xyz[3 * q + 2];
     const int K = a.K;
+    int32_t* nout = a.nbr + (q - a.nbr_q0) * a.n_scales * K;
     for (int s = 0; s < a.n_scales; ++s) {
-        // ---- exact kNN by rings of cells
         const ScaleGrid g = a.grid[s];
-        const float cs = 2.0f / (float)g.G;
-        const int cx = cell_of(x, g.G), cy = cell_of(y, g.G), cz = cell_of(z, g.G);
-        float bd[L_MAXK];
-        int bi[L_MAXK];
+        const int G = g.G;
+        const uint64_t* rows = lrows + g.row_off;
+        const float cs = 2.0f / (float)G;
+        const int cx = cell_of(x, G), cy = cell_of(y, G), cz = cell_of(z, G);
+        float bd[KC];
+        int bi[KC];
+#pragma unroll
+        for (int p = 0; p < KC; ++p) {
+            bd[p] = INFINITY;
+            bi[p] = 0x7fffffff;
+        }
         int cnt = 0;
         const float* an = a.anchors[s];
-        for (int r = 0; r < g.G; ++r) {
-            for (int i = cx - r; i <= cx + r; ++i) {
-                if (i < 0 || i >= g.G) continue;
-                for (int j = cy - r; j <= cy + r; ++j) {
-                    if (j < 0 || j >= g.G) continue;
-                    const bool edge_ij = i == cx - r || i == cx + r || j == cy - r || j == cy + r;
-                    for (int k = cz - r; k <= cz + r; k += (edge_ij ? 1 : 2 * r > 0 ? 2 * r : 1)) {
-                        if (k < 0 || k >= g.G) continue;
-                        const int c = (i * g.G + j) * g.G + k;
-                        for (int t = g.start[c]; t < g.start[c + 1]; ++t) {
+        for (int r = 0; r < G; ++r) {
+            // ring r: the cells at Chebyshev distance r from the query's cell
+            const int i0 = max(cx - r, 0), i1 = min(cx + r, G - 1);
+            const int j0 = max(cy - r, 0), j1 = min(cy + r, G - 1);
+            const int k0 = max(cz - r, 0), k1 = min(cz + r, G - 1);
+            const uint64_t span = (~0ull >> (63 - k1)) & (~0ull << k0);   // k in [k0, k1]
+            uint64_t ends = 0;                                              // k = cz - r, cz + r
+            if (cz - r >= 0) ends |= 1ull << (cz - r);
+            if (cz + r < G) ends |= 1ull << (cz + r);
+            for (int i = i0; i <= i1; ++i) {
+                const bool ei = i == cx - r || i == cx + r;
+                for (int j = j0; j <= j1; ++j) {
+                    uint64_t m = rows[i * G + j] & ((ei || j == cy - r || j == cy + r) ? span : ends);
+                    while (m) {
+                        const int k = __ffsll((long long)m) - 1;
+                        m &= m - 1;
+                        const int c = (i * G + j) * G + k;
+                        const int t1 = g.start[c + 1];
+                        for (int t = g.start[c]; t < t1; ++t) {
                             const int id = g.ids[t];
-                            knn_insert(bd, bi, cnt, K, d2_rn(an[3 * id], an[3 * id + 1], an[3 * id + 2], x, y, z), id);
+                            knn_insert<KC>(bd, bi, d2_rn(an[3 * id], an[3 * id + 1], an[3 * id + 2], x, y, z), id);
+                            ++cnt;
                         }
                     }
                 }
@@ -205,32 +230,76 @@ __global__ void __launch_bounds__(LQ_T) local_query_kernel(const LocalArgs a) {
             const float loy = -1.0f + (float)(cy - r) * cs, hiy = -1.0f + (float)(cy + r + 1) * cs;
             const float loz = -1.0f + (float)(cz - r) * cs, hiz = -1.0f + (float)(cz + r + 1) * cs;
             if (cx - r > 0) { all = false; bound = fminf(bound, x - lox); }
-            if (cx + r < g.G - 1) { all = false; bound = fminf(bound, hix - x); }
+            if (cx + r < G - 1) { all = false; bound = fminf(bound, hix - x); }
             if (cy - r > 0) { all = false; bound = fminf(bound, y - loy); }
-            if (cy + r < g.G - 1) { all = false; bound = fminf(bound, hiy - y); }
+            if (cy + r < G - 1) { all = false; bound = fminf(bound, hiy - y); }
             if (cz - r > 0) { all = false; bound = fminf(bound, z - loz); }
-            if (cz + r < g.G - 1) { all = false; bound = fminf(bound, hiz - z); }
+            if (cz + r < G - 1) { all = false; bound = fminf(bound, hiz - z); }
             if (all) break;
-            // margins: an anchor on a cell face may be binned to either side by rounding
-            const float b = bound - 1e-5f;
-            if (cnt == K && b > 0.f && bd[K - 1] < b * b * 0.99999f) break;
+            if (cnt >= K) {
+                float kth = bd[0];
+#pragma unroll
+                for (int p = 1; p < KC; ++p)
+                    if (p == K - 1) kth = bd[p];
+                // margins: an anchor on a cell face may be binned to either side by rounding
+                const float b = bound - 1e-5f;
+                if (b > 0.f && kth < b * b * 0.99999f) break;
+            }
         }
-        if (a.knn_out)
-            for (int t = 0; t < K; ++t) a.knn_out[(q * a.n_scales + s) * K + t] = t < cnt ? bi[t] : -1;
-        // ---- AVS-Conv of the scale
+#pragma unroll
+        for (int p = 0; p < KC; ++p)
+            if (p < K) nout[s * K + p] = p < cnt ? bi[p] : -1;
+    }
+}
+
+__global__ void __launch_bounds__(LQ_T) local_conv_kernel(const LocalArgs a) {
+    extern __shared__ float lsm[];
+    // staged weights: per scale W1 [hidden][3], b1, W2 [C][hidden], b2; then Wf, bf, wo; then the
+    // per-thread feature rows
+    const int hd = a.hidden;
+    for (int s = 0; s < a.n_scales; ++s) {
+        float* w = lsm + a.woff[s];
         const int C = a.C[s];
+        for (int i = threadIdx.x; i < hd * 3; i += LQ_T) w[i] = a.W1[s][i];
+        for (int i = threadIdx.x; i < hd; i += LQ_T) w[3 * hd + i] = a.b1[s][i];
+        for (int i = threadIdx.x; i < C * hd; i += LQ_T) w[4 * hd + i] = a.W2[s][i];
+        for (int i = threadIdx.x; i < C; i += LQ_T) w[4 * hd + C * hd + i] = a.b2[s][i];
+    }
+    float* wfs = lsm + a.woff[a.n_scales];
+    float* bfs = wfs + a.fuse_hidden * a.sumC;
+    float* wos = bfs + a.fuse_hidden;
+    float* frow = wos + a.fuse_hidden + threadIdx.x * (a.sumC + 1);   // odd row stride: rows in different banks
+    for (int i = threadIdx.x; i < a.fuse_hidden * a.sumC; i += LQ_T) wfs[i] = a.Wf[i];
+    for (int i = threadIdx.x; i < a.fuse_hidden; i += LQ_T) {
+        bfs[i] = a.bf[i];
+        wos[i] = a.wo[i];
+    }
+    __syncthreads();
+    const int64_t q = a.q0 + (int64_t)blockIdx.x * LQ_T + threadIdx.x;
+    if (q >= a.q1) return;
+    const float x = a.xyz[3 * q], y = a.xyz[3 * q + 1], z = a.xyz[3 * q + 2];
+    const int K = a.K;
+    const int32_t* nin = a.nbr + (q - a.nbr_q0) * a.n_scales * K;
+    for (int s = 0; s < a.n_scales; ++s) {
+        const float* an = a.anchors[s];
+        const int C = a.C[s];
+        const float* w1s = lsm + a.woff[s];
+        const float* b1s = w1s + 3 * hd;
+        const float* w2s = w1s + 4 * hd;
+        const float* b2s = w2s + C * hd;
         float acc[L_MAXC];
 #pragma unroll
         for (int c = 0; c < L_MAXC; ++c) acc[c] = 0.f;
         const float* F = a.feats[s];
-        for (int t = 0; t < cnt; ++t) {
-            const int id = bi[t];
+        for (int t = 0; t < K; ++t) {
+            const int id = nin[s * K + t];
+            if (id < 0) continue;
             const float rx = an[3 * id] - x, ry = an[3 * id + 1] - y, rz = an[3 * id + 2] - z;
             float hid[L_MAXH];
 #pragma unroll
             for (int h = 0; h < L_MAXH; ++h) {
-                if (h < a.hidden) {
-                    const float v = w1s[s][3 * h] * rx + w1s[s][3 * h + 1] * ry + w1s[s][3 * h + 2] * rz + b1s[s][h];
+                if (h < hd) {
+                    const float v = w1s[3 * h] * rx + w1s[3 * h + 1] * ry + w1s[3 * h + 2] * rz + b1s[h];
                     hid[h] = gelu_erf(v);
                 } else {
                     hid[h] = 0.f;
@@ -245,11 +314,11 @@ __global__ void __launch_bounds__(LQ_T) local_query_kernel(const LocalArgs a) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int c = 4 * c4 + e;
-                        float wv = b2s[s][c];
-                        const float* w2 = w2s[s] + c * a.hidden;
+                        float wv = b2s[c];
+                        const float* w2 = w2s + c * hd;
 #pragma unroll
                         for (int h = 0; h < L_MAXH; ++h)
-                            if (h < a.hidden) wv = fmaf(w2[h], hid[h], wv);
+                            if (h < hd) wv = fmaf(w2[h], hid[h], wv);
                         acc[c] = fmaf(wv + 1.0f, fv[e], acc[c]);
                     }
                 }
@@ -278,7 +347,7 @@ int grid_cells(int n) {
 }
 
 size_t local_ws_bytes(const vdm_local_decoder* d, size_t* off_cnt, size_t* off_start, size_t* off_cursor,
-                      size_t* off_ids, size_t* off_cell) {
+                      size_t* off_ids, size_t* off_cell, size_t* off_rows, size_t* off_nbr) {
     size_t o = 0;
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
     for (int s = 0; s < d->n_scales; ++s) {
@@ -289,7 +358,10 @@ size_t local_ws_bytes(const vdm_local_decoder* d, size_t* off_cnt, size_t* off_s
         off_cursor[s] = o; o = up(o + nc * 4);
         off_ids[s] = o;    o = up(o + (size_t)d->n_anchors[s] * 4);
         off_cell[s] = o;   o = up(o + (size_t)d->n_anchors[s] * 4);
+        off_rows[s] = o;   o = up(o + G * G * 8);
     }
+    *off_nbr = o;          // neighbour ids of one chunk of queries
+    o = up(o + (size_t)L_CHUNK * d->n_scales * d->K * 4);
     return o + 256;
 }
 
@@ -327,8 +399,8 @@ extern "C" {
 vdm_status vdm_local_workspace_size(const vdm_local_decoder* d, size_t* bytes) {
     VDM_TRY(check_local(d));
     if (!bytes) return fail(VDM_ERR_INVALID_ARG, "bytes is NULL");
-    size_t a[L_MAXS], b[L_MAXS], c[L_MAXS], e[L_MAXS], f[L_MAXS];
-    *bytes = local_ws_bytes(d, a, b, c, e, f);
+    size_t a[L_MAXS], b[L_MAXS], c[L_MAXS], e[L_MAXS], f[L_MAXS], g[L_MAXS], h;
+    *bytes = local_ws_bytes(d, a, b, c, e, f, g, &h);
     return VDM_OK;
 }
 
@@ -344,8 +416,8 @@ vdm_status vdm_decode_local(const vdm_local_decoder* d, const float* d_xyz, int6
     char* ws = reinterpret_cast<char*>(((uintptr_t)d_ws + 255) & ~(uintptr_t)255);
     if ((uintptr_t)ws - (uintptr_t)d_ws + need - 256 > ws_bytes)
         return fail(VDM_ERR_WORKSPACE, "workspace too small after alignment");
-    size_t o_cnt[L_MAXS], o_start[L_MAXS], o_cur[L_MAXS], o_ids[L_MAXS], o_cell[L_MAXS];
-    local_ws_bytes(d, o_cnt, o_start, o_cur, o_ids, o_cell);
+    size_t o_cnt[L_MAXS], o_start[L_MAXS], o_cur[L_MAXS], o_ids[L_MAXS], o_cell[L_MAXS], o_rows[L_MAXS], o_nbr;
+    local_ws_bytes(d, o_cnt, o_start, o_cur, o_ids, o_cell, o_rows, &o_nbr);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     LocalArgs a;
     memset(&a, 0, sizeof(a));
@@ -353,7 +425,7 @@ vdm_status vdm_decode_local(const vdm_local_decoder* d, const float* d_xyz, int6
     a.K = d->K;
     a.hidden = d->hidden;
     a.fuse_hidden = d->fuse_hidden;
-    int sumC = 0;
+    int sumC = 0, row_words = 0;
     for (int s = 0; s < d->n_scales; ++s) {
         a.C[s] = d->channels[s];
         a.coff[s] = sumC;
@@ -370,29 +442,50 @@ vdm_status vdm_decode_local(const vdm_local_decoder* d, const float* d_xyz, int6
         int32_t* cursor = reinterpret_cast<int32_t*>(ws + o_cur[s]);
         int32_t* ids = reinterpret_cast<int32_t*>(ws + o_ids[s]);
         int32_t* cell = reinterpret_cast<int32_t*>(ws + o_cell[s]);
+        uint64_t* rows = reinterpret_cast<uint64_t*>(ws + o_rows[s]);
         VDM_CUDA_TRY(cudaMemsetAsync(cnt, 0, (size_t)nc * 4, st));
         bin_count_kernel<<<(n + 255) / 256, 256, 0, st>>>(d->anchors[s], n, G, cnt, cell);
         bin_scan_kernel<<<1, 1024, 0, st>>>(cnt, nc, start, cursor);
         bin_place_kernel<<<(n + 255) / 256, 256, 0, st>>>(cell, n, cursor, ids);
+        row_mask_kernel<<<(G * G + 255) / 256, 256, 0, st>>>(cnt, G, rows);
         VDM_TRY(check_launch("local binning kernels"));
         a.grid[s].G = G;
         a.grid[s].start = start;
         a.grid[s].ids = ids;
+        a.grid[s].rows = rows;
+        a.grid[s].row_off = row_words;
+        row_words += G * G;
     }
     a.sumC = sumC;
+    a.row_words = row_words;
     a.Wf = d->Wf; a.bf = d->bf; a.wo = d->wo; a.bo = d->bo;
     a.xyz = d_xyz;
-    a.M = M;
     a.out = d_out;
-    a.knn_out = d_knn_out;
+    const size_t ksmem = (size_t)row_words * 8;
+    auto knn = d->K <= 8 ? local_knn_kernel<8> : local_knn_kernel<16>;
+    cudaError_t e = cudaFuncSetAttribute(knn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ksmem);
+    if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "local_knn smem attribute: %s", cudaGetErrorString(e));
     size_t smem = 0;
-    for (int s = 0; s < d->n_scales; ++s) smem += (size_t)(d->hidden * 4 + d->channels[s] * (d->hidden + 1));
+    for (int s = 0; s < d->n_scales; ++s) {
+        a.woff[s] = (int)smem;
+        smem += (size_t)(d->hidden * 4 + d->channels[s] * (d->hidden + 1));
+    }
+    a.woff[d->n_scales] = (int)smem;
     smem += (size_t)d->fuse_hidden * (sumC + 2) + (size_t)LQ_T * (sumC + 1);
     smem *= 4;
-    cudaError_t e = cudaFuncSetAttribute(local_query_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "local_query smem attribute: %s", cudaGetErrorString(e));
-    local_query_kernel<<<(unsigned)((M + LQ_T - 1) / LQ_T), LQ_T, smem, st>>>(a);
-    VDM_TRY(check_launch("local_query_kernel"));
+    e = cudaFuncSetAttribute(local_conv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "local_conv smem attribute: %s", cudaGetErrorString(e));
+    // with d_knn_out the neighbour ids go straight to it; else through the workspace, chunk by chunk
+    for (int64_t q0 = 0; q0 < M; q0 += L_CHUNK) {
+        a.q0 = q0;
+        a.q1 = q0 + L_CHUNK < M ? q0 + L_CHUNK : M;
+        a.nbr = d_knn_out ? d_knn_out : reinterpret_cast<int32_t*>(ws + o_nbr);
+        a.nbr_q0 = d_knn_out ? 0 : q0;
+        const unsigned nq = (unsigned)(a.q1 - a.q0);
+        knn<<<(nq + LK_T - 1) / LK_T, LK_T, ksmem, st>>>(a);
+        local_conv_kernel<<<(nq + LQ_T - 1) / LQ_T, LQ_T, smem, st>>>(a);
+        VDM_TRY(check_launch("local query kernels"));
+    }
     VDM_CUDA_TRY(cudaStreamSynchronize(st));
     return VDM_OK;
 }

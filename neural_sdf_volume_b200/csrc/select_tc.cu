@@ -58,6 +58,8 @@ struct SelArgs {
     const int32_t* tile_off;       // [T+1] parent offsets
     const int32_t* plist;
     const int32_t* qorder;
+    const float* probe_xyz;        // probes given as points (or NULL: hierarchical children)
+    const int32_t* probe_off;      // [T+1] with probe_xyz: probes of tile t are [probe_off[t], probe_off[t+1])
     const float* probe_ml;         // [T][n_probe][H][2]
     int R;
     int n_probe;
@@ -304,7 +306,16 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
             const bool valid = my_slot < tpu && t_idx < n_sel;
             const int t = valid ? a.sel_tiles[t_idx] : -1;
             float p[3] = {0.f, 0.f, 0.f};
-            if (valid) {
+            bool has_probe = valid;   // this row holds a probe of sub-volume t
+            if (valid && a.probe_xyz) {
+                const int beg = a.probe_off[t];
+                has_probe = my_i < a.probe_off[t + 1] - beg;
+                if (has_probe) {
+                    p[0] = a.probe_xyz[3 * (size_t)(beg + my_i)];
+                    p[1] = a.probe_xyz[3 * (size_t)(beg + my_i) + 1];
+                    p[2] = a.probe_xyz[3 * (size_t)(beg + my_i) + 2];
+                }
+            } else if (valid) {
                 const int e = a.qorder[8 * a.tile_off[t] + my_i];
                 voxel_point(child_index(a.plist[e >> 3], e & 7, a.R), a.R, p);
             }
@@ -316,7 +327,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
             }
             fence_proxy_async();
             arrive(&sh.bar_pe);
-            const float* ml = valid ? a.probe_ml + ((size_t)t * np + my_i) * H * 2 : nullptr;
+            const float* ml = has_probe ? a.probe_ml + ((size_t)t * np + my_i) * H * 2 : nullptr;
             // Q of every head: + bq, scale, bf16 pairs; warpgroup g packs head dims [32g, 32g+32) into
             // columns [32h + 16g, 32h + 16g + 16)
             for (int h0 = 0; h0 < H && ok; h0 += QROUND) {
@@ -350,7 +361,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                     tc_fence_after();
                     const uint32_t sb = trow + T_S0 + 128 * (i & 1) + 64 * wg;
                     // P = 2^(S - m) / l = 2^(S - m - log2 l); rows without a probe add 2^-inf = 0
-                    const float mo = valid ? ml[h * 2] + __log2f(ml[h * 2 + 1]) : INFINITY;
+                    const float mo = has_probe ? ml[h * 2] + __log2f(ml[h * 2 + 1]) : INFINITY;
                     auto accum = [&](const float (&x)[32], int c0) {
                         if (vcols >= c0 + 32) {
 #pragma unroll
@@ -486,7 +497,30 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// Probes given as points: probe p of tile t (p in [probe_off[t], probe_off[t+1])) keeps its
+// softmax statistics in row t * n_probe + (p - probe_off[t]); every tile is scored.
+__global__ void flat_probe_slots_kernel(const int32_t* __restrict__ probe_off, int T, int n_probe,
+                                        int32_t* __restrict__ ml_slot, int32_t* __restrict__ sel_tiles,
+                                        int32_t* __restrict__ n_sel) {
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    const int lane = threadIdx.x & 31;
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+        const int beg = probe_off[t], end = probe_off[t + 1];
+        for (int p = beg + lane; p < end; p += 32) ml_slot[p] = t * n_probe + (p - beg);
+        if (lane == 0) sel_tiles[t] = t;
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) *n_sel = T;
+}
+
 }  // namespace
+
+vdm_status launch_flat_probe_slots(const int32_t* probe_off, int T, int n_probe, int32_t* ml_slot,
+                                   int32_t* sel_tiles, int32_t* n_sel, cudaStream_t s) {
+    if (T <= 0) return VDM_OK;
+    const int grid = (T + 7) / 8 < 1184 ? (T + 7) / 8 : 1184;
+    flat_probe_slots_kernel<<<grid, 256, 0, s>>>(probe_off, T, n_probe, ml_slot, sel_tiles, n_sel);
+    return check_launch("flat_probe_slots_kernel");
+}
 
 static size_t select_tc_smem(int n_probe, int N) {
     return 1024 + 16384 + (size_t)NS * SLOT + (size_t)(128 / n_probe) * N * 4 + 2 * 4 * 128 * 4;
@@ -509,6 +543,8 @@ vdm_status launch_select_tc(const SelectTcLaunch& L, cudaStream_t st) {
     a.tile_off = L.tile_off;
     a.plist = L.plist;
     a.qorder = L.qorder;
+    a.probe_xyz = L.probe_xyz;
+    a.probe_off = L.probe_off;
     a.probe_ml = L.probe_ml;
     a.R = L.R;
     a.n_probe = L.n_probe;

@@ -270,26 +270,93 @@ vdm_status vdm_select_kv(const vdm_decoder* dec, const void* d_k, const void* d_
                          const float* d_probe_xyz, const int32_t* d_tile_off, int32_t T,
                          int64_t P_total, int32_t top_k, int32_t* d_sel_out, float* d_score_out,
                          vdm_stream stream) {
-    (void)d_v;
     VDM_TRY(check_decoder(dec, true));
     if (N < 1 || T < 0 || P_total < 0) return fail(VDM_ERR_INVALID_ARG, "bad N / T / P");
     if (N > kMaxN) return fail(VDM_ERR_UNSUPPORTED, "N = %d > %d", N, kMaxN);
     if (top_k < 1 || top_k > N) return fail(VDM_ERR_INVALID_ARG, "top_k must be in [1, N]");
     if (T == 0) return VDM_OK;
-    if (!d_k || !d_tile_off || !d_sel_out || (P_total > 0 && !d_probe_xyz))
-        return fail(VDM_ERR_INVALID_ARG, "null k / tile_off / sel / probe_xyz");
-    SelectArgs a;
-    memset(&a, 0, sizeof(a));
-    a.C = dec->C; a.H = dec->H; a.N = N;
-    a.Wq = dec->Wq; a.bq = dec->bq; a.K = d_k;
-    a.T = T;
-    a.probe_xyz = d_probe_xyz ? d_probe_xyz : reinterpret_cast<const float*>(d_tile_off);
-    a.probe_off = d_tile_off;
-    a.top_k = top_k;
-    a.sel = d_sel_out;
-    a.score = d_score_out;
+    if (!d_k || !d_v || !d_tile_off || !d_sel_out || (P_total > 0 && !d_probe_xyz))
+        return fail(VDM_ERR_INVALID_ARG, "null k / v / tile_off / sel / probe_xyz");
+    if (P_total > ((int64_t)1 << 31) - 1) return fail(VDM_ERR_UNSUPPORTED, "P too large");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    VDM_TRY(launch_select(a, dec->dtype, st));
+    // the offsets are checked on the host; the largest probe count picks the probe rows per sub-volume
+    std::vector<int32_t> off((size_t)T + 1);
+    VDM_CUDA_TRY(cudaMemcpyAsync(off.data(), d_tile_off, ((size_t)T + 1) * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+    VDM_CUDA_TRY(cudaStreamSynchronize(st));
+    if (off[0] != 0 || (int64_t)off[T] != P_total)
+        return fail(VDM_ERR_INVALID_ARG, "tile_off[0] must be 0 and tile_off[T] = P (%lld, got %d .. %d)",
+                    (long long)P_total, off[0], off[T]);
+    int max_count = 0;
+    for (int t = 0; t < T; ++t) {
+        const int c = off[t + 1] - off[t];
+        if (c < 0) return fail(VDM_ERR_INVALID_ARG, "tile_off must be non-decreasing (tile %d)", t);
+        max_count = std::max(max_count, c);
+    }
+    // Tensor-core route, the kernels of the hierarchical path: the probes are decoded with full
+    // attention (exporting their per-head softmax maximum and sum), then scored in one pass
+    DecodeArgs d = base_args(dec, d_k, d_v, N);
+    d.work = kWorkFlat;
+    d.qmode = kQueryXyz;
+    d.xyz = d_probe_xyz;
+    d.M = P_total;
+    int np = 0;
+    for (int c : {32, 64, 128})
+        if (np == 0 && max_count <= c && select_tc_supported(dec->C, c, N, dec->dtype)) np = c;
+    if (P_total > 0 && np > 0 && tc_supported(d, dec->dtype)) {
+        size_t o = 0;
+        const size_t o_ml = o;
+        o = align_up(o + (size_t)T * np * dec->H * 2 * sizeof(float));
+        const size_t o_slot = o;
+        o = align_up(o + (size_t)P_total * sizeof(int32_t));
+        const size_t o_tiles = o;
+        o = align_up(o + (size_t)T * sizeof(int32_t));
+        const size_t o_n = o;
+        o = align_up(o + sizeof(int32_t));
+        void* tmp = nullptr;
+        VDM_CUDA_TRY(cudaMallocAsync(&tmp, o, st));
+        auto run = [&]() -> vdm_status {
+            float* probe_ml = at<float>(tmp, o_ml);
+            int32_t* ml_slot = at<int32_t>(tmp, o_slot);
+            int32_t* sel_tiles = at<int32_t>(tmp, o_tiles);
+            int32_t* n_sel = at<int32_t>(tmp, o_n);
+            VDM_TRY(launch_flat_probe_slots(d_tile_off, T, np, ml_slot, sel_tiles, n_sel, st));
+            d.probe_ml = probe_ml;
+            d.ml_slot = ml_slot;
+            VDM_TRY(launch_decode_tc(d, st));
+            SelectTcLaunch L{};
+            L.C = dec->C; L.H = dec->H; L.N = N;
+            L.Wq = dec->Wq; L.bq = dec->bq; L.K = d_k;
+            L.T = T;
+            L.n_sel = n_sel;
+            L.sel_tiles = sel_tiles;
+            L.probe_xyz = d_probe_xyz;
+            L.probe_off = d_tile_off;
+            L.probe_ml = probe_ml;
+            L.n_probe = np;
+            L.top_k = top_k;
+            L.sel = d_sel_out;
+            L.score_out = d_score_out;
+            L.score_rows = d_score_out ? T : 0;
+            return launch_select_tc(L, st);
+        };
+        const vdm_status r = run();
+        const cudaError_t fe = cudaFreeAsync(tmp, st);
+        VDM_TRY(r);
+        if (fe != cudaSuccess) return fail(VDM_ERR_CUDA, "cudaFreeAsync: %s", cudaGetErrorString(fe));
+    } else {
+        // CUDA-core route: any dtype, width and probe count
+        SelectArgs a;
+        memset(&a, 0, sizeof(a));
+        a.C = dec->C; a.H = dec->H; a.N = N;
+        a.Wq = dec->Wq; a.bq = dec->bq; a.K = d_k;
+        a.T = T;
+        a.probe_xyz = d_probe_xyz ? d_probe_xyz : reinterpret_cast<const float*>(d_tile_off);
+        a.probe_off = d_tile_off;
+        a.top_k = top_k;
+        a.sel = d_sel_out;
+        a.score = d_score_out;
+        VDM_TRY(launch_select(a, dec->dtype, st));
+    }
     VDM_CUDA_TRY(cudaStreamSynchronize(st));
     return tc_check_error();
 }
@@ -582,7 +649,7 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
             }
             // selection
             if (sel_tc) {
-                SelectTcLaunch L;
+                SelectTcLaunch L{};
                 L.C = dec->C; L.H = dec->H; L.N = N;
                 L.Wq = dec->Wq; L.bq = dec->bq; L.K = K;
                 L.T = T;

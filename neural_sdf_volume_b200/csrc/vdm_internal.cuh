@@ -165,6 +165,8 @@ struct SelectTcLaunch {
     const int32_t* tile_off;
     const int32_t* plist;
     const int32_t* qorder;
+    const float* probe_xyz;     // probes as points [P][3] (or NULL: the first n_probe children in qorder)
+    const int32_t* probe_off;   // [T+1] with probe_xyz: tile t's probes, at most n_probe of them
     const float* probe_ml;      // [T][n_probe][H][2] from the dense pass
     int R, n_probe, top_k;
     int32_t* sel;               // [T][top_k]
@@ -172,6 +174,9 @@ struct SelectTcLaunch {
     int score_rows;
 };
 bool select_tc_supported(int C, int n_probe, int N, vdm_dtype dt);
+// probes given as points: statistics row of each probe (t * n_probe + rank), tile list 0..T-1
+vdm_status launch_flat_probe_slots(const int32_t* probe_off, int T, int n_probe, int32_t* ml_slot,
+                                   int32_t* sel_tiles, int32_t* n_sel, cudaStream_t s);
 vdm_status launch_select_tc(const SelectTcLaunch& L, cudaStream_t s);
 // picks the kernel for the decoder's dtype and shape; `slots` of tile modes follow its tile size
 vdm_status launch_decode(DecodeArgs a, vdm_dtype dt, cudaStream_t s);

@@ -81,12 +81,15 @@ __global__ void __launch_bounds__(PK_T, MAXV <= 4 ? 4 : 2) pack_kernel(const flo
 // clipped at the grid border (a voxel's own sign is in its cube, so "some neighbour has
 // the other sign" is "the cube holds both signs").  D = D_i o D_j o D_k, and along one
 // axis a word's dilation is its shifted copies plus the facing bit planes of its two
-// neighbour words.  One CTA computes the act words of an 8^3-word core from the sign
-// and near words of the core plus a 2-word halo (12^3 words in shared memory).
+// neighbour words.  One CTA computes the act words of an 8^3-word core.  The region it
+// stages has a 2-word halo along i and j and a 1-word halo along k (the first k step
+// reads the words' k neighbours from global memory): 12 x 12 x 10 words.
 constexpr int MW_T = 512;
 constexpr int MW_C = 8;                 // core edge (words)
-constexpr int MW_E = MW_C + 4;          // staged edge
-constexpr int MW_N = MW_E * MW_E * MW_E;
+constexpr int MW_EI = MW_C + 4;         // staged extent along i and j
+constexpr int MW_EK = MW_C + 2;         // staged extent along k
+constexpr int MW_N = MW_EI * MW_EI * MW_EK;
+constexpr int MW_SA = MW_EI * MW_EK, MW_SB = MW_EK;   // region strides of i and j
 constexpr uint64_t K0 = 0x1111111111111111ull, K3 = 0x8888888888888888ull;   // dk = 0 / 3
 constexpr uint64_t J0 = 0x000F000F000F000Full, J3 = 0xF000F000F000F000ull;   // dj = 0 / 3
 
@@ -99,21 +102,29 @@ __device__ __forceinline__ uint64_t dil(uint64_t x, uint64_t xp, uint64_t xn) {
     return x | (x >> 16) | (x << 16) | ((xn & 0xFFFFull) << 48) | (xp >> 48);
 }
 
-// the same step over staged words; neighbours outside the staged region count as empty
-// (such words are never used as valid)
+// the same step over staged words (both neighbours inside the region by construction)
 template <int AXIS>
 __device__ __forceinline__ uint64_t dil_at(const uint64_t* __restrict__ src, int r) {
-    constexpr int step = AXIS == 0 ? MW_E * MW_E : AXIS == 1 ? MW_E : 1;
-    const int c = AXIS == 0 ? r / (MW_E * MW_E) : AXIS == 1 ? (r / MW_E) % MW_E : r % MW_E;
-    return dil<AXIS>(src[r], c > 0 ? src[r - step] : 0ull, c < MW_E - 1 ? src[r + step] : 0ull);
+    constexpr int step = AXIS == 0 ? MW_SA : AXIS == 1 ? MW_SB : 1;
+    return dil<AXIS>(src[r], src[r - step], src[r + step]);
 }
 
-// Six passes: (1) load with the k step done on the fly from the words' global k
-// neighbours (adjacent in memory), for the inside and the outside words; (2) j step;
-// (3) i step and mark = near | (D(inside) & D(outside)); then, when dilating, (4) k,
-// (5) j and (6) i steps of the mark, the last written straight to the core's words.
-// Valid region after each pass: all, b in [1,10], a and b in [1,10], then e in [1,10],
-// b in [2,9], a in [2,9]: the 8^3 core at offset 2.
+// visit the region words of the box [A0,A1) x [B0,B1) x [E0,E1) (region coordinates)
+template <int A0, int A1, int B0, int B1, int E0, int E1, typename F>
+__device__ __forceinline__ void for_box(F f) {
+    constexpr int NA = A1 - A0, NB = B1 - B0, NE = E1 - E0;
+    for (int t = threadIdx.x; t < NA * NB * NE; t += MW_T) {
+        const int e = E0 + t % NE, b = B0 + (t / NE) % NB, a = A0 + t / (NE * NB);
+        f(a, b, e, (a * MW_EI + b) * MW_EK + e);
+    }
+}
+
+// Six passes, each over the box of the region that the passes after it read: (1) load,
+// with the k step done from global k neighbours, of the inside and outside words (all
+// of the region); (2) j step (b in [1,11)); (3) i step and mark = near | (D(inside) &
+// D(outside)) (a, b in [1,11)); then, when dilating, (4) k step (e in [1,9)), (5) j step
+// (b in [2,10)) and (6) i step of the mark over the core (a, b in [2,10), e in [1,9)),
+// written to the core's words.
 template <bool DILATE>
 __global__ void __launch_bounds__(MW_T) mark_words_kernel(const uint64_t* __restrict__ S,
                                                           const uint64_t* __restrict__ Nr, int nb,
@@ -129,18 +140,16 @@ __global__ void __launch_bounds__(MW_T) mark_words_kernel(const uint64_t* __rest
     const int ck = c % ncta; c /= ncta;
     const int cj = c % ncta; c /= ncta;
     const int ci = c;
-    const int i0 = ci * MW_C - 2, j0 = cj * MW_C - 2, k0 = ck * MW_C - 2;
-    auto on_grid = [&](int r, size_t& w) -> bool {
-        const int a = r / (MW_E * MW_E), b = (r / MW_E) % MW_E, e = r % MW_E;
+    const int i0 = ci * MW_C - 2, j0 = cj * MW_C - 2, k0 = ck * MW_C - 1;   // region origin (words)
+    auto on_grid = [&](int a, int b, int e) -> bool {
         const int bi = i0 + a, bj = j0 + b, bk = k0 + e;
-        w = ((size_t)bi * nb + bj) * nb + bk;
         return bi >= 0 && bi < nb && bj >= 0 && bj < nb && bk >= 0 && bk < nb;
     };
-    for (int r = threadIdx.x; r < MW_N; r += MW_T) {
-        size_t w;
+    for_box<0, MW_EI, 0, MW_EI, 0, MW_EK>([&](int a, int b, int e, int r) {
         uint64_t din = 0, dout = 0, n = 0;
-        if (on_grid(r, w)) {
-            const int bk = k0 + r % MW_E;
+        if (on_grid(a, b, e)) {
+            const int bk = k0 + e;
+            const size_t w = ((size_t)(i0 + a) * nb + (j0 + b)) * nb + bk;
             const uint64_t s = S[w];
             const bool hp = bk > 0, hn = bk + 1 < nb;
             const uint64_t sp = hp ? S[w - 1] : 0ull, sn = hn ? S[w + 1] : 0ull;
@@ -151,31 +160,29 @@ __global__ void __launch_bounds__(MW_T) mark_words_kernel(const uint64_t* __rest
         A[r] = din;
         B[r] = dout;
         Nw[r] = n;
-    }
+    });
     __syncthreads();
-    for (int r = threadIdx.x; r < MW_N; r += MW_T) {
+    for_box<0, MW_EI, 1, MW_EI - 1, 0, MW_EK>([&](int, int, int, int r) {
         X[r] = dil_at<1>(A, r);
         Y[r] = dil_at<1>(B, r);
-    }
+    });
     __syncthreads();
-    for (int r = threadIdx.x; r < MW_N; r += MW_T) {
-        size_t w;
-        A[r] = on_grid(r, w) ? (Nw[r] | (dil_at<0>(X, r) & dil_at<0>(Y, r))) : 0ull;   // mark, 0 off the grid
-    }
+    // mark; words off the grid stay empty (their dilated sign words are not)
+    for_box<1, MW_EI - 1, 1, MW_EI - 1, 0, MW_EK>([&](int a, int b, int e, int r) {
+        A[r] = on_grid(a, b, e) ? (Nw[r] | (dil_at<0>(X, r) & dil_at<0>(Y, r))) : 0ull;
+    });
     __syncthreads();
     if (DILATE) {
-        for (int r = threadIdx.x; r < MW_N; r += MW_T) B[r] = dil_at<2>(A, r);
+        for_box<1, MW_EI - 1, 1, MW_EI - 1, 1, MW_EK - 1>([&](int, int, int, int r) { B[r] = dil_at<2>(A, r); });
         __syncthreads();
-        for (int r = threadIdx.x; r < MW_N; r += MW_T) X[r] = dil_at<1>(B, r);
+        for_box<1, MW_EI - 1, 2, MW_EI - 2, 1, MW_EK - 1>([&](int, int, int, int r) { X[r] = dil_at<1>(B, r); });
         __syncthreads();
     }
-    for (int r = threadIdx.x; r < MW_C * MW_C * MW_C; r += MW_T) {
-        const int a = r / (MW_C * MW_C), b = (r / MW_C) % MW_C, e = r % MW_C;
-        const int bi = ci * MW_C + a, bj = cj * MW_C + b, bk = ck * MW_C + e;
-        const int rr = ((a + 2) * MW_E + (b + 2)) * MW_E + (e + 2);
+    for_box<2, MW_EI - 2, 2, MW_EI - 2, 1, MW_EK - 1>([&](int a, int b, int e, int r) {
+        const int bi = i0 + a, bj = j0 + b, bk = k0 + e;
         if (bi < nb && bj < nb && bk < nb)
-            act[((size_t)bi * nb + bj) * nb + bk] = DILATE ? dil_at<0>(X, rr) : A[rr];
-    }
+            act[((size_t)bi * nb + bj) * nb + bk] = DILATE ? dil_at<0>(X, r) : A[r];
+    });
 }
 
 // ------------------------------------------------------------------ compaction
@@ -334,38 +341,38 @@ __global__ void __launch_bounds__(CP_T) compact_kernel(const uint64_t* __restric
 
 // ------------------------------------------------------------------ inherit fill
 // Every voxel of the fine grid takes its parent's value (the decode that follows
-// overwrites the children of refined parents): 8 fine voxels along k per thread from
-// 4 parents (one 16-byte load), two 16-byte stores; no partial-sector writes.
+// overwrites the children of refined parents).  Item t = (coarse row (ci, cj), q): one
+// 8-byte load of parents 2q, 2q+1 and one 16-byte store of their 4 children along k in
+// each of the 4 fine rows (2ci + di, 2cj + dj); consecutive lanes take consecutive q, so
+// every load and store instruction of a warp covers one contiguous span.
 template <bool STREAM>
-__device__ __forceinline__ void fill_group(const float* __restrict__ fc, int R, float* __restrict__ ff, size_t t) {
-    const int R2 = 2 * R;
-    const int Q = R2 >> 3;   // groups of 8 fine voxels per row
-    const int q = (int)(t % Q);
-    const size_t ij = t / Q;
-    const int j = (int)(ij % R2), i = (int)(ij / R2);
-    const float4 p = *reinterpret_cast<const float4*>(fc + ((size_t)(i >> 1) * R + (j >> 1)) * R + 4 * q);
-    float4* dst = reinterpret_cast<float4*>(ff + ((size_t)i * R2 + j) * R2 + 8 * q);
-    const float4 a = make_float4(p.x, p.x, p.y, p.y), b = make_float4(p.z, p.z, p.w, p.w);
-    if (STREAM) {
-        __stcs(dst, a);
-        __stcs(dst + 1, b);
-    } else {
-        dst[0] = a;
-        dst[1] = b;
+__device__ __forceinline__ void fill_item(const float* __restrict__ fc, int R, float* __restrict__ ff, uint32_t t,
+                                          uint32_t Q) {
+    const uint32_t cr = t / Q, q = t - cr * Q;
+    const uint32_t ci = cr / (uint32_t)R, cj = cr - ci * (uint32_t)R;
+    const size_t R2 = 2 * (size_t)R;
+    const float2 p = *reinterpret_cast<const float2*>(fc + (size_t)cr * R + 2 * q);
+    const float4 v = make_float4(p.x, p.x, p.y, p.y);
+    float* row0 = ff + ((2 * ci) * R2 + 2 * cj) * R2 + 4 * q;
+#pragma unroll
+    for (int d = 0; d < 4; ++d) {
+        float4* dst = reinterpret_cast<float4*>(row0 + ((d >> 1) * R2 + (d & 1)) * R2);
+        if (STREAM) __stcs(dst, v);
+        else *dst = v;
     }
 }
 
-// two groups per thread and iteration (a grid-stride apart): more loads and stores in flight
 template <bool STREAM>
 __global__ void __launch_bounds__(256) fill_kernel(const float* __restrict__ fc, int R, float* __restrict__ ff) {
-    const size_t n = (size_t)(2 * R) * (2 * R) * ((2 * R) >> 3);
-    const size_t stride = (size_t)gridDim.x * blockDim.x;
-    size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
-    for (; t + stride < n; t += 2 * stride) {
-        fill_group<STREAM>(fc, R, ff, t);
-        fill_group<STREAM>(fc, R, ff, t + stride);
+    const uint32_t Q = (uint32_t)R >> 1;                   // parent pairs per coarse row
+    const uint32_t n = (uint32_t)R * (uint32_t)R * Q;
+    const uint32_t stride = gridDim.x * blockDim.x;
+    uint32_t t = blockIdx.x * blockDim.x + threadIdx.x;
+    for (; t + stride < n; t += 2 * stride) {            // two items in flight per thread
+        fill_item<STREAM>(fc, R, ff, t, Q);
+        fill_item<STREAM>(fc, R, ff, t + stride, Q);
     }
-    if (t < n) fill_group<STREAM>(fc, R, ff, t);
+    if (t < n) fill_item<STREAM>(fc, R, ff, t, Q);
 }
 
 // ------------------------------------------------------------------ probe order
@@ -504,7 +511,7 @@ vdm_status launch_mark_dilate(const float* f, const float* fn, int R, float thr,
     if (R % 4 || R < 4 || R > 1024) return fail(VDM_ERR_UNSUPPORTED, "mark: R = %d", R);
     const int nb = R >> 2;
     const size_t nw = (size_t)nb * nb * nb;
-    const int smem = 5 * MW_N * (int)sizeof(uint64_t);   // 69 KB: set for the current device
+    const int smem = 5 * MW_N * (int)sizeof(uint64_t);   // 57.6 KB: set for the current device
     cudaError_t e = cudaFuncSetAttribute(mark_words_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "mark_words smem attribute: %s", cudaGetErrorString(e));
     const int ncta = (nb + MW_C - 1) / MW_C;
@@ -550,14 +557,16 @@ vdm_status launch_compact(const uint64_t* words, int n_words, int R, int32_t* wo
 }
 
 vdm_status launch_fill(const float* f_coarse, int R, float* f_fine, cudaStream_t s) {
-    const size_t n = (size_t)(2 * R) * (2 * R) * ((2 * R) >> 3);
+    if (R < 2 || (R & 1)) return fail(VDM_ERR_INVALID_ARG, "fill needs an even resolution (R = %d)", R);
+    const size_t n = (size_t)R * R * (R / 2);   // items: 64 bytes of the fine grid each
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const size_t want = (n + 255) / 256;
     const int grid = (int)(want < (size_t)sms * 8 ? want : (size_t)sms * 8);
+    if (n + 2 * (size_t)grid * 256 > 0xFFFFFFFFull) return fail(VDM_ERR_UNSUPPORTED, "fill: R = %d too large", R);
     // a fine grid much larger than L2 is written with streaming stores
-    const bool stream = n * 32 > ((size_t)64 << 20);
+    const bool stream = n * 64 > ((size_t)64 << 20);
     prof_begin(kProfFill, s);
     if (stream) fill_kernel<true><<<grid, 256, 0, s>>>(f_coarse, R, f_fine);
     else fill_kernel<false><<<grid, 256, 0, s>>>(f_coarse, R, f_fine);

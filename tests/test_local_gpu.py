@@ -47,3 +47,28 @@ def test_local_decoder_empty_and_errors():
     with pytest.raises(vdm.VdmError) as ei:
         vdm.vdm_decode_local(ld, torch.zeros((4, 3), device="cuda"))
     assert ei.value.status == 2
+
+
+def test_local_decoder_several_chunks():
+    """More queries than one chunk of the neighbour buffer (65,536), with and
+    without the neighbour export: sampled rows against the oracle, and the
+    two calls' SDF values identical."""
+    import torch
+    import neural_sdf_volume_b200 as vdm
+    sp = W.make_spheres(6, seed=0, key=54)[0]
+    d = W.make_local_decoder(sp, n_anchors=(1024, 4096), channels=(32, 16), seed=0, key=55)
+    K = 8
+    ld = vdm.LocalDecoder.from_numpy(d, K)
+    rng = np.random.default_rng(7)
+    x = rng.uniform(-1.0, 1.0, (140_000, 3)).astype(np.float32)
+    xt = torch.from_numpy(x).cuda()
+    out, knn = vdm.vdm_decode_local(ld, xt, want_knn=True)
+    out2 = vdm.vdm_decode_local(ld, xt)
+    out, out2, knn = out.cpu().numpy(), out2.cpu().numpy(), knn.cpu().numpy()
+    assert np.array_equal(out, out2)
+    rows = np.concatenate([rng.choice(x.shape[0], 600, replace=False), [0, 65_535, 65_536, 131_071, 131_072,
+                                                                         x.shape[0] - 1]])
+    for s, a in enumerate(d["anchors"]):
+        assert np.array_equal(knn[rows, s, :], OL.knn(x[rows], a, K)), f"scale {s}"
+    want = OL.decode_local(x[rows], d["anchors"], d["feats"], d["scales"], d["fuse"], K)
+    assert np.abs(out[rows] - want).max() <= 1e-4 * max(1.0, np.abs(want).max())

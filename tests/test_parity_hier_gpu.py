@@ -140,8 +140,10 @@ def test_full_size_batched_slim_adaptive():
 
 
 def test_select_kv_scores_and_topk_given_the_same_scores():
-    """vdm_select_kv: scores within tolerance of the oracle's; the selection is
-    exactly the oracle's Top-K rule applied to the GPU's own scores."""
+    """vdm_select_kv with a sub-volume of 130 probes (more than the tensor-core
+    route's 128 rows, so the CUDA-core route): scores within tolerance of the
+    oracle's; the selection is exactly the oracle's Top-K rule applied to the
+    GPU's own scores."""
     import torch
     import neural_sdf_volume_b200 as vdm
     spec = W.DecoderSpec(C=512, H=8, F=2048, N=700, query_ln=True, dtype="bf16")
@@ -167,3 +169,61 @@ def test_select_kv_scores_and_topk_given_the_same_scores():
         assert np.abs(score[t] - want).max() <= 2e-2 * max(1.0, want.max())
         overlap = len(np.intersect1d(sel[t], OA.top_k(want, k))) / k
         assert overlap >= 0.9, overlap
+
+
+def test_select_kv_tensor_core_route_scores_and_topk():
+    """vdm_select_kv with at most 128 probes per sub-volume (the tensor-core
+    route, ragged counts including 0 and a full 128): scores within tolerance
+    of the oracle's, the selection exactly the Top-K rule on the GPU's scores."""
+    import torch
+    import neural_sdf_volume_b200 as vdm
+    spec = W.DecoderSpec(C=512, H=8, F=2048, N=700, query_ln=True, dtype="bf16")
+    case = Case(spec, key=2, stress=True)
+    counts = [0, 1, 31, 64, 100, 128, 0, 17]
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    pts = W.make_points(int(off[-1]), seed=5, key=3)[0]
+    k = 100
+    sel, score = vdm.vdm_select_kv(case.dec, case.K, case.V, torch.from_numpy(pts).cuda(),
+                                   torch.from_numpy(off).cuda(), k, want_scores=True)
+    sel = sel.cpu().numpy()
+    score = score.cpu().numpy().astype(np.float64)
+    K, V = case.okv()
+    for t in range(len(counts)):
+        assert np.array_equal(sel[t], OA.top_k(score[t], k)), f"tile {t}"
+        if counts[t] == 0:
+            assert np.array_equal(sel[t], np.arange(k))
+            assert not score[t].any()
+            continue
+        want = OA.token_scores(OA.query_vectors(pts[off[t]:off[t + 1]], case.w), K)
+        assert abs(score[t].sum() - counts[t] * 8) < 1e-3 * counts[t] * 8
+        assert np.abs(score[t] - want).max() <= 2e-2 * max(1.0, want.max())
+
+
+def test_select_kv_reproduces_the_hierarchical_selection():
+    """The public selection call run on a hierarchical level's own probes (as
+    points, in rank order) gives that level's scores and kept tokens bit for
+    bit: both run the same tensor-core kernels."""
+    import torch
+    import neural_sdf_volume_b200 as vdm
+    spec = W.DecoderSpec(C=512, H=8, F=2048, N=256, query_ln=True, dtype="bf16")
+    case = Case(spec, key=2, n_spheres=5, sphere_key=3, stress=True)
+    n_probe, k = 64, 64
+    grid, stats, dbg = _run(case, 1, 12, 3, True, n_probe=n_probe, top_k=k)
+    checked = 0
+    for l in (1, 2):
+        R = 12 << l
+        sel_h = dbg["sel"][l][0].cpu().numpy()
+        rows = np.flatnonzero(sel_h[:, 0] >= 0)          # sub-volumes that were scored
+        if rows.size == 0:
+            continue
+        vox = dbg["probes"][l][0].cpu().numpy()[rows].astype(np.int64)
+        assert (vox >= 0).all()
+        ijk = np.stack([vox // (R * R), (vox // R) % R, vox % R], axis=-1).reshape(-1, 3)
+        xyz = (np.float32(-1.0) + (2 * ijk + 1).astype(np.float32) / np.float32(R)).astype(np.float32)
+        off = (np.arange(rows.size + 1) * n_probe).astype(np.int32)
+        sel, score = vdm.vdm_select_kv(case.dec, case.K, case.V, torch.from_numpy(xyz).cuda(),
+                                       torch.from_numpy(off).cuda(), k, want_scores=True)
+        assert np.array_equal(sel.cpu().numpy(), sel_h[rows]), l
+        assert np.array_equal(score.cpu().numpy(), dbg["scores"][l][0].cpu().numpy()[rows]), l
+        checked += rows.size
+    assert checked > 0
