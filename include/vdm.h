@@ -228,7 +228,8 @@ typedef struct {
                                            of the non-empty sub-volumes       */
     int32_t* sel[VDM_MAX_LEVELS];       /* [B][max_tiles][top_k] kept tokens of
                                            sub-volume i (rows of sub-volumes
-                                           without a selection: untouched)   */
+                                           without a selection, those with at
+                                           most n_probe queries: unspecified) */
     int64_t max_tiles;                  /* capacity of the per-sub-volume rows */
     int32_t* probes[VDM_MAX_LEVELS];    /* [B][max_tiles][n_probe] fine voxel
                                            indices of the probes of sub-volume

@@ -213,7 +213,13 @@ def test_select_kv_reproduces_the_hierarchical_selection():
     for l in (1, 2):
         R = 12 << l
         sel_h = dbg["sel"][l][0].cpu().numpy()
-        rows = np.flatnonzero(sel_h[:, 0] >= 0)          # sub-volumes that were scored
+        # sub-volume i holds 8 children per refined parent of its 4^3 parent block (one mask word);
+        # those with more queries than probes were scored
+        tiles = dbg["tile_ids"][l][0].cpu().numpy()
+        tiles = tiles[tiles >= 0]
+        words = dbg["active"][l - 1][0].cpu().numpy().view(np.uint64)[tiles]
+        n_q = 8 * np.array([bin(int(w)).count("1") for w in words])
+        rows = np.flatnonzero(n_q > n_probe)
         if rows.size == 0:
             continue
         vox = dbg["probes"][l][0].cpu().numpy()[rows].astype(np.int64)
