@@ -202,7 +202,11 @@ __device__ __forceinline__ Unit unit_of(const DecodeArgs& a, int64_t unit) {
         u.nq = u.qbeg < M ? (int)(M - u.qbeg < BM ? M - u.qbeg : BM) : 0;
         return u;
     }
-    const int t = (int)(unit / a.slots), sl = (int)(unit - (int64_t)t * a.slots);
+    // slot-major order: units t, t + T, ... of one sub-volume are a grid stride apart, so the
+    // persistent CTAs' static round-robin deals every slot index to every CTA (a tile-major
+    // order with T * slots units would give CTA c only slot c mod slots, and the later slots
+    // of a sub-volume are often empty)
+    const int t = (int)(unit % a.T), sl = (int)(unit / a.T);
     const int cnt = 8 * (a.tile_off[t + 1] - a.tile_off[t]);
     int lo, n;
     if (a.work == kWorkTileDense) {
@@ -342,10 +346,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
     auto unit_at = [&](int64_t it, uint32_t r) -> Unit {
         if (!PAIR) return unit_of(a, it);
         if (a.work == kWorkFlat) return unit_of(a, 2 * it + r);
-        const int64_t t = it / spt;
-        const int sl = 2 * (int)(it - t * spt) + (int)r;
-        if (sl < a.slots) return unit_of(a, t * a.slots + sl);
-        Unit u = unit_of(a, t * a.slots);   // same sub-volume (same keys), no queries
+        const int64_t t = it % a.T;
+        const int sl = 2 * (int)(it / a.T) + (int)r;
+        if (sl < a.slots) return unit_of(a, (int64_t)sl * a.T + t);
+        Unit u = unit_of(a, t);   // same sub-volume (same keys), no queries
         u.nq = 0;
         return u;
     };

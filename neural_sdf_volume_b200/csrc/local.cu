@@ -23,15 +23,14 @@
 // can only search one ring more), which makes the result exact.
 //
 // Two kernels per chunk of queries.  local_knn_kernel: one thread per query,
-// the neighbour list sorted in registers (fixed capacity, static indices); the
-// cells are scanned through per-row occupancy words (bit k of row (i, j): cell
-// (i, j, k) holds an anchor) staged in shared memory, so empty cells cost a
-// few bit operations and only occupied cells are read from global memory --
-// a query far from every anchor scans many rings of cells.  local_conv_kernel:
-// one thread per query, the dynamic-weight hidden layer and the scale's
-// channel accumulators in registers, the scale outputs in its row of shared
-// memory, then the fusion MLP from shared memory; all weights are staged in
-// shared memory once per CTA.
+// the neighbour list sorted in registers (fixed capacity, static indices); a
+// ring of cells is walked through occupancy words staged in shared memory (one
+// bit per occupied plane, per occupied row of a plane, per occupied cell of a
+// row), so only occupied cells are visited and read from global memory -- a
+// query far from every anchor grows its ring many times over empty space.
+// local_conv_kernel: one warp per query (lanes over hidden units, channels and
+// fusion units; the neighbour's hidden values broadcast by shuffles), all
+// weights staged in shared memory once per CTA.
 #include <mutex>
 #include <string.h>
 
@@ -40,9 +39,9 @@
 namespace vdm {
 namespace {
 
-constexpr int LQ_T = 64;          // queries per CTA (AVS-Conv and fusion)
+constexpr int LQ_T = 256;         // threads per CTA (AVS-Conv and fusion: one warp per query)
 constexpr int LK_T = 128;         // queries per CTA (neighbour search)
-constexpr int L_CHUNK = 1 << 16;  // queries per chunk (neighbour ids kept in the workspace)
+constexpr int L_CHUNK = 1 << 18;  // queries per chunk (neighbour ids kept in the workspace)
 constexpr int L_MAXS = VDM_LOCAL_MAX_SCALES;
 constexpr int L_MAXK = 16, L_MAXH = 32, L_MAXC = 64, L_MAXSUMC = 128, L_MAXF = 64;
 
@@ -169,12 +168,39 @@ __device__ __forceinline__ void knn_insert(float (&bd)[KC], int (&bi)[KC], float
     }
 }
 
+// bits lo..hi of a word (0 <= lo <= hi <= 63)
+__device__ __forceinline__ uint64_t bit_span(int lo, int hi) {
+    return (~0ull >> (63 - hi)) & (~0ull << lo);
+}
+
+// Occupancy in shared memory, per scale from row_off: the G^2 row words, then per plane i a
+// word with bit j = row (i, j) occupied, then one word with bit i = plane i occupied.  A ring
+// visits occupied planes, their occupied rows and those rows' occupied cells only.
 template <int KC>
 __global__ void __launch_bounds__(LK_T) local_knn_kernel(const LocalArgs a) {
     extern __shared__ uint64_t lrows[];
     for (int s = 0; s < a.n_scales; ++s) {
         const int G = a.grid[s].G;
-        for (int i = threadIdx.x; i < G * G; i += LK_T) lrows[a.grid[s].row_off + i] = a.grid[s].rows[i];
+        uint64_t* r = lrows + a.grid[s].row_off;
+        for (int i = threadIdx.x; i < G * G; i += LK_T) r[i] = a.grid[s].rows[i];
+    }
+    __syncthreads();
+    for (int s = 0; s < a.n_scales; ++s) {
+        const int G = a.grid[s].G;
+        uint64_t* r = lrows + a.grid[s].row_off;
+        for (int i = threadIdx.x; i < G; i += LK_T) {
+            uint64_t pm = 0;
+            for (int j = 0; j < G; ++j) pm |= (uint64_t)(r[i * G + j] != 0) << j;
+            r[G * G + i] = pm;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < a.n_scales) {
+        const int G = a.grid[threadIdx.x].G;
+        uint64_t* r = lrows + a.grid[threadIdx.x].row_off;
+        uint64_t im = 0;
+        for (int i = 0; i < G; ++i) im |= (uint64_t)(r[G * G + i] != 0) << i;
+        r[G * G + G] = im;
     }
     __syncthreads();
     const int64_t q = a.q0 + (int64_t)blockIdx.x * LK_T + threadIdx.x;
@@ -186,6 +212,8 @@ __global__ void __launch_bounds__(LK_T) local_knn_kernel(const LocalArgs a) {
         const ScaleGrid g = a.grid[s];
         const int G = g.G;
         const uint64_t* rows = lrows + g.row_off;
+        const uint64_t* planes = rows + G * G;
+        const uint64_t occupied = planes[G];
         const float cs = 2.0f / (float)G;
         const int cx = cell_of(x, G), cy = cell_of(y, G), cz = cell_of(z, G);
         float bd[KC];
@@ -206,9 +234,12 @@ __global__ void __launch_bounds__(LK_T) local_knn_kernel(const LocalArgs a) {
             uint64_t ends = 0;                                              // k = cz - r, cz + r
             if (cz - r >= 0) ends |= 1ull << (cz - r);
             if (cz + r < G) ends |= 1ull << (cz + r);
-            for (int i = i0; i <= i1; ++i) {
+            const uint64_t jspan = bit_span(j0, j1);
+            for (uint64_t iv = occupied & bit_span(i0, i1); iv; iv &= iv - 1) {
+                const int i = __ffsll((long long)iv) - 1;
                 const bool ei = i == cx - r || i == cx + r;
-                for (int j = j0; j <= j1; ++j) {
+                for (uint64_t jv = planes[i] & jspan; jv; jv &= jv - 1) {
+                    const int j = __ffsll((long long)jv) - 1;
                     uint64_t m = rows[i * G + j] & ((ei || j == cy - r || j == cy + r) ? span : ends);
                     while (m) {
                         const int k = __ffsll((long long)m) - 1;
@@ -252,92 +283,92 @@ __global__ void __launch_bounds__(LK_T) local_knn_kernel(const LocalArgs a) {
     }
 }
 
+// One warp per query.  Lane h computes hidden unit h of a neighbour's dynamic-weight layer
+// (hidden <= 32), lanes take channels c = lane and lane + 32 of the per-channel weights and
+// features, the scale outputs go to the warp's row in shared memory, then lane o computes
+// fusion units o and o + 32.  Weights are staged transposed (W2^T [hidden][C], Wf^T
+// [sum C][fuse_hidden]) so that consecutive lanes read consecutive words.
 __global__ void __launch_bounds__(LQ_T) local_conv_kernel(const LocalArgs a) {
     extern __shared__ float lsm[];
-    // staged weights: per scale W1 [hidden][3], b1, W2 [C][hidden], b2; then Wf, bf, wo; then the
-    // per-thread feature rows
-    const int hd = a.hidden;
+    const int hd = a.hidden, FH = a.fuse_hidden, SC = a.sumC;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int s = 0; s < a.n_scales; ++s) {
         float* w = lsm + a.woff[s];
         const int C = a.C[s];
         for (int i = threadIdx.x; i < hd * 3; i += LQ_T) w[i] = a.W1[s][i];
         for (int i = threadIdx.x; i < hd; i += LQ_T) w[3 * hd + i] = a.b1[s][i];
-        for (int i = threadIdx.x; i < C * hd; i += LQ_T) w[4 * hd + i] = a.W2[s][i];
+        for (int i = threadIdx.x; i < C * hd; i += LQ_T) {   // W2 [C][hidden] -> [hidden][C]
+            const int c = i / hd, h = i - c * hd;
+            w[4 * hd + h * C + c] = a.W2[s][i];
+        }
         for (int i = threadIdx.x; i < C; i += LQ_T) w[4 * hd + C * hd + i] = a.b2[s][i];
     }
-    float* wfs = lsm + a.woff[a.n_scales];
-    float* bfs = wfs + a.fuse_hidden * a.sumC;
-    float* wos = bfs + a.fuse_hidden;
-    float* frow = wos + a.fuse_hidden + threadIdx.x * (a.sumC + 1);   // odd row stride: rows in different banks
-    for (int i = threadIdx.x; i < a.fuse_hidden * a.sumC; i += LQ_T) wfs[i] = a.Wf[i];
-    for (int i = threadIdx.x; i < a.fuse_hidden; i += LQ_T) {
+    float* wft = lsm + a.woff[a.n_scales];   // Wf [FH][SC] -> [SC][FH]
+    float* bfs = wft + FH * SC;
+    float* wos = bfs + FH;
+    float* frow = wos + FH + warp * SC;
+    for (int i = threadIdx.x; i < FH * SC; i += LQ_T) {
+        const int o = i / SC, c = i - o * SC;
+        wft[c * FH + o] = a.Wf[i];
+    }
+    for (int i = threadIdx.x; i < FH; i += LQ_T) {
         bfs[i] = a.bf[i];
         wos[i] = a.wo[i];
     }
     __syncthreads();
-    const int64_t q = a.q0 + (int64_t)blockIdx.x * LQ_T + threadIdx.x;
-    if (q >= a.q1) return;
-    const float x = a.xyz[3 * q], y = a.xyz[3 * q + 1], z = a.xyz[3 * q + 2];
     const int K = a.K;
-    const int32_t* nin = a.nbr + (q - a.nbr_q0) * a.n_scales * K;
-    for (int s = 0; s < a.n_scales; ++s) {
-        const float* an = a.anchors[s];
-        const int C = a.C[s];
-        const float* w1s = lsm + a.woff[s];
-        const float* b1s = w1s + 3 * hd;
-        const float* w2s = w1s + 4 * hd;
-        const float* b2s = w2s + C * hd;
-        float acc[L_MAXC];
-#pragma unroll
-        for (int c = 0; c < L_MAXC; ++c) acc[c] = 0.f;
-        const float* F = a.feats[s];
-        for (int t = 0; t < K; ++t) {
-            const int id = nin[s * K + t];
-            if (id < 0) continue;
-            const float rx = an[3 * id] - x, ry = an[3 * id + 1] - y, rz = an[3 * id + 2] - z;
-            float hid[L_MAXH];
-#pragma unroll
-            for (int h = 0; h < L_MAXH; ++h) {
-                if (h < hd) {
-                    const float v = w1s[3 * h] * rx + w1s[3 * h + 1] * ry + w1s[3 * h + 2] * rz + b1s[h];
-                    hid[h] = gelu_erf(v);
-                } else {
-                    hid[h] = 0.f;
+    const int64_t nq = a.q1 - a.q0;
+    const int wpc = LQ_T / 32;
+    for (int64_t qi = (int64_t)blockIdx.x * wpc + warp; qi < nq; qi += (int64_t)gridDim.x * wpc) {
+        const int64_t q = a.q0 + qi;
+        const float x = a.xyz[3 * q], y = a.xyz[3 * q + 1], z = a.xyz[3 * q + 2];
+        const int32_t* nin = a.nbr + (q - a.nbr_q0) * a.n_scales * K;
+        for (int s = 0; s < a.n_scales; ++s) {
+            const float* an = a.anchors[s];
+            const float* F = a.feats[s];
+            const int C = a.C[s];
+            const float* w1 = lsm + a.woff[s];
+            const float* b1 = w1 + 3 * hd;
+            const float* w2t = w1 + 4 * hd;
+            const float* b2 = w2t + C * hd;
+            const bool c0 = lane < C, c1 = lane + 32 < C;
+            const float bias0 = c0 ? b2[lane] : 0.f, bias1 = c1 ? b2[lane + 32] : 0.f;
+            const int my_id = lane < K ? nin[s * K + lane] : -1;
+            float acc0 = 0.f, acc1 = 0.f;
+            for (int t = 0; t < K; ++t) {
+                const int id = __shfl_sync(0xffffffffu, my_id, t);
+                if (id < 0) continue;
+                const float rx = an[3 * id] - x, ry = an[3 * id + 1] - y, rz = an[3 * id + 2] - z;
+                const float hv = lane < hd
+                    ? gelu_erf(w1[3 * lane] * rx + w1[3 * lane + 1] * ry + w1[3 * lane + 2] * rz + b1[lane])
+                    : 0.f;
+                const float f0 = c0 ? F[(size_t)id * C + lane] : 0.f;
+                const float f1 = c1 ? F[(size_t)id * C + lane + 32] : 0.f;
+                float wv0 = bias0, wv1 = bias1;
+                for (int h = 0; h < hd; ++h) {
+                    const float hh = __shfl_sync(0xffffffffu, hv, h);
+                    if (c0) wv0 = fmaf(w2t[h * C + lane], hh, wv0);
+                    if (c1) wv1 = fmaf(w2t[h * C + lane + 32], hh, wv1);
                 }
+                acc0 = fmaf(wv0 + 1.0f, f0, acc0);
+                acc1 = fmaf(wv1 + 1.0f, f1, acc1);
             }
-            const float4* Fj = reinterpret_cast<const float4*>(F + (size_t)id * C);
-#pragma unroll
-            for (int c4 = 0; c4 < L_MAXC / 4; ++c4) {
-                if (4 * c4 < C) {
-                    const float4 f = Fj[c4];
-                    const float fv[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c = 4 * c4 + e;
-                        float wv = b2s[c];
-                        const float* w2 = w2s + c * hd;
-#pragma unroll
-                        for (int h = 0; h < L_MAXH; ++h)
-                            if (h < hd) wv = fmaf(w2[h], hid[h], wv);
-                        acc[c] = fmaf(wv + 1.0f, fv[e], acc[c]);
-                    }
-                }
-            }
+            const float invk = 1.0f / (float)K;
+            if (c0) frow[a.coff[s] + lane] = acc0 * invk;
+            if (c1) frow[a.coff[s] + lane + 32] = acc1 * invk;
         }
-        const float invk = 1.0f / (float)K;
-#pragma unroll
-        for (int c = 0; c < L_MAXC; ++c)
-            if (c < C) frow[a.coff[s] + c] = acc[c] * invk;
+        __syncwarp();
+        // fusion: wo . GELU(Wf f + bf) + bo
+        float part = 0.f;
+        for (int o = lane; o < FH; o += 32) {
+            float v = bfs[o];
+            for (int c = 0; c < SC; ++c) v = fmaf(wft[c * FH + o], frow[c], v);
+            part = fmaf(wos[o], gelu_erf(v), part);
+        }
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) a.out[q] = a.bo[0] + part;
+        __syncwarp();   // frow is rewritten by the warp's next query
     }
-    // ---- fusion: wo . GELU(Wf f + bf) + bo
-    float sdf = a.bo[0];
-    for (int o = 0; o < a.fuse_hidden; ++o) {
-        float v = bfs[o];
-        const float* wf = wfs + o * a.sumC;
-        for (int c = 0; c < a.sumC; ++c) v = fmaf(wf[c], frow[c], v);
-        sdf = fmaf(wos[o], gelu_erf(v), sdf);
-    }
-    a.out[q] = sdf;
 }
 
 int grid_cells(int n) {
@@ -454,7 +485,7 @@ vdm_status vdm_decode_local(const vdm_local_decoder* d, const float* d_xyz, int6
         a.grid[s].ids = ids;
         a.grid[s].rows = rows;
         a.grid[s].row_off = row_words;
-        row_words += G * G;
+        row_words += G * G + G + 1;
     }
     a.sumC = sumC;
     a.row_words = row_words;
@@ -471,7 +502,7 @@ vdm_status vdm_decode_local(const vdm_local_decoder* d, const float* d_xyz, int6
         smem += (size_t)(d->hidden * 4 + d->channels[s] * (d->hidden + 1));
     }
     a.woff[d->n_scales] = (int)smem;
-    smem += (size_t)d->fuse_hidden * (sumC + 2) + (size_t)LQ_T * (sumC + 1);
+    smem += (size_t)d->fuse_hidden * (sumC + 2) + (size_t)(LQ_T / 32) * sumC;
     smem *= 4;
     e = cudaFuncSetAttribute(local_conv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return fail(VDM_ERR_CUDA, "local_conv smem attribute: %s", cudaGetErrorString(e));
@@ -483,7 +514,8 @@ vdm_status vdm_decode_local(const vdm_local_decoder* d, const float* d_xyz, int6
         a.nbr_q0 = d_knn_out ? 0 : q0;
         const unsigned nq = (unsigned)(a.q1 - a.q0);
         knn<<<(nq + LK_T - 1) / LK_T, LK_T, ksmem, st>>>(a);
-        local_conv_kernel<<<(nq + LQ_T - 1) / LQ_T, LQ_T, smem, st>>>(a);
+        const unsigned conv_ctas = (nq + LQ_T / 32 - 1) / (LQ_T / 32);
+        local_conv_kernel<<<conv_ctas < 148u * 8u ? conv_ctas : 148u * 8u, LQ_T, smem, st>>>(a);
         VDM_TRY(check_launch("local query kernels"));
     }
     VDM_CUDA_TRY(cudaStreamSynchronize(st));

@@ -50,7 +50,7 @@ def test_local_decoder_empty_and_errors():
 
 
 def test_local_decoder_several_chunks():
-    """More queries than one chunk of the neighbour buffer (65,536), with and
+    """More queries than one chunk of the neighbour buffer (262,144), with and
     without the neighbour export: sampled rows against the oracle, and the
     two calls' SDF values identical."""
     import torch
@@ -60,14 +60,13 @@ def test_local_decoder_several_chunks():
     K = 8
     ld = vdm.LocalDecoder.from_numpy(d, K)
     rng = np.random.default_rng(7)
-    x = rng.uniform(-1.0, 1.0, (140_000, 3)).astype(np.float32)
+    x = rng.uniform(-1.0, 1.0, (300_000, 3)).astype(np.float32)
     xt = torch.from_numpy(x).cuda()
     out, knn = vdm.vdm_decode_local(ld, xt, want_knn=True)
     out2 = vdm.vdm_decode_local(ld, xt)
     out, out2, knn = out.cpu().numpy(), out2.cpu().numpy(), knn.cpu().numpy()
     assert np.array_equal(out, out2)
-    rows = np.concatenate([rng.choice(x.shape[0], 600, replace=False), [0, 65_535, 65_536, 131_071, 131_072,
-                                                                         x.shape[0] - 1]])
+    rows = np.concatenate([rng.choice(x.shape[0], 600, replace=False), [0, 262_143, 262_144, x.shape[0] - 1]])
     for s, a in enumerate(d["anchors"]):
         assert np.array_equal(knn[rows, s, :], OL.knn(x[rows], a, K)), f"scale {s}"
     want = OL.decode_local(x[rows], d["anchors"], d["feats"], d["scales"], d["fuse"], K)
