@@ -22,7 +22,10 @@
 // the query to every cell not yet visited (with a relative margin, so rounding
 // can only search one ring more), which makes the result exact.
 //
-// Two kernels per chunk of queries.  local_knn_kernel: one thread per query,
+// Per chunk of queries: a counting sort of the queries by cell of a 32^3 grid
+// (neighbouring threads then walk rings of similar size: the search cost of a
+// query grows with its distance to the anchors), then two kernels.
+// local_knn_kernel: one thread per query,
 // the neighbour list sorted in registers (fixed capacity, static indices); a
 // ring of cells is walked through occupancy words staged in shared memory (one
 // bit per occupied plane, per occupied row of a plane, per occupied cell of a
@@ -42,6 +45,7 @@ namespace {
 constexpr int LQ_T = 256;         // threads per CTA (AVS-Conv and fusion: one warp per query)
 constexpr int LK_T = 128;         // queries per CTA (neighbour search)
 constexpr int L_CHUNK = 1 << 18;  // queries per chunk (neighbour ids kept in the workspace)
+constexpr int L_QG = 32;          // cells per axis of the grid the queries are sorted by
 constexpr int L_MAXS = VDM_LOCAL_MAX_SCALES;
 constexpr int L_MAXK = 16, L_MAXH = 32, L_MAXC = 64, L_MAXSUMC = 128, L_MAXF = 64;
 
@@ -64,6 +68,7 @@ struct LocalArgs {
     ScaleGrid grid[L_MAXS];
     const float* xyz;
     int64_t q0, q1;        // this chunk's queries [q0, q1)
+    const int32_t* perm;   // the chunk's queries in cell order: thread t takes query q0 + perm[t]
     float* out;
     int32_t* nbr;          // neighbour ids of query q at nbr[(q - nbr_q0) * n_scales * K]
     int64_t nbr_q0;
@@ -203,8 +208,9 @@ __global__ void __launch_bounds__(LK_T) local_knn_kernel(const LocalArgs a) {
         r[G * G + G] = im;
     }
     __syncthreads();
-    const int64_t q = a.q0 + (int64_t)blockIdx.x * LK_T + threadIdx.x;
-    if (q >= a.q1) return;
+    const int64_t tq = (int64_t)blockIdx.x * LK_T + threadIdx.x;
+    if (tq >= a.q1 - a.q0) return;
+    const int64_t q = a.q0 + a.perm[tq];
     const float x = a.xyz[3 * q], y = a.xyz[3 * q + 1], z = a.xyz[3 * q + 2];
     const int K = a.K;
     int32_t* nout = a.nbr + (q - a.nbr_q0) * a.n_scales * K;
@@ -320,7 +326,7 @@ __global__ void __launch_bounds__(LQ_T) local_conv_kernel(const LocalArgs a) {
     const int64_t nq = a.q1 - a.q0;
     const int wpc = LQ_T / 32;
     for (int64_t qi = (int64_t)blockIdx.x * wpc + warp; qi < nq; qi += (int64_t)gridDim.x * wpc) {
-        const int64_t q = a.q0 + qi;
+        const int64_t q = a.q0 + a.perm[qi];
         const float x = a.xyz[3 * q], y = a.xyz[3 * q + 1], z = a.xyz[3 * q + 2];
         const int32_t* nin = a.nbr + (q - a.nbr_q0) * a.n_scales * K;
         for (int s = 0; s < a.n_scales; ++s) {
@@ -378,7 +384,7 @@ int grid_cells(int n) {
 }
 
 size_t local_ws_bytes(const vdm_local_decoder* d, size_t* off_cnt, size_t* off_start, size_t* off_cursor,
-                      size_t* off_ids, size_t* off_cell, size_t* off_rows, size_t* off_nbr) {
+                      size_t* off_ids, size_t* off_cell, size_t* off_rows, size_t* off_nbr, size_t* off_q) {
     size_t o = 0;
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
     for (int s = 0; s < d->n_scales; ++s) {
@@ -393,6 +399,14 @@ size_t local_ws_bytes(const vdm_local_decoder* d, size_t* off_cnt, size_t* off_s
     }
     *off_nbr = o;          // neighbour ids of one chunk of queries
     o = up(o + (size_t)L_CHUNK * d->n_scales * d->K * 4);
+    off_q[0] = o;          // query cells of a chunk
+    o = up(o + (size_t)L_CHUNK * 4);
+    off_q[1] = o;          // the chunk's order
+    o = up(o + (size_t)L_CHUNK * 4);
+    const size_t nqc = (size_t)L_QG * L_QG * L_QG;
+    off_q[2] = o; o = up(o + nqc * 4);          // counts
+    off_q[3] = o; o = up(o + (nqc + 1) * 4);    // starts
+    off_q[4] = o; o = up(o + nqc * 4);          // cursors
     return o + 256;
 }
 
@@ -430,8 +444,8 @@ extern "C" {
 vdm_status vdm_local_workspace_size(const vdm_local_decoder* d, size_t* bytes) {
     VDM_TRY(check_local(d));
     if (!bytes) return fail(VDM_ERR_INVALID_ARG, "bytes is NULL");
-    size_t a[L_MAXS], b[L_MAXS], c[L_MAXS], e[L_MAXS], f[L_MAXS], g[L_MAXS], h;
-    *bytes = local_ws_bytes(d, a, b, c, e, f, g, &h);
+    size_t a[L_MAXS], b[L_MAXS], c[L_MAXS], e[L_MAXS], f[L_MAXS], g[L_MAXS], h, qo[5];
+    *bytes = local_ws_bytes(d, a, b, c, e, f, g, &h, qo);
     return VDM_OK;
 }
 
@@ -447,8 +461,9 @@ vdm_status vdm_decode_local(const vdm_local_decoder* d, const float* d_xyz, int6
     char* ws = reinterpret_cast<char*>(((uintptr_t)d_ws + 255) & ~(uintptr_t)255);
     if ((uintptr_t)ws - (uintptr_t)d_ws + need - 256 > ws_bytes)
         return fail(VDM_ERR_WORKSPACE, "workspace too small after alignment");
-    size_t o_cnt[L_MAXS], o_start[L_MAXS], o_cur[L_MAXS], o_ids[L_MAXS], o_cell[L_MAXS], o_rows[L_MAXS], o_nbr;
-    local_ws_bytes(d, o_cnt, o_start, o_cur, o_ids, o_cell, o_rows, &o_nbr);
+    size_t o_cnt[L_MAXS], o_start[L_MAXS], o_cur[L_MAXS], o_ids[L_MAXS], o_cell[L_MAXS], o_rows[L_MAXS], o_nbr,
+        o_q[5];
+    local_ws_bytes(d, o_cnt, o_start, o_cur, o_ids, o_cell, o_rows, &o_nbr, o_q);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     LocalArgs a;
     memset(&a, 0, sizeof(a));
@@ -513,6 +528,18 @@ vdm_status vdm_decode_local(const vdm_local_decoder* d, const float* d_xyz, int6
         a.nbr = d_knn_out ? d_knn_out : reinterpret_cast<int32_t*>(ws + o_nbr);
         a.nbr_q0 = d_knn_out ? 0 : q0;
         const unsigned nq = (unsigned)(a.q1 - a.q0);
+        // sort the chunk's queries by cell: neighbouring threads then walk similar rings
+        int32_t* qcell = reinterpret_cast<int32_t*>(ws + o_q[0]);
+        int32_t* perm = reinterpret_cast<int32_t*>(ws + o_q[1]);
+        int32_t* qcnt = reinterpret_cast<int32_t*>(ws + o_q[2]);
+        int32_t* qstart = reinterpret_cast<int32_t*>(ws + o_q[3]);
+        int32_t* qcur = reinterpret_cast<int32_t*>(ws + o_q[4]);
+        const int nqc = L_QG * L_QG * L_QG;
+        VDM_CUDA_TRY(cudaMemsetAsync(qcnt, 0, (size_t)nqc * 4, st));
+        bin_count_kernel<<<(nq + 255) / 256, 256, 0, st>>>(d_xyz + 3 * q0, (int)nq, L_QG, qcnt, qcell);
+        bin_scan_kernel<<<1, 1024, 0, st>>>(qcnt, nqc, qstart, qcur);
+        bin_place_kernel<<<(nq + 255) / 256, 256, 0, st>>>(qcell, (int)nq, qcur, perm);
+        a.perm = perm;
         knn<<<(nq + LK_T - 1) / LK_T, LK_T, ksmem, st>>>(a);
         const unsigned conv_ctas = (nq + LQ_T / 32 - 1) / (LQ_T / 32);
         local_conv_kernel<<<conv_ctas < 148u * 8u ? conv_ctas : 148u * 8u, LQ_T, smem, st>>>(a);
