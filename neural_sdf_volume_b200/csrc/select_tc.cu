@@ -351,6 +351,17 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
             }
             int pb = 0;   // partial-sum buffer
             int i = 0;    // S index: key block j, head h -> i = j H + h
+            // A column of a sub-volume sums the partials of the warps that hold its rows in the
+            // column's warpgroup: one warp (32 probes) or two (64), added straight into the score
+            // row (a shared-memory atomic add of two terms onto zero gives the same value in
+            // either order), so no barrier per key block; four (128) go through the partial
+            // buffer in a fixed order.
+            const bool direct = warps_per_tile <= 2;
+            const int my_sv = (32 * (warp & 3)) / np;
+            if (direct && warps_per_tile == 2) {
+                for (int idx = tid; idx < tpu * N; idx += NCOMP) score[idx] = 0.f;
+                if (!(ok = csync(97))) break;
+            }
             for (int j = 0; j < nb && ok; ++j) {
                 const int vcols = N - j * 128 - 64 * wg;   // own columns < vcols are real tokens
                 float acc[64];
@@ -386,6 +397,18 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                 if (!ok) break;
                 float cs[2];
                 warp_colsum64(acc, lane, cs);
+                if (direct) {
+                    const int col = j * 128 + 64 * wg + 2 * lane;
+                    float* dst = score + (size_t)my_sv * N + col;
+                    if (warps_per_tile == 1) {
+                        if (col < N) dst[0] = cs[0];
+                        if (col + 1 < N) dst[1] = cs[1];
+                    } else {
+                        if (col < N) atomicAdd(dst, cs[0]);
+                        if (col + 1 < N) atomicAdd(dst + 1, cs[1]);
+                    }
+                    continue;
+                }
                 float* pw = part + (pb * 8 + warp) * 64;
                 pw[2 * lane] = cs[0];
                 pw[2 * lane + 1] = cs[1];
@@ -399,16 +422,21 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                         float sum = 0.f;
                         for (int w = 0; w < warps_per_tile; ++w) sum += pp[w * 64];
                         score[(size_t)sv * N + j * 128 + col] = sum;
-                        if (a.score_out && unit * tpu + sv < n_sel) {
-                            const int ts = a.sel_tiles[unit * tpu + sv];
-                            if (ts < a.score_rows) a.score_out[(size_t)ts * N + j * 128 + col] = sum;
-                        }
                     }
                 }
                 pb ^= 1;
             }
             if (!ok) break;
             if (!(ok = csync(89))) break;
+            if (a.score_out) {   // debug export of the unit's score rows
+                for (int idx = tid; idx < tpu * N; idx += NCOMP) {
+                    const int sv = idx / N;
+                    if (unit * tpu + sv < n_sel) {
+                        const int ts = a.sel_tiles[unit * tpu + sv];
+                        if (ts < a.score_rows) a.score_out[(size_t)ts * N + (idx - sv * N)] = score[idx];
+                    }
+                }
+            }
             // ------------------------------------------------ Top-K per sub-volume
             const int k = a.top_k;
             for (int s = 0; s < tpu && ok; ++s) {
