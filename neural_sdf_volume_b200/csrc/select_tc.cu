@@ -382,17 +382,17 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                             for (int c = 0; c < 32; ++c) acc[c0 + c] += c0 + c < vcols ? ex2(x[c] - mo) : 0.f;
                         }
                     };
-                    float s0[32];
+                    // both 32-column halves in flight at once, one wait
+                    float s0[32], s1[32];
                     tmem_ld32(sb, s0);
+                    tmem_ld32(sb + 32, s1);
                     tmem_wait_ld();
                     reg_fence(s0);
-                    accum(s0, 0);
-                    tmem_ld32(sb + 32, s0);
-                    tmem_wait_ld();
-                    reg_fence(s0);
+                    reg_fence(s1);
                     tc_fence_before();
                     arrive(&sh.bar_p[i & 1]);   // this half of S_i consumed
-                    accum(s0, 32);
+                    accum(s0, 0);
+                    accum(s1, 32);
                 }
                 if (!ok) break;
                 float cs[2];
