@@ -360,24 +360,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
     // barriers of the MMA-issuing CTA, and commits that reach both CTAs
     auto lead_bar = [&](uint64_t* b) -> uint32_t { return PAIR ? mapa(smem_u32(b), 0u) : smem_u32(b); };
     // (issued by the whole MMA warp; one elected lane commits)
-    // (single CTAs: lane 0 issues every MMA and commit, so a commit always covers the MMAs
-    // issued before it)
     auto commit_both = [&](uint64_t* b) {
         if (PAIR) {
             mma_commit_pair_w(mapa(smem_u32(b), 0u));
             mma_commit_pair_w(mapa(smem_u32(b), 1u));
         } else {
-            if (lane == 0) mma_commit(smem_u32(b));
-            __syncwarp();
+            mma_commit_w(smem_u32(b));
         }
     };
     auto commit_own = [&](uint64_t* b) {
-        if (PAIR) {
-            mma_commit_pair_w(smem_u32(b));
-        } else {
-            if (lane == 0) mma_commit(smem_u32(b));
-            __syncwarp();
-        }
+        if (PAIR) mma_commit_pair_w(smem_u32(b));
+        else mma_commit_w(smem_u32(b));
     };
     // items a unit pushes through the ring (producer, MMA and forwarder agree on it)
     auto n_items = [&](int nb) -> int {
@@ -599,20 +592,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             auto release = [&](int slot) { commit_both(&sh.empty[slot]); };
             constexpr int MR = 128 * CG;   // MMA rows
             auto mma_s = [&](uint32_t d, uint64_t da, uint64_t db, uint32_t id, uint32_t acc) {
-                if (PAIR) {
-                    mma_ss_pair_w(d, da, db, id, acc);
-                } else {
-                    if (lane == 0) mma_ss(d, da, db, id, acc);
-                    __syncwarp();
-                }
+                if (PAIR) mma_ss_pair_w(d, da, db, id, acc);
+                else mma_ss_w(d, da, db, id, acc);
             };
             auto mma_t = [&](uint32_t d, uint32_t ta_, uint64_t db, uint32_t id, uint32_t acc) {
-                if (PAIR) {
-                    mma_ts_pair_w(d, ta_, db, id, acc);
-                } else {
-                    if (lane == 0) mma_ts(d, ta_, db, id, acc);
-                    __syncwarp();
-                }
+                if (PAIR) mma_ts_pair_w(d, ta_, db, id, acc);
+                else mma_ts_w(d, ta_, db, id, acc);
             };
             int64_t n_done = 0;
             for (int64_t it = it0; it < n_iter && ok; it += it_step) {
@@ -644,19 +629,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         if (u.sel) fence_proxy_async();
                         const uint64_t da = desc_sw128(s_abuf + h * 16384), db = desc_sw128(s_ring + sl * RS);
                         const uint32_t sd = tmem + T_S0 + 128 * (j % NSB);
-                        if (!PAIR) {
-                            // one lane issues the block's MMAs and commits back to back (an elect per
-                            // instruction cost the issuing warp more than the tensor time of a block)
-                            if (lane == 0) {
-                                #pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    mma_ss(sd, da + 2 * kk, db + 2 * kk, idesc_bf16(MR, 128, false), kk > 0);
-                                mma_commit(smem_u32(&sh.empty[sl]));
-                                mma_commit(smem_u32(&sh.bar_s[j % 6]));
-                            }
-                            __syncwarp();
-                            return true;
-                        }
                         #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             mma_s(sd, da + 2 * kk, db + 2 * kk, idesc_bf16(MR, 128, false), kk > 0);
@@ -677,29 +649,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         const uint64_t dv = PAIR ? desc_sw64(s_ring + slot * RS) : desc_sw128(s_ring + slot * RS);
                         constexpr int vstep = PAIR ? 64 : 128;
                         const uint32_t pa = tmem + T_S0 + 128 * (j % NSB);
-                        if (!PAIR) {
-                            if (lane == 0) {
-                                #pragma unroll
-                                for (int kk = 0; kk < 8; ++kk)
-                                    mma_ts(tmem + (g ? T_O1 : T_O0), pa + 32 * (kk >> 1) + 8 * (kk & 1), dv + vstep * kk,
-                                           idesc_bf16(MR, 64, true), (j >= 2 || kk > 0));
-                                mma_commit(smem_u32(&sh.empty[slot]));
-                                if (j + 2 < nb) mma_commit(smem_u32(&sh.bar_pvg[g]));
-                                if (j + NSB < nb) mma_commit(smem_u32(&sh.bar_pvm));
-                            }
-                            __syncwarp();
-                        } else {
-                            #pragma unroll
-                            for (int kk = 0; kk < 8; ++kk)
-                                mma_t(tmem + (g ? T_O1 : T_O0), pa + 32 * (kk >> 1) + 8 * (kk & 1), dv + vstep * kk,
-                                      idesc_bf16(MR, 64, true), (j >= 2 || kk > 0));
-                            release(slot);
-                            // O_g is final for this block once the PV is done (the owner waits before its next)
-                            if (j + 2 < nb) commit_both(&sh.bar_pvg[g]);
-                            if (j + NSB < nb) commit_own(&sh.bar_pvm);
-                        }
+                        #pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_t(tmem + (g ? T_O1 : T_O0), pa + 32 * (kk >> 1) + 8 * (kk & 1), dv + vstep * kk,
+                                  idesc_bf16(MR, 64, true), (j >= 2 || kk > 0));
+                        release(slot);
+                        // O_g is final for this block once the PV is done (the owner waits before its next)
+                        if (j + 2 < nb) commit_both(&sh.bar_pvg[g]);
                         if (j + NSB < nb) {
                             // S_{j+3} overwrites the columns this PV reads: let the PV finish first
+                            commit_own(&sh.bar_pvm);
                             if (!(ok = W.wait(&sh.bar_pvm, ph_pvm, 66))) break;
                             tc_fence_after();
                             ok = issue_s(j + NSB);
