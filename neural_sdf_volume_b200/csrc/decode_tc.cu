@@ -7,7 +7,7 @@
 // One persistent CTA per SM decodes 128-query tiles; nothing but the final
 // SDF value (and, for probe queries, their softmax statistics) leaves the SM.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads; 320 for CTA pairs):
 //   warps 0-7  compute: two warpgroups; thread (g, r) owns TMEM lane r and
 //              half g of the row's columns (head dims, hidden units, LayerNorm
 //              columns), so every SM sub-partition runs two compute warps; in
@@ -18,6 +18,10 @@
 //   warp 9     producer: TMA loads of weights and of contiguous K/V blocks,
 //              cp.async gathers of a sub-volume's selected K/V rows (each lane's
 //              copies arrive on the slot's barrier when they land);
+//   warp 10    (single CTAs) the attention's P V MMAs, from a ring of values of
+//              their own, so that block j's P V and the S of block j+3 (which
+//              waits for that P V to have read P_j) are issued by different
+//              warps and the issue chain of one block no longer holds the next;
 // connected only by mbarriers (no CTA-wide barrier inside a tile).
 // Compiled twice per width: one CTA per 128-row MMA, or (cta_group::2) a CTA
 // pair of a cluster per 256-row MMA, each CTA holding half of every B tile.
@@ -74,8 +78,9 @@ using namespace ptx;
 
 constexpr int BM = 128;        // queries per tile (TMEM lanes)
 constexpr int NCOMP = 256;     // compute threads (two warpgroups)
-constexpr int NT = 320;        // + MMA warp + producer warp
-constexpr int WARP_MMA = 8, WARP_PROD = 9;
+constexpr int NT = 320;        // + MMA warp + producer warp (CTA pairs)
+constexpr int NT_SPLIT = 352;  // single CTAs: + a second MMA-issue warp for the P V products
+constexpr int WARP_MMA = 8, WARP_PROD = 9, WARP_PV = 10;
 constexpr int SLOT = 16384;    // ring slot bytes
 constexpr int MAX_NS = 16;   // ring slots (CTA pairs use twice as many, half as large)
 constexpr int RING_ARRIVALS = 32;   // arrivals completing a ring slot: one per producer lane
@@ -111,7 +116,9 @@ struct Shared {
     uint64_t full[MAX_NS], empty[MAX_NS];
     // MMA commits (count 1); bar_hd and bar_w2 are waited on by the MMA warp only
     // bar_s[j mod 6]: S_j ready (block j's buffer and owner both follow from j mod 6)
-    uint64_t bar_q, bar_s[6], bar_pvg[2], bar_pvm, bar_pv, bar_x, bar_h[2], bar_acc, bar_hd, bar_w2, bar_fin;
+    // bar_pvm[e mod 3]: the e-th P V product that an S issue waits for is complete
+    uint64_t bar_q, bar_s[6], bar_pvg[2], bar_pvm[3], bar_pv, bar_x, bar_h[2], bar_acc, bar_hd, bar_w2, bar_fin,
+        bar_fin2;
     // compute-warp arrivals (count 128)
     uint64_t bar_pe, bar_qc, bar_p[2], bar_a, bar_hin, bar_r, bar_g[2], bar_cs, bar_wg;
     uint32_t tmem_base;
@@ -227,7 +234,7 @@ __device__ __forceinline__ Unit unit_of(const DecodeArgs& a, int64_t unit) {
 
 // ---------------------------------------------------------------- the kernel
 template <int CC, int CG>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(CG == 2 ? NT : NT_SPLIT, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_wq64,
                  const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_w1,
                  const __grid_constant__ CUtensorMap tm_w2, const __grid_constant__ CUtensorMap tm_k,
@@ -261,6 +268,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
     // carries two consecutive 64-wide K atoms (8 MMA k-steps per wait and release)
     constexpr int RS = SLOT;
     constexpr int NR = NS;
+    // Single CTAs split the MMA issue over two warps: the P V products of the attention run on
+    // WARP_PV, everything else on WARP_MMA, so a block's P V and the S of a later block are issued
+    // side by side.  The values then travel in a ring of their own (slots NRA..NR-1, consumed by
+    // WARP_PV), the other items in slots 0..NRA-1 (consumed by WARP_MMA); each ring has one
+    // producer and one consumer in FIFO order.
+    constexpr bool SPLIT = !PAIR;
+    constexpr int NRB = SPLIT ? 2 : 0;
+    constexpr int NRA = NR - NRB;
+    static_assert(NRA >= 2, "ring too small");
     constexpr int AT = PAIR ? 2 : 1;      // K atoms per weight item
     constexpr int KA = NA + 1;            // output-projection K atoms: embedding + attention
 
@@ -280,8 +296,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             mbar_init(smem_u32(&sh.empty[i]), 1);
         }
         uint64_t* one[] = {&sh.bar_q, &sh.bar_s[0], &sh.bar_s[1], &sh.bar_s[2], &sh.bar_s[3], &sh.bar_s[4],
-                           &sh.bar_s[5], &sh.bar_pvg[0], &sh.bar_pvg[1], &sh.bar_pvm, &sh.bar_pv, &sh.bar_x,
-                           &sh.bar_h[0], &sh.bar_h[1], &sh.bar_acc, &sh.bar_hd, &sh.bar_w2, &sh.bar_fin};
+                           &sh.bar_s[5], &sh.bar_pvg[0], &sh.bar_pvg[1], &sh.bar_pvm[0], &sh.bar_pvm[1],
+                           &sh.bar_pvm[2], &sh.bar_pv, &sh.bar_x, &sh.bar_h[0], &sh.bar_h[1], &sh.bar_acc,
+                           &sh.bar_hd, &sh.bar_w2, &sh.bar_fin, &sh.bar_fin2};
         for (auto* b : one) mbar_init(smem_u32(b), 1);
         // compute -> MMA: one arrival per compute thread, or per compute warp of both CTAs
         uint64_t* to_mma[] = {&sh.bar_pe, &sh.bar_qc, &sh.bar_a,
@@ -380,28 +397,44 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
 
     // ==================================================================== producer
     if (warp == WARP_PROD) {
-        uint32_t ring_head = 0;
+        uint32_t head_a = 0, head_b = 0;   // items pushed into each ring
         const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.K);
         const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.V);
         bool ok = true;
-        int p_slot = 0;
-        uint32_t p_ph = 1;   // parity of the empty-phase a reused slot waits for (first pass: none)
-        auto take_slot = [&](int& slot) -> bool {
-            slot = p_slot;
-            if (ring_head >= (uint32_t)NR) {
-                uint32_t ph = p_ph;
+        int pa_slot = 0, pb_slot = 0;
+        uint32_t pa_ph = 1, pb_ph = 1;   // parity of the empty-phase a reused slot waits for (first pass: none)
+        // ring B (values, single CTAs) when `vring`, else ring A
+        auto take_slot = [&](int& slot, bool vring) -> bool {
+            if constexpr (NRB > 0) {
+                if (vring) {
+                    slot = NRA + pb_slot;
+                    if (head_b >= (uint32_t)NRB) {
+                        uint32_t ph = pb_ph;
+                        if (!W.wait(&sh.empty[slot], ph, 41)) return false;
+                    }
+                    ++head_b;
+                    if (++pb_slot == NRB) {
+                        pb_slot = 0;
+                        pb_ph ^= 1;
+                    }
+                    return true;
+                }
+            }
+            slot = pa_slot;
+            if (head_a >= (uint32_t)NRA) {
+                uint32_t ph = pa_ph;
                 if (!W.wait(&sh.empty[slot], ph, 40)) return false;
             }
-            ++ring_head;
-            if (++p_slot == NR) {
-                p_slot = 0;
-                p_ph ^= 1;
+            ++head_a;
+            if (++pa_slot == NRA) {
+                pa_slot = 0;
+                pa_ph ^= 1;
             }
             return true;
         };
-        auto push_tma = [&](const CUtensorMap* m, int x, int y, uint32_t bytes) -> bool {
+        auto push_tma = [&](const CUtensorMap* m, int x, int y, uint32_t bytes, bool vring = false) -> bool {
             int slot;
-            if (!take_slot(slot)) return false;
+            if (!take_slot(slot, vring)) return false;
             if (lane == 0) {
                 const uint32_t fb = smem_u32(&sh.full[slot]);
                 mbar_expect_tx_only(fb, bytes);
@@ -415,7 +448,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
         auto push_tma2 = [&](const CUtensorMap* m0, int x0, int y0, const CUtensorMap* m1, int x1, int y1,
                              uint32_t bytes, int nbox) -> bool {
             int slot;
-            if (!take_slot(slot)) return false;
+            if (!take_slot(slot, false)) return false;
             if (lane == 0) {
                 const uint32_t fb = smem_u32(&sh.full[slot]);
                 mbar_expect_tx_only(fb, bytes * nbox);
@@ -429,7 +462,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
         auto push_gather = [&](bool isv, const __nv_bfloat16* src, const int32_t* sel, int h, int j,
                                int nk) -> bool {
             int slot;
-            if (!take_slot(slot)) return false;
+            if (!take_slot(slot, SPLIT && isv)) return false;
             const uint32_t dst = s_ring + slot * RS;
             if (!PAIR) {
                 // 128 rows x 8 chunks of 16 B: lane l copies chunk l % 8 of rows 4i + l / 8; the
@@ -491,7 +524,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             const int nb = (nk + 127) / 128;
             auto push_kv = [&](bool isv, int h, int j) -> bool {
                 if (u.sel) return push_gather(isv, isv ? Vg : Kg, u.sel, h, j, nk);
-                if (isv) return push_tma(&tm_v, PAIR ? 32 * (int)crank : 0, h * N + j * 128, PAIR ? 8192 : SLOT);
+                if (isv) return push_tma(&tm_v, PAIR ? 32 * (int)crank : 0, h * N + j * 128, PAIR ? 8192 : SLOT, SPLIT);
                 return push_tma(&tm_k, 0, h * N + j * 128 + rb, BR * 128);
             };
             for (int h = 0; h < H && ok; ++h) {
@@ -535,8 +568,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
         // complete; consumed or not, the last use of each slot is awaited;
         // in the even CTA of a pair that includes the odd CTA's forwarded half)
         if (lane == 0) {
-            const uint32_t first = ring_head > (uint32_t)NR ? ring_head - NR : 0;
-            for (uint32_t i = first; i < ring_head; ++i) drain_wait(smem_u32(&sh.full[i % NR]), (i / NR) & 1, ta.timeout);
+            const uint32_t first = head_a > (uint32_t)NRA ? head_a - NRA : 0;
+            for (uint32_t i = first; i < head_a; ++i) drain_wait(smem_u32(&sh.full[i % NRA]), (i / NRA) & 1, ta.timeout);
+            if constexpr (NRB > 0) {
+                const uint32_t fb = head_b > (uint32_t)NRB ? head_b - NRB : 0;
+                for (uint32_t i = fb; i < head_b; ++i)
+                    drain_wait(smem_u32(&sh.full[NRA + i % NRB]), (i / NRB) & 1, ta.timeout);
+            }
         }
         __syncwarp();
     }
@@ -573,7 +611,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             W.cluster_acq = PAIR;
             uint32_t ring_tail = 0;
             uint32_t ph_pe = 0, ph_qc = 0, ph_p[2] = {0, 0}, ph_a = 0, ph_hin = 0, ph_r = 0, ph_g[2] = {0, 0};
-            uint32_t ph_hd = 0, ph_w2 = 0, ph_pvm = 0;
+            uint32_t ph_hd = 0, ph_w2 = 0, ph_pvm = 0 /* bit k: phase of bar_pvm[k] (bit 0 alone: pairs) */;
+            int ev_pvm = 0;   // P V completions awaited so far (single CTAs)
             bool ok = true;
             int c_slot = 0;
             uint32_t c_ph = 0;
@@ -583,7 +622,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 if (!W.wait(&sh.full[slot], ph, 50)) return false;
                 tc_fence_after();
                 ++ring_tail;
-                if (++c_slot == NR) {
+                if (++c_slot == NRA) {
                     c_slot = 0;
                     c_ph ^= 1;
                 }
@@ -637,6 +676,22 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         return true;
                     };
                     for (int j = 0; j < nb && j < NSB && ok; ++j) ok = issue_s(j);
+                    if constexpr (SPLIT) {
+                        // S_{j+3} overwrites the columns P V_j reads (issued by WARP_PV): wait for it
+                        for (int j = 0; j + NSB < nb && ok; ++j) {
+                            const int e = ev_pvm % 3;
+                            uint32_t ph = (ph_pvm >> e) & 1u;
+                            if (!(ok = W.wait(&sh.bar_pvm[e], ph, 66))) break;
+                            ph_pvm ^= 1u << e;
+                            ++ev_pvm;
+                            tc_fence_after();
+                            ok = issue_s(j + NSB);
+                        }
+                        if (!ok) break;
+                        // the next head's Q projection accumulates in S2, which this head's P V read
+                        if (!(ok = W.wait(&sh.bar_hd, ph_hd, 54))) break;
+                        tc_fence_after();
+                    } else {
                     for (int j = 0; j < nb && ok; ++j) {
                         const int g = j & 1;   // block j belongs to warpgroup j mod 2
                         if (!(ok = W.wait(&sh.bar_p[g], ph_p[g], 53))) break;
@@ -658,8 +713,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         if (j + 2 < nb) commit_both(&sh.bar_pvg[g]);
                         if (j + NSB < nb) {
                             // S_{j+3} overwrites the columns this PV reads: let the PV finish first
-                            commit_own(&sh.bar_pvm);
-                            if (!(ok = W.wait(&sh.bar_pvm, ph_pvm, 66))) break;
+                            commit_own(&sh.bar_pvm[0]);
+                            if (!(ok = W.wait(&sh.bar_pvm[0], ph_pvm, 66))) break;
                             tc_fence_after();
                             ok = issue_s(j + NSB);
                         }
@@ -670,6 +725,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     commit_own(&sh.bar_hd);
                     if (!(ok = W.wait(&sh.bar_hd, ph_hd, 54))) break;
                     tc_fence_after();
+                    }
                 }
                 if (!ok) break;
                 // ---- X = PE Wq^T + a Wo^T
@@ -760,6 +816,63 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             commit_own(&sh.bar_fin);
             drain_wait(smem_u32(&sh.bar_fin), 0, ta.timeout);
         }
+    }
+    // ==================================================================== P V issue (single CTAs)
+    else if (SPLIT && warp == WARP_PV) {
+      if constexpr (SPLIT) {
+        // O_g += P_j V_j for every block: P_j from its warpgroup, V_j from the value ring
+        uint32_t ph_p[2] = {0, 0};
+        int v_slot = 0;
+        uint32_t v_ph = 0;
+        int ev = 0;   // completions the S issue waits for (bar_pvm[ev mod 3])
+        bool ok = true;
+        for (int64_t it = it0; it < n_iter && ok; it += it_step) {
+            if (!active(it)) continue;
+            const Unit u = unit_at(it, crank);
+            const int nk = u.sel ? a.ksel : N;
+            const int nb = (nk + 127) / 128;
+            for (int h = 0; h < H && ok; ++h) {
+                for (int j = 0; j < nb && ok; ++j) {
+                    const int g = j & 1;   // block j belongs to warpgroup j mod 2
+                    if (!(ok = W.wait(&sh.bar_p[g], ph_p[g], 53))) break;
+                    tc_fence_after();
+                    const int slot = NRA + v_slot;
+                    {
+                        uint32_t ph = v_ph;
+                        if (!(ok = W.wait(&sh.full[slot], ph, 91))) break;
+                    }
+                    tc_fence_after();
+                    if (++v_slot == NRB) {
+                        v_slot = 0;
+                        v_ph ^= 1;
+                    }
+                    // gathered rows were written by cp.async (generic proxy): order them before the MMA's reads
+                    if (u.sel) fence_proxy_async();
+                    // P_j is read in place: the bf16 pairs of tokens [32i, 32i+32) occupy columns
+                    // [32i, 32i+16) of its S buffer; V is N-major, 16 tokens (rows of 128 B) per k-step
+                    const uint64_t dv = desc_sw128(s_ring + slot * RS);
+                    const uint32_t pa = tmem + T_S0 + 128 * (j % NSB);
+                    #pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts_w(tmem + (g ? T_O1 : T_O0), pa + 32 * (kk >> 1) + 8 * (kk & 1), dv + 128 * kk,
+                                 idesc_bf16(128, 64, true), (j >= 2 || kk > 0));
+                    mma_commit_w(smem_u32(&sh.empty[slot]));
+                    // O_g is final for this block once the P V is done (the owner waits before its next)
+                    if (j + 2 < nb) mma_commit_w(smem_u32(&sh.bar_pvg[g]));
+                    if (j + NSB < nb) {
+                        mma_commit_w(smem_u32(&sh.bar_pvm[ev % 3]));
+                        ++ev;
+                    }
+                }
+                if (!ok) break;
+                mma_commit_w(smem_u32(&sh.bar_pv));   // the head's P V are complete: O0 and O1 final
+                mma_commit_w(smem_u32(&sh.bar_hd));   // and S2 is free for the next head's Q projection
+            }
+        }
+        // nothing of ours may run on the tensor cores once TMEM is released
+        mma_commit_w(smem_u32(&sh.bar_fin2));
+        drain_wait(smem_u32(&sh.bar_fin2), 0, ta.timeout);
+      }
     }
     // ==================================================================== compute warps
     else {
@@ -1382,7 +1495,7 @@ vdm_status launch_decode_tc(const DecodeArgs& d, cudaStream_t st) {
     const unsigned grid = (unsigned)(per * (n_iter < groups ? n_iter : groups));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(NT);
+    cfg.blockDim = dim3(pair ? NT : NT_SPLIT);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
