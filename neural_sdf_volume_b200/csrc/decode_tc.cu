@@ -355,13 +355,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
     // Work: units of 128 queries; a CTA pair takes two units that attend to the same keys
     // (consecutive flat units, or two slots of one sub-volume) and skips a pair only when
     // both are empty.
-    const int64_t n_units = a.work == kWorkFlat ? (a.M + BM - 1) / BM : (int64_t)a.T * a.slots;
+    // single CTAs in the sparse pass take the non-empty units from a list (equal shares per CTA)
+    const bool listed = !PAIR && a.work == kWorkTileSparse && a.unit_list != nullptr;
+    const int64_t n_units = a.work == kWorkFlat ? (a.M + BM - 1) / BM
+                            : listed             ? (int64_t)*a.n_units_dev
+                                                 : (int64_t)a.T * a.slots;
     const int spt = PAIR ? (a.slots + 1) / 2 : a.slots;   // slot pairs per sub-volume
     const int64_t n_iter = !PAIR ? n_units : a.work == kWorkFlat ? (n_units + 1) / 2 : (int64_t)a.T * spt;
     const int64_t it0 = PAIR ? blockIdx.x / 2 : blockIdx.x;
     const int64_t it_step = PAIR ? gridDim.x / 2 : gridDim.x;
     auto unit_at = [&](int64_t it, uint32_t r) -> Unit {
-        if (!PAIR) return unit_of(a, it);
+        if (!PAIR) return unit_of(a, listed ? (int64_t)a.unit_list[it] : it);
         if (a.work == kWorkFlat) return unit_of(a, 2 * it + r);
         const int64_t t = it % a.T;
         const int sl = 2 * (int)(it / a.T) + (int)r;

@@ -110,7 +110,7 @@ struct Plan {
     size_t off_grid[VDM_MAX_LEVELS];
     size_t off_tgrid[VDM_MAX_LEVELS];   // tSDF grids of levels 0 .. L-2 (decoders with a tSDF head)
     size_t off_words, off_bits, off_word_off, off_tile_ids, off_tile_off, off_counts, off_scan, off_plist,
-        off_qorder, off_sel, off_seltiles, off_ml, off_dense, off_dense_ml;
+        off_qorder, off_sel, off_seltiles, off_ml, off_dense, off_dense_ml, off_units, off_units_n;
     int nw_max;
     int k;
     size_t ml_bytes;
@@ -168,6 +168,9 @@ vdm_status make_plan(const vdm_hier_params* p, int N, int ml_heads, bool tsdf, P
     const size_t dense_max = p->adaptive ? (size_t)nw_max * (p->n_probe < 512 ? p->n_probe : 512) : 0;
     pl.off_dense = o;     o = align_up(o + dense_max * 4);
     pl.off_dense_ml = o;  o = align_up(o + dense_max * 4);
+    // the sparse pass's non-empty (sub-volume, slot) units: at most 512 / 128 slots per sub-volume
+    pl.off_units = o;     o = align_up(o + (p->adaptive ? (size_t)nw_max * 4 * 4 : 0));
+    pl.off_units_n = o;   o = align_up(o + 4);
     pl.total = o + 256;
     return VDM_OK;
 }
@@ -681,6 +684,11 @@ vdm_status vdm_decode_hierarchical(const vdm_decoder* dec, const void* d_k, cons
                 a.work = kWorkTileSparse;
                 a.sel = sel;
                 a.ksel = pl.k;
+                int32_t* units = at<int32_t>(ws, pl.off_units);
+                int32_t* units_n = at<int32_t>(ws, pl.off_units_n);
+                VDM_TRY(launch_sparse_units(tile_off, T, p->n_probe, kTcTile, units, units_n, st));
+                a.unit_list = units;
+                a.n_units_dev = units_n;
                 VDM_TRY(launch_decode(a, dec->dtype, st));
             }
             if (dbg && dbg->tile_ids[l + 1] && dbg->max_tiles > 0) {

@@ -75,6 +75,8 @@ struct DecodeArgs {
     int slots;                  // chunks per tile
     const int32_t* sel;         // [T][ksel]
     int ksel;
+    const int32_t* unit_list;   // kWorkTileSparse, single CTAs: the non-empty units (slot * T + tile) or NULL
+    const int32_t* n_units_dev; //   and their number (device)
     // outputs
     float* probe_ml;            // kWorkTileDense: per (tile, probe, head) softmax max and sum (log2 units) or NULL
     float* out;                 // out[q] (flat work only) or NULL
@@ -203,6 +205,9 @@ vdm_status launch_fill(const float* f_coarse, int R, float* f_fine, cudaStream_t
 vdm_status launch_probe_export(const int32_t* tile_off, int n_tiles, const int32_t* plist,
                                const int32_t* qorder, int R2, int n_probe, int32_t* out,
                                cudaStream_t s);
+// the sparse pass's non-empty (sub-volume, slot) units, `tile_q` queries per slot
+vdm_status launch_sparse_units(const int32_t* tile_off, int T, int n_probe, int tile_q, int32_t* list,
+                               int32_t* n_units, cudaStream_t s);
 vdm_status launch_probe_order(const int32_t* tile_off, int n_tiles, const int32_t* plist, int R2,
                               int n_probe, uint64_t salt, int32_t* qorder, int32_t* counters,
                               int32_t* sel_tiles, int32_t* dense_q, int32_t* dense_ml, cudaStream_t s);

@@ -574,6 +574,31 @@ vdm_status launch_fill(const float* f_coarse, int R, float* f_fine, cudaStream_t
     return check_launch("fill_kernel");
 }
 
+// The sparse pass's work units: unit (sub-volume t, slot s) for every slot that holds queries
+// (the queries after the first n_probe, 128 per slot), as s * T + t.  The units of a sub-volume
+// differ in number, so a static share of all T * slots (unit, slot) pairs per persistent CTA
+// gives the CTAs unequal work; a list of the non-empty units shares them evenly.  The order of
+// the list does not matter (units are independent).
+__global__ void sparse_units_kernel(const int32_t* __restrict__ tile_off, int T, int n_probe, int tile_q,
+                                    int32_t* __restrict__ list, int32_t* __restrict__ n_units) {
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= T) return;
+    const int cnt = 8 * (tile_off[t + 1] - tile_off[t]);
+    const int n = cnt > n_probe ? cnt - n_probe : 0;
+    const int units = (n + tile_q - 1) / tile_q;
+    if (units == 0) return;
+    const int base = atomicAdd(n_units, units);
+    for (int sl = 0; sl < units; ++sl) list[base + sl] = sl * T + t;
+}
+
+vdm_status launch_sparse_units(const int32_t* tile_off, int T, int n_probe, int tile_q, int32_t* list,
+                               int32_t* n_units, cudaStream_t s) {
+    VDM_CUDA_TRY(cudaMemsetAsync(n_units, 0, sizeof(int32_t), s));
+    if (T <= 0) return VDM_OK;
+    sparse_units_kernel<<<(T + 255) / 256, 256, 0, s>>>(tile_off, T, n_probe, tile_q, list, n_units);
+    return check_launch("sparse_units_kernel");
+}
+
 vdm_status launch_probe_order(const int32_t* tile_off, int n_tiles, const int32_t* plist, int R2,
                               int n_probe, uint64_t salt, int32_t* qorder, int32_t* counters,
                               int32_t* sel_tiles, int32_t* dense_q, int32_t* dense_ml, cudaStream_t s) {
