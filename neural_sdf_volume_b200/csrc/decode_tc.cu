@@ -7,7 +7,7 @@
 // One persistent CTA per SM decodes 128-query tiles; nothing but the final
 // SDF value (and, for probe queries, their softmax statistics) leaves the SM.
 //
-// Warp roles (352 threads; 320 for CTA pairs):
+// Warp roles (384 threads; 320 for CTA pairs):
 //   warps 0-7  compute: two warpgroups; thread (g, r) owns TMEM lane r and
 //              half g of the row's columns (head dims, hidden units, LayerNorm
 //              columns), so every SM sub-partition runs two compute warps; in
@@ -22,6 +22,8 @@
 //              their own, so that block j's P V and the S of block j+3 (which
 //              waits for that P V to have read P_j) are issued by different
 //              warps and the issue chain of one block no longer holds the next;
+//   warp 11    (single CTAs) the values' producer (TMA or gathers), so that the
+//              value ring refills without waiting behind the other ring;
 // connected only by mbarriers (no CTA-wide barrier inside a tile).
 // Compiled twice per width: one CTA per 128-row MMA, or (cta_group::2) a CTA
 // pair of a cluster per 256-row MMA, each CTA holding half of every B tile.
@@ -79,8 +81,8 @@ using namespace ptx;
 constexpr int BM = 128;        // queries per tile (TMEM lanes)
 constexpr int NCOMP = 256;     // compute threads (two warpgroups)
 constexpr int NT = 320;        // + MMA warp + producer warp (CTA pairs)
-constexpr int NT_SPLIT = 352;  // single CTAs: + a second MMA-issue warp for the P V products
-constexpr int WARP_MMA = 8, WARP_PROD = 9, WARP_PV = 10;
+constexpr int NT_SPLIT = 384;  // single CTAs: + a P V issue warp and a value producer warp
+constexpr int WARP_MMA = 8, WARP_PROD = 9, WARP_PV = 10, WARP_VPROD = 11;
 constexpr int SLOT = 16384;    // ring slot bytes
 constexpr int MAX_NS = 16;   // ring slots (CTA pairs use twice as many, half as large)
 constexpr int RING_ARRIVALS = 32;   // arrivals completing a ring slot: one per producer lane
@@ -400,7 +402,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
     };
 
     // ==================================================================== producer
-    if (warp == WARP_PROD) {
+    if (warp == WARP_PROD || (SPLIT && warp == WARP_VPROD)) {
+        // single CTAs: WARP_PROD fills ring A (weights, keys), WARP_VPROD ring B (values)
+        const bool vprod = SPLIT && warp == WARP_VPROD;
         uint32_t head_a = 0, head_b = 0;   // items pushed into each ring
         const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.K);
         const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.V);
@@ -532,13 +536,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 return push_tma(&tm_k, 0, h * N + j * 128 + rb, BR * 128);
             };
             for (int h = 0; h < H && ok; ++h) {
-                ok = push_tma(&tm_wq64, 0, h * 64 + (PAIR ? 32 * (int)crank : 0), PAIR ? 32 * 128 : 64 * 128);
-                for (int j = 0; j < nb && j < NSB && ok; ++j) ok = push_kv(false, h, j);
+                if (!vprod) {
+                    ok = push_tma(&tm_wq64, 0, h * 64 + (PAIR ? 32 * (int)crank : 0), PAIR ? 32 * 128 : 64 * 128);
+                    for (int j = 0; j < nb && j < NSB && ok; ++j) ok = push_kv(false, h, j);
+                }
                 for (int j = 0; j < nb && ok; ++j) {
-                    ok = push_kv(true, h, j);
-                    if (j + NSB < nb) ok = ok && push_kv(false, h, j + NSB);
+                    if (vprod || !SPLIT) ok = push_kv(true, h, j);
+                    if (!vprod && j + NSB < nb) ok = ok && push_kv(false, h, j + NSB);
                 }
             }
+            if (vprod) continue;   // the value producer has no weight items
             // X = PE Wq^T + a Wo^T : items of AT K atoms (atom 0: Wq, atom ka > 0: Wo columns ka-1)
             for (int nc = 0; nc < C / 128 && ok; ++nc)
                 for (int ka = 0; ka < KA && ok; ka += AT) {
