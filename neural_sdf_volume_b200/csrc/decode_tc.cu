@@ -122,7 +122,8 @@ struct Shared {
     uint64_t bar_q, bar_s[6], bar_pvg[2], bar_pvm[3], bar_pv, bar_x, bar_h[2], bar_acc, bar_hd, bar_w2, bar_fin,
         bar_fin2;
     // compute-warp arrivals (count 128)
-    uint64_t bar_pe, bar_qc, bar_p[2], bar_a, bar_hin, bar_r, bar_g[2], bar_cs, bar_wg;
+    // bar_cmb (single CTAs): a head's combine has read O0 and O1 (the next head's first P V may overwrite them)
+    uint64_t bar_pe, bar_qc, bar_p[2], bar_a, bar_hin, bar_r, bar_g[2], bar_cs, bar_wg, bar_cmb;
     uint32_t tmem_base;
     int abort;
     float G, Bc;     // SDF head folded with LN2's affine: sum w g, sum w b + b_head
@@ -310,6 +311,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
         for (auto* b : {&sh.bar_p[0], &sh.bar_p[1]}) mbar_init(smem_u32(b), PAIR ? 2 * (BM / 32) : BM);
         mbar_init(smem_u32(&sh.bar_cs), NCOMP);
         mbar_init(smem_u32(&sh.bar_wg), NCOMP);
+        mbar_init(smem_u32(&sh.bar_cmb), NCOMP);
         sh.abort = 0;
         fence_mbar_init();
         fence_proxy_async();
@@ -535,14 +537,26 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 if (isv) return push_tma(&tm_v, PAIR ? 32 * (int)crank : 0, h * N + j * 128, PAIR ? 8192 : SLOT, SPLIT);
                 return push_tma(&tm_k, 0, h * N + j * 128 + rb, BR * 128);
             };
-            for (int h = 0; h < H && ok; ++h) {
+            if constexpr (SPLIT) {
+                // blocks b = h nb + j of all heads in one stream: the Q projection of every head first
+                // (C/128 items of Wq rows), keys three blocks ahead of their values
+                const int nbt = H * nb;
                 if (!vprod) {
+                    for (int i = 0; i < C / 128 && ok; ++i) ok = push_tma(&tm_wq, 0, i * 128, 128 * 128);
+                    for (int b = 0; b < nbt && b < NSB && ok; ++b) ok = push_kv(false, b / nb, b % nb);
+                }
+                for (int b = 0; b < nbt && ok; ++b) {
+                    if (vprod) ok = push_kv(true, b / nb, b % nb);
+                    else if (b + NSB < nbt) ok = push_kv(false, (b + NSB) / nb, (b + NSB) % nb);
+                }
+            } else {
+                for (int h = 0; h < H && ok; ++h) {
                     ok = push_tma(&tm_wq64, 0, h * 64 + (PAIR ? 32 * (int)crank : 0), PAIR ? 32 * 128 : 64 * 128);
                     for (int j = 0; j < nb && j < NSB && ok; ++j) ok = push_kv(false, h, j);
-                }
-                for (int j = 0; j < nb && ok; ++j) {
-                    if (vprod || !SPLIT) ok = push_kv(true, h, j);
-                    if (!vprod && j + NSB < nb) ok = ok && push_kv(false, h, j + NSB);
+                    for (int j = 0; j < nb && ok; ++j) {
+                        ok = push_kv(true, h, j);
+                        if (j + NSB < nb) ok = ok && push_kv(false, h, j + NSB);
+                    }
                 }
             }
             if (vprod) continue;   // the value producer has no weight items
@@ -658,6 +672,53 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 const int nb = (nk + 127) / 128;
                 if (!(ok = W.wait(&sh.bar_pe, ph_pe, 51))) break;
                 tc_fence_after();
+                if constexpr (SPLIT) {
+                    // Q of every head first: PE Wq^T in C/128 items of 128 output rows, into TMEM [0, C)
+                    for (int i = 0; i < C / 128 && ok; ++i) {
+                        int slot;
+                        if (!(ok = consume(slot))) break;
+                        const uint64_t da = desc_sw128(s_pe), db = desc_sw128(s_ring + slot * RS);
+                        #pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_s(tmem + 128 * i, da + 2 * kk, db + 2 * kk, idesc_bf16(MR, 128, false), kk > 0);
+                        release(slot);
+                    }
+                    if (!ok) break;
+                    if (!(ta.inject && first_unit)) commit_both(&sh.bar_q);
+                    // every head's packed Q is in shared memory (and the accumulators are read)
+                    if (!(ok = W.wait(&sh.bar_qc, ph_qc, 52))) break;
+                    tc_fence_after();
+                    // then the blocks b = h nb + j of all heads as one stream: S_b into buffer b mod 3,
+                    // signalled on bar_s[(b mod 3) * 2 + j mod 2] (one waiting warpgroup per barrier);
+                    // S_{b+3} waits for P V_b, which reads P_b from the same columns
+                    const int nbt = H * nb;
+                    auto issue_sb = [&](int b) -> bool {
+                        const int h = b / nb, j = b - h * nb;
+                        int sl;
+                        if (!consume(sl)) return false;
+                        // gathered rows were written by cp.async (generic proxy): order them before the MMA's reads
+                        if (u.sel) fence_proxy_async();
+                        const uint64_t da = desc_sw128(s_abuf + h * 16384), db = desc_sw128(s_ring + sl * RS);
+                        const uint32_t sd = tmem + T_S0 + 128 * (b % NSB);
+                        #pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_s(sd, da + 2 * kk, db + 2 * kk, idesc_bf16(MR, 128, false), kk > 0);
+                        release(sl);
+                        commit_both(&sh.bar_s[(b % NSB) * 2 + (j & 1)]);
+                        return true;
+                    };
+                    for (int b = 0; b < nbt && b < NSB && ok; ++b) ok = issue_sb(b);
+                    for (int b = 0; b + NSB < nbt && ok; ++b) {
+                        const int e = ev_pvm % 3;
+                        uint32_t ph = (ph_pvm >> e) & 1u;
+                        if (!(ok = W.wait(&sh.bar_pvm[e], ph, 66))) break;
+                        ph_pvm ^= 1u << e;
+                        ++ev_pvm;
+                        tc_fence_after();
+                        ok = issue_sb(b + NSB);
+                    }
+                    if (!ok) break;
+                } else
                 for (int h = 0; h < H && ok; ++h) {
                     int slot;
                     // Q_h = PE Wq_h^T (M=128, N=64, K=64)
@@ -687,22 +748,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         return true;
                     };
                     for (int j = 0; j < nb && j < NSB && ok; ++j) ok = issue_s(j);
-                    if constexpr (SPLIT) {
-                        // S_{j+3} overwrites the columns P V_j reads (issued by WARP_PV): wait for it
-                        for (int j = 0; j + NSB < nb && ok; ++j) {
-                            const int e = ev_pvm % 3;
-                            uint32_t ph = (ph_pvm >> e) & 1u;
-                            if (!(ok = W.wait(&sh.bar_pvm[e], ph, 66))) break;
-                            ph_pvm ^= 1u << e;
-                            ++ev_pvm;
-                            tc_fence_after();
-                            ok = issue_s(j + NSB);
-                        }
-                        if (!ok) break;
-                        // the next head's Q projection accumulates in S2, which this head's P V read
-                        if (!(ok = W.wait(&sh.bar_hd, ph_hd, 54))) break;
-                        tc_fence_after();
-                    } else {
+                    {
                     for (int j = 0; j < nb && ok; ++j) {
                         const int g = j & 1;   // block j belongs to warpgroup j mod 2
                         if (!(ok = W.wait(&sh.bar_p[g], ph_p[g], 53))) break;
@@ -832,7 +878,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
     else if (SPLIT && warp == WARP_PV) {
       if constexpr (SPLIT) {
         // O_g += P_j V_j for every block: P_j from its warpgroup, V_j from the value ring
-        uint32_t ph_p[2] = {0, 0};
+        uint32_t ph_p[2] = {0, 0}, ph_cmb = 0;
         int v_slot = 0;
         uint32_t v_ph = 0;
         int ev = 0;   // completions the S issue waits for (bar_pvm[ev mod 3])
@@ -842,7 +888,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
             const Unit u = unit_at(it, crank);
             const int nk = u.sel ? a.ksel : N;
             const int nb = (nk + 127) / 128;
+            const int nbt = H * nb;
             for (int h = 0; h < H && ok; ++h) {
+                if (h > 0) {
+                    // the first two P V of a head overwrite O0 and O1: the previous head's combine has read them
+                    if (!(ok = W.wait(&sh.bar_cmb, ph_cmb, 56))) break;
+                    tc_fence_after();
+                }
                 for (int j = 0; j < nb && ok; ++j) {
                     const int g = j & 1;   // block j belongs to warpgroup j mod 2
                     if (!(ok = W.wait(&sh.bar_p[g], ph_p[g], 53))) break;
@@ -862,7 +914,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     // P_j is read in place: the bf16 pairs of tokens [32i, 32i+32) occupy columns
                     // [32i, 32i+16) of its S buffer; V is N-major, 16 tokens (rows of 128 B) per k-step
                     const uint64_t dv = desc_sw128(s_ring + slot * RS);
-                    const uint32_t pa = tmem + T_S0 + 128 * (j % NSB);
+                    const uint32_t pa = tmem + T_S0 + 128 * ((h * nb + j) % NSB);   // block b = h nb + j of the stream
                     #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         mma_ts_w(tmem + (g ? T_O1 : T_O0), pa + 32 * (kk >> 1) + 8 * (kk & 1), dv + 128 * kk,
@@ -870,14 +922,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     mma_commit_w(smem_u32(&sh.empty[slot]));
                     // O_g is final for this block once the P V is done (the owner waits before its next)
                     if (j + 2 < nb) mma_commit_w(smem_u32(&sh.bar_pvg[g]));
-                    if (j + NSB < nb) {
+                    if (h * nb + j + NSB < nbt) {   // S of the block three later in the stream waits for it
                         mma_commit_w(smem_u32(&sh.bar_pvm[ev % 3]));
                         ++ev;
                     }
                 }
                 if (!ok) break;
                 mma_commit_w(smem_u32(&sh.bar_pv));   // the head's P V are complete: O0 and O1 final
-                mma_commit_w(smem_u32(&sh.bar_hd));   // and S2 is free for the next head's Q projection
             }
         }
         // nothing of ours may run on the tensor cores once TMEM is released
@@ -953,7 +1004,35 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 else if (a.ml_slot) ml_out = a.probe_ml + (size_t)a.ml_slot[u.qbeg + row] * H * 2;
             }
             // ================================================= attention
+            if constexpr (SPLIT) {
+                // Q of every head at once (TMEM [64 h, 64 h + 64)): + bq, scaled, bf16 into
+                // attention-output atom h, which the head's combine overwrites
+                if (!(ok = W.wait(&sh.bar_q, ph_q, 60))) break;
+                tc_fence_after();
+                for (int h = 0; h < H; ++h) {
+                    float q[32], b[32];
+                    tmem_ld32(trow + 64 * h + 32 * wg, q);
+                    ldg32(a.bq + h * 64 + 32 * wg, b);
+                    tmem_wait_ld();
+                    reg_fence(q);
+                    const uint32_t qa = s_abuf + h * 16384;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const int d = 8 * c + 2 * v;
+                            w[v] = pack_bf16((q[d] + b[d]) * qscale, (q[d + 1] + b[d + 1]) * qscale);
+                        }
+                        st_shared_v4(swz(qa, row, 4 * wg + c), w);
+                    }
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                arrive_mma(&sh.bar_qc);
+            }
             for (int h = 0; h < H && ok; ++h) {
+              if constexpr (!SPLIT) {
                 if (!(ok = W.wait(&sh.bar_q, ph_q, 60))) break;
                 tc_fence_after();
                 {
@@ -979,16 +1058,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 fence_proxy_async();
                 tc_fence_before();
                 arrive_mma(&sh.bar_qc);
+              }
                 float m_ref = -INFINITY, l_part = 0.f;
                 for (int j = wg; j < nb; j += 2) {
+                    // single CTAs: block b = h nb + j of the stream, in buffer b mod 3
+                    const int bstr = SPLIT ? h * nb + j : j;
                     {
-                        const int sb = j % 6;
+                        const int sb = SPLIT ? (bstr % NSB) * 2 + (j & 1) : j % 6;
                         uint32_t ph = (ph_s >> sb) & 1u;
                         if (!(ok = W.wait(&sh.bar_s[sb], ph, 61))) break;
                         ph_s ^= 1u << sb;
                     }
                     tc_fence_after();
-                    const uint32_t sbase = trow + T_S0 + 128 * (j % NSB);
+                    const uint32_t sbase = trow + T_S0 + 128 * (bstr % NSB);
                     const bool first = j < 2;
                     const int valid = nk - j * 128;   // columns < valid are real tokens
                     // block maximum, 64 columns at a time
@@ -1074,16 +1156,34 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 if (!ok) break;
                 if (!(ok = W.wait(&sh.bar_pv, ph_pv, 63))) break;   // PV_{nb-1}
                 tc_fence_after();
-                // combine the halves: exchange (maximum, sum) through TMEM (S0 is idle until the
-                // next head's S_0), then O = (O0 2^(m0-M) + O1 2^(m1-M)) / (l0 2^(m0-M) + l1 2^(m1-M))
-                tmem_st1(trow + T_S0 + 2 * wg, __float_as_uint(m_ref));
-                tmem_st1(trow + T_S0 + 2 * wg + 1, __float_as_uint(l_part));
+                // combine the halves: exchange (maximum, sum), then
+                // O = (O0 2^(m0-M) + O1 2^(m1-M)) / (l0 2^(m0-M) + l1 2^(m1-M)).
+                // CTA pairs exchange through S0, idle until the next head's S_0. Single CTAs stream
+                // the next head's scores into the S buffers already, so each thread first reads its
+                // first 16 dims of O0 and O1 and then exchanges through the first two of those
+                // columns of its own warpgroup's O (which the other warpgroup does not read).
+                float o0a[16], o1a[16];
+                uint32_t x_own, x_oth;
+                if constexpr (SPLIT) {
+                    tmem_ld16(trow + T_O0 + 32 * wg, o0a);
+                    tmem_ld16(trow + T_O1 + 32 * wg, o1a);
+                    tmem_wait_ld();
+                    reg_fence16(o0a);
+                    reg_fence16(o1a);
+                    x_own = trow + (wg ? T_O1 : T_O0) + 32 * wg;
+                    x_oth = trow + (wg ? T_O0 : T_O1) + 32 * (wg ^ 1);
+                } else {
+                    x_own = trow + T_S0 + 2 * wg;
+                    x_oth = trow + T_S0 + 2 * (wg ^ 1);
+                }
+                tmem_st1(x_own, __float_as_uint(m_ref));
+                tmem_st1(x_own + 1, __float_as_uint(l_part));
                 tmem_wait_st();
                 tc_fence_before();
                 if (!(ok = wg_sync(70))) break;
                 tc_fence_after();
-                uint32_t mo_bits = tmem_ld1(trow + T_S0 + 2 * (wg ^ 1));
-                uint32_t lo_bits = tmem_ld1(trow + T_S0 + 2 * (wg ^ 1) + 1);
+                uint32_t mo_bits = tmem_ld1(x_oth);
+                uint32_t lo_bits = tmem_ld1(x_oth + 1);
                 tmem_wait_ld();
                 asm volatile("" : "+r"(mo_bits), "+r"(lo_bits));
                 const float m_oth = __uint_as_float(mo_bits), l_oth = __uint_as_float(lo_bits);
@@ -1103,11 +1203,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {   // 16 of this warpgroup's 32 head dims at a time
                         float o0[16], o1[16];
-                        tmem_ld16(trow + T_O0 + 32 * wg + 16 * hh, o0);
-                        tmem_ld16(trow + T_O1 + 32 * wg + 16 * hh, o1);
-                        tmem_wait_ld();
-                        reg_fence16(o0);
-                        reg_fence16(o1);
+                        if (SPLIT && hh == 0) {
+                            #pragma unroll
+                            for (int c = 0; c < 16; ++c) {
+                                o0[c] = o0a[c];
+                                o1[c] = o1a[c];
+                            }
+                        } else {
+                            tmem_ld16(trow + T_O0 + 32 * wg + 16 * hh, o0);
+                            tmem_ld16(trow + T_O1 + 32 * wg + 16 * hh, o1);
+                            tmem_wait_ld();
+                            reg_fence16(o0);
+                            reg_fence16(o1);
+                        }
                         #pragma unroll
                         for (int c = 0; c < 2; ++c) {
                             uint32_t w[4];
@@ -1129,6 +1237,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 if (ml_out) {
                     ml_out[h * 2] = M;
                     ml_out[h * 2 + 1] = l_tot;
+                }
+                if constexpr (SPLIT) {
+                    if (h + 1 < H) {   // O0 and O1 are read: the next head's first P V may overwrite them
+                        tc_fence_before();
+                        arrive(&sh.bar_cmb);
+                    }
                 }
             }
             if (!ok) break;
