@@ -41,6 +41,9 @@
 //   per 128-token block j, owned by warpgroup g = j mod 2: S_j = Q_h K_j^T into
 //   S_{j mod 3} ; softmax of the block -> P_j (bf16, in place) ; O_g += P_j V_j ;
 //   end of head: combine the two (max, sum, O_g) -> a[:, h] (bf16 smem).
+//   (Single CTAs project Q for every head at the start of the tile and run the
+//   blocks of all heads as one stream b = h nb + j, S_b in S_{b mod 3}, so the
+//   next head's scores are computed during a head's combine.)
 //   X = PE Wq^T + a Wo^T ; LN1 -> bf16 smem ; MLP hidden chunks:
 //   H_c = LN1(x1) W1_c^T, GELU, X += GELU(H_c) W2_c^T ; LN2 . w_head -> SDF.
 //
