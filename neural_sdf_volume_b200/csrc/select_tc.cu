@@ -14,14 +14,15 @@
 // over the heads in registers (key blocks outer, heads inner: the packed Q of
 // every head stays in TMEM), then per key block the column sums over each
 // sub-volume's probe rows by a warp transpose-reduce (5 shuffle rounds; lane L
-// ends with columns 2L, 2L+1) plus a fixed-order sum over the sub-volume's warps
+// ends with column L of the warp's 32) plus a fixed-order sum over the sub-volume's warps
 // -- deterministic.  Then a radix select of the k largest scores (ties to the
 // smaller token) per sub-volume, in shared memory.
 //
 // Rows: 128 TMEM lanes hold 128 / n_probe sub-volumes' probes (n_probe in
-// {32, 64, 128}).  Roles: warps 0-7 compute in two warpgroups (thread (g, r)
-// owns row r and the 64 columns of half g of each 128-token block, so every
-// SM sub-partition runs two compute warps), warp 8 MMA issue, warp 9 TMA.
+// {32, 64, 128}).  Roles: warps 0-15 compute in four warpgroups (thread (g, r)
+// owns row r and the 32 columns [32g, 32g+32) of each 128-token block, so every
+// SM sub-partition runs four compute warps to hide the TMEM and exponential
+// latencies), warp 16 MMA issue, warp 17 TMA.
 #include <cuda.h>
 
 #include "tc_ptx.cuh"
@@ -36,9 +37,9 @@ namespace {
 
 using namespace ptx;
 
-constexpr int NT = 320;
-constexpr int NCOMP = 256;
-constexpr int WARP_MMA = 8, WARP_PROD = 9;
+constexpr int NT = 576;
+constexpr int NCOMP = 512;   // compute threads: four warpgroups, 32 of the 128 columns of a block each
+constexpr int WARP_MMA = 16, WARP_PROD = 17;
 constexpr int SLOT = 16384;
 constexpr int NS = 6;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -113,48 +114,42 @@ __device__ __forceinline__ uint32_t swz(uint32_t base, int r, int c) {
     return base + r * 128 + ((c ^ (r & 7)) << 4);
 }
 
-// Sum of v over the 32 lanes for each of 64 columns; lane L returns the sums of
-// columns 2L and 2L+1 (the same recursive halving as below, one round fewer).
-__device__ __forceinline__ void warp_colsum64(const float (&v)[64], int lane, float (&out)[2]) {
-    float a32[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const bool up = lane & 16;
-        const float send = up ? v[i] : v[i + 32];
-        const float keep = up ? v[i + 32] : v[i];
-        a32[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
+// Sum of v over the 32 lanes for each of 32 columns; lane L returns the sum of column L.
+__device__ __forceinline__ float warp_colsum32(const float (&v)[32], int lane) {
     float a16[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-        const bool up = lane & 8;
-        const float send = up ? a32[i] : a32[i + 16];
-        const float keep = up ? a32[i + 16] : a32[i];
-        a16[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        const bool up = lane & 16;
+        const float send = up ? v[i] : v[i + 16];
+        const float keep = up ? v[i + 16] : v[i];
+        a16[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
     }
     float a8[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const bool up = lane & 4;
+        const bool up = lane & 8;
         const float send = up ? a16[i] : a16[i + 8];
         const float keep = up ? a16[i + 8] : a16[i];
-        a8[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+        a8[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
     }
     float a4[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const bool up = lane & 2;
+        const bool up = lane & 4;
         const float send = up ? a8[i] : a8[i + 4];
         const float keep = up ? a8[i + 4] : a8[i];
-        a4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+        a4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
     }
+    float a2[2];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-        const bool up = lane & 1;
+        const bool up = lane & 2;
         const float send = up ? a4[i] : a4[i + 2];
         const float keep = up ? a4[i + 2] : a4[i];
-        out[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+        a2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
     }
+    const bool up = lane & 1;
+    return (up ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, up ? a2[0] : a2[1], 1);
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -169,7 +164,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
     const uint32_t s_pe = dyn0;
     const uint32_t s_ring = s_pe + 16384;
     float* score = reinterpret_cast<float*>(dyn_raw + (dyn0 - smem_u32(dyn_raw)) + 16384 + NS * SLOT);  // [tpu][N]
-    float* part = score + (size_t)tpu * N;    // [2][8 warps][64]
+    float* part = score + (size_t)tpu * N;    // [2][16 warps][32]
     Waiter W{&sh, a.err, a.timeout};
 
     if (tid == 0) {
@@ -319,7 +314,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                 const int e = a.qorder[8 * a.tile_off[t] + my_i];
                 voxel_point(child_index(a.plist[e >> 3], e & 7, a.R), a.R, p);
             }
-            for (int c = 4 * wg; c < 4 * wg + 4; ++c) {
+            for (int c = 2 * wg; c < 2 * wg + 2; ++c) {
                 uint32_t w[4];
                 for (int v = 0; v < 4; ++v) w[v] = pack_bf16(pe_lane(p, c * 8 + 2 * v), pe_lane(p, c * 8 + 2 * v + 1));
                 asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(swz(s_pe, row, c)), "r"(w[0]),
@@ -328,22 +323,22 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
             fence_proxy_async();
             arrive(&sh.bar_pe);
             const float* ml = has_probe ? a.probe_ml + ((size_t)t * np + my_i) * H * 2 : nullptr;
-            // Q of every head: + bq, scale, bf16 pairs; warpgroup g packs head dims [32g, 32g+32) into
-            // columns [32h + 16g, 32h + 16g + 16)
+            // Q of every head: + bq, scale, bf16 pairs; warpgroup g packs head dims [16g, 16g+16) into
+            // columns [32h + 8g, 32h + 8g + 8)
             for (int h0 = 0; h0 < H && ok; h0 += QROUND) {
                 if (!(ok = W.wait(&sh.bar_q, ph_q, 86))) break;
                 tc_fence_after();
                 for (int h = h0; h < H && h < h0 + QROUND; ++h) {
-                    float q[32];
-                    tmem_ld32(trow + T_QA + 64 * (h - h0) + 32 * wg, q);
+                    float q[16];
+                    tmem_ld16(trow + T_QA + 64 * (h - h0) + 16 * wg, q);
                     tmem_wait_ld();
-                    reg_fence(q);
-                    uint32_t pk[16];
-                    for (int v = 0; v < 16; ++v) {
-                        const int c0 = h * 64 + 32 * wg + 2 * v;
+                    reg_fence16(q);
+                    uint32_t pk[8];
+                    for (int v = 0; v < 8; ++v) {
+                        const int c0 = h * 64 + 16 * wg + 2 * v;
                         pk[v] = pack_bf16((q[2 * v] + a.bq[c0]) * qscale, (q[2 * v + 1] + a.bq[c0 + 1]) * qscale);
                     }
-                    tmem_st16(trow + T_QP + 32 * h + 16 * wg, pk);
+                    tmem_st8(trow + T_QP + 32 * h + 8 * wg, pk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -363,64 +358,51 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                 if (!(ok = csync(97))) break;
             }
             for (int j = 0; j < nb && ok; ++j) {
-                const int vcols = N - j * 128 - 64 * wg;   // own columns < vcols are real tokens
-                float acc[64];
+                const int vcols = N - j * 128 - 32 * wg;   // own columns < vcols are real tokens
+                float acc[32];
 #pragma unroll
-                for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+                for (int c = 0; c < 32; ++c) acc[c] = 0.f;
                 for (int h = 0; h < H; ++h, ++i) {
                     if (!(ok = W.wait(&sh.bar_s[i & 1], ph_s[i & 1], 87))) break;
                     tc_fence_after();
-                    const uint32_t sb = trow + T_S0 + 128 * (i & 1) + 64 * wg;
+                    const uint32_t sb = trow + T_S0 + 128 * (i & 1) + 32 * wg;
                     // P = 2^(S - m) / l = 2^(S - m - log2 l); rows without a probe add 2^-inf = 0
                     const float mo = has_probe ? ml[h * 2] + __log2f(ml[h * 2 + 1]) : INFINITY;
-                    auto accum = [&](const float (&x)[32], int c0) {
-                        if (vcols >= c0 + 32) {
-#pragma unroll
-                            for (int c = 0; c < 32; ++c) acc[c0 + c] += ex2(x[c] - mo);
-                        } else {
-#pragma unroll
-                            for (int c = 0; c < 32; ++c) acc[c0 + c] += c0 + c < vcols ? ex2(x[c] - mo) : 0.f;
-                        }
-                    };
-                    // both 32-column halves in flight at once, one wait
-                    float s0[32], s1[32];
+                    float s0[32];
                     tmem_ld32(sb, s0);
-                    tmem_ld32(sb + 32, s1);
                     tmem_wait_ld();
                     reg_fence(s0);
-                    reg_fence(s1);
                     tc_fence_before();
-                    arrive(&sh.bar_p[i & 1]);   // this half of S_i consumed
-                    accum(s0, 0);
-                    accum(s1, 32);
+                    arrive(&sh.bar_p[i & 1]);   // this quarter of S_i consumed
+                    if (vcols >= 32) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) acc[c] += ex2(s0[c] - mo);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) acc[c] += c < vcols ? ex2(s0[c] - mo) : 0.f;
+                    }
                 }
                 if (!ok) break;
-                float cs[2];
-                warp_colsum64(acc, lane, cs);
+                const float cs = warp_colsum32(acc, lane);
                 if (direct) {
-                    const int col = j * 128 + 64 * wg + 2 * lane;
-                    float* dst = score + (size_t)my_sv * N + col;
-                    if (warps_per_tile == 1) {
-                        if (col < N) dst[0] = cs[0];
-                        if (col + 1 < N) dst[1] = cs[1];
-                    } else {
-                        if (col < N) atomicAdd(dst, cs[0]);
-                        if (col + 1 < N) atomicAdd(dst + 1, cs[1]);
+                    const int col = j * 128 + 32 * wg + lane;
+                    if (col < N) {
+                        float* dst = score + (size_t)my_sv * N + col;
+                        if (warps_per_tile == 1) *dst = cs;
+                        else atomicAdd(dst, cs);
                     }
                     continue;
                 }
-                float* pw = part + (pb * 8 + warp) * 64;
-                pw[2 * lane] = cs[0];
-                pw[2 * lane + 1] = cs[1];
+                part[(pb * 16 + warp) * 32 + lane] = cs;
                 if (!(ok = csync(88))) break;
                 // column col of sub-volume s: its warps of the column's warpgroup, in order
                 for (int idx = tid; idx < tpu * 128; idx += NCOMP) {
                     const int sv = idx >> 7, col = idx & 127;
                     if (j * 128 + col < N) {
-                        const int g = col >> 6;
-                        const float* pp = part + (pb * 8 + 4 * g + sv * warps_per_tile) * 64 + (col & 63);
+                        const int g = col >> 5;
+                        const float* pp = part + (pb * 16 + 4 * g + sv * warps_per_tile) * 32 + (col & 31);
                         float sum = 0.f;
-                        for (int w = 0; w < warps_per_tile; ++w) sum += pp[w * 64];
+                        for (int w = 0; w < warps_per_tile; ++w) sum += pp[w * 32];
                         score[(size_t)sv * N + j * 128 + col] = sum;
                     }
                 }
