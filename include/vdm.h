@@ -160,6 +160,9 @@ VDM_API vdm_status vdm_decode_dense(const vdm_decoder* dec, const void* d_k, con
  *   P_total       P (host value; must match d_tile_off[T])
  *   d_sel_out     [T][top_k] int32 (device)
  *   d_score_out   [T][N] float32 or NULL
+ *   d_probe_dec_out [P] float32 or NULL: the raw decoder output at every
+ *                 probe (full attention; the probes' values are final in the
+ *                 adaptive procedure, section 4.1 item 2 step 3)
  * Sub-volumes with no probe select tokens 0..top_k-1.  top_k >= N selects
  * every token.
  * Kernels: with a bf16 decoder of width 128, 256 or 512 and at most 128
@@ -178,7 +181,7 @@ VDM_API vdm_status vdm_decode_dense(const vdm_decoder* dec, const void* d_k, con
 VDM_API vdm_status vdm_select_kv(const vdm_decoder* dec, const void* d_k, const void* d_v, int32_t N,
                          const float* d_probe_xyz, const int32_t* d_tile_off, int32_t T,
                          int64_t P_total, int32_t top_k, int32_t* d_sel_out, float* d_score_out,
-                         vdm_stream stream);
+                         float* d_probe_dec_out, vdm_stream stream);
 
 /* Hierarchical volume decoding parameters (section 4.1 items 1-2).        */
 typedef struct {
@@ -469,7 +472,7 @@ VDM_API vdm_status vdm_profile_end(vdm_profile* out);
 
 VDM_API const char* vdm_status_string(vdm_status s);
 VDM_API const char* vdm_last_error(void);   /* thread-local message of the last error */
-VDM_API int32_t vdm_abi_version(void);      /* 2                                      */
+VDM_API int32_t vdm_abi_version(void);      /* 3                                      */
 
 #ifdef __cplusplus
 }

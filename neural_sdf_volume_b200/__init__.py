@@ -110,7 +110,7 @@ _lib.vdm_precompute_kv.argtypes = [C.POINTER(CDecoder), _vp, _i32, _i32, _vp, _v
 _lib.vdm_decode_dense.argtypes = [C.POINTER(CDecoder), _vp, _vp, _i32, _i32, _vp, _i64, _i32,
                                   C.POINTER(CAnalytic), _vp, _vp]
 _lib.vdm_select_kv.argtypes = [C.POINTER(CDecoder), _vp, _vp, _i32, _vp, _vp, _i32, _i64, _i32,
-                               _vp, _vp, _vp]
+                               _vp, _vp, _vp, _vp]
 _lib.vdm_hierarchical_workspace_size.argtypes = [C.POINTER(CDecoder), C.POINTER(CHierParams), _i32,
                                                  C.POINTER(C.c_size_t)]
 _lib.vdm_decode_hierarchical.argtypes = [C.POINTER(CDecoder), _vp, _vp, _i32, _i32,
@@ -254,19 +254,26 @@ def vdm_decode_dense(dec: Decoder, K, V, xyz=None, grid_R: int = 0, spheres=None
 
 
 def vdm_select_kv(dec: Decoder, K, V, probe_xyz, tile_off, top_k: int, want_scores: bool = False,
-                  stream=None):
-    """Per sub-volume Top-K token ids ``[T, top_k]`` (and scores ``[T, N]``)."""
+                  stream=None, want_probe_dec: bool = False):
+    """Per sub-volume Top-K token ids ``[T, top_k]``, then (when asked) scores
+    ``[T, N]`` and the probes' raw decoder output ``[P]``, in that order."""
     torch = _torch()
     N = K.shape[-2]
     T = int(tile_off.numel()) - 1
     P = int(probe_xyz.shape[0]) if probe_xyz is not None else 0
     sel = torch.empty((max(T, 0), top_k), device=K.device, dtype=torch.int32)
     score = torch.empty((max(T, 0), N), device=K.device, dtype=torch.float32) if want_scores else None
+    pdec = torch.empty((P,), device=K.device, dtype=torch.float32) if want_probe_dec else None
     cd = dec.cstruct()
     _check(_lib.vdm_select_kv(C.byref(cd), K.data_ptr(), V.data_ptr(), N, _ptr(probe_xyz),
-                              tile_off.data_ptr(), T, P, top_k, sel.data_ptr(), _ptr(score),
+                              tile_off.data_ptr(), T, P, top_k, sel.data_ptr(), _ptr(score), _ptr(pdec),
                               _stream(stream)))
-    return (sel, score) if want_scores else sel
+    out = (sel,)
+    if want_scores:
+        out += (score,)
+    if want_probe_dec:
+        out += (pdec,)
+    return out if len(out) > 1 else sel
 
 
 def hier_params(r0: int, n_levels: int, adaptive: bool = False, tile: int = 8, n_probe: int = 64,

@@ -186,7 +186,7 @@ using namespace vdm;
 
 extern "C" {
 
-int32_t vdm_abi_version(void) { return 2; }
+int32_t vdm_abi_version(void) { return 3; }
 
 const char* vdm_last_error(void) { return g_err; }
 
@@ -272,7 +272,7 @@ vdm_status vdm_decode_dense(const vdm_decoder* dec, const void* d_k, const void*
 vdm_status vdm_select_kv(const vdm_decoder* dec, const void* d_k, const void* d_v, int32_t N,
                          const float* d_probe_xyz, const int32_t* d_tile_off, int32_t T,
                          int64_t P_total, int32_t top_k, int32_t* d_sel_out, float* d_score_out,
-                         vdm_stream stream) {
+                         float* d_probe_dec_out, vdm_stream stream) {
     VDM_TRY(check_decoder(dec, true));
     if (N < 1 || T < 0 || P_total < 0) return fail(VDM_ERR_INVALID_ARG, "bad N / T / P");
     if (N > kMaxN) return fail(VDM_ERR_UNSUPPORTED, "N = %d > %d", N, kMaxN);
@@ -325,6 +325,7 @@ vdm_status vdm_select_kv(const vdm_decoder* dec, const void* d_k, const void* d_
             VDM_TRY(launch_flat_probe_slots(d_tile_off, T, np, ml_slot, sel_tiles, n_sel, st));
             d.probe_ml = probe_ml;
             d.ml_slot = ml_slot;
+            d.out = d_probe_dec_out;   // the probes' decoded values, when asked for
             VDM_TRY(launch_decode_tc(d, st));
             SelectTcLaunch L{};
             L.C = dec->C; L.H = dec->H; L.N = N;
@@ -359,6 +360,10 @@ vdm_status vdm_select_kv(const vdm_decoder* dec, const void* d_k, const void* d_
         a.sel = d_sel_out;
         a.score = d_score_out;
         VDM_TRY(launch_select(a, dec->dtype, st));
+        if (d_probe_dec_out && P_total > 0) {
+            d.out = d_probe_dec_out;
+            VDM_TRY(launch_decode(d, dec->dtype, st));
+        }
     }
     VDM_CUDA_TRY(cudaStreamSynchronize(st));
     return tc_check_error();

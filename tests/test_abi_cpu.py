@@ -26,7 +26,7 @@ def test_every_declared_function_is_exported():
 
 
 def test_status_strings_and_version():
-    assert vdm.abi_version() == 2
+    assert vdm.abi_version() == 3
     assert vdm._lib.vdm_status_string(0) == b"ok"
     assert vdm._lib.vdm_status_string(3) == b"workspace too small"
 
@@ -77,7 +77,7 @@ def test_null_arguments_are_rejected():
 
 def test_select_rejects_bad_top_k():
     d = _fake_decoder()
-    st = vdm._lib.vdm_select_kv(C.byref(d), 0x1000, 0x2000, 64, 0x3000, 0x4000, 2, 10, 65, 0x5000, None, None)
+    st = vdm._lib.vdm_select_kv(C.byref(d), 0x1000, 0x2000, 64, 0x3000, 0x4000, 2, 10, 65, 0x5000, None, None, None)
     assert st == 1
 
 

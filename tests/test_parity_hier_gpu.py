@@ -152,10 +152,12 @@ def test_select_kv_scores_and_topk_given_the_same_scores():
     off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
     pts = W.make_points(int(off[-1]), seed=3, key=3)[0]
     k = 100
-    sel, score = vdm.vdm_select_kv(case.dec, case.K, case.V, torch.from_numpy(pts).cuda(),
-                                   torch.from_numpy(off).cuda(), k, want_scores=True)
+    sel, score, pdec = vdm.vdm_select_kv(case.dec, case.K, case.V, torch.from_numpy(pts).cuda(),
+                                         torch.from_numpy(off).cuda(), k, want_scores=True, want_probe_dec=True)
     sel = sel.cpu().numpy()
     score = score.cpu().numpy().astype(np.float64)
+    # the probes' decoded values (full attention)
+    assert np.abs(pdec.cpu().numpy() - case.oracle_dec(pts)).max() <= TOL["bf16"]
     K, V = case.okv()
     for t in range(len(counts)):
         assert np.array_equal(sel[t], OA.top_k(score[t], k)), f"tile {t}"
@@ -183,10 +185,11 @@ def test_select_kv_tensor_core_route_scores_and_topk():
     off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
     pts = W.make_points(int(off[-1]), seed=5, key=3)[0]
     k = 100
-    sel, score = vdm.vdm_select_kv(case.dec, case.K, case.V, torch.from_numpy(pts).cuda(),
-                                   torch.from_numpy(off).cuda(), k, want_scores=True)
+    sel, score, pdec = vdm.vdm_select_kv(case.dec, case.K, case.V, torch.from_numpy(pts).cuda(),
+                                         torch.from_numpy(off).cuda(), k, want_scores=True, want_probe_dec=True)
     sel = sel.cpu().numpy()
     score = score.cpu().numpy().astype(np.float64)
+    assert np.abs(pdec.cpu().numpy() - case.oracle_dec(pts)).max() <= TOL["bf16"]
     K, V = case.okv()
     for t in range(len(counts)):
         assert np.array_equal(sel[t], OA.top_k(score[t], k)), f"tile {t}"
