@@ -637,7 +637,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
         {   // the whole warp runs the issue loop; one elected lane issues each instruction
             // the MMA issuer of a pair waits on barriers that the other CTA arrives at
             W.cluster_acq = PAIR;
-            uint32_t ring_tail = 0;
             uint32_t ph_pe = 0, ph_qc = 0, ph_p[2] = {0, 0}, ph_a = 0, ph_hin = 0, ph_r = 0, ph_g[2] = {0, 0};
             uint32_t ph_hd = 0, ph_w2 = 0, ph_pvm = 0 /* bit k: phase of bar_pvm[k] (bit 0 alone: pairs) */;
             int ev_pvm = 0;   // P V completions awaited so far (single CTAs)
@@ -649,7 +648,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                 uint32_t ph = c_ph;
                 if (!W.wait(&sh.full[slot], ph, 50)) return false;
                 tc_fence_after();
-                ++ring_tail;
                 if (++c_slot == NRA) {
                     c_slot = 0;
                     c_ph ^= 1;
