@@ -1092,11 +1092,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                             }
                         }
 #pragma unroll
-                        for (int c = 0; c < 32; c += 2) {
-                            m0 = fmaxf(m0, sa[c]);
-                            m1 = fmaxf(m1, sa[c + 1]);
-                            m2 = fmaxf(m2, sb[c]);
-                            m3 = fmaxf(m3, sb[c + 1]);
+                        for (int c = 0; c < 32; c += 4) {
+                            m0 = fmax3(m0, sa[c], sa[c + 1]);
+                            m1 = fmax3(m1, sa[c + 2], sa[c + 3]);
+                            m2 = fmax3(m2, sb[c], sb[c + 1]);
+                            m3 = fmax3(m3, sb[c + 2], sb[c + 3]);
                         }
                     }
                     const float mb = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
@@ -1107,7 +1107,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                     const float m_use = m_ref == -INFINITY ? 0.f : m_ref;   // no real token yet: P = 0
                     // exponentials, 32 columns at a time; P of columns [c0, c0+32) goes to columns
                     // [c0, c0+16), which are read already
-                    float la = 0.f, lb = 0.f;
+                    // (even and odd columns summed separately, as fp32 pairs)
+                    uint64_t lab = f32x2(0.f, 0.f);
+                    const uint64_t mm = f32x2(m_use, m_use);
                     #pragma unroll 1
                     for (int c0 = 0; c0 < 128; c0 += 32) {
                         float x[32];
@@ -1122,13 +1124,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         uint32_t pk[16];
 #pragma unroll
                         for (int v = 0; v < 16; ++v) {
-                            const float e0 = ex2(x[2 * v] - m_use), e1 = ex2(x[2 * v + 1] - m_use);
-                            la += e0;
-                            lb += e1;
+                            float d0, d1;
+                            f32x2_split(sub_f32x2(f32x2(x[2 * v], x[2 * v + 1]), mm), d0, d1);
+                            const float e0 = ex2(d0), e1 = ex2(d1);
+                            lab = add_f32x2(lab, f32x2(e0, e1));
                             pk[v] = pack_bf16(e0, e1);
                         }
                         tmem_st16(sbase + c0, pk);
                     }
+                    float la, lb;
+                    f32x2_split(lab, la, lb);
                     if (need && !first) l_part *= f;
                     l_part += la + lb;
                     if (!first) {   // the PV of this warpgroup's previous block is done: O_g is stable
@@ -1366,7 +1371,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                         uint32_t w[16];
 #pragma unroll
                         for (int e = 0; e < 16; ++e)
-                            w[e] = pack_bf16(gelu_as(v[2 * e] + bb[2 * e]), gelu_as(v[2 * e + 1] + bb[2 * e + 1]));
+                            w[e] = gelu_as_pack(v[2 * e] + bb[2 * e], v[2 * e + 1] + bb[2 * e + 1]);
                         tmem_st16(hb + 16 * part, w);
                     }
                     tmem_wait_st();

@@ -375,8 +375,15 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tm_wq64, const __grid_const
                     tc_fence_before();
                     arrive(&sh.bar_p[i & 1]);   // this quarter of S_i consumed
                     if (vcols >= 32) {
+                        const uint64_t mm = f32x2(mo, mo);
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) acc[c] += ex2(s0[c] - mo);
+                        for (int c = 0; c < 32; c += 2) {
+                            float d0, d1, a0, a1;
+                            f32x2_split(sub_f32x2(f32x2(s0[c], s0[c + 1]), mm), d0, d1);
+                            f32x2_split(add_f32x2(f32x2(acc[c], acc[c + 1]), f32x2(ex2(d0), ex2(d1))), a0, a1);
+                            acc[c] = a0;
+                            acc[c + 1] = a1;
+                        }
                     } else {
 #pragma unroll
                         for (int c = 0; c < 32; ++c) acc[c] += c < vcols ? ex2(s0[c] - mo) : 0.f;

@@ -361,10 +361,71 @@ __device__ __forceinline__ float gelu_as(float x) {
     const float erf_abs = fmaf(-q, e, 1.0f);
     return 0.5f * x * (1.0f + copysignf(erf_abs, x));
 }
+// Three-input maximum (sm_100): one instruction for two fmaxf steps.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): each lane of the pair is rounded exactly
+// as the scalar instruction would round it, so these are bit-identical to two scalar ops.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f32x2_split(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
+}
+// gelu_as of two values at once, packed to bf16: the same operations in the same order as
+// gelu_as on each (the multiplies, adds and fused multiply-adds as fp32 pairs, the reciprocal
+// and the exponential per value), so the result equals pack_bf16(gelu_as(x0), gelu_as(x1)).
+__device__ __forceinline__ uint32_t gelu_as_pack(float x0, float x1) {
+    constexpr uint64_t SIGN = 0x8000000080000000ull;
+    const auto splat = [](float c) { return f32x2(c, c); };
+    const uint64_t x = f32x2(x0, x1);
+    const uint64_t z = mul_f32x2(x & ~SIGN, splat(0.70710678118654752f));
+    float u0, u1;
+    f32x2_split(fma_f32x2(splat(0.3275911f), z, splat(1.0f)), u0, u1);
+    const uint64_t t = f32x2(rcp_approx(u0), rcp_approx(u1));
+    uint64_t q = fma_f32x2(splat(1.061405429f), t, splat(-1.453152027f));
+    q = fma_f32x2(q, t, splat(1.421413741f));
+    q = fma_f32x2(q, t, splat(-0.284496736f));
+    q = fma_f32x2(q, t, splat(0.254829592f));
+    q = mul_f32x2(q, t);
+    float w0, w1;
+    f32x2_split(mul_f32x2(mul_f32x2(z ^ SIGN, z), splat(1.4426950408889634f)), w0, w1);
+    const uint64_t e = f32x2(ex2(w0), ex2(w1));
+    const uint64_t erf_abs = fma_f32x2(q ^ SIGN, e, splat(1.0f));
+    const uint64_t r = mul_f32x2(mul_f32x2(splat(0.5f), x), add_f32x2(splat(1.0f), (erf_abs & ~SIGN) | (x & SIGN)));
+    float r0, r1;
+    f32x2_split(r, r0, r1);
+    return pack_bf16(r0, r1);
 }
 
 }  // namespace ptx
