@@ -97,6 +97,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 // and hand-offs; one O accumulator per warpgroup (its blocks, all 64 head dims); the Q
 // projection accumulates in S2 before the head's first block, the packed Q waits in shared
 // memory
+#ifndef VDM_EMU_PAIRS
+#define VDM_EMU_PAIRS 0x8888u
+#endif
+// Column pairs (bit v: columns 2v, 2v+1 of every 32) whose softmax exponentials run on the
+// FMA pipe (exp2_pair_poly) instead of the special-function unit.
+constexpr uint32_t kEmuPairs = VDM_EMU_PAIRS;
 constexpr uint32_t T_S0 = 0, T_O0 = 384, T_O1 = 448, T_QACC = 256;
 constexpr int NSB = 3;   // S buffers
 
@@ -1122,13 +1128,33 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constan
                                 if (c0 + c >= valid) x[c] = -INFINITY;
                         }
                         uint32_t pk[16];
+                        if (valid >= c0 + 32) {
+                            // the column pairs in kEmuPairs on the FMA pipe, the rest on ex2
 #pragma unroll
-                        for (int v = 0; v < 16; ++v) {
-                            float d0, d1;
-                            f32x2_split(sub_f32x2(f32x2(x[2 * v], x[2 * v + 1]), mm), d0, d1);
-                            const float e0 = ex2(d0), e1 = ex2(d1);
-                            lab = add_f32x2(lab, f32x2(e0, e1));
-                            pk[v] = pack_bf16(e0, e1);
+                            for (int v = 0; v < 16; ++v) {
+                                const uint64_t d = sub_f32x2(f32x2(x[2 * v], x[2 * v + 1]), mm);
+                                uint64_t e;
+                                if ((kEmuPairs >> v) & 1u) {
+                                    e = exp2_pair_poly(d);
+                                } else {
+                                    float d0, d1;
+                                    f32x2_split(d, d0, d1);
+                                    e = f32x2(ex2(d0), ex2(d1));
+                                }
+                                lab = add_f32x2(lab, e);
+                                float e0, e1;
+                                f32x2_split(e, e0, e1);
+                                pk[v] = pack_bf16(e0, e1);
+                            }
+                        } else {
+#pragma unroll
+                            for (int v = 0; v < 16; ++v) {
+                                float d0, d1;
+                                f32x2_split(sub_f32x2(f32x2(x[2 * v], x[2 * v + 1]), mm), d0, d1);
+                                const float e0 = ex2(d0), e1 = ex2(d1);
+                                lab = add_f32x2(lab, f32x2(e0, e1));
+                                pk[v] = pack_bf16(e0, e1);
+                            }
                         }
                         tmem_st16(sbase + c0, pk);
                     }

@@ -402,6 +402,30 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
+// 2^x of a pair of values on the FMA and integer pipes instead of the special-function
+// unit (which computes one exponential per lane every 8 cycles per sub-partition).
+// Range reduction in the manner of Cody and Waite: x = n + f with n = round(x), taken from
+// the low mantissa bits of x + 1.5 * 2^23, and f = x - n in [-1/2, 1/2]; 2^f by a cubic
+// whose coefficients were fitted for this function by iteratively reweighted least squares
+// (Lawson's minimax method) on [-1/2, 1/2]: relative error <= 7.5e-5 in fp32 Horner form,
+// below the bf16 rounding of the probabilities (2^-9); 2^n by adding n to the exponent
+// field.  Inputs are clamped below at -126, where the result is at most 2^-126 (not 0), so
+// the caller keeps masked (-inf) columns on ex2.
+__device__ __forceinline__ uint64_t exp2_pair_poly(uint64_t x) {
+    constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
+    const auto splat = [](float c) { return f32x2(c, c); };
+    float x0, x1;
+    f32x2_split(x, x0, x1);
+    const uint64_t xc = f32x2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+    const uint64_t t = add_f32x2(xc, splat(kShift));
+    const uint64_t f = sub_f32x2(xc, sub_f32x2(t, splat(kShift)));
+    uint64_t p = fma_f32x2(splat(0.055171627551317215f), f, splat(0.2426111400127411f));
+    p = fma_f32x2(p, f, splat(0.6932609677314758f));
+    p = fma_f32x2(p, f, splat(0.9999280571937561f));
+    const uint32_t t0 = (uint32_t)t, t1 = (uint32_t)(t >> 32);
+    const uint32_t p0 = (uint32_t)p, p1 = (uint32_t)(p >> 32);
+    return (uint64_t)(p0 + (t0 << 23)) | ((uint64_t)(p1 + (t1 << 23)) << 32);
+}
 // gelu_as of two values at once, packed to bf16: the same operations in the same order as
 // gelu_as on each (the multiplies, adds and fused multiply-adds as fp32 pairs, the reciprocal
 // and the exponential per value), so the result equals pack_bf16(gelu_as(x0), gelu_as(x1)).
