@@ -52,7 +52,7 @@ def _peaks():
 # dram__bytes_read.sum + dram__bytes_write.sum per decode launch of one shape of a
 # workload (mean over the shape's decode launches), from ncu's one-pass DRAM counters on
 # this script's own launches; None until captured for the current decoder kernel.
-DECODE_DRAM_BYTES_PER_LAUNCH = {4: 39.54e6}
+DECODE_DRAM_BYTES_PER_LAUNCH = {4: 39.48e6}
 
 
 def decode_flops_per_query(spec: W.DecoderSpec, n_tokens: int) -> float:
