@@ -457,10 +457,7 @@ def run_vdm(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"config {cfg.cid}: {cfg.name}, N={cfg.dec.N}, C={cfg.dec.C}, "
-                               f"H={cfg.dec.H}, F={cfg.dec.F}, top_k={cfg.top_k}, {cfg.n_spheres} spheres",
-                   "shapes_per_gpu": B, "final_resolution": Rf, "l2": "flushed between timed steps",
-                   "parallelism": f"shape-sharded x{world}"},
+        "config": hier_config(cfg, world),
         "ms_per_shape": ms / B,
         "decoded_points_per_shape": decoded / B,
         "queries_saved_vs_dense": 1.0 - decoded / (B * Rf ** 3),
@@ -663,6 +660,14 @@ def cpu_baseline(cfg, seconds: float = 15.0):
                       f"float64 dense decode, {dt:.1f} s"}
 
 
+def hier_config(cfg, world):
+    """The `config` object of a hierarchical workload's line (both arms print the same one)."""
+    return {"workload": f"config {cfg.cid}: {cfg.name}, N={cfg.dec.N}, C={cfg.dec.C}, "
+                        f"H={cfg.dec.H}, F={cfg.dec.F}, top_k={cfg.top_k}, {cfg.n_spheres} spheres",
+            "shapes_per_gpu": cfg.B, "final_resolution": cfg.r_final, "l2": "flushed between timed steps",
+            "parallelism": f"shape-sharded x{world}"}
+
+
 def run_reference(args, world, rank):
     cfg = W.CONFIGS[args.config]
     if rank != 0:
@@ -680,7 +685,7 @@ def run_reference(args, world, rank):
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"config {cfg.cid}: {cfg.name}", "sample_points_per_step": n},
+            "config": hier_config(cfg, world) if cfg.mode == "hier" else {"workload": f"config {cfg.cid}: {cfg.name}"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": f"{n} query points per step, float64 dense decode"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
