@@ -49,8 +49,9 @@
 //
 // TMEM (512 columns x 128 lanes):
 //   attention: S0 [0,128) S1 [128,256) S2 [256,384) (P_j overwrites the first 16 of
-//              each 32 S columns once they are read; the Q accumulator sits in S2
-//              before the head's first block) O0 [384,448) O1 [448,512)
+//              each 32 S columns once they are read; CTA pairs accumulate Q_h in S2
+//              before the head's first block, single CTAs every head's Q in [0, C)
+//              at the start of the tile) O0 [384,448) O1 [448,512)
 //   output projection: X [0, C)
 //   MLP, C <= 256: acc [0, C); hidden chunks (128 wide) at [256,384) [384,512)
 //   MLP, C == 512: the 128 x 512 fp32 residual alone fills TMEM, so the MLP
@@ -61,7 +62,8 @@
 //
 // Softmax: logits in log2 units (the 1/8 scale and log2 e folded into Q);
 // the running maximum is only raised when a block exceeds it by more than 8
-// (then O and the sum are rescaled), so P stays <= 2^8.
+// (then O and the sum are rescaled), so P stays <= 2^8.  A quarter of the
+// exponentials run on the FMA pipe (exp2_pair_poly), the rest on ex2.approx.
 //
 // Barrier protocol: waits are parity based, so every waiter observes every
 // phase of the barriers it uses, and no barrier can run two phases ahead of a
@@ -94,9 +96,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 // attention: three S buffers in rotation (block j in S_{j mod 3}; its P overwrites the S
 // columns already read), so the next block's scores are ready before a warpgroup needs them;
 // the warpgroups alternate blocks, so one's exponentials overlap the other's loads, maximum
-// and hand-offs; one O accumulator per warpgroup (its blocks, all 64 head dims); the Q
-// projection accumulates in S2 before the head's first block, the packed Q waits in shared
-// memory
+// and hand-offs; one O accumulator per warpgroup (its blocks, all 64 head dims); the packed
+// Q of a head waits in shared memory
 #ifndef VDM_EMU_PAIRS
 #define VDM_EMU_PAIRS 0x8888u
 #endif
