@@ -444,6 +444,18 @@ VDM_API vdm_status vdm_surface_case_table(uint8_t* ntri, uint8_t* tri);
  * restores normal operation.                                                */
 VDM_API vdm_status vdm_debug_inject(int32_t mode, int64_t timeout_cycles);
 
+/* Test hook for the decoder's softmax arithmetic (not needed for decoding):
+ * d_y[i] = 2^d_x[i] (device float32 arrays of n elements, n >= 0) computed the
+ * way the tensor-core decoder computes a quarter of its softmax exponentials:
+ * x = m + f with m = round(x) and f in [-1/2, 1/2] (range reduction in the
+ * manner of Cody and Waite), 2^f by a cubic fitted for this function (relative
+ * error <= 7.5e-5 for -125 <= x <= 9), 2^m added to the exponent field.
+ * Inputs below -125 (and -inf) give a result in [0, 2^-124] (not 0, and not
+ * accurate once it leaves the normal range); NaN is not an input the decoder
+ * produces and gives no meaningful result.
+ * Asynchronous on `stream`.  Errors: INVALID_ARG, CUDA.                     */
+VDM_API vdm_status vdm_debug_exp2(const float* d_x, float* d_y, int64_t n, vdm_stream stream);
+
 /* Tensor-core decoding on CTA pairs: with enable = 1, each 256-query MMA runs
  * on the two CTAs of a cluster (cta_group::2); each CTA holds 128 query rows
  * and loads half of every weight and key/value tile, which halves the bytes

@@ -39,7 +39,7 @@ EXPORTS = ("vdm_precompute_kv", "vdm_decode_dense", "vdm_select_kv",
            "vdm_surface_workspace_size", "vdm_extract_surface", "vdm_surface_case_table",
            "vdm_refine_workspace_size", "vdm_refine_level",
            "vdm_encode_workspace_size", "vdm_encode", "vdm_local_workspace_size", "vdm_decode_local",
-           "vdm_debug_inject", "vdm_set_cta_pairs",
+           "vdm_debug_inject", "vdm_debug_exp2", "vdm_set_cta_pairs",
            "vdm_profile_begin", "vdm_profile_end",
            "vdm_status_string", "vdm_last_error", "vdm_abi_version")
 PROF_CLASSES = ("kv", "decode", "select", "mark", "scan", "list", "fill", "probe")
@@ -132,6 +132,8 @@ _lib.vdm_decode_local.argtypes = [C.POINTER(CLocalDecoder), _vp, _i64, _vp, _vp,
 _lib.vdm_encode.argtypes = [C.POINTER(CDecoder), _vp, _vp, _vp, _i32, _i32, _vp, _i32, _vp, _vp, C.c_size_t, _vp]
 _lib.vdm_debug_inject.argtypes = [_i32, _i64]
 _lib.vdm_debug_inject.restype = C.c_int
+_lib.vdm_debug_exp2.argtypes = [C.c_void_p, C.c_void_p, _i64, C.c_void_p]
+_lib.vdm_debug_exp2.restype = C.c_int
 _lib.vdm_set_cta_pairs.argtypes = [_i32]
 _lib.vdm_set_cta_pairs.restype = C.c_int
 _lib.vdm_profile_begin.argtypes = []
@@ -504,6 +506,18 @@ def vdm_debug_inject(mode: int, timeout_cycles: int = 0):
     """Test hook: mode 1 withholds one completion signal in the next
     tensor-core decode launch (its bounded waits then report a timeout)."""
     _check(_lib.vdm_debug_inject(mode, timeout_cycles))
+
+
+def vdm_debug_exp2(x, stream=None):
+    """Test hook: 2^x (float32 CUDA tensor) by the decoder softmax's polynomial form."""
+    import torch
+
+    x = x.contiguous()
+    if x.dtype != torch.float32 or not x.is_cuda:
+        raise ValueError("x must be a float32 CUDA tensor")
+    y = torch.empty_like(x)
+    _check(_lib.vdm_debug_exp2(x.data_ptr(), y.data_ptr(), x.numel(), _stream(stream)))
+    return y
 
 
 def vdm_set_cta_pairs(enable: bool):

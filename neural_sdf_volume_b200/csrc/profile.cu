@@ -3,10 +3,23 @@
 
 #include <vector>
 
+#include "tc_ptx.cuh"
 #include "vdm_internal.cuh"
 
 namespace vdm {
 namespace {
+
+// the decoder's polynomial 2^x on pairs of elements (the last element of an odd n is paired
+// with itself)
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+    const int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : x0;
+    float y0, y1;
+    ptx::f32x2_split(ptx::exp2_pair_poly(ptx::f32x2(x0, x1)), y0, y1);
+    y[i] = y0;
+    if (i + 1 < n) y[i + 1] = y1;
+}
 
 struct Rec {
     cudaEvent_t a, b;
@@ -58,6 +71,17 @@ vdm_status vdm_debug_inject(int32_t mode, int64_t timeout_cycles) {
     g_debug.inject = mode;
     g_debug.timeout = timeout_cycles > 0 ? timeout_cycles : 0;
     return VDM_OK;
+}
+
+vdm_status vdm_debug_exp2(const float* d_x, float* d_y, int64_t n, vdm_stream stream) {
+    if (n < 0) return fail(VDM_ERR_INVALID_ARG, "n must be >= 0, got %lld", (long long)n);
+    if (n == 0) return VDM_OK;
+    if (!d_x || !d_y) return fail(VDM_ERR_INVALID_ARG, "null array");
+    const int64_t pairs = (n + 1) / 2;
+    const int64_t blocks = (pairs + 255) / 256;
+    if (blocks > 0x7fffffffLL) return fail(VDM_ERR_INVALID_ARG, "n too large: %lld", (long long)n);
+    exp2_poly_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(d_x, d_y, n);
+    return check_launch("exp2_poly_kernel");
 }
 
 vdm_status vdm_set_cta_pairs(int32_t enable) {

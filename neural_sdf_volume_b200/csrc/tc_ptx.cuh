@@ -408,9 +408,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // the low mantissa bits of x + 1.5 * 2^23, and f = x - n in [-1/2, 1/2]; 2^f by a cubic
 // whose coefficients were fitted for this function by iteratively reweighted least squares
 // (Lawson's minimax method) on [-1/2, 1/2]: relative error <= 7.5e-5 in fp32 Horner form,
-// below the bf16 rounding of the probabilities (2^-9); 2^n by adding n to the exponent
-// field.  Inputs are clamped below at -126, where the result is at most 2^-126 (not 0), so
-// the caller keeps masked (-inf) columns on ex2.
+// below the bf16 rounding of the probabilities (2^-9), for -125 <= x <= 9; 2^n by adding n
+// to the exponent field.  Inputs are clamped below at -126; below -125 the result is at most
+// 2^-124 (not 0, and inaccurate once it leaves the normal range), so the caller keeps masked
+// (-inf) columns on ex2.
 __device__ __forceinline__ uint64_t exp2_pair_poly(uint64_t x) {
     constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
     const auto splat = [](float c) { return f32x2(c, c); };
