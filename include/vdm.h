@@ -456,6 +456,15 @@ VDM_API vdm_status vdm_debug_inject(int32_t mode, int64_t timeout_cycles);
  * Asynchronous on `stream`.  Errors: INVALID_ARG, CUDA.                     */
 VDM_API vdm_status vdm_debug_exp2(const float* d_x, float* d_y, int64_t n, vdm_stream stream);
 
+/* Test hook for the decoder's GELU (not needed for decoding): for the n inputs
+ * d_x (device float32), d_y[i] = the tensor-core decoder's GELU of x_i as it
+ * feeds the MLP's second matrix (bf16, widened to float32; computed on pairs of
+ * inputs), and d_y[n + i] = the same GELU in scalar float32 before rounding.
+ * GELU(x) = x Phi(x), with erf by Abramowitz & Stegun formula 7.1.26 (absolute
+ * error <= 1.5e-7).  d_y holds 2 n floats.  Asynchronous on `stream`.
+ * Errors: INVALID_ARG, CUDA.                                                */
+VDM_API vdm_status vdm_debug_gelu(const float* d_x, float* d_y, int64_t n, vdm_stream stream);
+
 /* Tensor-core decoding on CTA pairs: with enable = 1, each 256-query MMA runs
  * on the two CTAs of a cluster (cta_group::2); each CTA holds 128 query rows
  * and loads half of every weight and key/value tile, which halves the bytes

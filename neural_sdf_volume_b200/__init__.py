@@ -39,7 +39,7 @@ EXPORTS = ("vdm_precompute_kv", "vdm_decode_dense", "vdm_select_kv",
            "vdm_surface_workspace_size", "vdm_extract_surface", "vdm_surface_case_table",
            "vdm_refine_workspace_size", "vdm_refine_level",
            "vdm_encode_workspace_size", "vdm_encode", "vdm_local_workspace_size", "vdm_decode_local",
-           "vdm_debug_inject", "vdm_debug_exp2", "vdm_set_cta_pairs",
+           "vdm_debug_inject", "vdm_debug_exp2", "vdm_debug_gelu", "vdm_set_cta_pairs",
            "vdm_profile_begin", "vdm_profile_end",
            "vdm_status_string", "vdm_last_error", "vdm_abi_version")
 PROF_CLASSES = ("kv", "decode", "select", "mark", "scan", "list", "fill", "probe")
@@ -134,6 +134,8 @@ _lib.vdm_debug_inject.argtypes = [_i32, _i64]
 _lib.vdm_debug_inject.restype = C.c_int
 _lib.vdm_debug_exp2.argtypes = [C.c_void_p, C.c_void_p, _i64, C.c_void_p]
 _lib.vdm_debug_exp2.restype = C.c_int
+_lib.vdm_debug_gelu.argtypes = [C.c_void_p, C.c_void_p, _i64, C.c_void_p]
+_lib.vdm_debug_gelu.restype = C.c_int
 _lib.vdm_set_cta_pairs.argtypes = [_i32]
 _lib.vdm_set_cta_pairs.restype = C.c_int
 _lib.vdm_profile_begin.argtypes = []
@@ -518,6 +520,18 @@ def vdm_debug_exp2(x, stream=None):
     y = torch.empty_like(x)
     _check(_lib.vdm_debug_exp2(x.data_ptr(), y.data_ptr(), x.numel(), _stream(stream)))
     return y
+
+
+def vdm_debug_gelu(x, stream=None):
+    """Test hook: the decoder's GELU of x (float32 CUDA tensor) as ``(bf16 pair form, float32 scalar form)``."""
+    import torch
+
+    x = x.contiguous()
+    if x.dtype != torch.float32 or not x.is_cuda:
+        raise ValueError("x must be a float32 CUDA tensor")
+    y = torch.empty(2 * x.numel(), dtype=torch.float32, device=x.device)
+    _check(_lib.vdm_debug_gelu(x.data_ptr(), y.data_ptr(), x.numel(), _stream(stream)))
+    return y[: x.numel()].view_as(x), y[x.numel():].view_as(x)
 
 
 def vdm_set_cta_pairs(enable: bool):

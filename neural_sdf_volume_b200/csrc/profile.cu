@@ -42,6 +42,20 @@ cudaEvent_t take() {
     return e;
 }
 
+// the decoder's GELU: the pair form that feeds the MLP (bf16) and the scalar form (float32)
+__global__ void gelu_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+    const int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : x0;
+    const uint32_t pk = ptx::gelu_as_pack(x0, x1);
+    y[i] = __uint_as_float(pk << 16);
+    y[n + i] = ptx::gelu_as(x0);
+    if (i + 1 < n) {
+        y[i + 1] = __uint_as_float(pk & 0xffff0000u);
+        y[n + i + 1] = ptx::gelu_as(x1);
+    }
+}
+
 }  // namespace
 
 void prof_begin(int cls, cudaStream_t s) {
@@ -82,6 +96,16 @@ vdm_status vdm_debug_exp2(const float* d_x, float* d_y, int64_t n, vdm_stream st
     if (blocks > 0x7fffffffLL) return fail(VDM_ERR_INVALID_ARG, "n too large: %lld", (long long)n);
     exp2_poly_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(d_x, d_y, n);
     return check_launch("exp2_poly_kernel");
+}
+
+vdm_status vdm_debug_gelu(const float* d_x, float* d_y, int64_t n, vdm_stream stream) {
+    if (n < 0) return fail(VDM_ERR_INVALID_ARG, "n must be >= 0, got %lld", (long long)n);
+    if (n == 0) return VDM_OK;
+    if (!d_x || !d_y) return fail(VDM_ERR_INVALID_ARG, "null array");
+    const int64_t blocks = ((n + 1) / 2 + 255) / 256;
+    if (blocks > 0x7fffffffLL) return fail(VDM_ERR_INVALID_ARG, "n too large: %lld", (long long)n);
+    gelu_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(d_x, d_y, n);
+    return check_launch("gelu_kernel");
 }
 
 vdm_status vdm_set_cta_pairs(int32_t enable) {
